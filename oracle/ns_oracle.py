@@ -1,0 +1,382 @@
+"""Plain, slow, fp64 CPU oracle for the Newton-Schulz msign family.
+
+TEST INFRASTRUCTURE ONLY. Nothing in the product package may import this
+module. Its only callers are the test-suite, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py``.  It shares
+no code, constants or tables with the CUDA path; the only thing both sides
+consume is the seeded input generator module, which holds none of the
+method's arithmetic.
+
+Sources (cited by page title and section/equation):
+
+* [P2] "msign算子的Newton-Schulz迭代（上）" (kexue.fm/archives/10922):
+  definition of msign via the SVD (eq. 1-2), the normalised start
+  X0 = M/||M||_F and the quintic iteration (eq. 4, 6), Jordan's
+  coefficients (eq. 7), the batched reference routine in section
+  "参考实现" (cast to bf16, transpose when rows > cols, eps inside the
+  square root), the scalar reduction in section "原理分析" and the per-step
+  coefficient idea in section "解开约束" (eq. 12).
+* [P3] "Gram Newton-Schulz" (zifeng-mai.github.io, 2026/04/05): the muon
+  update (section 1.1), FLOP accounting (sections 1.2, 2.4, 3.4),
+  Algorithm 1 (Naive Gram Newton-Schulz, section 2.3), Algorithm 2
+  (Stabilized Gram Newton-Schulz, section 3.4), Theorem 1 (section 2.2).
+
+Conventions (readings of the pages, each listed in the design doc):
+
+* Arithmetic is fp64 throughout.  The only roundings are the explicit
+  casts the pages prescribe: the input cast to the compute dtype of [P2]
+  "参考实现" (``input_cast='bf16'``) and the fp16 cast of step 2 of
+  Algorithm 2 in [P3] section 3.4 (``cast_fp16=True``).
+* Orientation: the iteration runs on the side with fewer rows; a matrix
+  with rows > cols is transposed first and transposed back at the end
+  (square matrices are not transposed) ([P2] "参考实现").
+* Standard NS normalises with sqrt(sum(x^2) + eps), eps = 1e-20 ([P2]
+  "参考实现"); Gram NS with ||X||_F + eps, eps = 1e-7 ([P3] Alg. 1 step 1,
+  Alg. 2 step 1).
+* Coefficients are a list of (a_t, b_t, c_t) triples, one per step; the
+  default is Jordan's triple repeated T = 5 times ([P2] eq. 7).
+
+Parity pins: every public function here is checked in
+``tests/test_oracle_*.py`` against closed forms, invariants, special cases
+and the figures the pages print; none is "parity unpinned" except the ones
+whose docstring says so.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Iterable, Sequence
+
+import numpy as np
+
+# Jordan's quintic coefficients and step count, [P2] eq. (7).
+JORDAN_ABC = (3.4445, -4.7750, 2.0315)
+JORDAN_STEPS = 5
+
+
+def jordan_schedule(steps: int = JORDAN_STEPS) -> list[tuple[float, float, float]]:
+    """Jordan's constant triple repeated ``steps`` times ([P2] eq. 7)."""
+    return [JORDAN_ABC] * steps
+
+
+# ----------------------------------------------------------------------------
+# Casts the pages prescribe (the only non-fp64 roundings in this oracle)
+# ----------------------------------------------------------------------------
+
+def round_to_bf16(x) -> np.ndarray:
+    """Round to the nearest bfloat16 value (ties to even); returns float64.
+
+    bfloat16 keeps the top 16 bits of an IEEE float32.  The input is first
+    taken as float32 (the inputs the method receives are float32 or already
+    bfloat16-valued), then the low 16 bits are rounded away: add 0x7FFF plus
+    the lowest kept bit, and clear the low half.  This is the cast of
+    ``x.astype('bfloat16')`` in [P2] "参考实现".
+    """
+    f = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    keep_lsb = (u >> np.uint64(16)) & np.uint64(1)
+    u = ((u + np.uint64(0x7FFF) + keep_lsb) >> np.uint64(16)) << np.uint64(16)
+    out = (u & np.uint64(0xFFFFFFFF)).astype(np.uint32).view(np.float32)
+    return out.astype(np.float64).reshape(f.shape)
+
+
+def round_to_fp16(x) -> np.ndarray:
+    """Round to the nearest IEEE half (ties to even); returns float64.
+
+    This is the ``float16(X)`` cast of [P3] Algorithm 2, step 2.
+    """
+    return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
+def _apply_input_cast(x, input_cast):
+    if input_cast is None:
+        return np.array(x, dtype=np.float64, copy=True)
+    if input_cast == "bf16":
+        return round_to_bf16(x)
+    if input_cast == "fp16":
+        return round_to_fp16(x)
+    raise ValueError(f"unknown input_cast {input_cast!r}")
+
+
+def _as_schedule(coeffs) -> list[tuple[float, float, float]]:
+    if coeffs is None:
+        return jordan_schedule()
+    sched = [tuple(float(v) for v in abc) for abc in coeffs]
+    for abc in sched:
+        if len(abc) != 3:
+            raise ValueError("each step needs an (a, b, c) triple")
+    return sched
+
+
+# ----------------------------------------------------------------------------
+# Closed forms
+# ----------------------------------------------------------------------------
+
+def msign_svd(M) -> np.ndarray:
+    """msign(M) = U[:, :r] V[:, :r]^T from the SVD ([P2] eq. 1).
+
+    Every non-zero singular value becomes 1; zero singular values stay 0.
+    Rank r is decided with the usual numerical threshold
+    max(shape) * eps * sigma_max.
+    """
+    M = np.asarray(M, dtype=np.float64)
+    U, s, Vt = np.linalg.svd(M, full_matrices=False)
+    if s.size == 0 or s[0] == 0.0:
+        return np.zeros_like(M)
+    tol = max(M.shape) * np.finfo(np.float64).eps * s[0]
+    r = int(np.sum(s > tol))
+    return U[:, :r] @ Vt[:r, :]
+
+
+def ns_scalar(x, coeffs=None) -> np.ndarray:
+    """The scalar map the iteration applies to each singular value.
+
+    x_{t+1} = a_t x_t + b_t x_t^3 + c_t x_t^5  ([P2] section 原理分析 and the
+    per-step form of section 解开约束).  Returns x_T for each entry of x.
+    """
+    x = np.asarray(x, dtype=np.float64).copy()
+    for a, b, c in _as_schedule(coeffs):
+        x = a * x + b * x ** 3 + c * x ** 5
+    return x
+
+
+def msign_ns_closed_form(M, coeffs=None, eps: float = 1e-20) -> np.ndarray:
+    """U phi_T(Sigma / ||M||_F) V^T: what T exact NS steps return.
+
+    [P2] section 原理分析 (and [P3] Proposition 1): the iteration keeps the
+    singular vectors and maps every normalised singular value through the
+    scalar polynomial composed T times.  Uses the same eps convention as
+    ``msign_ns`` so the two agree to rounding.
+    """
+    M = np.asarray(M, dtype=np.float64)
+    U, s, Vt = np.linalg.svd(M, full_matrices=False)
+    nrm = math.sqrt(float(np.sum(M * M)) + eps)
+    return (U * ns_scalar(s / nrm, coeffs)) @ Vt
+
+
+# ----------------------------------------------------------------------------
+# Standard Newton-Schulz msign
+# ----------------------------------------------------------------------------
+
+def msign_ns(M, coeffs=None, eps: float = 1e-20, input_cast=None) -> np.ndarray:
+    """Quintic Newton-Schulz msign, batched over leading dims, in fp64.
+
+    Steps ([P2] eq. 4 and 6, section 参考实现):
+      1. cast the input to the compute dtype (``input_cast``; None = none);
+      2. if rows > cols work on the transpose (the side with the smaller
+         Gram matrix);
+      3. X = X / sqrt(sum(X^2) + eps);
+      4. for each (a, b, c):  A = X X^T;  B = b A + c A A;  X = a X + B X
+         (the left form of the quintic, as in the flash-muon post of
+         nil9.net, which is the same polynomial as [P2] eq. 6 written on
+         the other side);
+      5. transpose back.
+    """
+    X = _apply_input_cast(M, input_cast)
+    if X.ndim < 2:
+        raise ValueError("msign needs at least a matrix")
+    flip = X.shape[-2] > X.shape[-1]
+    if flip:
+        X = np.swapaxes(X, -1, -2)
+    X = np.array(X, dtype=np.float64, copy=True)
+    norm = np.sqrt(np.sum(X * X, axis=(-2, -1), keepdims=True) + eps)
+    X = X / norm
+    XT = lambda Y: np.swapaxes(Y, -1, -2)  # noqa: E731
+    for a, b, c in _as_schedule(coeffs):
+        A = X @ XT(X)
+        B = b * A + c * (A @ A)
+        X = a * X + B @ X
+    if flip:
+        X = XT(X)
+    return np.ascontiguousarray(X)
+
+
+# ----------------------------------------------------------------------------
+# Gram product
+# ----------------------------------------------------------------------------
+
+def gram_xxt(X) -> np.ndarray:
+    """A = X X^T, batched over leading dims, fp64 (the symmetric Gram
+    product of the flash-muon ``matmul_transpose`` post, nil9.net).
+    The result is symmetrised by construction: entry (i, j) and (j, i)
+    are the same dot product, so the oracle returns exactly symmetric A."""
+    X = np.asarray(X, dtype=np.float64)
+    A = X @ np.swapaxes(X, -1, -2)
+    upper = np.triu(np.ones(A.shape[-2:], dtype=bool))
+    return np.where(upper, A, np.swapaxes(A, -1, -2))
+
+
+def gram_xxt_bruteforce(X) -> np.ndarray:
+    """Triple loop version of X X^T for tiny inputs (a pin for gram_xxt)."""
+    X = np.asarray(X, dtype=np.float64)
+    n, m = X.shape
+    A = np.zeros((n, n))
+    for i in range(n):
+        for j in range(n):
+            acc = 0.0
+            for k in range(m):
+                acc += X[i, k] * X[j, k]
+            A[i, j] = acc
+    return A
+
+
+# ----------------------------------------------------------------------------
+# Gram Newton-Schulz ([P3] sections 2.3 and 3.4)
+# ----------------------------------------------------------------------------
+
+def _orient(X):
+    flip = X.shape[-2] > X.shape[-1]
+    return (np.swapaxes(X, -1, -2) if flip else X), flip
+
+
+def gram_ns_naive(M, coeffs=None, eps: float = 1e-7, input_cast=None) -> np.ndarray:
+    """[P3] Algorithm 1 (Naive Gram Newton-Schulz), fp64.
+
+      X <- X / (||X||_F + eps);  R_0 = X X^T;  Q_0 = I;
+      for t: Z_t = a_t I + b_t R + c_t R^2;  Q_t = Q_{t-1} Z_t;
+             R_t = Z_t R_{t-1} Z_t;
+      return Q_T X.
+    Wide orientation (n <= m) as in the standard routine.
+    """
+    X, flip = _orient(_apply_input_cast(M, input_cast))
+    X = np.array(X, dtype=np.float64)
+    n = X.shape[-2]
+    I = np.eye(n)
+    X = X / (np.sqrt(np.sum(X * X, axis=(-2, -1), keepdims=True)) + eps)
+    R = X @ np.swapaxes(X, -1, -2)
+    Q = np.broadcast_to(I, R.shape).copy()
+    for a, b, c in _as_schedule(coeffs):
+        Z = a * I + b * R + c * (R @ R)
+        Q = Q @ Z
+        R = Z @ R @ Z
+    out = Q @ X
+    return np.swapaxes(out, -1, -2) if flip else out
+
+
+def gram_ns(M, coeffs=None, restart_after: Iterable[int] = (2,), eps: float = 1e-7,
+            input_cast=None, cast_fp16: bool = True) -> np.ndarray:
+    """[P3] Algorithm 2 (Stabilized Gram Newton-Schulz), fp64 arithmetic.
+
+      1. X <- X / (||X||_F + eps)
+      2. X <- float16(X)                     (``cast_fp16``)
+      3. for each segment of steps between restarts:
+           R <- X X^T ;  Q <- I
+           for t in the segment:
+             Z  <- b_t R + c_t R^2
+             Q  <- Q Z + a_t Q
+             RZ <- R Z + a_t R
+             R  <- Z RZ + a_t RZ
+           X <- Q X                          (the restart)
+      4. return X  (= Q X of the last segment)
+    ``restart_after`` lists the step numbers after which the Gram matrix is
+    recomputed; the page's schedule restarts after step 2 ([P3] section
+    3.2).  An empty list gives the unrestarted iteration, and restarting
+    after every step reproduces standard NS ([P3] end of section 3.4).
+    Every product written in the algorithm is performed, including Q = I Z
+    at the first step of a segment; skipping it is a FLOP saving the page
+    describes, not a change of result.
+    """
+    sched = _as_schedule(coeffs)
+    T = len(sched)
+    cuts = sorted({int(t) for t in restart_after if 0 < int(t) < T})
+    bounds = [0] + cuts + [T]
+    X, flip = _orient(_apply_input_cast(M, input_cast))
+    X = np.array(X, dtype=np.float64)
+    n = X.shape[-2]
+    I = np.eye(n)
+    XT = lambda Y: np.swapaxes(Y, -1, -2)  # noqa: E731
+    X = X / (np.sqrt(np.sum(X * X, axis=(-2, -1), keepdims=True)) + eps)
+    if cast_fp16:
+        X = round_to_fp16(X)
+    for s0, s1 in zip(bounds[:-1], bounds[1:]):
+        R = X @ XT(X)
+        Q = np.broadcast_to(I, R.shape).copy()
+        for a, b, c in sched[s0:s1]:
+            Z = b * R + c * (R @ R)
+            Q = Q @ Z + a * Q
+            RZ = R @ Z + a * R
+            R = Z @ RZ + a * RZ
+        X = Q @ X
+    return XT(X) if flip else X
+
+
+def gram_ns_scalar(x, coeffs=None):
+    """[P3] Theorem 1 in scalar form: r_0 = x^2, q_0 = 1,
+    z_t = h_t(r_{t-1}) with h_t(y) = a_t + b_t y + c_t y^2 (Lemma 1),
+    q_t = q_{t-1} z_t, r_t = r_{t-1} z_t^2.  Returns (q_T, r_T)."""
+    x = np.asarray(x, dtype=np.float64)
+    r = x * x
+    q = np.ones_like(x)
+    for a, b, c in _as_schedule(coeffs):
+        z = a + b * r + c * r * r
+        q = q * z
+        r = r * z * z
+    return q, r
+
+
+# ----------------------------------------------------------------------------
+# Muon update ([P3] section 1.1, formula lost in extraction; reading below)
+# ----------------------------------------------------------------------------
+
+def muon_step(W, M, G, momentum: float = 0.95, lr: float = 0.02, coeffs=None,
+              eps: float = 1e-20, input_cast="bf16"):
+    """One Muon update of one weight matrix, fp64.
+
+    M <- momentum * M + G;  O = msign_NS(M);  W <- W - lr * sqrt(max(1, rows/cols)) * O.
+    The momentum recursion with M_0 = 0 is the one [P3] section 1.1 names
+    (mu, eta); the sqrt(max(1, rows/cols)) factor is the spectral scaling
+    of the Muon update used by the Llama-shaped workload.  Returns
+    (W_new, M_new, O).
+    """
+    W = np.asarray(W, dtype=np.float64)
+    M_new = momentum * np.asarray(M, dtype=np.float64) + np.asarray(G, dtype=np.float64)
+    O = msign_ns(M_new, coeffs=coeffs, eps=eps, input_cast=input_cast)
+    rows, cols = W.shape[-2], W.shape[-1]
+    scale = math.sqrt(max(1.0, rows / cols))
+    return W - lr * scale * O, M_new, O
+
+
+# ----------------------------------------------------------------------------
+# FLOP bookkeeping ([P3] sections 1.2, 2.4, 3.4)
+# ----------------------------------------------------------------------------
+
+def ns_flops(n: int, m: int, steps: int = 5, symmetric: bool = True) -> float:
+    """FLOPs of standard NS on an n x m matrix (n <= m).
+
+    Per step ([P3] section 1.2): X X^T costs 2 m n^2, A^2 costs 2 n^3 and
+    B X costs 2 m n^2.  With symmetric products (only one triangle of the
+    two symmetric outputs is needed) the first two halve, giving
+    T (3 alpha + 1) n^3 in total ([P3] section 2.4)."""
+    sym = 0.5 if symmetric else 1.0
+    per = sym * 2 * m * n * n + sym * 2 * n ** 3 + 2 * m * n * n
+    return steps * per
+
+
+def gram_ns_plan(n: int, m: int, steps: int = 5, restart_after: Sequence[int] = (2,)):
+    """The list of products a Gram-NS run performs after the savings the
+    page lists, with their FLOP cost under the symmetric-GEMM model.
+
+    Per step ([P3] section 2.4): R^2 costs n^3, Q Z costs n^3, Z R Z costs
+    2 n^3 (as R Z then Z (R Z)).  Start and end: X X^T costs m n^2 and
+    Q X costs 2 m n^2.  Savings: the first Q Z of a segment is Q = Z
+    (Q = I), and the last R update of a segment is never used.  A restart
+    adds Q X (2 m n^2) and X X^T (m n^2) ([P3] section 3.4).
+    Returns a list of (name, flops)."""
+    cuts = sorted({int(t) for t in restart_after if 0 < int(t) < steps})
+    bounds = [0] + cuts + [steps]
+    plan = []
+    for s0, s1 in zip(bounds[:-1], bounds[1:]):
+        plan.append(("XXt", m * n * n))
+        for t in range(s0, s1):
+            plan.append((f"R2[{t + 1}]", n ** 3))
+            if t != s0:
+                plan.append((f"QZ[{t + 1}]", n ** 3))
+            if t != s1 - 1:
+                plan.append((f"RZ[{t + 1}]", n ** 3))
+                plan.append((f"ZRZ[{t + 1}]", n ** 3))
+        plan.append(("QX", 2 * m * n * n))
+    return plan
+
+
+def gram_ns_flops(n: int, m: int, steps: int = 5, restart_after: Sequence[int] = (2,)) -> float:
+    return float(sum(f for _, f in gram_ns_plan(n, m, steps, restart_after)))
