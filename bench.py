@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark of the hot path: one 5-step Newton-Schulz msign of a 4096 x 4096
+bf16 matrix (Jordan's coefficients), reported as ms per msign call and
+useful TFLOP/s against the measured dense BF16 tensor-core peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1).  Every rank runs its own msign
+calls on its own matrix (the problems are independent: weak scaling, no
+collective on the data path); the step time is the max over ranks.
+
+Timing: W untimed warm-up calls, then K timed calls.  Before each timed call
+an L2 flush writes a 256 MiB buffer (larger than the 126 MB L2); each call is
+bracketed by CUDA events on the launching stream and the K durations are
+summed.  The library's launch records time every kernel of the timed calls
+on the same stream for the roofline of the dominant kernel.
+
+The reference arm (--impl reference) times the fp64 CPU oracle on the host
+cores, rank 0 only, on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ms per msign call and useful TFLOP/s (% of B200 dense BF16 peak), 4096² bf16"
+N_ROWS = N_COLS = 4096
+T_STEPS = 5
+FLUSH_BYTES = 256 << 20
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of gemm_sm100_kernel,
+# averaged over the 15 GEMM launches of one 4096^2 msign call, from the ncu
+# capture summarised in profiles/gemm_sm100_msign4096.md; valid only for the
+# kernel source whose hash is recorded with it.
+NCU_TRAFFIC = {"bytes_per_launch": None, "kernel_sha": None}
+
+
+def useful_flops(n: int, m: int, steps: int) -> float:
+    """Triangle-counted useful FLOPs of one NS call on an oriented n x m matrix:
+    per step X X^T (m n (n+1)), A A (n^2 (n+1)) and B X (2 n^2 m)."""
+    return float(steps * (m * n * (n + 1) + n * n * (n + 1) + 2 * n * n * m))
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("gemm_sm100.cuh", "ptx_sm100.cuh"):
+        with open(os.path.join(ROOT, "newton_schulz_msign_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"bf16_tflops": d.get("bf16_tflops"), "bf16_tflops_sustained": d.get("bf16_tflops_sustained"),
+                "hbm_gbs": d.get("hbm_gbs"), "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- ranks
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(world: int, backend: str = "nccl"):
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity on one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Polls NVML (read-only) every 20 ms: SM clock, max SM clock, power and
+    the active clock-event reasons, for the duration of the timed region."""
+
+    REASONS = {
+        "hw_slowdown": 0x0000000000000008,
+        "hw_thermal_slowdown": 0x0000000000000040,
+        "hw_power_brake_slowdown": 0x0000000000000080,
+        "sw_thermal_slowdown": 0x0000000000000020,
+        "sw_power_cap": 0x0000000000000004,
+    }
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no clocks rather than fail the run
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                power = nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+                self.samples.append((mhz, reasons, power))
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def start(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self) -> dict:
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        reasons = sorted({name for _, r, _ in self.samples for name, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "power_w_max": max(s[2] for s in self.samples)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def time_oracle(target_s: float = 20.0):
+    """Times the fp64 oracle's msign on the host.  Runs 4096^2 itself when a
+    1024^2 probe predicts it fits in ~target_s, else the largest power-of-two
+    size that does, scaled by the FLOP ratio.  Returns (ms per 4096^2 call,
+    cores, sample description)."""
+    import numpy as np
+
+    from oracle import ns_oracle as O
+
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count() or 1])
+    except Exception:
+        cores = os.cpu_count() or 1
+
+    def run(n):
+        x = np.random.default_rng(0).standard_normal((n, n)).astype(np.float32)
+        t0 = time.perf_counter()
+        O.msign_ns(x, input_cast="bf16")
+        return time.perf_counter() - t0
+
+    n = 1024
+    t = run(n)
+    while n < N_ROWS and t * 8 < target_s:
+        n *= 2
+        t = run(n)
+    scale = useful_flops(N_ROWS, N_COLS, T_STEPS) / useful_flops(n, n, T_STEPS)
+    desc = (f"one {n}x{n} fp64 NS msign (5 steps) on the host"
+            + ("" if n == N_ROWS else f", scaled x{scale:.0f} by the FLOP ratio to 4096^2"))
+    return t * scale * 1e3, cores, desc, t
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import newton_schulz_msign_b200 as msb
+    from newton_schulz_msign_b200 import synth
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init(world)
+    stream = torch.cuda.current_stream()
+
+    x = synth.momentum_like_torch(N_ROWS, N_COLS, seed=1000 + rank, device=dev).to(torch.bfloat16).contiguous()
+    out = torch.empty_like(x)
+    ws = torch.empty(msb.msign_ns_workspace_size(1, N_ROWS, N_COLS), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    for _ in range(args.warmup):
+        msb.msign_ns(x, out, workspace=ws)
+    msb.sync_status()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    msb.profile_reset()
+    msb.profile_enable(True)
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        ev[k][0].record(stream)
+        msb.msign_ns(x, out, workspace=ws)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    msb.profile_enable(False)
+    msb.sync_status()
+    per_call = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(per_call)
+    kinds = {k: msb.profile_read(k) for k in ("gemm", "norm", "ingest", "elementwise")}
+    msb.profile_reset()
+
+    # end to end through the public call with host buffers: pinned input
+    # copied in and the result copied out inside the timed region
+    host_in = x.cpu().pin_memory()
+    host_out = torch.empty_like(host_in).pin_memory()
+    dev_in = torch.empty_like(x)
+    for _ in range(2):
+        dev_in.copy_(host_in, non_blocking=True)
+        msb.msign_ns(dev_in, out, workspace=ws)
+        host_out.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        e2e_ev[k][0].record(stream)
+        dev_in.copy_(host_in, non_blocking=True)
+        msb.msign_ns(dev_in, out, workspace=ws)
+        host_out.copy_(out, non_blocking=True)
+        e2e_ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    msb.sync_status()
+
+    max_total = max_over_ranks(total_ms, world, dev)
+    max_e2e = max_over_ranks(e2e_ms, world, dev)
+    units = world * args.steps
+    ms_per_call = max_total / units
+    e2e_per_call = max_e2e / units
+    flops = useful_flops(N_ROWS, N_COLS, T_STEPS)
+    tflops = flops * units / (max_total / 1e3) / 1e12
+
+    peaks = measured_peaks()
+    g = kinds["gemm"]
+    achieved = g["flops"] / (g["ms"] / 1e3) / 1e12 if g["ms"] > 0 else None
+    traffic = NCU_TRAFFIC["bytes_per_launch"] if NCU_TRAFFIC["kernel_sha"] == kernel_sha() else None
+    roofline = {
+        "bound": "tensor", "kernel": "gemm_sm100_kernel", "achieved": achieved, "peak": peaks["bf16_tflops"],
+        "unit": "TFLOP/s", "frac": (achieved / peaks["bf16_tflops"]) if achieved else None, "traffic": traffic,
+        "peak_source": f"{peaks['source']} bf16 burst",
+        "launches": g["launches"], "avg_launch_ms": g["ms"] / max(g["launches"], 1),
+        "flops_per_launch": g["flops"] / max(g["launches"], 1),
+        "share_of_call_time": g["ms"] / total_ms if total_ms > 0 else None,
+    }
+    launches = sum(v["launches"] for v in kinds.values())
+
+    result = {
+        "metric": METRIC, "value": ms_per_call, "unit": "ms/call", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_call * world, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "msign_ns 4096x4096 bf16, 5-step quintic NS, Jordan (3.4445, -4.7750, 2.0315)",
+                   "rows": N_ROWS, "cols": N_COLS, "ns_steps": T_STEPS, "batch_per_gpu": 1,
+                   "input": "momentum-like U diag(i^-0.8) V^T + N(0,1e-3^2) noise, seed 1000+rank",
+                   "l2": "flushed (256 MiB write) before every timed call", "parallelism": f"replicas x{world}"},
+        "useful_tflops": tflops, "frac_of_peak": tflops / peaks["bf16_tflops"],
+        "useful_flops_per_call": flops,
+        "roofline": roofline,
+        "e2e": {"value": e2e_per_call, "unit": "ms/call", "h2d_bytes_per_step": host_in.numel() * 2,
+                "d2h_bytes_per_step": host_out.numel() * 2},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "other_kernels": {k: {"launches": v["launches"], "ms": v["ms"], "bytes": v["bytes"]}
+                          for k, v in kinds.items() if k != "gemm"},
+        "per_call_ms": {"min": min(per_call), "median": statistics.median(per_call), "max": max(per_call)},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ms, cores, desc, secs = time_oracle()
+        result["cpu_baseline"] = {"value": ms, "unit": "ms/call", "cores": cores, "kind": "oracle", "sample": desc,
+                                  "sample_seconds": secs}
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+
+    from oracle import ns_oracle as O
+
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count() or 1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    # each step: one bounded sample of the workload, an n x n fp64 NS msign,
+    # with n chosen so the whole run stays within a few minutes
+    budget_s = 150.0
+    n = 512
+    x = np.random.default_rng(0).standard_normal((n, n)).astype(np.float32)
+    t0 = time.perf_counter()
+    O.msign_ns(x, input_cast="bf16")
+    t = time.perf_counter() - t0
+    while n < N_ROWS and t * 8 * (args.steps + args.warmup) < budget_s:
+        n *= 2
+        x = np.random.default_rng(0).standard_normal((n, n)).astype(np.float32)
+        t0 = time.perf_counter()
+        O.msign_ns(x, input_cast="bf16")
+        t = time.perf_counter() - t0
+    x = np.random.default_rng(0).standard_normal((n, n)).astype(np.float32)
+    for _ in range(args.warmup):
+        O.msign_ns(x, input_cast="bf16")
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.msign_ns(x, input_cast="bf16")
+        times.append(time.perf_counter() - t0)
+    scale = useful_flops(N_ROWS, N_COLS, T_STEPS) / useful_flops(n, n, T_STEPS)
+    ms = sum(times) / len(times) * scale * 1e3
+    sample = (f"one {n}x{n} fp64 NS msign per step on {cores} host threads"
+              + ("" if n == N_ROWS else f", scaled x{scale:.0f} by the FLOP ratio to 4096^2"))
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": ms, "unit": "ms/call", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "msign_ns 4096x4096, 5-step quintic NS, Jordan (3.4445, -4.7750, 2.0315)",
+                   "rows": N_ROWS, "cols": N_COLS, "ns_steps": T_STEPS, "parallelism": "host cores"},
+        "cpu_baseline": {"value": ms, "unit": "ms/call", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": ms, "unit": "ms/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the host oracle timing")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

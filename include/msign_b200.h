@@ -1,0 +1,211 @@
+/*
+ * msign_b200.h - C ABI of the B200 (sm_100a) Newton-Schulz msign library.
+ *
+ * The operation is msign(M) = (M M^T)^{-1/2} M = U V^T, the polar factor of
+ * M, approximated by the quintic Newton-Schulz iteration that the Muon
+ * optimizer uses.  Sources, cited by page title and section:
+ *
+ *   [P1] nil9.net blog, flash-muon post: the symmetric X X^T operator
+ *        ("matmul_transpose") that computes one triangle and mirrors it.
+ *   [P2] "msign算子的Newton-Schulz迭代（上）" (kexue.fm/archives/10922):
+ *        definition (eq. 1-2), iteration X0 = M/||M||_F,
+ *        X <- aX + bX(X^T X) + cX(X^T X)^2 (eq. 4, 6), Jordan's
+ *        coefficients (a,b,c) = (3.4445, -4.7750, 2.0315), T = 5 (eq. 7),
+ *        batched routine with bf16 cast, transpose when rows > cols and
+ *        eps = 1e-20 under the square root (section 参考实现), per-step
+ *        coefficients (section 解开约束, eq. 12).
+ *   [P3] "Gram Newton-Schulz" (zifeng-mai.github.io, 2026/04/05): Muon
+ *        update (section 1.1), Algorithm 2 "Stabilized Gram Newton-Schulz"
+ *        (section 3.4) with its restart (section 3.2), fp16 arithmetic
+ *        (section 3.3), and the fused symmetric kernel C <- aAB + bC + gI
+ *        (section 4).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Matrices are dense, row-major, batched back to back: matrix i of a batch
+ *   of rows x cols starts at element i*rows*cols.  All pointers passed as
+ *   matrices are DEVICE pointers unless stated otherwise.
+ * - The caller owns every buffer.  The library allocates nothing: it works
+ *   in the caller's workspace, whose size the *_workspace_size() query gives
+ *   (a workspace must be 256-byte aligned).  Inputs are never written
+ *   unless stated.  Outputs must not overlap inputs or the workspace.
+ * - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *   the legacy default stream).  Argument checks happen on the host before
+ *   anything is enqueued; on any error status nothing has been enqueued,
+ *   except for MSIGN_ERR_CUDA, which reports a failed launch.
+ * - Kernels never wait without a time limit.  A wait that runs out sets a
+ *   device-side error word and the kernel returns; msign_sync_status()
+ *   reports it as MSIGN_ERR_TIMEOUT.
+ * - Coefficient schedules are HOST arrays.  NULL selects Jordan's triple
+ *   for T = 5 steps ([P2] eq. 7).
+ * - Empty problems (batch, rows or cols = 0) are valid and do nothing.
+ */
+#ifndef MSIGN_B200_H
+#define MSIGN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *msign_stream_t;
+
+typedef enum {
+  MSIGN_OK = 0,
+  MSIGN_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad coefficient count */
+  MSIGN_ERR_UNSUPPORTED = 2,  /* dtype combination or size outside what is built */
+  MSIGN_ERR_WORKSPACE = 3,    /* workspace missing, too small or misaligned */
+  MSIGN_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed */
+  MSIGN_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (see msign_sync_status) */
+} msign_status;
+
+typedef enum {
+  MSIGN_BF16 = 0,
+  MSIGN_FP16 = 1,
+  MSIGN_FP32 = 2
+} msign_dtype;
+
+/* Coefficient schedule: steps triples (a_t, b_t, c_t), one per iteration,
+ * laid out a_1 b_1 c_1 a_2 b_2 c_2 ... in a HOST array.  abc == NULL means
+ * Jordan's triple repeated `steps` times (steps <= 0 then means 5).
+ * eps < 0 selects the default of the routine (1e-20 for msign_ns, 1e-7 for
+ * gram_ns). */
+typedef struct {
+  int steps;
+  const float *abc;
+  float eps;
+} msign_coeffs;
+
+/* Library ABI version (major * 100 + minor). */
+int msign_abi_version(void);
+
+/* Human-readable name of a status code (static storage). */
+const char *msign_status_string(msign_status status);
+
+/* Waits for `stream`, then reads and clears the device-side error word that
+ * bounded waits set.  Returns MSIGN_OK, MSIGN_ERR_TIMEOUT, or
+ * MSIGN_ERR_CUDA if the stream reports an error. */
+msign_status msign_sync_status(msign_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Launch records, for benchmarks (no counterpart on the pages).
+ *
+ * msign_profile_enable(1) makes every later kernel launch of the library
+ * record a CUDA event on its stream before and after the kernel, tagged with
+ * a kind and with the launch's algorithmic work: useful FLOPs (symmetric
+ * outputs count one triangle) and compulsory HBM bytes (operands, epilogue
+ * input and outputs once each).  msign_profile_read() waits for the records
+ * of one kind and returns their count, summed device time in milliseconds,
+ * FLOPs and bytes; msign_profile_reset() drops all records.  Kinds: 0 =
+ * tensor-core GEMM, 1 = Frobenius-norm reduction, 2 = cast/orient/scale
+ * ingest, 3 = Muon elementwise (momentum, weight update).  Not thread-safe
+ * with concurrent library calls on other host threads.
+ * ------------------------------------------------------------------------ */
+msign_status msign_profile_enable(int enable);
+
+msign_status msign_profile_read(int kind, int *launches, double *total_ms, double *flops, double *bytes);
+
+msign_status msign_profile_reset(void);
+
+/* ------------------------------------------------------------------------
+ * msign_ns: batched standard Newton-Schulz msign ([P2] eq. 4-7, section
+ * 参考实现).
+ *
+ * For each of `batch` matrices M (rows x cols): cast to the compute dtype,
+ * work on M^T when rows > cols, X0 = M / sqrt(sum(M^2) + eps), then for
+ * t = 1..T:  A = X X^T;  B = b_t A + c_t A A;  X = a_t X + B X;  finally
+ * transpose back and write X in io_dtype.
+ *
+ *   in, out        device pointers, batch x rows x cols in io_dtype
+ *   io_dtype       MSIGN_BF16, MSIGN_FP16 or MSIGN_FP32
+ *   compute_dtype  MSIGN_BF16: bf16 tensor-core operands, fp32 accumulation,
+ *                  fp32 epilogue arithmetic and an fp32 copy of X between
+ *                  steps.  (MSIGN_FP32 is reserved for the fp32-accurate
+ *                  path and returns MSIGN_ERR_UNSUPPORTED when not built.)
+ *   coeffs         schedule (NULL: Jordan, T = 5, eps = 1e-20)
+ *   workspace      device scratch of at least msign_ns_workspace_size() bytes
+ * ------------------------------------------------------------------------ */
+size_t msign_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute_dtype);
+
+msign_status msign_ns(const void *in, void *out, msign_dtype io_dtype, msign_dtype compute_dtype,
+                      int64_t batch, int64_t rows, int64_t cols, const msign_coeffs *coeffs,
+                      void *workspace, size_t workspace_bytes, msign_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * gram_xxt: symmetric Gram product A = X X^T ([P1] flash-muon
+ * matmul_transpose; [P3] section 4, triangular scheduling).
+ *
+ * Only output tiles on or above the diagonal are computed; each is stored
+ * and its transpose is stored into the mirrored position from the same
+ * fp32 accumulators, so A is bit-exactly symmetric.
+ *
+ *   X   device pointer, batch x n x m, dtype x_dtype (MSIGN_BF16 or MSIGN_FP16)
+ *   A   device pointer, batch x n x n, dtype a_dtype (BF16, FP16 or FP32)
+ *   workspace  needed only when X is not 16-byte aligned or m is not a
+ *              multiple of 8 (X is then staged into the workspace); the
+ *              query returns 0 otherwise.
+ * ------------------------------------------------------------------------ */
+size_t gram_xxt_workspace_size(int64_t batch, int64_t n, int64_t m, msign_dtype x_dtype, const void *X);
+
+msign_status gram_xxt(const void *X, msign_dtype x_dtype, void *A, msign_dtype a_dtype,
+                      int64_t batch, int64_t n, int64_t m,
+                      void *workspace, size_t workspace_bytes, msign_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * gram_ns: batched Stabilized Gram Newton-Schulz ([P3] Algorithm 2,
+ * sections 3.2-3.4).
+ *
+ * For each matrix (oriented so that n <= m as in msign_ns):
+ * X <- X / (||X||_F + eps); X <- float16(X); then for each segment of steps
+ * between restarts: R = X X^T, Q = I; per step Z = b R + c R^2,
+ * Q <- QZ + aQ, RZ <- RZ + aR, R <- Z RZ + a RZ; then X <- Q X.  The n x n
+ * products are symmetric (polynomials in one Gram matrix) and use the
+ * triangle schedule; the a_t terms are added in fp32 epilogues.  Operands
+ * are fp16, accumulation fp32.
+ *
+ *   restart_after  HOST array of step numbers after which to restart
+ *                  (values in 1..T-1); NULL with n_restart < 0 selects the
+ *                  page's schedule {2}; n_restart == 0 means no restart.
+ * ------------------------------------------------------------------------ */
+size_t gram_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols);
+
+msign_status gram_ns(const void *in, void *out, msign_dtype io_dtype,
+                     int64_t batch, int64_t rows, int64_t cols, const msign_coeffs *coeffs,
+                     const int *restart_after, int n_restart,
+                     void *workspace, size_t workspace_bytes, msign_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * muon_step: one Muon update of a list of weight matrices ([P3] section
+ * 1.1; momentum M_0 = 0, no Nesterov term, no weight decay).
+ *
+ * For each matrix i (rows[i] x cols[i]):
+ *   M_i <- momentum * M_i + G_i                           (fp32)
+ *   O_i  = msign_ns(M_i)  with bf16 compute, `coeffs` schedule
+ *   W_i <- W_i - lr * sqrt(max(1, rows_i / cols_i)) * O_i
+ * Matrices of equal (oriented) shape share grouped launches; all shapes in
+ * one call are scheduled together.
+ *
+ *   W, M, G     HOST arrays of `num` DEVICE pointers.  W_i in w_dtype
+ *               (BF16 or FP32) is updated in place; M_i is fp32 and updated
+ *               in place; G_i is in g_dtype (BF16 or FP32) and read only.
+ *   rows, cols  HOST arrays of `num` sizes.
+ *   workspace   at least muon_step_workspace_size() bytes; a smaller one
+ *               (but at least the size for the largest single matrix) makes
+ *               the call process the list in several groups.
+ * ------------------------------------------------------------------------ */
+size_t muon_step_workspace_size(int num, const int64_t *rows, const int64_t *cols);
+
+msign_status muon_step(int num, void *const *W, float *const *M, const void *const *G,
+                       const int64_t *rows, const int64_t *cols,
+                       msign_dtype w_dtype, msign_dtype g_dtype,
+                       float momentum, float lr, const msign_coeffs *coeffs,
+                       void *workspace, size_t workspace_bytes, msign_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSIGN_B200_H */

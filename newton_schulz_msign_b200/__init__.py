@@ -1,0 +1,228 @@
+"""B200 (sm_100a) Newton-Schulz msign: thin PyTorch binding of the C ABI.
+
+Each function marshals tensors into the pointer/size arguments of the C entry
+point of the same name (include/msign_b200.h) and enqueues it on the current
+CUDA stream.  Every step of the computation runs in the library's kernels;
+PyTorch only supplies device memory and the stream.  There is no CPU path:
+calling these without the built library or without a CUDA tensor raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+
+from . import _lib
+from ._lib import BF16, FP16, FP32, MsignError, check, make_coeffs
+
+__all__ = [
+    "MsignError", "msign_ns", "msign_ns_workspace_size", "gram_xxt", "gram_xxt_workspace_size", "gram_ns",
+    "gram_ns_workspace_size", "muon_step", "muon_step_workspace_size", "sync_status", "library_path",
+]
+
+
+def library_path() -> str:
+    return _lib.LIB_PATH
+
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    m = {torch.bfloat16: BF16, torch.float16: FP16, torch.float32: FP32}
+    if t.dtype not in m:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return m[t.dtype]
+
+
+def _compute_code(name) -> int:
+    return {"bf16": BF16, "fp16": FP16, "fp32": FP32}[name]
+
+
+def _stream(stream) -> int:
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _need_cuda(t, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _workspace(nbytes, device, workspace):
+    torch = _torch()
+    if nbytes == 0:
+        return workspace, (0 if workspace is None else workspace.numel() * workspace.element_size())
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def sync_status(stream=None) -> None:
+    """Waits for the stream and raises MsignError if a kernel's bounded wait ran out."""
+    check(_lib.lib().msign_sync_status(_stream(stream)), "msign_sync_status")
+
+
+# ---------------------------------------------------------------- msign_ns
+
+def msign_ns_workspace_size(batch: int, rows: int, cols: int, compute: str = "bf16") -> int:
+    return int(_lib.lib().msign_ns_workspace_size(batch, rows, cols, _compute_code(compute)))
+
+
+def msign_ns(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, workspace=None, stream=None):
+    """Newton-Schulz msign of the last two dims of ``x`` (bf16/fp16/fp32 CUDA tensor)."""
+    torch = _torch()
+    _need_cuda(x, "x")
+    if x.dim() < 2:
+        raise ValueError("x needs at least two dims")
+    rows, cols = x.shape[-2], x.shape[-1]
+    batch = math.prod(x.shape[:-2])
+    if out is None:
+        out = torch.empty_like(x)
+    _need_cuda(out, "out")
+    if out.shape != x.shape or out.dtype != x.dtype:
+        raise ValueError("out must match x in shape and dtype")
+    ws, wsb = _workspace(msign_ns_workspace_size(batch, rows, cols, compute), x.device, workspace)
+    c, keep = make_coeffs(coeffs, eps)
+    st = _lib.lib().msign_ns(x.data_ptr(), out.data_ptr(), _dtype_code(x), _compute_code(compute), batch, rows,
+                             cols, ctypes.byref(c) if c is not None else None, _ptr(ws), wsb, _stream(stream))
+    del keep
+    check(st, "msign_ns")
+    return out
+
+
+# ---------------------------------------------------------------- gram_xxt
+
+def gram_xxt_workspace_size(x) -> int:
+    n, m = x.shape[-2], x.shape[-1]
+    batch = math.prod(x.shape[:-2])
+    return int(_lib.lib().gram_xxt_workspace_size(batch, n, m, _dtype_code(x), x.data_ptr()))
+
+
+def gram_xxt(x, out=None, *, out_dtype=None, workspace=None, stream=None):
+    """A = X X^T over the last two dims of ``x`` (bf16 or fp16), exactly symmetric."""
+    torch = _torch()
+    _need_cuda(x, "x")
+    n, m = x.shape[-2], x.shape[-1]
+    batch = math.prod(x.shape[:-2])
+    if out is None:
+        out = torch.empty(*x.shape[:-2], n, n, dtype=out_dtype or x.dtype, device=x.device)
+    _need_cuda(out, "out")
+    if tuple(out.shape) != tuple(x.shape[:-2]) + (n, n):
+        raise ValueError("out must be (..., n, n)")
+    ws, wsb = _workspace(gram_xxt_workspace_size(x), x.device, workspace)
+    st = _lib.lib().gram_xxt(x.data_ptr(), _dtype_code(x), out.data_ptr(), _dtype_code(out), batch, n, m, _ptr(ws),
+                             wsb, _stream(stream))
+    check(st, "gram_xxt")
+    return out
+
+
+# ---------------------------------------------------------------- gram_ns
+
+def gram_ns_workspace_size(batch: int, rows: int, cols: int) -> int:
+    return int(_lib.lib().gram_ns_workspace_size(batch, rows, cols))
+
+
+def gram_ns(x, out=None, *, coeffs=None, eps=None, restart_after=(2,), workspace=None, stream=None):
+    """Stabilized Gram Newton-Schulz (fp16 inner iteration) of the last two dims of ``x``."""
+    torch = _torch()
+    _need_cuda(x, "x")
+    rows, cols = x.shape[-2], x.shape[-1]
+    batch = math.prod(x.shape[:-2])
+    if out is None:
+        out = torch.empty_like(x)
+    _need_cuda(out, "out")
+    ws, wsb = _workspace(gram_ns_workspace_size(batch, rows, cols), x.device, workspace)
+    c, keep = make_coeffs(coeffs, eps)
+    if restart_after is None:
+        rbuf, nr = None, -1
+    else:
+        r = [int(v) for v in restart_after]
+        rbuf, nr = (ctypes.c_int * max(1, len(r)))(*r), len(r)
+    st = _lib.lib().gram_ns(x.data_ptr(), out.data_ptr(), _dtype_code(x), batch, rows, cols,
+                            ctypes.byref(c) if c is not None else None,
+                            ctypes.cast(rbuf, ctypes.POINTER(ctypes.c_int)) if rbuf is not None else None, nr,
+                            _ptr(ws), wsb, _stream(stream))
+    del keep
+    check(st, "gram_ns")
+    return out
+
+
+# ---------------------------------------------------------------- muon_step
+
+def _i64_array(vals):
+    return (ctypes.c_int64 * len(vals))(*[int(v) for v in vals])
+
+
+def muon_step_workspace_size(shapes) -> int:
+    rows = _i64_array([s[0] for s in shapes])
+    cols = _i64_array([s[1] for s in shapes])
+    return int(_lib.lib().muon_step_workspace_size(len(shapes), rows, cols))
+
+
+def muon_step(weights, momenta, grads, *, momentum: float = 0.95, lr: float = 0.02, coeffs=None, eps=None,
+              workspace=None, stream=None):
+    """In-place Muon update of lists of weights (bf16/fp32), fp32 momenta and grads (bf16/fp32)."""
+    torch = _torch()
+    num = len(weights)
+    if not (len(momenta) == num and len(grads) == num):
+        raise ValueError("weights, momenta and grads must have the same length")
+    if num == 0:
+        return
+    for w, m, g in zip(weights, momenta, grads):
+        for t, nm in ((w, "weight"), (m, "momentum"), (g, "grad")):
+            _need_cuda(t, nm)
+        if w.dim() != 2 or w.shape != m.shape or w.shape != g.shape:
+            raise ValueError("each weight, momentum and grad must be the same 2-D shape")
+        if m.dtype != torch.float32:
+            raise TypeError("momenta must be float32")
+    wdt = {_dtype_code(w) for w in weights}
+    gdt = {_dtype_code(g) for g in grads}
+    if len(wdt) != 1 or len(gdt) != 1:
+        raise TypeError("all weights (and all grads) must share one dtype")
+    shapes = [tuple(w.shape) for w in weights]
+    ws, wsb = _workspace(muon_step_workspace_size(shapes), weights[0].device, workspace)
+    W = (ctypes.c_void_p * num)(*[w.data_ptr() for w in weights])
+    M = (ctypes.c_void_p * num)(*[m.data_ptr() for m in momenta])
+    G = (ctypes.c_void_p * num)(*[g.data_ptr() for g in grads])
+    rows = _i64_array([s[0] for s in shapes])
+    cols = _i64_array([s[1] for s in shapes])
+    c, keep = make_coeffs(coeffs, eps)
+    st = _lib.lib().muon_step(num, W, M, G, rows, cols, wdt.pop(), gdt.pop(), float(momentum), float(lr),
+                              ctypes.byref(c) if c is not None else None, _ptr(ws), wsb, _stream(stream))
+    del keep
+    check(st, "muon_step")
+
+
+# ---------------------------------------------------------------- launch records
+
+PROFILE_KINDS = {"gemm": 0, "norm": 1, "ingest": 2, "elementwise": 3}
+
+
+def profile_enable(enable: bool = True) -> None:
+    check(_lib.lib().msign_profile_enable(1 if enable else 0), "msign_profile_enable")
+
+
+def profile_reset() -> None:
+    check(_lib.lib().msign_profile_reset(), "msign_profile_reset")
+
+
+def profile_read(kind: str) -> dict:
+    """{'launches', 'ms', 'flops', 'bytes'} summed over the recorded launches of one kind."""
+    n = ctypes.c_int()
+    ms, fl, by = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    check(_lib.lib().msign_profile_read(PROFILE_KINDS[kind], ctypes.byref(n), ctypes.byref(ms), ctypes.byref(fl),
+                                        ctypes.byref(by)), "msign_profile_read")
+    return {"launches": n.value, "ms": ms.value, "flops": fl.value, "bytes": by.value}

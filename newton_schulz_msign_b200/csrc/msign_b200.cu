@@ -1,0 +1,952 @@
+// msign_b200.cu - C ABI of the library (declared in include/msign_b200.h):
+// argument checks, workspace layout, TMA descriptor construction and the
+// launch sequences of msign_ns, gram_xxt, gram_ns and muon_step.
+//
+// Every step of every entry point runs in the kernels of gemm_sm100.cuh and
+// elementwise.cuh; the host only plans and enqueues.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <vector>
+
+#include "msign_b200.h"
+#include "elementwise.cuh"
+#include "gemm_sm100.cuh"
+
+namespace msb {
+
+// Device error word raised by bounded waits (bit 0).
+__device__ int g_err_word;
+
+constexpr float kJordanA = 3.4445f, kJordanB = -4.7750f, kJordanC = 2.0315f;  // [P2] eq. 7
+constexpr int kJordanSteps = 5;
+constexpr float kNsEps = 1e-20f;    // [P2] section 参考实现, under the square root
+constexpr float kGramEps = 1e-7f;   // [P3] Algorithm 2 step 1, added to the norm
+constexpr int kMaxSteps = 64;
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per wait
+
+// ---------------------------------------------------------------- device state
+
+struct DeviceState {
+  bool ready = false;
+  int sms = 0;
+  int* err = nullptr;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[64];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+msign_status device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MSIGN_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MSIGN_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return MSIGN_ERR_CUDA;
+    if (major != 10 || minor != 0) return MSIGN_ERR_UNSUPPORTED;  // built for sm_100a only
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MSIGN_ERR_CUDA;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_err_word) != cudaSuccess) return MSIGN_ERR_CUDA;
+    if (cudaFuncSetAttribute(gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaSuccess)
+      return MSIGN_ERR_CUDA;
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return MSIGN_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    d.ready = true;
+  }
+  *out = &d;
+  return MSIGN_OK;
+}
+
+// ---------------------------------------------------------------- launch records
+//
+// While enabled (msign_profile_enable), every kernel the library enqueues is
+// bracketed by two CUDA events on its own stream, tagged with its kind and
+// its algorithmic work (useful FLOPs, compulsory HBM bytes).
+
+struct ProfRec {
+  int kind;
+  cudaEvent_t e0, e1;
+  double flops, bytes;
+};
+
+bool g_prof = false;
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_event_pool;
+cudaEvent_t g_pending = nullptr;
+
+cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+void prof_begin(cudaStream_t s) {
+  if (!g_prof) return;
+  g_pending = pool_event();
+  cudaEventRecord(g_pending, s);
+}
+
+void prof_end(int kind, cudaStream_t s, double flops, double bytes) {
+  if (!g_prof || g_pending == nullptr) return;
+  cudaEvent_t e1 = pool_event();
+  cudaEventRecord(e1, s);
+  g_prof_recs.push_back({kind, g_pending, e1, flops, bytes});
+  g_pending = nullptr;
+}
+
+// ---------------------------------------------------------------- helpers
+
+inline int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+int to_dt(msign_dtype d) { return d == MSIGN_BF16 ? DT_BF16 : d == MSIGN_FP16 ? DT_FP16 : DT_FP32; }
+
+bool valid_dtype(msign_dtype d) { return d == MSIGN_BF16 || d == MSIGN_FP16 || d == MSIGN_FP32; }
+
+// Workspace carving: the same routine sizes and slices the workspace.
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  void* take(size_t bytes) {
+    off = (off + 1023) & ~size_t(1023);
+    void* p = base ? base + off : nullptr;
+    off += bytes;
+    return p;
+  }
+};
+
+struct Schedule {
+  std::vector<float> abc;
+  float eps;
+  int steps() const { return static_cast<int>(abc.size() / 3); }
+};
+
+msign_status read_schedule(const msign_coeffs* c, float default_eps, Schedule* s) {
+  int T = kJordanSteps;
+  const float* abc = nullptr;
+  float eps = default_eps;
+  if (c != nullptr) {
+    if (c->abc != nullptr) {
+      if (c->steps <= 0) return MSIGN_ERR_INVALID_ARG;
+      T = c->steps;
+      abc = c->abc;
+    } else if (c->steps > 0) {
+      T = c->steps;
+    }
+    if (c->eps >= 0.0f) eps = c->eps;
+    if (!std::isfinite(eps)) return MSIGN_ERR_INVALID_ARG;
+  }
+  if (T > kMaxSteps) return MSIGN_ERR_UNSUPPORTED;
+  s->abc.resize(3 * T);
+  for (int t = 0; t < T; ++t) {
+    s->abc[3 * t + 0] = abc ? abc[3 * t + 0] : kJordanA;
+    s->abc[3 * t + 1] = abc ? abc[3 * t + 1] : kJordanB;
+    s->abc[3 * t + 2] = abc ? abc[3 * t + 2] : kJordanC;
+    for (int j = 0; j < 3; ++j)
+      if (!std::isfinite(s->abc[3 * t + j])) return MSIGN_ERR_INVALID_ARG;
+  }
+  s->eps = eps;
+  return MSIGN_OK;
+}
+
+// A dense batched matrix: rows x cols, leading dimension ld, batch stride bs
+// (both in elements).
+struct Mat {
+  const void* ptr;
+  int dt;
+  int64_t rows, cols, ld, bs;
+};
+
+bool tma_ok(const Mat& m) {
+  const int es = dtype_size(m.dt);
+  return m.dt != DT_FP32 && (reinterpret_cast<uintptr_t>(m.ptr) % 16) == 0 && (m.ld * es) % 16 == 0 &&
+         (m.bs * es) % 16 == 0;
+}
+
+bool encode(CUtensorMap* tm, const Mat& m, bool kmajor_rows_box, int box_rows, int64_t batch) {
+  // dims: (cols, rows, batch); box: (64, box_rows, 1)
+  const int es = dtype_size(m.dt);
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(m.cols), static_cast<cuuint64_t>(m.rows),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(m.ld * es), static_cast<cuuint64_t>(m.bs * es)};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  (void)kmajor_rows_box;
+  CUresult r = g_encode(tm, m.dt == DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                        const_cast<void*>(m.ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+EpiOut out_to(void* ptr, int dt, int64_t ld, int64_t bs, bool transposed, float gamma = 0.0f) {
+  EpiOut e;
+  std::memset(&e, 0, sizeof(e));
+  e.ptr = ptr;
+  e.dtype = dt;
+  e.ld = ld;
+  e.bs = bs;
+  e.transposed = transposed ? 1 : 0;
+  e.gamma = gamma;
+  return e;
+}
+
+// One class of a grouped launch: D (M x N) = epilogue(A_op * B_op^T).
+//   A: rows M, cols K (K-major).
+//   B: if !b_mn: rows N, cols K (K-major); if b_mn: rows K, cols N.
+struct ClassSpec {
+  Mat A, B;
+  bool b_mn = false;
+  bool symmetric = false;
+  int64_t M = 0, N = 0, K = 0, batch = 0;
+  float alpha = 1.0f, beta = 0.0f;
+  const float* alpha_scale = nullptr;
+  const float* beta_scale = nullptr;
+  const void* C = nullptr;
+  int c_dt = DT_FP32;
+  int64_t ldc = 0, c_bs = 0;
+  std::vector<EpiOut> outs;
+};
+
+int64_t triangle_tiles(int64_t n) {
+  const int64_t tm_n = (n + kBM - 1) / kBM, tn_n = (n + kBN - 1) / kBN;
+  int64_t c = 0;
+  for (int64_t tm = 0; tm < tm_n; ++tm) c += tn_n - tm / 2;
+  return c;
+}
+
+int64_t class_tiles(const ClassSpec& s) {
+  if (s.M <= 0 || s.N <= 0 || s.batch <= 0) return 0;
+  const int64_t per = s.symmetric ? triangle_tiles(s.M) : ((s.M + kBM - 1) / kBM) * ((s.N + kBN - 1) / kBN);
+  return per * s.batch;
+}
+
+// Encodes and launches up to kMaxClasses classes of one operand dtype.
+msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_t stream) {
+  DeviceState* dev = nullptr;
+  msign_status st = device_state(&dev);
+  if (st != MSIGN_OK) return st;
+  specs.erase(std::remove_if(specs.begin(), specs.end(), [](const ClassSpec& s) { return class_tiles(s) == 0; }),
+              specs.end());
+  if (specs.empty()) return MSIGN_OK;
+  if (specs.size() > static_cast<size_t>(kMaxClasses)) return MSIGN_ERR_UNSUPPORTED;
+  // longest reduction first: its tiles are the longest-running work items
+  std::stable_sort(specs.begin(), specs.end(), [](const ClassSpec& a, const ClassSpec& b) { return a.K > b.K; });
+
+  static thread_local GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  int64_t total = 0;
+  for (size_t i = 0; i < specs.size(); ++i) {
+    const ClassSpec& s = specs[i];
+    GemmClass& c = p.cls[i];
+    if (s.K <= 0 || s.outs.empty() || s.outs.size() > static_cast<size_t>(kMaxOuts)) return MSIGN_ERR_INVALID_ARG;
+    if (s.symmetric && s.M != s.N) return MSIGN_ERR_INVALID_ARG;
+    if (!tma_ok(s.A) || !tma_ok(s.B) || s.A.dt != ab_dt || s.B.dt != ab_dt) return MSIGN_ERR_UNSUPPORTED;
+    if (s.M > INT32_MAX || s.N > INT32_MAX || s.K > INT32_MAX || s.batch > 65535) return MSIGN_ERR_UNSUPPORTED;
+    Mat a = s.A;
+    a.rows = s.M;
+    a.cols = s.K;
+    if (!encode(&c.tmA, a, true, kBM, s.batch)) return MSIGN_ERR_CUDA;
+    Mat b = s.B;
+    if (!s.b_mn) {
+      b.rows = s.N;
+      b.cols = s.K;
+      if (!encode(&c.tmB, b, true, kBN, s.batch)) return MSIGN_ERR_CUDA;
+    } else {
+      b.rows = s.K;
+      b.cols = s.N;
+      if (!encode(&c.tmB, b, false, kBK, s.batch)) return MSIGN_ERR_CUDA;
+    }
+    c.M = static_cast<int>(s.M);
+    c.N = static_cast<int>(s.N);
+    c.K = static_cast<int>(s.K);
+    c.batch = static_cast<int>(s.batch);
+    c.tiles_m = static_cast<int>((s.M + kBM - 1) / kBM);
+    c.tiles_n = static_cast<int>((s.N + kBN - 1) / kBN);
+    c.tiles_per_batch = static_cast<int>(class_tiles(s) / s.batch);
+    c.tile_begin = static_cast<int>(total);
+    c.symmetric = s.symmetric ? 1 : 0;
+    c.b_mn_major = s.b_mn ? 1 : 0;
+    c.num_out = static_cast<int>(s.outs.size());
+    c.alpha = s.alpha;
+    c.beta = s.beta;
+    c.alpha_scale = s.alpha_scale;
+    c.beta_scale = s.beta_scale;
+    c.C = s.C;
+    c.c_dtype = s.c_dt;
+    c.ldc = s.ldc;
+    c.c_bs = s.c_bs;
+    for (size_t o = 0; o < s.outs.size(); ++o) c.out[o] = s.outs[o];
+    total += class_tiles(s);
+  }
+  if (total > INT32_MAX) return MSIGN_ERR_UNSUPPORTED;
+  p.num_classes = static_cast<int>(specs.size());
+  p.total_tiles = static_cast<int>(total);
+  const uint32_t fmt = (ab_dt == DT_BF16) ? 1u : 0u;
+  p.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
+            (static_cast<uint32_t>(kBM >> 4) << 24);
+  p.err = dev->err;
+  p.timeout_ns = kWaitLimitNs;
+  const int grid = static_cast<int>(std::min<int64_t>(total, dev->sms));
+  double flops = 0.0, bytes = 0.0;
+  for (const ClassSpec& s : specs) {
+    const double bt = static_cast<double>(s.batch);
+    // useful FLOPs: the triangle only for symmetric outputs
+    flops += s.symmetric ? bt * s.K * static_cast<double>(s.M) * (s.M + 1) : bt * 2.0 * s.M * s.N * s.K;
+    // compulsory traffic: both operands once, C once, every output once
+    const double es = dtype_size(s.A.dt);
+    bytes += bt * es * (static_cast<double>(s.M) * s.K + (s.A.ptr == s.B.ptr ? 0.0 : static_cast<double>(s.N) * s.K));
+    if (s.C) bytes += bt * dtype_size(s.c_dt) * static_cast<double>(s.M) * s.N;
+    for (const EpiOut& e : s.outs)
+      bytes += bt * dtype_size(e.dtype) * static_cast<double>(s.M) * s.N * (s.symmetric ? 0.5 : 1.0);
+  }
+  prof_begin(stream);
+  gemm_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
+  prof_end(0, stream, flops, bytes);
+  return cudaGetLastError() == cudaSuccess ? MSIGN_OK : MSIGN_ERR_CUDA;
+}
+
+msign_status launch_ok() { return cudaGetLastError() == cudaSuccess ? MSIGN_OK : MSIGN_ERR_CUDA; }
+
+// Frobenius normalisation factor of every matrix of a batch into scale[].
+msign_status launch_norm(const void* in, int in_dt, int64_t per, int64_t batch, int cast_dt, float eps, int mode,
+                         float* partials, float* scale, cudaStream_t stream) {
+  dim3 g(kNormParts, static_cast<unsigned>(batch));
+  prof_begin(stream);
+  sumsq_partial_kernel<<<g, kNormThreads, 0, stream>>>(in, in_dt, per, cast_dt, partials);
+  prof_end(1, stream, 0.0, static_cast<double>(batch) * per * dtype_size(in_dt));
+  prof_begin(stream);
+  norm_finalize_kernel<<<static_cast<unsigned>(batch), kNormParts, 0, stream>>>(partials, kNormParts, eps, mode,
+                                                                                scale);
+  prof_end(1, stream, 0.0, static_cast<double>(batch) * kNormParts * 4);
+  return launch_ok();
+}
+
+msign_status launch_ingest(const void* in, int in_dt, int64_t rows, int64_t cols, bool transpose, const float* scale,
+                           int cast_dt, void* xop, int op_dt, int64_t ld_op, int64_t op_bs, float* master,
+                           int64_t ld_m, int64_t m_bs, int64_t batch, cudaStream_t stream) {
+  const int64_t n = transpose ? cols : rows, m = transpose ? rows : cols;
+  dim3 g(static_cast<unsigned>((m + 31) / 32), static_cast<unsigned>((n + 31) / 32), static_cast<unsigned>(batch));
+  prof_begin(stream);
+  ingest_kernel<<<g, dim3(32, 8), 0, stream>>>(in, in_dt, static_cast<int>(rows), static_cast<int>(cols),
+                                               transpose ? 1 : 0, scale, cast_dt, xop, op_dt, ld_op, op_bs, master,
+                                               ld_m, m_bs);
+  prof_end(2, stream, 0.0,
+           static_cast<double>(batch) * rows * cols * (dtype_size(in_dt) + dtype_size(op_dt) + (master ? 4 : 0)));
+  return launch_ok();
+}
+
+// ---------------------------------------------------------------- msign_ns plan
+
+struct NsBuffers {
+  float* partials;
+  float* scale;
+  void* P[2];     // bf16 operand copies of X (n x ldm)
+  float* master;  // fp32 X (n x ldm)
+  void* A;        // bf16 n x ldn
+  void* B;        // bf16 n x ldn
+};
+
+void carve_ns(Carver& cv, int64_t batch, int64_t n, int64_t m, NsBuffers* b) {
+  const int64_t ldm = round_up(m, 8), ldn = round_up(n, 8);
+  b->partials = static_cast<float*>(cv.take(sizeof(float) * kNormParts * batch));
+  b->scale = static_cast<float*>(cv.take(sizeof(float) * batch));
+  b->P[0] = cv.take(2ull * batch * n * ldm);
+  b->P[1] = cv.take(2ull * batch * n * ldm);
+  b->master = static_cast<float*>(cv.take(4ull * batch * n * ldm));
+  b->A = cv.take(2ull * batch * n * ldn);
+  b->B = cv.take(2ull * batch * n * ldn);
+}
+
+// Launches a list of classes of one operand dtype, kMaxClasses at a time.
+msign_status launch_all(const std::vector<ClassSpec>& specs, int ab_dt, cudaStream_t stream) {
+  for (size_t i = 0; i < specs.size(); i += kMaxClasses) {
+    std::vector<ClassSpec> chunk(specs.begin() + i, specs.begin() + std::min(specs.size(), i + kMaxClasses));
+    msign_status st = launch_grouped(chunk, ab_dt, stream);
+    if (st != MSIGN_OK) return st;
+  }
+  return MSIGN_OK;
+}
+
+// One shape class of a standard-NS run: `batch` oriented n x m matrices.
+struct NsClass {
+  NsBuffers w;
+  int64_t batch, n, m;
+  std::vector<EpiOut> final_outs;  // outputs of the last step's B X product
+};
+
+// The three products of one NS step ([P2] eq. 6, left form), each launched
+// once for all classes:
+//   SYRK   A = X X^T                  (symmetric, mirror store)
+//   SQR    B = b A + c A A            (symmetric; A A = A A^T as A = A^T)
+//   BX     X' = a X + B X             (X read MN-major; the a X term uses
+//                                      the fp32 copy of X)
+msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b, float c, bool last,
+                     cudaStream_t stream) {
+  std::vector<ClassSpec> syrk, sqr, bx;
+  for (const NsClass& k : cls) {
+    const int64_t n = k.n, m = k.m, ldm = round_up(m, 8), ldn = round_up(n, 8);
+    const Mat X{k.w.P[cur], DT_BF16, n, m, ldm, n * ldm};
+    const Mat A{k.w.A, DT_BF16, n, n, ldn, n * ldn};
+    const Mat B{k.w.B, DT_BF16, n, n, ldn, n * ldn};
+    ClassSpec s;
+    s.A = X, s.B = X, s.symmetric = true;
+    s.M = n, s.N = n, s.K = m, s.batch = k.batch;
+    s.outs = {out_to(k.w.A, DT_BF16, ldn, n * ldn, false), out_to(k.w.A, DT_BF16, ldn, n * ldn, true)};
+    syrk.push_back(s);
+
+    ClassSpec q;
+    q.A = A, q.B = A, q.symmetric = true;
+    q.M = n, q.N = n, q.K = n, q.batch = k.batch;
+    q.alpha = c, q.beta = b;
+    q.C = k.w.A, q.c_dt = DT_BF16, q.ldc = ldn, q.c_bs = n * ldn;
+    q.outs = {out_to(k.w.B, DT_BF16, ldn, n * ldn, false), out_to(k.w.B, DT_BF16, ldn, n * ldn, true)};
+    sqr.push_back(q);
+
+    ClassSpec x;
+    x.A = B, x.B = X, x.b_mn = true;
+    x.M = n, x.N = m, x.K = n, x.batch = k.batch;
+    x.alpha = 1.0f, x.beta = a;
+    x.C = k.w.master, x.c_dt = DT_FP32, x.ldc = ldm, x.c_bs = n * ldm;
+    if (!last)
+      x.outs = {out_to(k.w.master, DT_FP32, ldm, n * ldm, false),
+                out_to(k.w.P[cur ^ 1], DT_BF16, ldm, n * ldm, false)};
+    else
+      x.outs = k.final_outs;
+    bx.push_back(x);
+  }
+  msign_status st = launch_all(syrk, DT_BF16, stream);
+  if (st == MSIGN_OK) st = launch_all(sqr, DT_BF16, stream);
+  if (st == MSIGN_OK) st = launch_all(bx, DT_BF16, stream);
+  return st;
+}
+
+// Runs all steps of the schedule on classes whose P[0] / master already hold X0.
+msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cudaStream_t stream) {
+  const int T = sch.steps();
+  int cur = 0;
+  for (int t = 0; t < T; ++t) {
+    msign_status st = ns_step(cls, cur, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == T - 1, stream);
+    if (st != MSIGN_OK) return st;
+    cur ^= 1;
+  }
+  return MSIGN_OK;
+}
+
+// ---------------------------------------------------------------- gram_ns plan
+
+struct GramBuffers {
+  float* partials;
+  float* scale;
+  void* P[2];  // fp16 X (n x ldm)
+  void* R;     // fp16 n x ldn
+  void* Z;
+  void* Q[2];
+  void* RZ;
+};
+
+void carve_gram(Carver& cv, int64_t batch, int64_t n, int64_t m, GramBuffers* b) {
+  const int64_t ldm = round_up(m, 8), ldn = round_up(n, 8);
+  b->partials = static_cast<float*>(cv.take(sizeof(float) * kNormParts * batch));
+  b->scale = static_cast<float*>(cv.take(sizeof(float) * batch));
+  b->P[0] = cv.take(2ull * batch * n * ldm);
+  b->P[1] = cv.take(2ull * batch * n * ldm);
+  b->R = cv.take(2ull * batch * n * ldn);
+  b->Z = cv.take(2ull * batch * n * ldn);
+  b->Q[0] = cv.take(2ull * batch * n * ldn);
+  b->Q[1] = cv.take(2ull * batch * n * ldn);
+  b->RZ = cv.take(2ull * batch * n * ldn);
+}
+
+// Restart schedule -> segment bounds [0, r1, r2, ..., T].
+msign_status gram_segments(int T, const int* restart_after, int n_restart, std::vector<int>* bounds) {
+  std::vector<int> cuts;
+  if (restart_after == nullptr && n_restart < 0) {
+    if (T > 2) cuts.push_back(2);  // [P3] section 3.2: restart after the second step
+  } else {
+    if (n_restart < 0 || (n_restart > 0 && restart_after == nullptr)) return MSIGN_ERR_INVALID_ARG;
+    for (int i = 0; i < n_restart; ++i) {
+      if (restart_after[i] < 1 || restart_after[i] > T - 1) return MSIGN_ERR_INVALID_ARG;
+      cuts.push_back(restart_after[i]);
+    }
+    std::sort(cuts.begin(), cuts.end());
+    cuts.erase(std::unique(cuts.begin(), cuts.end()), cuts.end());
+  }
+  bounds->clear();
+  bounds->push_back(0);
+  for (int c : cuts) bounds->push_back(c);
+  bounds->push_back(T);
+  return MSIGN_OK;
+}
+
+}  // namespace msb
+
+using namespace msb;
+
+
+// ================================================================ C ABI
+
+extern "C" {
+
+int msign_abi_version(void) { return 100; }
+
+const char* msign_status_string(msign_status s) {
+  switch (s) {
+    case MSIGN_OK: return "ok";
+    case MSIGN_ERR_INVALID_ARG: return "invalid argument";
+    case MSIGN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MSIGN_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case MSIGN_ERR_CUDA: return "CUDA error";
+    case MSIGN_ERR_TIMEOUT: return "a bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+msign_status msign_sync_status(msign_stream_t stream) {
+  DeviceState* dev = nullptr;
+  msign_status st = device_state(&dev);
+  if (st != MSIGN_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MSIGN_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, dev->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MSIGN_ERR_CUDA;
+  if (word != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(dev->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MSIGN_ERR_CUDA;
+    return MSIGN_ERR_TIMEOUT;
+  }
+  return MSIGN_OK;
+}
+
+msign_status msign_profile_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_prof = enable != 0;
+  return MSIGN_OK;
+}
+
+msign_status msign_profile_read(int kind, int* launches, double* total_ms, double* flops, double* bytes) {
+  if (launches == nullptr || total_ms == nullptr || flops == nullptr || bytes == nullptr) return MSIGN_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  *launches = 0;
+  *total_ms = 0.0;
+  *flops = 0.0;
+  *bytes = 0.0;
+  for (const ProfRec& r : g_prof_recs) {
+    if (r.kind != kind) continue;
+    if (cudaEventSynchronize(r.e1) != cudaSuccess) return MSIGN_ERR_CUDA;
+    float ms = 0.0f;
+    if (cudaEventElapsedTime(&ms, r.e0, r.e1) != cudaSuccess) return MSIGN_ERR_CUDA;
+    *launches += 1;
+    *total_ms += ms;
+    *flops += r.flops;
+    *bytes += r.bytes;
+  }
+  return MSIGN_OK;
+}
+
+msign_status msign_profile_reset(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (const ProfRec& r : g_prof_recs) {
+    cudaEventSynchronize(r.e1);
+    g_event_pool.push_back(r.e0);
+    g_event_pool.push_back(r.e1);
+  }
+  g_prof_recs.clear();
+  return MSIGN_OK;
+}
+
+size_t msign_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute_dtype) {
+  (void)compute_dtype;
+  if (batch <= 0 || rows <= 0 || cols <= 0) return 0;
+  const int64_t n = std::min(rows, cols), m = std::max(rows, cols);
+  Carver cv(nullptr);
+  NsBuffers b;
+  carve_ns(cv, batch, n, m, &b);
+  return cv.off + 1024;
+}
+
+msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dtype compute_dtype, int64_t batch,
+                      int64_t rows, int64_t cols, const msign_coeffs* coeffs, void* workspace,
+                      size_t workspace_bytes, msign_stream_t stream_) {
+  if (!valid_dtype(io_dtype) || !valid_dtype(compute_dtype)) return MSIGN_ERR_INVALID_ARG;
+  if (batch < 0 || rows < 0 || cols < 0) return MSIGN_ERR_INVALID_ARG;
+  Schedule sch;
+  msign_status st = read_schedule(coeffs, kNsEps, &sch);
+  if (st != MSIGN_OK) return st;
+  if (batch == 0 || rows == 0 || cols == 0) return MSIGN_OK;
+  if (in == nullptr || out == nullptr) return MSIGN_ERR_INVALID_ARG;
+  if (compute_dtype != MSIGN_BF16) return MSIGN_ERR_UNSUPPORTED;
+  if (batch > 65535 || rows > (1 << 30) || cols > (1 << 30)) return MSIGN_ERR_UNSUPPORTED;
+  const size_t need = msign_ns_workspace_size(batch, rows, cols, compute_dtype);
+  if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
+    return MSIGN_ERR_WORKSPACE;
+  DeviceState* dev = nullptr;
+  st = device_state(&dev);
+  if (st != MSIGN_OK) return st;
+
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const bool tr = rows > cols;  // iterate on the side with the smaller Gram matrix
+  const int64_t n = tr ? cols : rows, m = tr ? rows : cols;
+  const int64_t ldm = round_up(m, 8);
+  const int io = to_dt(io_dtype);
+  Carver cv(workspace);
+  NsBuffers w;
+  carve_ns(cv, batch, n, m, &w);
+
+  st = launch_norm(in, io, rows * cols, batch, DT_BF16, sch.eps, 0, w.partials, w.scale, stream);
+  if (st != MSIGN_OK) return st;
+  st = launch_ingest(in, io, rows, cols, tr, w.scale, DT_BF16, w.P[0], DT_BF16, ldm, n * ldm, w.master, ldm, n * ldm,
+                     batch, stream);
+  if (st != MSIGN_OK) return st;
+  std::vector<NsClass> cls(1);
+  cls[0].w = w;
+  cls[0].batch = batch, cls[0].n = n, cls[0].m = m;
+  cls[0].final_outs = {out_to(out, io, cols, rows * cols, tr)};
+  return ns_iterate(cls, sch, stream);
+}
+
+size_t gram_xxt_workspace_size(int64_t batch, int64_t n, int64_t m, msign_dtype x_dtype, const void* X) {
+  if (batch <= 0 || n <= 0 || m <= 0) return 0;
+  const int es = x_dtype == MSIGN_FP32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(X) % 16) == 0 && (m * es) % 16 == 0) return 0;
+  return 2ull * batch * n * round_up(m, 8) + 2048;
+}
+
+msign_status gram_xxt(const void* X, msign_dtype x_dtype, void* A, msign_dtype a_dtype, int64_t batch, int64_t n,
+                      int64_t m, void* workspace, size_t workspace_bytes, msign_stream_t stream_) {
+  if (!valid_dtype(x_dtype) || !valid_dtype(a_dtype)) return MSIGN_ERR_INVALID_ARG;
+  if (batch < 0 || n < 0 || m < 0) return MSIGN_ERR_INVALID_ARG;
+  if (batch == 0 || n == 0) return MSIGN_OK;
+  if (X == nullptr && m > 0) return MSIGN_ERR_INVALID_ARG;
+  if (A == nullptr) return MSIGN_ERR_INVALID_ARG;
+  if (x_dtype == MSIGN_FP32) return MSIGN_ERR_UNSUPPORTED;
+  if (batch > 65535 || n > (1 << 30) || m > (1 << 30)) return MSIGN_ERR_UNSUPPORTED;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (m == 0) {  // empty inner dimension: A = 0
+    const size_t bytes = static_cast<size_t>(batch) * n * n * (a_dtype == MSIGN_FP32 ? 4 : 2);
+    return cudaMemsetAsync(A, 0, bytes, stream) == cudaSuccess ? MSIGN_OK : MSIGN_ERR_CUDA;
+  }
+  const int xd = to_dt(x_dtype);
+  Mat Xm{X, xd, n, m, m, n * m};
+  const size_t need = gram_xxt_workspace_size(batch, n, m, x_dtype, X);
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
+      return MSIGN_ERR_WORKSPACE;
+    const int64_t ldm = round_up(m, 8);
+    msign_status st = launch_ingest(X, xd, n, m, false, nullptr, DT_FP32, workspace, xd, ldm, n * ldm, nullptr, 0, 0,
+                                    batch, stream);
+    if (st != MSIGN_OK) return st;
+    Xm = Mat{workspace, xd, n, m, ldm, n * ldm};
+  }
+  ClassSpec s;
+  s.A = Xm;
+  s.B = Xm;
+  s.symmetric = true;
+  s.M = n, s.N = n, s.K = m, s.batch = batch;
+  const int ad = to_dt(a_dtype);
+  s.outs = {out_to(A, ad, n, n * n, false), out_to(A, ad, n, n * n, true)};
+  return launch_grouped({s}, xd, stream);
+}
+
+
+size_t gram_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols) {
+  if (batch <= 0 || rows <= 0 || cols <= 0) return 0;
+  const int64_t n = std::min(rows, cols), m = std::max(rows, cols);
+  Carver cv(nullptr);
+  GramBuffers b;
+  carve_gram(cv, batch, n, m, &b);
+  return cv.off + 1024;
+}
+
+msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t batch, int64_t rows, int64_t cols,
+                     const msign_coeffs* coeffs, const int* restart_after, int n_restart, void* workspace,
+                     size_t workspace_bytes, msign_stream_t stream_) {
+  if (!valid_dtype(io_dtype)) return MSIGN_ERR_INVALID_ARG;
+  if (batch < 0 || rows < 0 || cols < 0) return MSIGN_ERR_INVALID_ARG;
+  Schedule sch;
+  msign_status st = read_schedule(coeffs, kGramEps, &sch);
+  if (st != MSIGN_OK) return st;
+  const int T = sch.steps();
+  std::vector<int> bounds;
+  st = gram_segments(T, restart_after, n_restart, &bounds);
+  if (st != MSIGN_OK) return st;
+  if (batch == 0 || rows == 0 || cols == 0) return MSIGN_OK;
+  if (in == nullptr || out == nullptr) return MSIGN_ERR_INVALID_ARG;
+  if (batch > 65535 || rows > (1 << 30) || cols > (1 << 30)) return MSIGN_ERR_UNSUPPORTED;
+  const size_t need = gram_ns_workspace_size(batch, rows, cols);
+  if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
+    return MSIGN_ERR_WORKSPACE;
+  DeviceState* dev = nullptr;
+  st = device_state(&dev);
+  if (st != MSIGN_OK) return st;
+
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const bool tr = rows > cols;
+  const int64_t n = tr ? cols : rows, m = tr ? rows : cols;
+  const int64_t ldm = round_up(m, 8), ldn = round_up(n, 8);
+  const int io = to_dt(io_dtype);
+  Carver cv(workspace);
+  GramBuffers w;
+  carve_gram(cv, batch, n, m, &w);
+  const int64_t sq = n * ldn, rect = n * ldm;
+  auto sym_out = [&](void* p, float gamma) {
+    return std::vector<EpiOut>{out_to(p, DT_FP16, ldn, sq, false, gamma), out_to(p, DT_FP16, ldn, sq, true, gamma)};
+  };
+  auto sqm = [&](void* p) { return Mat{p, DT_FP16, n, n, ldn, sq}; };
+
+  // [P3] Algorithm 2 steps 1-2: X <- X / (||X||_F + eps); X <- float16(X)
+  st = launch_norm(in, io, rows * cols, batch, DT_FP32, sch.eps, 1, w.partials, w.scale, stream);
+  if (st != MSIGN_OK) return st;
+  st = launch_ingest(in, io, rows, cols, tr, w.scale, DT_FP32, w.P[0], DT_FP16, ldm, rect, nullptr, 0, 0, batch,
+                     stream);
+  if (st != MSIGN_OK) return st;
+
+  int cur = 0;
+  for (size_t seg = 0; seg + 1 < bounds.size(); ++seg) {
+    const int s0 = bounds[seg], s1 = bounds[seg + 1];
+    const Mat X{w.P[cur], DT_FP16, n, m, ldm, rect};
+    {  // R = X X^T
+      ClassSpec s;
+      s.A = X, s.B = X, s.symmetric = true;
+      s.M = n, s.N = n, s.K = m, s.batch = batch;
+      s.outs = sym_out(w.R, 0.0f);
+      st = launch_grouped({s}, DT_FP16, stream);
+      if (st != MSIGN_OK) return st;
+    }
+    int q = -1;  // Q = I until the first step of the segment sets it
+    for (int t = s0; t < s1; ++t) {
+      const float a = sch.abc[3 * t], b = sch.abc[3 * t + 1], c = sch.abc[3 * t + 2];
+      const bool first = (t == s0), last = (t == s1 - 1);
+      {  // Z = b R + c R^2; on the first step also Q = Z + a I (Q Z with Q = I)
+        ClassSpec s;
+        s.A = sqm(w.R), s.B = sqm(w.R), s.symmetric = true;
+        s.M = n, s.N = n, s.K = n, s.batch = batch;
+        s.alpha = c, s.beta = b;
+        s.C = w.R, s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
+        s.outs = sym_out(w.Z, 0.0f);
+        if (first) {
+          std::vector<EpiOut> qo = sym_out(w.Q[0], a);
+          s.outs.insert(s.outs.end(), qo.begin(), qo.end());
+        }
+        st = launch_grouped({s}, DT_FP16, stream);
+        if (st != MSIGN_OK) return st;
+        if (first) q = 0;
+      }
+      std::vector<ClassSpec> pair;
+      if (!first) {  // Q <- Q Z + a Q
+        ClassSpec s;
+        s.A = sqm(w.Q[q]), s.B = sqm(w.Z), s.symmetric = true;
+        s.M = n, s.N = n, s.K = n, s.batch = batch;
+        s.alpha = 1.0f, s.beta = a;
+        s.C = w.Q[q], s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
+        s.outs = sym_out(w.Q[q ^ 1], 0.0f);
+        pair.push_back(s);
+      }
+      if (!last) {  // RZ <- R Z + a R
+        ClassSpec s;
+        s.A = sqm(w.R), s.B = sqm(w.Z), s.symmetric = true;
+        s.M = n, s.N = n, s.K = n, s.batch = batch;
+        s.alpha = 1.0f, s.beta = a;
+        s.C = w.R, s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
+        s.outs = sym_out(w.RZ, 0.0f);
+        pair.push_back(s);
+      }
+      if (!pair.empty()) {
+        st = launch_grouped(pair, DT_FP16, stream);
+        if (st != MSIGN_OK) return st;
+      }
+      if (!first) q ^= 1;
+      if (!last) {  // R <- Z RZ + a RZ
+        ClassSpec s;
+        s.A = sqm(w.Z), s.B = sqm(w.RZ), s.symmetric = true;
+        s.M = n, s.N = n, s.K = n, s.batch = batch;
+        s.alpha = 1.0f, s.beta = a;
+        s.C = w.RZ, s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
+        s.outs = sym_out(w.R, 0.0f);
+        st = launch_grouped({s}, DT_FP16, stream);
+        if (st != MSIGN_OK) return st;
+      }
+    }
+    {  // X <- Q X (the restart), or the output after the last segment
+      ClassSpec s;
+      s.A = sqm(w.Q[q]), s.B = X, s.b_mn = true;
+      s.M = n, s.N = m, s.K = n, s.batch = batch;
+      if (seg + 2 == bounds.size())
+        s.outs = {out_to(out, io, cols, rows * cols, tr)};
+      else
+        s.outs = {out_to(w.P[cur ^ 1], DT_FP16, ldm, rect, false)};
+      st = launch_grouped({s}, DT_FP16, stream);
+      if (st != MSIGN_OK) return st;
+    }
+    cur ^= 1;
+  }
+  return MSIGN_OK;
+}
+
+// Workspace of one group of Muon matrices: one NsBuffers set per distinct
+// oriented shape, in first-seen order.
+static size_t muon_group_bytes(const std::vector<std::pair<int64_t, int64_t>>& shapes,
+                               const std::vector<int64_t>& counts) {
+  Carver cv(nullptr);
+  for (size_t i = 0; i < shapes.size(); ++i) {
+    NsBuffers b;
+    carve_ns(cv, counts[i], shapes[i].first, shapes[i].second, &b);
+  }
+  return cv.off + 1024;
+}
+
+static void muon_group_shapes(const int64_t* rows, const int64_t* cols, int begin, int end,
+                              std::vector<std::pair<int64_t, int64_t>>* shapes, std::vector<int64_t>* counts,
+                              std::vector<int>* cls_of, std::vector<int64_t>* slot_of) {
+  shapes->clear();
+  counts->clear();
+  cls_of->assign(end - begin, -1);
+  slot_of->assign(end - begin, -1);
+  for (int i = begin; i < end; ++i) {
+    if (rows[i] == 0 || cols[i] == 0) continue;
+    const std::pair<int64_t, int64_t> sh{std::min(rows[i], cols[i]), std::max(rows[i], cols[i])};
+    size_t c = 0;
+    while (c < shapes->size() && (*shapes)[c] != sh) ++c;
+    if (c == shapes->size()) {
+      shapes->push_back(sh);
+      counts->push_back(0);
+    }
+    (*cls_of)[i - begin] = static_cast<int>(c);
+    (*slot_of)[i - begin] = (*counts)[c]++;
+  }
+}
+
+size_t muon_step_workspace_size(int num, const int64_t* rows, const int64_t* cols) {
+  if (num <= 0 || rows == nullptr || cols == nullptr) return 0;
+  std::vector<std::pair<int64_t, int64_t>> shapes;
+  std::vector<int64_t> counts, slots;
+  std::vector<int> cls;
+  muon_group_shapes(rows, cols, 0, num, &shapes, &counts, &cls, &slots);
+  if (shapes.empty()) return 0;
+  return muon_group_bytes(shapes, counts);
+}
+
+msign_status muon_step(int num, void* const* W, float* const* M, const void* const* G, const int64_t* rows,
+                       const int64_t* cols, msign_dtype w_dtype, msign_dtype g_dtype, float momentum, float lr,
+                       const msign_coeffs* coeffs, void* workspace, size_t workspace_bytes,
+                       msign_stream_t stream_) {
+  if (num < 0) return MSIGN_ERR_INVALID_ARG;
+  if (num == 0) return MSIGN_OK;
+  if (W == nullptr || M == nullptr || G == nullptr || rows == nullptr || cols == nullptr) return MSIGN_ERR_INVALID_ARG;
+  if (!valid_dtype(w_dtype) || !valid_dtype(g_dtype)) return MSIGN_ERR_INVALID_ARG;
+  if (w_dtype == MSIGN_FP16 || g_dtype == MSIGN_FP16) return MSIGN_ERR_UNSUPPORTED;
+  if (!std::isfinite(momentum) || !std::isfinite(lr)) return MSIGN_ERR_INVALID_ARG;
+  Schedule sch;
+  msign_status st = read_schedule(coeffs, kNsEps, &sch);
+  if (st != MSIGN_OK) return st;
+  size_t largest = 0;
+  for (int i = 0; i < num; ++i) {
+    if (rows[i] < 0 || cols[i] < 0) return MSIGN_ERR_INVALID_ARG;
+    if (rows[i] == 0 || cols[i] == 0) continue;
+    if (W[i] == nullptr || M[i] == nullptr || G[i] == nullptr) return MSIGN_ERR_INVALID_ARG;
+    if (rows[i] > (1 << 30) || cols[i] > (1 << 30)) return MSIGN_ERR_UNSUPPORTED;
+    largest = std::max(largest, muon_step_workspace_size(1, rows + i, cols + i));
+  }
+  if (largest == 0) return MSIGN_OK;
+  if (workspace == nullptr || workspace_bytes < largest || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
+    return MSIGN_ERR_WORKSPACE;
+  DeviceState* dev = nullptr;
+  st = device_state(&dev);
+  if (st != MSIGN_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const int wd = to_dt(w_dtype), gd = to_dt(g_dtype);
+
+  int begin = 0;
+  while (begin < num) {
+    // the longest prefix of the remaining list whose workspace fits
+    int end = begin + 1;
+    std::vector<std::pair<int64_t, int64_t>> shapes;
+    std::vector<int64_t> counts, slots;
+    std::vector<int> cls;
+    while (end < num) {
+      muon_group_shapes(rows, cols, begin, end + 1, &shapes, &counts, &cls, &slots);
+      if (muon_group_bytes(shapes, counts) > workspace_bytes) break;
+      ++end;
+    }
+    muon_group_shapes(rows, cols, begin, end, &shapes, &counts, &cls, &slots);
+    if (shapes.empty()) {
+      begin = end;
+      continue;
+    }
+    Carver cv(workspace);
+    std::vector<NsClass> ns(shapes.size());
+    for (size_t c = 0; c < shapes.size(); ++c) {
+      carve_ns(cv, counts[c], shapes[c].first, shapes[c].second, &ns[c].w);
+      ns[c].batch = counts[c];
+      ns[c].n = shapes[c].first;
+      ns[c].m = shapes[c].second;
+      const int64_t ldm = round_up(ns[c].m, 8);
+      ns[c].final_outs = {out_to(ns[c].w.master, DT_FP32, ldm, ns[c].n * ldm, false)};
+    }
+    // M <- mu M + G; X0 = bf16(M) / ||bf16(M)||_F into the class slot
+    for (int i = begin; i < end; ++i) {
+      const int c = cls[i - begin];
+      if (c < 0) continue;
+      const int64_t slot = slots[i - begin];
+      const NsClass& k = ns[c];
+      const int64_t count = rows[i] * cols[i];
+      const int blocks = static_cast<int>(std::min<int64_t>((count + 1023) / 1024, 4 * dev->sms));
+      prof_begin(stream);
+      momentum_kernel<<<std::max(blocks, 1), 256, 0, stream>>>(M[i], G[i], gd, count, momentum);
+      prof_end(3, stream, 0.0, static_cast<double>(count) * (8 + dtype_size(gd)));
+      st = launch_ok();
+      if (st != MSIGN_OK) return st;
+      st = launch_norm(M[i], DT_FP32, count, 1, DT_BF16, sch.eps, 0, k.w.partials + slot * kNormParts,
+                       k.w.scale + slot, stream);
+      if (st != MSIGN_OK) return st;
+      const bool tr = rows[i] > cols[i];
+      const int64_t ldm = round_up(k.m, 8), per = k.n * ldm;
+      st = launch_ingest(M[i], DT_FP32, rows[i], cols[i], tr, k.w.scale + slot, DT_BF16,
+                         static_cast<char*>(k.w.P[0]) + 2 * slot * per, DT_BF16, ldm, per, k.w.master + slot * per,
+                         ldm, per, 1, stream);
+      if (st != MSIGN_OK) return st;
+    }
+    st = ns_iterate(ns, sch, stream);
+    if (st != MSIGN_OK) return st;
+    // W <- W - lr * sqrt(max(1, rows/cols)) * O
+    for (int i = begin; i < end; ++i) {
+      const int c = cls[i - begin];
+      if (c < 0) continue;
+      const NsClass& k = ns[c];
+      const int64_t ldm = round_up(k.m, 8), per = k.n * ldm;
+      const float coef = lr * std::sqrt(std::max(1.0f, static_cast<float>(rows[i]) / static_cast<float>(cols[i])));
+      dim3 g(static_cast<unsigned>((cols[i] + 31) / 32), static_cast<unsigned>((rows[i] + 31) / 32));
+      prof_begin(stream);
+      apply_update_kernel<<<g, dim3(32, 8), 0, stream>>>(W[i], wd, static_cast<int>(rows[i]),
+                                                         static_cast<int>(cols[i]), k.w.master + slots[i - begin] * per,
+                                                         ldm, rows[i] > cols[i] ? 1 : 0, coef);
+      prof_end(3, stream, 0.0, static_cast<double>(rows[i]) * cols[i] * (4 + 2 * dtype_size(wd)));
+      st = launch_ok();
+      if (st != MSIGN_OK) return st;
+    }
+    begin = end;
+  }
+  return MSIGN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every
+function the header declares, and rejects bad arguments on the host before
+touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+from newton_schulz_msign_b200 import _lib, build
+
+HEADER = os.path.join(ROOT, "include", "msign_b200.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w \*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "sizeof")))
+
+
+def test_header_declares_the_boundary():
+    assert header_functions() == sorted(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in header_functions():
+        assert hasattr(L, name), name
+
+
+def test_exported_symbols_match_nm(L):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in header_functions():
+        assert name in exported
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.msign_abi_version() == 100
+    assert L.msign_status_string(_lib.OK) == b"ok"
+    assert b"timed out" in L.msign_status_string(_lib.ERR_TIMEOUT)
+    assert L.msign_status_string(99) == b"unknown status"
+
+
+def test_workspace_queries_are_host_only(L):
+    assert L.msign_ns_workspace_size(0, 16, 16, _lib.BF16) == 0
+    a = L.msign_ns_workspace_size(1, 256, 512, _lib.BF16)
+    b = L.msign_ns_workspace_size(1, 512, 256, _lib.BF16)
+    assert a == b > 0  # the tall case is oriented to the wide one
+    # two X operand copies + A + B (bf16) + fp32 X, 4096 x 4096
+    big = L.msign_ns_workspace_size(1, 4096, 4096, _lib.BF16)
+    assert 4096 * 4096 * (2 + 2 + 4 + 2 + 2) <= big < 4096 * 4096 * 12 + 2 ** 20
+    assert L.gram_ns_workspace_size(2, 1024, 4096) > 0
+    rows = (ctypes.c_int64 * 3)(4096, 1024, 14336)
+    cols = (ctypes.c_int64 * 3)(4096, 4096, 4096)
+    assert L.muon_step_workspace_size(3, rows, cols) > L.msign_ns_workspace_size(1, 4096, 14336, _lib.BF16)
+    # aligned X with m % 8 == 0 needs no staging workspace
+    assert L.gram_xxt_workspace_size(1, 100, 64, _lib.BF16, 1 << 20) == 0
+    assert L.gram_xxt_workspace_size(1, 100, 63, _lib.BF16, 1 << 20) > 0
+
+
+def test_invalid_arguments_rejected_on_host(L):
+    # negative sizes and bad dtypes fail before any CUDA call
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, -1, 4, 4, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.msign_ns(None, None, 7, _lib.BF16, 1, 4, 4, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    # empty problems are a no-op
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 0, 4, 4, None, None, 0, None) == _lib.OK
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 3, 0, 4, None, None, 0, None) == _lib.OK
+    # null data pointers with a non-empty problem
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 1, 4, 4, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    # a coefficient table needs a positive step count
+    c = _lib.MsignCoeffs()
+    buf = (ctypes.c_float * 3)(1.0, 0.0, 0.0)
+    c.steps, c.abc, c.eps = 0, ctypes.cast(buf, ctypes.POINTER(ctypes.c_float)), -1.0
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == \
+        _lib.ERR_INVALID_ARG
+    c.steps = 100  # beyond the built maximum
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == \
+        _lib.ERR_UNSUPPORTED
+    # workspace missing for a real problem (pointer values are never dereferenced on this path)
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, None, None, 0, None) == _lib.ERR_WORKSPACE
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.FP32, 1, 4, 4, None, None, 0, None) == _lib.ERR_UNSUPPORTED
+
+
+def test_gram_ns_restart_validation(L):
+    r = (ctypes.c_int * 1)(5)  # must lie in 1..T-1
+    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, None, ctypes.cast(r, ctypes.POINTER(ctypes.c_int)), 1, None, 0,
+                     None) == _lib.ERR_INVALID_ARG
+    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, None, None, 2, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, None, None, -1, None, 0, None) == _lib.ERR_WORKSPACE
+
+
+def test_muon_step_validation(L):
+    assert L.muon_step(0, None, None, None, None, None, _lib.BF16, _lib.BF16, 0.95, 0.02, None, None, 0,
+                       None) == _lib.OK
+    assert L.muon_step(-1, None, None, None, None, None, _lib.BF16, _lib.BF16, 0.95, 0.02, None, None, 0,
+                       None) == _lib.ERR_INVALID_ARG
+    one = (ctypes.c_void_p * 1)(16)
+    rows = (ctypes.c_int64 * 1)(8)
+    cols = (ctypes.c_int64 * 1)(8)
+    assert L.muon_step(1, one, one, one, rows, cols, _lib.FP16, _lib.BF16, 0.95, 0.02, None, None, 0,
+                       None) == _lib.ERR_UNSUPPORTED
+    assert L.muon_step(1, one, one, one, rows, cols, _lib.BF16, _lib.BF16, float("nan"), 0.02, None, None, 0,
+                       None) == _lib.ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    import newton_schulz_msign_b200 as msb
+    with pytest.raises(ValueError, match="CUDA"):
+        msb.msign_ns(torch.zeros(4, 4))

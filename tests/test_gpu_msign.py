@@ -1,0 +1,112 @@
+"""msign_ns on the GPU against the fp64 oracle, through the C ABI."""
+
+import numpy as np
+import pytest
+import torch
+
+import newton_schulz_msign_b200 as msb
+from newton_schulz_msign_b200 import synth
+from oracle import ns_oracle as O
+
+from helpers import TOL_BF16, rel_fro, to_np
+
+pytestmark = pytest.mark.gpu
+
+TDT = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}
+
+
+def run_case(x_np, io="bf16", coeffs=None):
+    x = torch.from_numpy(np.ascontiguousarray(x_np, dtype=np.float32)).to(TDT[io]).cuda()
+    y = msb.msign_ns(x, coeffs=coeffs)
+    msb.sync_status()
+    # the oracle gets exactly the values the GPU received, then casts to bf16
+    # itself (the compute dtype's input cast)
+    ref = O.msign_ns(to_np(x), coeffs, input_cast="bf16")
+    return to_np(y), ref
+
+
+def test_gaussian_256x512_fp32_in():
+    # the single-matrix workload: 256 x 512 fp32 N(0,1), seed 0, bf16 compute
+    x = np.random.default_rng(0).standard_normal((256, 512)).astype(np.float32)
+    got, ref = run_case(x, io="fp32")
+    err = rel_fro(got, ref)
+    assert err < TOL_BF16, err
+    # the output keeps the band NS reaches (Jordan's triple does not converge to 1)
+    s = np.linalg.svd(got, compute_uv=False)
+    assert 0.6 < s.min() and s.max() < 1.2
+    exact = O.msign_svd(x.astype(np.float64))
+    assert 0.05 < rel_fro(got, exact) < 0.3
+
+
+@pytest.mark.parametrize("shape", [(64, 64), (128, 384), (384, 128), (100, 300), (300, 100), (1, 64), (64, 1),
+                                   (7, 129), (129, 7), (256, 2048), (520, 600), (1000, 1000)])
+def test_shapes(shape):
+    x = synth.gaussian(shape, seed=shape[0] * 131 + shape[1])
+    got, ref = run_case(x)
+    assert rel_fro(got, ref) < TOL_BF16
+
+
+@pytest.mark.parametrize("io", ["bf16", "fp16", "fp32"])
+def test_io_dtypes(io):
+    x = synth.gaussian((192, 320), seed=3)
+    got, ref = run_case(x, io=io)
+    assert rel_fro(got, ref) < TOL_BF16
+
+
+def test_batched_mixed_orientation_values():
+    x = synth.gaussian((4, 160, 96), seed=4)
+    got, ref = run_case(x)
+    assert rel_fro(got, ref) < TOL_BF16
+
+
+@pytest.mark.parametrize("table", ["youjiacheng_6step", "dion_5step", "su_ours_x3_5step", "cubic_bernstein"])
+def test_coefficient_tables(coeff_tables, table):
+    x = synth.gaussian((128, 512), seed=5)
+    got, ref = run_case(x, coeffs=coeff_tables[table])
+    assert rel_fro(got, ref) < TOL_BF16
+
+
+def test_momentum_like_spectrum():
+    x = synth.momentum_like(512, 1024, seed=6)
+    got, ref = run_case(x)
+    assert rel_fro(got, ref) < TOL_BF16
+
+
+def test_zero_input_gives_zero():
+    x = torch.zeros(3, 64, 96, dtype=torch.bfloat16, device="cuda")
+    y = msb.msign_ns(x)
+    msb.sync_status()
+    assert torch.count_nonzero(y).item() == 0
+
+
+def test_rank_one_input():
+    u = synth.gaussian((200, 1), seed=7)
+    v = synth.gaussian((1, 300), seed=8)
+    got, ref = run_case(u @ v)
+    assert rel_fro(got, ref) < TOL_BF16
+
+
+def test_repeat_calls_identical():
+    x = torch.from_numpy(synth.gaussian((256, 768), seed=9)).to(torch.bfloat16).cuda()
+    a = msb.msign_ns(x)
+    b = msb.msign_ns(x)
+    msb.sync_status()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("rows,cols,batch", [(4096, 4096, 8), (4096, 11008, 4)])
+def test_momentum_like_full_size(rows, cols, batch):
+    # the batched workload: momentum-like matrices U diag(i^-0.8) V^T + noise,
+    # bf16; the whole batch runs, the first and last matrix are checked
+    # against the oracle, all are checked for finiteness.
+    xs = torch.stack([synth.momentum_like_torch(rows, cols, seed=100 + i, device="cuda") for i in (0, 1)])
+    x = torch.empty(batch, rows, cols, dtype=torch.bfloat16, device="cuda")
+    for i in range(batch):
+        x[i] = xs[0 if i < batch - 1 else 1]
+    y = msb.msign_ns(x)
+    msb.sync_status()
+    assert torch.isfinite(y).all()
+    for i in (0, batch - 1):
+        ref = O.msign_ns(to_np(x[i]), input_cast="bf16")
+        assert rel_fro(to_np(y[i]), ref) < TOL_BF16
+    assert torch.equal(y[0], y[1])

@@ -1,0 +1,105 @@
+"""muon_step on the GPU against the fp64 oracle."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import newton_schulz_msign_b200 as msb
+from newton_schulz_msign_b200 import synth
+from oracle import ns_oracle as O
+
+from helpers import TOL_BF16, rel_fro, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def make(shapes, wdt, gdt, seed):
+    W, M, G = [], [], []
+    for i, (r, c) in enumerate(shapes):
+        W.append(synth.gaussian_torch((r, c), seed=seed + 3 * i, device="cuda", std=0.02).to(wdt))
+        M.append(synth.gaussian_torch((r, c), seed=seed + 3 * i + 1, device="cuda", std=1e-3))
+        G.append(synth.gaussian_torch((r, c), seed=seed + 3 * i + 2, device="cuda", std=1e-4).to(gdt))
+    return W, M, G
+
+
+def check_matrix(W0, M0, G, W1, M1, lr, mu=0.95):
+    r, c = W0.shape
+    Wr, Mr, Or = O.muon_step(to_np(W0), to_np(M0), to_np(G), momentum=mu, lr=lr, input_cast="bf16")
+    # momentum: fp32 fused multiply-add of exact inputs
+    assert rel_fro(to_np(M1), Mr) < 1e-6
+    scale = math.sqrt(max(1.0, r / c))
+    dW_ref = Wr - to_np(W0)
+    dW = to_np(W1) - to_np(W0)
+    if W1.dtype == torch.float32:
+        assert rel_fro(dW, dW_ref) < TOL_BF16
+    else:
+        # bf16 weights: the update is rounded into W; every element must lie
+        # within one bf16 rounding of the exact update, plus the NS error
+        slack = 2.0 ** -8 * np.abs(to_np(W1)) + 0.1 * lr * scale * np.abs(Or) + 1e-7
+        assert np.all(np.abs(to_np(W1) - Wr) <= slack)
+        assert rel_fro(dW, dW_ref) < 0.1
+
+
+@pytest.mark.parametrize("wdt,gdt", [(torch.float32, torch.float32), (torch.float32, torch.bfloat16),
+                                     (torch.bfloat16, torch.bfloat16)])
+def test_muon_small_mixed_shapes(wdt, gdt):
+    shapes = [(64, 128), (128, 64), (96, 96), (200, 72), (64, 128), (33, 257)]
+    W, M, G = make(shapes, wdt, gdt, seed=100)
+    W0 = [w.clone() for w in W]
+    M0 = [m.clone() for m in M]
+    msb.muon_step(W, M, G, momentum=0.95, lr=0.02)
+    msb.sync_status()
+    for i in range(len(shapes)):
+        check_matrix(W0[i], M0[i], G[i], W[i], M[i], 0.02)
+
+
+def test_muon_equals_msign_composition():
+    # the fused step equals momentum + msign_ns + scaled update done by hand
+    shapes = [(256, 128), (128, 384)]
+    W, M, G = make(shapes, torch.float32, torch.float32, seed=200)
+    W0 = [w.clone() for w in W]
+    M0 = [m.clone() for m in M]
+    msb.muon_step(W, M, G, momentum=0.9, lr=0.05)
+    msb.sync_status()
+    for i, (r, c) in enumerate(shapes):
+        Mn = 0.9 * M0[i] + G[i]
+        assert torch.allclose(M[i], Mn, rtol=1e-6, atol=1e-9)
+        O_ = msb.msign_ns(Mn)
+        Wn = W0[i] - 0.05 * math.sqrt(max(1.0, r / c)) * O_
+        assert torch.allclose(W[i], Wn, rtol=1e-5, atol=1e-6)
+
+
+def test_muon_small_workspace_processes_in_groups():
+    shapes = [(128, 256), (256, 128), (128, 256), (64, 64)]
+    W, M, G = make(shapes, torch.float32, torch.float32, seed=300)
+    Wb, Mb = [w.clone() for w in W], [m.clone() for m in M]
+    msb.muon_step(W, M, G)
+    need_one = max(msb.muon_step_workspace_size([s]) for s in shapes)
+    ws = torch.empty(need_one, dtype=torch.uint8, device="cuda")
+    msb.muon_step(Wb, Mb, G, workspace=ws)
+    msb.sync_status()
+    for a, b in zip(W, Wb):
+        assert torch.equal(a, b)
+    for a, b in zip(M, Mb):
+        assert torch.equal(a, b)
+
+
+def test_muon_llama_layer_full_size():
+    # one Llama-3-8B decoder layer (q, k, v, o, gate, up, down) at full size,
+    # bf16 weights, fp32 momentum, G ~ N(0, 1e-4^2); the q, k and down
+    # matrices (one per distinct oriented shape class) are checked against
+    # the oracle, the rest for finiteness.
+    shapes = [(r, c) for _, r, c in synth.llama3_8b_layer_shapes()]
+    W, M, G = make(shapes, torch.bfloat16, torch.bfloat16, seed=400)
+    for m in M:
+        m.zero_()
+    W0 = [w.clone() for w in W]
+    M0 = [m.clone() for m in M]
+    msb.muon_step(W, M, G, momentum=0.95, lr=0.02)
+    msb.sync_status()
+    for w in W:
+        assert torch.isfinite(w).all()
+    for i in (0, 1, 6):
+        check_matrix(W0[i], M0[i], G[i], W[i], M[i], 0.02)
