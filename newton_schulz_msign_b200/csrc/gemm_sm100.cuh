@@ -7,30 +7,58 @@
 // concatenation of the classes' tiles (the host orders classes by K, longest
 // first, so short tiles fill the tail of the last wave).
 //
-// Roles inside a 192-thread CTA (one CTA per SM, persistent over tiles):
-//   warp 0      TMA producer: fills a kStages-deep ring of 128-byte-swizzled
-//               shared-memory stages (A 128x64, B 256x64 elements).
-//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators)
-//               and issues tcgen05.mma (M=128, N=256, K=16) from one thread;
-//               tcgen05.commit releases a stage / publishes an accumulator.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32*(w%4)..+31 = tile rows), fused arithmetic
-//               v = alpha*acc + beta*C, then up to kMaxOuts stores, each
-//               direct or transposed (through a padded shared-memory
-//               transpose) and each with its own gamma*I diagonal term.
+// The kernel runs on CTA pairs (clusters of two CTAs on one TPC) that share
+// a tcgen05.mma.cta_group::2 instruction stream: a 256 x 256 output tile is
+// one M = 256, N = 256 MMA per 16-wide K slice, with A's rows 0..127 and B's
+// rows 0..127 staged in the leader CTA and the other halves in the peer.
+// Each SM thus streams half of B per FLOP compared with a one-SM 128 x 256
+// tile, which is what keeps the tensor pipe fed from L2.
+//
+// Roles inside each 192-thread CTA (one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer, in both CTAs: loads this CTA's halves of A and
+//               B (128 x 64 elements each, 128-byte swizzle) into a
+//               kStages-deep ring; completion is counted on the LEADER's
+//               stage barrier, which expects the bytes of both CTAs.
+//   warp 1      allocates 512 TMEM columns in both CTAs (two 128 x 256 fp32
+//               accumulators per CTA); in the leader one thread issues the
+//               MMAs and tcgen05.commit-multicasts stage releases and
+//               accumulator-ready signals to both CTAs.
+//   warps 2..5  epilogue, in both CTAs: tcgen05.ld of this CTA's 128
+//               accumulator rows (warp w reads TMEM lanes 32*(w%4)..+31),
+//               fused arithmetic v = alpha*acc + beta*C, then up to
+//               kMaxOuts stores, each direct or transposed and each with its
+//               own gamma*I term.  Every 32x32 block moves between registers
+//               and global memory through a swizzled shared-memory block, so
+//               all global accesses are coalesced 16-byte row segments.  One
+//               lane per warp then releases the accumulator on the leader's
+//               barrier.
 //
 // Symmetric classes ([P1] flash-muon matmul_transpose; [P3] section 4,
-// triangular scheduler) enumerate only tiles that touch the upper triangle
-// (tile (tm, tn) with tn >= tm/2 for 128x256 tiles).  In them, 32x32 blocks
-// strictly below the diagonal are skipped, blocks above it are stored
-// directly and transposed into the mirrored position, and diagonal blocks
-// store their upper part directly and their strict upper part transposed.
-// Both copies come from the same fp32 value with the same rounding, so the
-// stored matrix is bit-exactly symmetric.
+// triangular scheduler) enumerate only tiles (tm, tn) with tn >= tm.  A
+// mirrored tile (every tile in mirror mode, the diagonal tiles otherwise)
+// skips its 32x32 blocks strictly below the diagonal, stores the blocks
+// above it directly and transposed into the mirrored position, and stores
+// the upper part of diagonal blocks directly and their strict upper part
+// transposed.  Both copies come from the same fp32 value with the same
+// rounding, so the stored matrix is bit-exactly symmetric.
 //
 // The B operand is read K-major (rows of B_op are the output columns) or
 // MN-major (B_op^T stored row-major as K x N, e.g. X in B*X), the latter via
 // the UMMA descriptor's MN-major mode, so X is never transposed in memory.
+//
+// Symmetric intermediates (A and B of standard NS; R, Z, Q and RZ of Gram
+// NS) are stored by upper 256 x 256 blocks only: a triangle-scheduled
+// product writes its tiles (tm, tn >= tm) and nothing else, the diagonal
+// tiles symmetrised from their upper triangle (Gram NS needs its
+// intermediates exactly symmetric: products of commuting matrices such as
+// Q Z are symmetric only up to rounding, and that asymmetry grows).  A
+// consumer that needs rows [R, R+256) x K slice [k0, k0+64) of such a matrix
+// with k0 + 64 <= R reads the stored transpose S[k0.., R..] instead and
+// feeds it to the MMA through an MN-major descriptor (decided per K slice,
+// identically for both CTAs of the pair).  Only the user-facing X X^T keeps
+// exact mirror stores.
+//
+// No load anywhere uses cluster multicast: each CTA fetches its own halves.
 #pragma once
 
 #include <cuda.h>
@@ -44,25 +72,30 @@
 
 namespace msb {
 
-constexpr int kBM = 128;
-constexpr int kBN = 256;
-constexpr int kBK = 64;  // 64 16-bit elements = one 128-byte swizzle row
-constexpr int kStages = 4;
+constexpr int kBM = 256;      // output tile rows per CTA pair
+constexpr int kHalfM = 128;   // rows per CTA (= TMEM lanes)
+constexpr int kBN = 256;      // output tile columns
+constexpr int kHalfN = 128;   // B rows staged per CTA
+constexpr int kBK = 64;       // 64 16-bit elements = one 128-byte swizzle row
+constexpr int kStages = 6;
 constexpr int kThreads = 192;
-constexpr int kATileBytes = kBM * kBK * 2;  // 16 KB
-constexpr int kBTileBytes = kBN * kBK * 2;  // 32 KB
+constexpr int kATileBytes = kHalfM * kBK * 2;  // 16 KB
+constexpr int kBTileBytes = kHalfN * kBK * 2;  // 16 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
-constexpr int kEpiStride = 33;  // padded row of the 32x32 transpose buffer
-constexpr int kEpiWarpFloats = 32 * kEpiStride;
+constexpr int kScratchStride = 33;  // padded row of the per-warp 32 x 32 fp32 transpose scratch
+constexpr int kStageOutBytes = 32 * kScratchStride * 4;
+constexpr int kEpiBytes = 4 * kStageOutBytes;  // one scratch block per epilogue warp
 constexpr int kTmemCols = 512;
 constexpr int kMaxClasses = 8;
 constexpr int kNumBarriers = 2 * kStages + 2 + 2 + 1;
-constexpr int kSmemBytes = 1024 /* alignment slack */ + kStages * kStageBytes + 4 * kEpiWarpFloats * 4 +
-                           kNumBarriers * 8 + 16;
+constexpr int kSmemBytes = 1024 /* alignment slack */ + kStages * kStageBytes + kEpiBytes + kNumBarriers * 8 + 16;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum : int { DT_BF16 = 0, DT_FP16 = 1, DT_FP32 = 2 };
 
 __host__ __device__ inline int dtype_size(int dt) { return dt == DT_FP32 ? 4 : 2; }
+
+constexpr int kMaxOuts = 4;
 
 // One epilogue output.  Direct: D[row][col] = w; transposed: D[col][row] = w,
 // where w = v + gamma * [row == col] and v = alpha*acc + beta*C.
@@ -75,21 +108,31 @@ struct EpiOut {
   int pad;
 };
 
-constexpr int kMaxOuts = 4;
-
-struct alignas(64) GemmClass {
-  CUtensorMap tmA;  // (k, row, batch), K-major, box 64 x 128
-  CUtensorMap tmB;  // K-major: (k, col, batch) box 64 x 256; MN-major: (col, k, batch) box 64 x 64
+// Per-class scalars: tile schedule and epilogue (read through the constant
+// cache of the kernel parameters).
+struct ClassInfo {
   int M, N, K, batch;
   int tiles_m, tiles_n, tiles_per_batch, tile_begin;
-  int symmetric, b_mn_major, num_out, pad0;
+  int symmetric;   // output tiles (tm, tn) with tn >= tm only
+  int mirror;      // symmetric: every tile also stores its mirror (full, exactly symmetric matrix)
+  int a_sym;       // A operand is a symmetric matrix stored by upper 256-blocks
+  int b_sym;       // same for the B operand (K-major)
+  int b_mn_major;  // B operand stored K x N (MN-major)
+  int num_out, c_dtype, pad0;
   float alpha, beta;
   const float* alpha_scale;  // optional per-batch factor on alpha
   const float* beta_scale;   // optional per-batch factor on beta
   const void* C;             // optional epilogue input, C[row][col]
   long long ldc, c_bs;
-  int c_dtype, pad1;
   EpiOut out[kMaxOuts];
+};
+
+struct alignas(64) GemmClass {
+  CUtensorMap tmA;   // (k, row, batch), K-major, box 64 x 128
+  CUtensorMap tmB;   // K-major: (k, col, batch) box 64 x 128; MN-major: (col, k, batch) box 64 x 64
+  CUtensorMap tmA2;  // a_sym: the same matrix with a 64 x 64 box, for transposed K slices
+  CUtensorMap tmB2;  // b_sym: likewise
+  ClassInfo info;
 };
 
 struct GemmParams {
@@ -107,8 +150,8 @@ struct TileCoord {
 
 __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
   int c = 0;
-  while (c + 1 < p.num_classes && t >= p.cls[c + 1].tile_begin) ++c;
-  const GemmClass& k = p.cls[c];
+  while (c + 1 < p.num_classes && t >= p.cls[c + 1].info.tile_begin) ++c;
+  const ClassInfo& k = p.cls[c].info;
   int l = t - k.tile_begin;
   int b = l / k.tiles_per_batch;
   int r = l - b * k.tiles_per_batch;
@@ -117,14 +160,15 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
     tm = r / k.tiles_n;
     tn = r - tm * k.tiles_n;
   } else {
+    // square 256 x 256 tiles on or above the diagonal, row by row
     tm = 0;
     while (true) {
-      int cnt = k.tiles_n - (tm >> 1);
+      int cnt = k.tiles_n - tm;
       if (r < cnt) break;
       r -= cnt;
       ++tm;
     }
-    tn = (tm >> 1) + r;
+    tn = tm + r;
   }
   return {c, b, tm, tn};
 }
@@ -224,58 +268,84 @@ __device__ __forceinline__ char* row_ptr(void* base, int dt, long long ld, long 
 }
 
 // ---------------------------------------------------------------- epilogue
+//
+// Each lane owns one accumulator row (TMEM lane = tile row) and moves its 32
+// consecutive elements of a block with 16-byte accesses.  Transposed outputs
+// go through a 32 x 32 fp32 scratch block in shared memory whose rows are
+// padded to 33 words, so that writing by rows and reading by columns are both
+// conflict-free with one instruction per access.
+
+__device__ __forceinline__ char* gaddr(const void* p, int dt, long long ld, long long bs, int b, long long r,
+                                       long long c) {
+  return const_cast<char*>(reinterpret_cast<const char*>(p)) +
+         (static_cast<long long>(b) * bs + r * ld + c) * dtype_size(dt);
+}
+
+__device__ __forceinline__ uint32_t lane_mask(int n) { return n >= 32 ? 0xFFFFFFFFu : ((1u << n) - 1u); }
+
+// Epilogue input of the block at (row0, col0) for this lane's row.
+__device__ __forceinline__ void load_c(const ClassInfo& k, int b, int row0, int col0, int lane, float (&cv)[32]) {
+  const int r = row0 + lane;
+  const uint32_t m = (r < k.M) ? lane_mask(k.N - col0) : 0u;
+  load_row32(gaddr(k.C, k.c_dtype, k.ldc, k.c_bs, b, r, col0), k.c_dtype, m, cv);
+}
 
 // One 32x32 block: this lane owns output row `row0 + lane`, columns
-// col0..col0+31, whose fp32 accumulators are in `acc`.
-__device__ __forceinline__ void epilogue_block(const GemmClass& k, int b, int row0, int col0, float (&acc)[32],
-                                               float* stage, int lane) {
+// col0..col0+31, whose fp32 accumulators are in `acc` and epilogue input in
+// `cv` (when the class has one).  `mirror`: the block is stored together
+// with its transpose at the mirrored position (symmetric classes: every
+// block of mirror classes, and the blocks of diagonal tiles); on a diagonal
+// block the upper part and its mirror fill the block, so the stored matrix
+// is exactly symmetric there.
+__device__ __forceinline__ void epilogue_block(const ClassInfo& k, int b, int row0, int col0, bool mirror,
+                                               float (&acc)[32], const float (&cv)[32], float* scratch, int lane) {
   const int r = row0 + lane;
-  const bool diag = k.symmetric && (col0 == row0);
-  const uint32_t colmask = (k.N - col0 >= 32) ? 0xFFFFFFFFu : ((1u << (k.N - col0)) - 1u);
-  const uint32_t rowmask = (k.M - row0 >= 32) ? 0xFFFFFFFFu : ((1u << (k.M - row0)) - 1u);
+  const bool diag = mirror && (col0 == row0);
+  const uint32_t colmask = lane_mask(k.N - col0);
+  const uint32_t rowmask = lane_mask(k.M - row0);
 
   float alpha = k.alpha;
   if (k.alpha_scale != nullptr) alpha *= k.alpha_scale[b];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] *= alpha;
-
   if (k.C != nullptr) {
     float beta = k.beta;
     if (k.beta_scale != nullptr) beta *= k.beta_scale[b];
-    float cv[32];
-    const uint32_t m = (r < k.M) ? colmask : 0u;
-    load_row32(row_ptr(const_cast<void*>(k.C), k.c_dtype, k.ldc, k.c_bs, b, r, col0), k.c_dtype, m, cv);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = fmaf(beta, cv[i], acc[i]);
+    for (int i = 0; i < 32; ++i) acc[i] = fmaf(alpha, acc[i], beta * cv[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] *= alpha;
   }
 
 #pragma unroll 1
   for (int o = 0; o < k.num_out; ++o) {
     const EpiOut& e = k.out[o];
     float w[32];
+    const float g = (col0 == row0) ? e.gamma : 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) w[i] = (col0 + i == r) ? acc[i] + e.gamma : acc[i];
-    if (!e.transposed) {
-      if (r < k.M) {
-        uint32_t m = colmask;
-        if (diag) m &= (0xFFFFFFFFu << lane);  // keep columns c >= r
-        store_row32(row_ptr(e.ptr, e.dtype, e.ld, e.bs, b, r, col0), e.dtype, m, w);
-      }
-    } else {
-      // stage[i][lane] = w(row0 + lane, col0 + i); read back transposed so
-      // that lane l owns row col0 + l of D, columns row0..row0+31.
+    for (int i = 0; i < 32; ++i) w[i] = (i == lane) ? acc[i] + g : acc[i];
+    const bool direct = !e.transposed;
+    const bool trans = e.transposed || mirror;
+    if (direct && r < k.M) {
+      uint32_t m = colmask;
+      if (diag) m &= (0xFFFFFFFFu << lane);  // columns c >= r; the mirror supplies c < r
+      store_row32(gaddr(e.ptr, e.dtype, e.ld, e.bs, b, r, col0), e.dtype, m, w);
+    }
+    if (trans) {
+      // scratch[i][lane] = w(row0 + lane, col0 + i) in rows padded to 33
+      // words (conflict-free both ways); lane l then reads its column l,
+      // which is row col0 + l of the transposed block
 #pragma unroll
-      for (int i = 0; i < 32; ++i) stage[i * kEpiStride + lane] = w[i];
+      for (int i = 0; i < 32; ++i) scratch[i * kScratchStride + lane] = w[i];
       __syncwarp();
       float t[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) t[j] = stage[lane * kEpiStride + j];
+      for (int j = 0; j < 32; ++j) t[j] = scratch[lane * kScratchStride + j];
       __syncwarp();
-      const int tr = col0 + lane;
+      const int tr = col0 + lane;  // row of the transposed block
       if (tr < k.N) {
         uint32_t m = rowmask;
-        if (diag) m &= (lane == 0) ? 0u : (0xFFFFFFFFu >> (32 - lane));  // keep rows r < c (strict)
-        store_row32(row_ptr(e.ptr, e.dtype, e.ld, e.bs, b, tr, row0), e.dtype, m, t);
+        if (diag) m &= (lane == 0) ? 0u : (0xFFFFFFFFu >> (32 - lane));  // rows r < c (strict)
+        store_row32(gaddr(e.ptr, e.dtype, e.ld, e.bs, b, tr, row0), e.dtype, m, t);
       }
     }
   }
@@ -283,23 +353,29 @@ __device__ __forceinline__ void epilogue_block(const GemmClass& k, int b, int ro
 
 // ---------------------------------------------------------------- kernel
 
-__global__ void __launch_bounds__(kThreads, 1) gemm_sm100_kernel(const __grid_constant__ GemmParams p) {
+// Launched with clusters of 2 CTAs along x; gridDim.x is even.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_sm100_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kATileBytes;
-  float* sEpi = reinterpret_cast<float*>(sB + kStages * kBTileBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + 4 * kEpiWarpFloats);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  uint64_t* tfull = bars + 2 * kStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint8_t* sOut = sB + kStages * kBTileBytes;  // epilogue staging, kEpiBytes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + kEpiBytes);
+  uint64_t* full = bars;             // leader: both CTAs' loads of a stage landed
+  uint64_t* empty = bars + kStages;  // both: the MMAs reading a stage finished
+  uint64_t* tfull = bars + 2 * kStages;  // both: accumulator buffer ready
+  uint64_t* tempty = tfull + 2;          // leader: both epilogues drained a buffer
+  uint64_t* drain = tempty + 2;          // leader: every issued MMA finished
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + kNumBarriers);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
   const uint64_t limit = p.timeout_ns;
 
   if (threadIdx.x == 0) {
@@ -309,15 +385,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_sm100_kernel(const __grid_co
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4 * 32);
+      mbar_init(&tempty[i], 2 * 4);  // one arrival per epilogue warp of each CTA
     }
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(s_tmem, kTmemCols);
+    tmem_relinquish_pair();
   }
   if (warp == 0 && lane == 0) {
     for (int c = 0; c < p.num_classes; ++c) {
@@ -327,35 +403,60 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_sm100_kernel(const __grid_co
   }
   tc_fence_before();
   __syncthreads();
+  // both CTAs' barriers are initialised before either signals the other's
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t used = 0, last_phase = 0;  // per-stage bits
+      uint32_t used = 0, last_phase = 0;  // per-stage bits (leader only)
       bool ok = true;
-      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+      const uint32_t sA0 = smem_u32(sA), sB0 = smem_u32(sB);
+      for (int t = pair; t < p.total_tiles && ok; t += num_pairs) {
         const TileCoord tc = decode_tile(p, t);
-        const GemmClass& k = p.cls[tc.c];
+        const ClassInfo& k = p.cls[tc.c].info;
+        // per-tile state in registers
         const int nk = (k.K + kBK - 1) / kBK;
+        const int arow = tc.tm * kBM + static_cast<int>(rank) * kHalfM;
+        const int bcol = tc.tn * kBN + static_cast<int>(rank) * kHalfN;
+        const int a_tr = k.a_sym ? (tc.tm * kBM) / kBK : 0;  // K slices below this read A transposed
+        const int b_tr = k.b_sym ? (tc.tn * kBN) / kBK : 0;
+        const bool b_mn = k.b_mn_major != 0;
+        const GemmClass& g = p.cls[tc.c];
+        const void* tmA = &g.tmA;
+        const void* tmA2 = &g.tmA2;
+        const void* tmB = &g.tmB;
+        const void* tmB2 = &g.tmB2;
+        const int bz = tc.b;
         for (int kb = 0; kb < nk; ++kb) {
           if (!wait_bounded(&empty[stage], phase ^ 1u, s_abort, p.err, limit)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+          const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = sA + stage * kATileBytes;
           uint8_t* b_dst = sB + stage * kBTileBytes;
-          tma_load_3d(a_dst, &k.tmA, &full[stage], kb * kBK, tc.tm * kBM, tc.b);
-          if (!k.b_mn_major) {
-            tma_load_3d(b_dst, &k.tmB, &full[stage], kb * kBK, tc.tn * kBN, tc.b);
+          const int k0 = kb * kBK;
+          if (kb < a_tr) {
+            // stored transpose: rows k0.. of S, columns arow..arow+127 (MN-major)
+            tma_load_3d_pair(a_dst, tmA2, fbar, arow, k0, bz);
+            tma_load_3d_pair(a_dst + kBK * 64 * 2, tmA2, fbar, arow + 64, k0, bz);
           } else {
-#pragma unroll
-            for (int c = 0; c < kBN / 64; ++c)
-              tma_load_3d(b_dst + c * (kBK * 64 * 2), &k.tmB, &full[stage], tc.tn * kBN + c * 64, kb * kBK, tc.b);
+            tma_load_3d_pair(a_dst, tmA, fbar, k0, arow, bz);
+          }
+          if (kb < b_tr) {
+            tma_load_3d_pair(b_dst, tmB2, fbar, bcol, k0, bz);
+            tma_load_3d_pair(b_dst + kBK * 64 * 2, tmB2, fbar, bcol + 64, k0, bz);
+          } else if (!b_mn) {
+            tma_load_3d_pair(b_dst, tmB, fbar, k0, bcol, bz);
+          } else {
+            tma_load_3d_pair(b_dst, tmB, fbar, bcol, k0, bz);
+            tma_load_3d_pair(b_dst + kBK * 64 * 2, tmB, fbar, bcol + 64, k0, bz);
           }
           used |= 1u << stage;
           last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
@@ -365,25 +466,36 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_sm100_kernel(const __grid_co
           }
         }
       }
-      // Never leave the CTA with bulk copies still landing in its shared
-      // memory: wait (bounded, ignoring the abort word) for the last load
-      // issued into every stage.
-      for (int s = 0; s < kStages; ++s)
-        if ((used >> s) & 1u) wait_bounded(&full[s], (last_phase >> s) & 1u, nullptr, p.err, limit);
+      (void)sA0;
+      (void)sB0;
+      // Never leave the pair with bulk copies still landing: the leader's
+      // stage barriers count both CTAs' bytes, so the leader waits (bounded,
+      // ignoring the abort word) for the last phase issued into each stage.
+      if (leader)
+        for (int s = 0; s < kStages; ++s)
+          if ((used >> s) & 1u) wait_bounded(&full[s], (last_phase >> s) & 1u, nullptr, p.err, limit);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
       uint32_t bphase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+      const uint32_t idesc0 = p.idesc;
+      const uint32_t sA0 = smem_u32(sA), sB0 = smem_u32(sB);
+      // K-major and MN-major descriptors of stage 0; stage s adds s * tile
+      // bytes and K step kk adds 32 (K-major) or 2048 (MN-major) bytes, all
+      // in the 16-byte-unit start-address field.
+      const uint64_t dA_k = smem_desc_sw128(sA0, 16, 1024), dA_mn = smem_desc_sw128(sA0, kBK * 64 * 2, 1024);
+      const uint64_t dB_k = smem_desc_sw128(sB0, 16, 1024), dB_mn = smem_desc_sw128(sB0, kBK * 64 * 2, 1024);
+      for (int t = pair; t < p.total_tiles && ok; t += num_pairs) {
         const TileCoord tc = decode_tile(p, t);
-        const GemmClass& k = p.cls[tc.c];
+        const ClassInfo& k = p.cls[tc.c].info;
         const int nk = (k.K + kBK - 1) / kBK;
-        const uint32_t idesc = p.idesc | (static_cast<uint32_t>(k.b_mn_major) << 16);
+        const int a_tr = k.a_sym ? (tc.tm * kBM) / kBK : 0;
+        const int b_tr = k.b_sym ? (tc.tn * kBN) / kBK : (k.b_mn_major ? nk : 0);
         if (!wait_bounded(&tempty[buf], bphase ^ 1u, s_abort, p.err, limit)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
@@ -393,50 +505,63 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_sm100_kernel(const __grid_co
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + stage * kATileBytes);
-          const uint32_t b_base = smem_u32(sB + stage * kBTileBytes);
+          const bool a_mn = kb < a_tr;
+          const bool b_mn = kb < b_tr;
+          const uint32_t idesc = idesc0 | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16);
+          const uint64_t da = (a_mn ? dA_mn : dA_k) + static_cast<uint64_t>((stage * kATileBytes) >> 4);
+          const uint64_t db = (b_mn ? dB_mn : dB_k) + static_cast<uint64_t>((stage * kBTileBytes) >> 4);
+          const uint32_t sa = a_mn ? (2048 >> 4) : (32 >> 4);
+          const uint32_t sb = b_mn ? (2048 >> 4) : (32 >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(a_base + kk * 32, 16, 1024);
-            const uint64_t bdesc = k.b_mn_major ? smem_desc_sw128(b_base + kk * 2048, kBK * 64 * 2, 1024)
-                                                : smem_desc_sw128(b_base + kk * 32, 16, 1024);
-            umma_f16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
-          }
-          umma_commit(&empty[stage]);
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_f16_pair(d_tmem, da + kk * sa, db + kk * sb, idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[buf]);
+        umma_commit_pair_mc(&tfull[buf], 0x3);
         buf ^= 1;
         if (buf == 0) bphase ^= 1u;
       }
       // every MMA issued so far has finished before TMEM is released
-      umma_commit(drain);
+      umma_commit_pair_mc(drain, 0x1);
       wait_bounded(drain, 0, nullptr, p.err, limit);
     }
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;  // TMEM lane quarter this warp may read
-    float* stage_buf = sEpi + (warp - 2) * kEpiWarpFloats;
+    float* scratch = reinterpret_cast<float*>(sOut + (warp - 2) * kStageOutBytes);
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
     int buf = 0;
     uint32_t bphase = 0;
-    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+    for (int t = pair; t < p.total_tiles; t += num_pairs) {
       const TileCoord tc = decode_tile(p, t);
-      const GemmClass& k = p.cls[tc.c];
+      const ClassInfo& k = p.cls[tc.c].info;
+      const int row0 = tc.tm * kBM + static_cast<int>(rank) * kHalfM + q * 32;
+      // mirrored tiles visit only blocks on or above the diagonal
+      const bool mirror = k.symmetric && (k.mirror || tc.tm == tc.tn);
+      int jfirst = 0;
+      if (mirror)
+        while (jfirst < kBN / 32 && tc.tn * kBN + jfirst * 32 < row0) ++jfirst;
+      // the epilogue input of the first block is read before the
+      // accumulator is ready
+      const bool has_c = k.C != nullptr;
+      float cv[32];
+      if (has_c && row0 < k.M && jfirst < kBN / 32 && tc.tn * kBN + jfirst * 32 < k.N)
+        load_c(k, tc.b, row0, tc.tn * kBN + jfirst * 32, lane, cv);
       int ok = 1;
       if (lane == 0) ok = wait_bounded(&tfull[buf], bphase, s_abort, p.err, limit) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const int row0 = tc.tm * kBM + q * 32;
 #pragma unroll 1
-      for (int j = 0; j < kBN / 32; ++j) {
+      for (int j = jfirst; j < kBN / 32; ++j) {
         const int col0 = tc.tn * kBN + j * 32;
-        if (row0 >= k.M || col0 >= k.N) continue;
-        if (k.symmetric && col0 < row0) continue;
+        if (row0 >= k.M || col0 >= k.N) break;
         uint32_t raw[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * kBN + j * 32),
                            raw);
@@ -444,20 +569,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_sm100_kernel(const __grid_co
         float acc[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) acc[i] = __uint_as_float(raw[i]);
-        epilogue_block(k, tc.b, row0, col0, acc, stage_buf, lane);
+        if (has_c && j != jfirst) load_c(k, tc.b, row0, col0, lane, cv);
+        epilogue_block(k, tc.b, row0, col0, mirror, acc, cv, scratch, lane);
       }
       tc_fence_before();
-      mbar_arrive(&tempty[buf]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
       buf ^= 1;
       if (buf == 0) bphase ^= 1u;
     }
   }
 
+  // Reconverge every warp first: in the producer and MMA warps only lane 0
+  // ran the role loop, and a block barrier reached by a warp in two pieces
+  // would let the CTA go on (and release TMEM) while others still work.
+  __syncwarp();
   __syncthreads();
+  // no CTA of the pair leaves while the other may still signal it
+  cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 

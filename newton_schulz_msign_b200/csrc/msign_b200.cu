@@ -36,6 +36,7 @@ constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per wait
 struct DeviceState {
   bool ready = false;
   int sms = 0;
+  int max_pairs = 0;  // CTA pairs of the GEMM kernel that fit on the GPU at once
   int* err = nullptr;
 };
 
@@ -58,6 +59,25 @@ msign_status device_state(DeviceState** out) {
     if (cudaFuncSetAttribute(gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
         cudaSuccess)
       return MSIGN_ERR_CUDA;
+    {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(static_cast<unsigned>(d.sms & ~1), 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, gemm_sm100_kernel, &cfg) != cudaSuccess || clusters < 1) {
+        (void)cudaGetLastError();
+        clusters = d.sms / 2;
+      }
+      d.max_pairs = clusters;
+    }
     if (g_encode == nullptr) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -218,7 +238,10 @@ EpiOut out_to(void* ptr, int dt, int64_t ld, int64_t bs, bool transposed, float 
 struct ClassSpec {
   Mat A, B;
   bool b_mn = false;
-  bool symmetric = false;
+  bool symmetric = false;  // triangle schedule (M == N)
+  bool mirror = false;     // symmetric: write exact mirrors (else upper 256-blocks only)
+  bool a_sym = false;      // A is a symmetric matrix stored by upper 256-blocks
+  bool b_sym = false;      // B likewise
   int64_t M = 0, N = 0, K = 0, batch = 0;
   float alpha = 1.0f, beta = 0.0f;
   const float* alpha_scale = nullptr;
@@ -229,11 +252,10 @@ struct ClassSpec {
   std::vector<EpiOut> outs;
 };
 
+// Square kBM x kBN tiles on or above the diagonal.
 int64_t triangle_tiles(int64_t n) {
-  const int64_t tm_n = (n + kBM - 1) / kBM, tn_n = (n + kBN - 1) / kBN;
-  int64_t c = 0;
-  for (int64_t tm = 0; tm < tm_n; ++tm) c += tn_n - tm / 2;
-  return c;
+  const int64_t t = (n + kBN - 1) / kBN;
+  return t * (t + 1) / 2;
 }
 
 int64_t class_tiles(const ClassSpec& s) {
@@ -267,37 +289,48 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     Mat a = s.A;
     a.rows = s.M;
     a.cols = s.K;
-    if (!encode(&c.tmA, a, true, kBM, s.batch)) return MSIGN_ERR_CUDA;
+    if (!encode(&c.tmA, a, true, kHalfM, s.batch)) return MSIGN_ERR_CUDA;
+    if (s.a_sym && (s.M != s.K || !encode(&c.tmA2, a, false, kBK, s.batch))) return MSIGN_ERR_INVALID_ARG;
     Mat b = s.B;
+    if (s.b_sym) {
+      if (s.b_mn || s.N != s.K) return MSIGN_ERR_INVALID_ARG;
+      b.rows = s.N;
+      b.cols = s.K;
+      if (!encode(&c.tmB2, b, false, kBK, s.batch)) return MSIGN_ERR_CUDA;
+    }
     if (!s.b_mn) {
       b.rows = s.N;
       b.cols = s.K;
-      if (!encode(&c.tmB, b, true, kBN, s.batch)) return MSIGN_ERR_CUDA;
+      if (!encode(&c.tmB, b, true, kHalfN, s.batch)) return MSIGN_ERR_CUDA;
     } else {
       b.rows = s.K;
       b.cols = s.N;
       if (!encode(&c.tmB, b, false, kBK, s.batch)) return MSIGN_ERR_CUDA;
     }
-    c.M = static_cast<int>(s.M);
-    c.N = static_cast<int>(s.N);
-    c.K = static_cast<int>(s.K);
-    c.batch = static_cast<int>(s.batch);
-    c.tiles_m = static_cast<int>((s.M + kBM - 1) / kBM);
-    c.tiles_n = static_cast<int>((s.N + kBN - 1) / kBN);
-    c.tiles_per_batch = static_cast<int>(class_tiles(s) / s.batch);
-    c.tile_begin = static_cast<int>(total);
-    c.symmetric = s.symmetric ? 1 : 0;
-    c.b_mn_major = s.b_mn ? 1 : 0;
-    c.num_out = static_cast<int>(s.outs.size());
-    c.alpha = s.alpha;
-    c.beta = s.beta;
-    c.alpha_scale = s.alpha_scale;
-    c.beta_scale = s.beta_scale;
-    c.C = s.C;
-    c.c_dtype = s.c_dt;
-    c.ldc = s.ldc;
-    c.c_bs = s.c_bs;
-    for (size_t o = 0; o < s.outs.size(); ++o) c.out[o] = s.outs[o];
+    ClassInfo& ci = c.info;
+    ci.M = static_cast<int>(s.M);
+    ci.N = static_cast<int>(s.N);
+    ci.K = static_cast<int>(s.K);
+    ci.batch = static_cast<int>(s.batch);
+    ci.tiles_m = static_cast<int>((s.M + kBM - 1) / kBM);
+    ci.tiles_n = static_cast<int>((s.N + kBN - 1) / kBN);
+    ci.tiles_per_batch = static_cast<int>(class_tiles(s) / s.batch);
+    ci.tile_begin = static_cast<int>(total);
+    ci.symmetric = s.symmetric ? 1 : 0;
+    ci.mirror = (s.symmetric && s.mirror) ? 1 : 0;
+    ci.a_sym = s.a_sym ? 1 : 0;
+    ci.b_sym = s.b_sym ? 1 : 0;
+    ci.b_mn_major = s.b_mn ? 1 : 0;
+    ci.num_out = static_cast<int>(s.outs.size());
+    ci.alpha = s.alpha;
+    ci.beta = s.beta;
+    ci.alpha_scale = s.alpha_scale;
+    ci.beta_scale = s.beta_scale;
+    ci.C = s.C;
+    ci.c_dtype = s.c_dt;
+    ci.ldc = s.ldc;
+    ci.c_bs = s.c_bs;
+    for (size_t o = 0; o < s.outs.size(); ++o) ci.out[o] = s.outs[o];
     total += class_tiles(s);
   }
   if (total > INT32_MAX) return MSIGN_ERR_UNSUPPORTED;
@@ -308,7 +341,8 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
             (static_cast<uint32_t>(kBM >> 4) << 24);
   p.err = dev->err;
   p.timeout_ns = kWaitLimitNs;
-  const int grid = static_cast<int>(std::min<int64_t>(total, dev->sms));
+  // one CTA pair per co-resident cluster slot, never more pairs than tiles
+  const int grid = 2 * static_cast<int>(std::min<int64_t>(total, dev->max_pairs));
   double flops = 0.0, bytes = 0.0;
   for (const ClassSpec& s : specs) {
     const double bt = static_cast<double>(s.batch);
@@ -410,22 +444,22 @@ msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b,
     const Mat X{k.w.P[cur], DT_BF16, n, m, ldm, n * ldm};
     const Mat A{k.w.A, DT_BF16, n, n, ldn, n * ldn};
     const Mat B{k.w.B, DT_BF16, n, n, ldn, n * ldn};
-    ClassSpec s;
+    ClassSpec s;  // A: upper 256-blocks of X X^T
     s.A = X, s.B = X, s.symmetric = true;
     s.M = n, s.N = n, s.K = m, s.batch = k.batch;
-    s.outs = {out_to(k.w.A, DT_BF16, ldn, n * ldn, false), out_to(k.w.A, DT_BF16, ldn, n * ldn, true)};
+    s.outs = {out_to(k.w.A, DT_BF16, ldn, n * ldn, false)};
     syrk.push_back(s);
 
-    ClassSpec q;
-    q.A = A, q.B = A, q.symmetric = true;
+    ClassSpec q;  // B: upper 256-blocks of b A + c A A, both operands read from A's upper blocks
+    q.A = A, q.B = A, q.symmetric = true, q.a_sym = true, q.b_sym = true;
     q.M = n, q.N = n, q.K = n, q.batch = k.batch;
     q.alpha = c, q.beta = b;
     q.C = k.w.A, q.c_dt = DT_BF16, q.ldc = ldn, q.c_bs = n * ldn;
-    q.outs = {out_to(k.w.B, DT_BF16, ldn, n * ldn, false), out_to(k.w.B, DT_BF16, ldn, n * ldn, true)};
+    q.outs = {out_to(k.w.B, DT_BF16, ldn, n * ldn, false)};
     sqr.push_back(q);
 
-    ClassSpec x;
-    x.A = B, x.B = X, x.b_mn = true;
+    ClassSpec x;  // X' = a X + B X with B read from its upper blocks
+    x.A = B, x.a_sym = true, x.B = X, x.b_mn = true;
     x.M = n, x.N = m, x.K = n, x.batch = k.batch;
     x.alpha = 1.0f, x.beta = a;
     x.C = k.w.master, x.c_dt = DT_FP32, x.ldc = ldm, x.c_bs = n * ldm;
@@ -662,9 +696,10 @@ msign_status gram_xxt(const void* X, msign_dtype x_dtype, void* A, msign_dtype a
   s.A = Xm;
   s.B = Xm;
   s.symmetric = true;
+  s.mirror = true;  // the user gets the full, exactly symmetric matrix
   s.M = n, s.N = n, s.K = m, s.batch = batch;
   const int ad = to_dt(a_dtype);
-  s.outs = {out_to(A, ad, n, n * n, false), out_to(A, ad, n, n * n, true)};
+  s.outs = {out_to(A, ad, n, n * n, false)};
   return launch_grouped({s}, xd, stream);
 }
 
@@ -709,9 +744,8 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
   GramBuffers w;
   carve_gram(cv, batch, n, m, &w);
   const int64_t sq = n * ldn, rect = n * ldm;
-  auto sym_out = [&](void* p, float gamma) {
-    return std::vector<EpiOut>{out_to(p, DT_FP16, ldn, sq, false, gamma), out_to(p, DT_FP16, ldn, sq, true, gamma)};
-  };
+  // every n x n intermediate is symmetric and kept as its upper 256-blocks
+  auto sym_out = [&](void* p, float gamma) { return std::vector<EpiOut>{out_to(p, DT_FP16, ldn, sq, false, gamma)}; };
   auto sqm = [&](void* p) { return Mat{p, DT_FP16, n, n, ldn, sq}; };
 
   // [P3] Algorithm 2 steps 1-2: X <- X / (||X||_F + eps); X <- float16(X)
@@ -739,7 +773,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
       const bool first = (t == s0), last = (t == s1 - 1);
       {  // Z = b R + c R^2; on the first step also Q = Z + a I (Q Z with Q = I)
         ClassSpec s;
-        s.A = sqm(w.R), s.B = sqm(w.R), s.symmetric = true;
+        s.A = sqm(w.R), s.B = sqm(w.R), s.symmetric = true, s.a_sym = true, s.b_sym = true;
         s.M = n, s.N = n, s.K = n, s.batch = batch;
         s.alpha = c, s.beta = b;
         s.C = w.R, s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
@@ -755,7 +789,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
       std::vector<ClassSpec> pair;
       if (!first) {  // Q <- Q Z + a Q
         ClassSpec s;
-        s.A = sqm(w.Q[q]), s.B = sqm(w.Z), s.symmetric = true;
+        s.A = sqm(w.Q[q]), s.B = sqm(w.Z), s.symmetric = true, s.a_sym = true, s.b_sym = true;
         s.M = n, s.N = n, s.K = n, s.batch = batch;
         s.alpha = 1.0f, s.beta = a;
         s.C = w.Q[q], s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
@@ -764,7 +798,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
       }
       if (!last) {  // RZ <- R Z + a R
         ClassSpec s;
-        s.A = sqm(w.R), s.B = sqm(w.Z), s.symmetric = true;
+        s.A = sqm(w.R), s.B = sqm(w.Z), s.symmetric = true, s.a_sym = true, s.b_sym = true;
         s.M = n, s.N = n, s.K = n, s.batch = batch;
         s.alpha = 1.0f, s.beta = a;
         s.C = w.R, s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
@@ -778,7 +812,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
       if (!first) q ^= 1;
       if (!last) {  // R <- Z RZ + a RZ
         ClassSpec s;
-        s.A = sqm(w.Z), s.B = sqm(w.RZ), s.symmetric = true;
+        s.A = sqm(w.Z), s.B = sqm(w.RZ), s.symmetric = true, s.a_sym = true, s.b_sym = true;
         s.M = n, s.N = n, s.K = n, s.batch = batch;
         s.alpha = 1.0f, s.beta = a;
         s.C = w.RZ, s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
@@ -789,7 +823,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
     }
     {  // X <- Q X (the restart), or the output after the last segment
       ClassSpec s;
-      s.A = sqm(w.Q[q]), s.B = X, s.b_mn = true;
+      s.A = sqm(w.Q[q]), s.a_sym = true, s.B = X, s.b_mn = true;
       s.M = n, s.N = m, s.K = n, s.batch = batch;
       if (seg + 2 == bounds.size())
         s.outs = {out_to(out, io, cols, rows * cols, tr)};
@@ -948,5 +982,6 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
   }
   return MSIGN_OK;
 }
+
 
 }  // extern "C"
