@@ -135,6 +135,38 @@ msign_status msign_ns(const void *in, void *out, msign_dtype io_dtype, msign_dty
                       void *workspace, size_t workspace_bytes, msign_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * msign_ns_noalloc: msign_ns for callers that cannot allocate device memory.
+ * The pages have no counterpart of this entry point.
+ *
+ * Some callers may not call cudaMalloc where they need msign: code being
+ * captured into a CUDA graph (an allocation there can synchronise the device
+ * and is not captured), plugins hosted by a framework that reserves all GPU
+ * memory for its own pool, and loops that forbid allocation after start-up.
+ * This variant takes no workspace: it computes exactly what msign_ns does
+ * with compute_dtype MSIGN_BF16, in a scratch array built into the library
+ * (a file-scope __device__ array of msign_ns_noalloc_max_bytes() = 32 MiB,
+ * held on every GPU that loads the library until the process exits).  It
+ * makes no device allocation of its own; inputs and outputs are the caller's.
+ *
+ * - A problem whose msign_ns_workspace_size(batch, rows, cols, MSIGN_BF16)
+ *   exceeds the built-in scratch is rejected with MSIGN_ERR_WORKSPACE before
+ *   anything is enqueued (e.g. 1024 x 2048 fits, 2048 x 2048 does not).
+ * - The first call on a device looks up that device's address of the array
+ *   (cudaGetSymbolAddress) with the device current; make that first call
+ *   before any stream capture that contains later calls.
+ * - All calls on a device share the one array and leave their intermediate
+ *   results in it; nothing in it needs to start at zero.  Calls whose
+ *   executions overlap on the GPU (different streams, or different host
+ *   threads without ordering) race on the array and give wrong results:
+ *   order them on one stream.
+ * ------------------------------------------------------------------------ */
+size_t msign_ns_noalloc_max_bytes(void);
+
+msign_status msign_ns_noalloc(const void *in, void *out, msign_dtype io_dtype,
+                              int64_t batch, int64_t rows, int64_t cols, const msign_coeffs *coeffs,
+                              msign_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * gram_xxt: symmetric Gram product A = X X^T ([P1] flash-muon
  * matmul_transpose; [P3] section 4, triangular scheduling).
  *

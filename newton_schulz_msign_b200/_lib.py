@@ -24,6 +24,7 @@ EXPORTS = (
     "gram_ns_workspace_size", "gram_ns",
     "muon_step_workspace_size", "muon_step",
     "msign_profile_enable", "msign_profile_read", "msign_profile_reset",
+    "msign_ns_noalloc_max_bytes", "msign_ns_noalloc",
 )
 
 
@@ -86,6 +87,10 @@ def lib() -> ctypes.CDLL:
                                          ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
         L.msign_profile_reset.restype = I32
         L.msign_profile_reset.argtypes = []
+        L.msign_ns_noalloc_max_bytes.restype = SZ
+        L.msign_ns_noalloc_max_bytes.argtypes = []
+        L.msign_ns_noalloc.restype = I32
+        L.msign_ns_noalloc.argtypes = [P, P, I32, I64, I64, I64, ctypes.POINTER(MsignCoeffs), P]
         _lib = L
     return _lib
 

@@ -985,3 +985,55 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
 
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation variant
+//
+// Some callers cannot allocate device memory at the point where they need
+// msign: code inside a stream capture that must not call cudaMalloc (which
+// may synchronise the device), plugins hosted by a framework that owns all of
+// the GPU's memory through its own pool, or real-time loops that forbid any
+// allocation after start-up.  msign_ns_noalloc() serves them from a fixed
+// scratch array that lives in the library's own device image.
+
+namespace msb {
+
+// Built-in scratch for msign_ns_noalloc: 32 MiB, resident on every GPU that
+// loads this library until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+}  // namespace msb
+
+extern "C" {
+
+size_t msign_ns_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
+
+msign_status msign_ns_noalloc(const void* in, void* out, msign_dtype io_dtype, int64_t batch, int64_t rows,
+                              int64_t cols, const msign_coeffs* coeffs, msign_stream_t stream) {
+  if (!valid_dtype(io_dtype) || batch < 0 || rows < 0 || cols < 0) return MSIGN_ERR_INVALID_ARG;
+  if (batch == 0 || rows == 0 || cols == 0) return MSIGN_OK;
+  if (in == nullptr || out == nullptr) return MSIGN_ERR_INVALID_ARG;
+  if (msign_ns_workspace_size(batch, rows, cols, MSIGN_BF16) > kNoAllocScratchBytes) return MSIGN_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MSIGN_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    // The array's host-side name is only a stand-in; the device address of
+    // this device's copy comes from cudaGetSymbolAddress, once per device.
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MSIGN_ERR_CUDA;
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  // Every buffer msign_ns carves from its workspace is written before it is
+  // read, so the contents left by an earlier call need no clearing.
+  return msign_ns(in, out, io_dtype, MSIGN_BF16, batch, rows, cols, coeffs, scratch, kNoAllocScratchBytes, stream);
+}
+
+}  // extern "C"
