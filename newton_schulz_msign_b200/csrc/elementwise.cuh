@@ -3,14 +3,16 @@
 //   sumsq_partial_kernel   per-matrix sum of squares of the (compute-dtype
 //                          cast) input: grid-stride, 16-byte loads, warp
 //                          shuffle + block reduction into one partial per
-//                          block (no atomics: the result is deterministic).
+//                          block (no atomics: the result is deterministic);
+//                          the grid grows with the matrix to keep HBM busy.
 //   norm_finalize_kernel   sums the partials in a fixed order and writes the
 //                          normalisation factor of [P2] section 参考实现
 //                          (1/sqrt(sum + eps)) or of [P3] Algorithm 2 step 1
 //                          (1/(sqrt(sum) + eps)).
 //   ingest_kernel          cast + orient + scale: X0 = cast(cast(M) * s),
 //                          transposed through a 32x32 shared-memory tile
-//                          when rows > cols, plus the fp32 copy of X0.
+//                          when rows > cols, plus the fp32 copy of X0;
+//   ingest_rows_kernel     the same without transposition, 16-byte accesses.
 //   momentum_kernel        M <- mu M + G in fp32 (Muon, [P3] section 1.1).
 //   apply_update_kernel    W <- W - lr * scale * O^(T) with the oriented O.
 #pragma once
@@ -25,8 +27,15 @@
 
 namespace msb {
 
-constexpr int kNormParts = 128;  // partial sums per matrix
+constexpr int kNormParts = 2048;  // maximum partial sums per matrix
 constexpr int kNormThreads = 256;
+constexpr int kNormElemsPerBlock = kNormThreads * 16;  // 16 elements per thread per pass
+
+// Blocks per matrix for the sum of squares: enough to keep HBM busy, at most kNormParts.
+__host__ __device__ inline int norm_parts(long long per) {
+  long long b = (per + kNormElemsPerBlock - 1) / kNormElemsPerBlock;
+  return static_cast<int>(b < 1 ? 1 : (b > kNormParts ? kNormParts : b));
+}
 
 // Rounds v to the compute dtype (bf16 / fp16) and back; DT_FP32 keeps it.
 __device__ __forceinline__ float round_to(float v, int dt) {
@@ -102,10 +111,10 @@ __global__ void __launch_bounds__(kNormThreads) sumsq_partial_kernel(const void*
   if (threadIdx.x == 0) partials[static_cast<long long>(b) * gridDim.x + blockIdx.x] = acc;
 }
 
-// One block of kNormParts threads per matrix.  mode 0: s = 1/sqrt(sum + eps);
-// mode 1: s = 1/(sqrt(sum) + eps).
-__global__ void __launch_bounds__(kNormParts) norm_finalize_kernel(const float* partials, int nparts, float eps,
-                                                                   int mode, float* scale) {
+// One block of 1024 threads per matrix sums the nparts partials in a fixed
+// order.  mode 0: s = 1/sqrt(sum + eps); mode 1: s = 1/(sqrt(sum) + eps).
+__global__ void __launch_bounds__(1024) norm_finalize_kernel(const float* partials, int nparts, float eps,
+                                                             int mode, float* scale) {
   __shared__ float red[32];
   const int b = blockIdx.x;
   float v = 0.0f;
@@ -169,6 +178,65 @@ __global__ void __launch_bounds__(256) ingest_kernel(const void* in, int in_dt, 
                      (static_cast<long long>(b) * op_bs + static_cast<long long>(i) * ld_op + j) * dtype_size(op_dt),
                  op_dt, xs);
       if (master) master[static_cast<long long>(b) * m_bs + static_cast<long long>(i) * ld_m + j] = xs;
+    }
+  }
+}
+
+// Row-wise ingest without transposition, 8 elements per thread with 16-byte
+// accesses: rows x cols input (leading dimension cols) to the operand copy and
+// the fp32 copy (leading dimensions ld_op, ld_m).  Requires cols % 8 == 0 and
+// 16-byte aligned bases and rows on every side.
+template <int IN_DT, int OP_DT>
+__global__ void __launch_bounds__(256) ingest_rows_kernel(const void* in, long long rows, int cols,
+                                                          const float* scale, int cast_dt, void* xop, long long ld_op,
+                                                          long long op_bs, float* master, long long ld_m,
+                                                          long long m_bs) {
+  const int b = blockIdx.y;
+  const int vpr = cols / 8;  // vectors per row
+  const long long nvec = rows * vpr;
+  const float s = scale ? scale[b] : 1.0f;
+  const char* src = reinterpret_cast<const char*>(in) + static_cast<long long>(b) * rows * cols * dtype_size(IN_DT);
+  for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < nvec;
+       v += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long i = v / vpr;
+    const int j = static_cast<int>(v - i * vpr) * 8;
+    float x[8];
+    if (IN_DT == DT_FP32) {
+      const float4* q = reinterpret_cast<const float4*>(src + (i * cols + j) * 4);
+      const float4 a = q[0], c = q[1];
+      x[0] = a.x, x[1] = a.y, x[2] = a.z, x[3] = a.w, x[4] = c.x, x[5] = c.y, x[6] = c.z, x[7] = c.w;
+    } else {
+      const uint4 u = *reinterpret_cast<const uint4*>(src + (i * cols + j) * 2);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        float2 f;
+        if (IN_DT == DT_BF16)
+          f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+        else
+          f = __half22float2(*reinterpret_cast<const __half2*>(&w[t]));
+        x[2 * t] = f.x, x[2 * t + 1] = f.y;
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) x[t] = round_to(x[t], cast_dt) * s;
+    uint32_t o[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      if (OP_DT == DT_BF16) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * t], x[2 * t + 1]);
+        o[t] = *reinterpret_cast<uint32_t*>(&h);
+      } else {
+        __half2 h = __floats2half2_rn(x[2 * t], x[2 * t + 1]);
+        o[t] = *reinterpret_cast<uint32_t*>(&h);
+      }
+    }
+    *reinterpret_cast<uint4*>(reinterpret_cast<char*>(xop) + (static_cast<long long>(b) * op_bs + i * ld_op + j) * 2) =
+        make_uint4(o[0], o[1], o[2], o[3]);
+    if (master) {
+      float4* d = reinterpret_cast<float4*>(master + static_cast<long long>(b) * m_bs + i * ld_m + j);
+      d[0] = make_float4(x[0], x[1], x[2], x[3]);
+      d[1] = make_float4(x[4], x[5], x[6], x[7]);
     }
   }
 }

@@ -366,14 +366,14 @@ msign_status launch_ok() { return cudaGetLastError() == cudaSuccess ? MSIGN_OK :
 // Frobenius normalisation factor of every matrix of a batch into scale[].
 msign_status launch_norm(const void* in, int in_dt, int64_t per, int64_t batch, int cast_dt, float eps, int mode,
                          float* partials, float* scale, cudaStream_t stream) {
-  dim3 g(kNormParts, static_cast<unsigned>(batch));
+  const int parts = norm_parts(per);
+  dim3 g(static_cast<unsigned>(parts), static_cast<unsigned>(batch));
   prof_begin(stream);
   sumsq_partial_kernel<<<g, kNormThreads, 0, stream>>>(in, in_dt, per, cast_dt, partials);
   prof_end(1, stream, 0.0, static_cast<double>(batch) * per * dtype_size(in_dt));
   prof_begin(stream);
-  norm_finalize_kernel<<<static_cast<unsigned>(batch), kNormParts, 0, stream>>>(partials, kNormParts, eps, mode,
-                                                                                scale);
-  prof_end(1, stream, 0.0, static_cast<double>(batch) * kNormParts * 4);
+  norm_finalize_kernel<<<static_cast<unsigned>(batch), 1024, 0, stream>>>(partials, parts, eps, mode, scale);
+  prof_end(1, stream, 0.0, static_cast<double>(batch) * parts * 4);
   return launch_ok();
 }
 
@@ -381,13 +381,38 @@ msign_status launch_ingest(const void* in, int in_dt, int64_t rows, int64_t cols
                            int cast_dt, void* xop, int op_dt, int64_t ld_op, int64_t op_bs, float* master,
                            int64_t ld_m, int64_t m_bs, int64_t batch, cudaStream_t stream) {
   const int64_t n = transpose ? cols : rows, m = transpose ? rows : cols;
+  const double bytes =
+      static_cast<double>(batch) * rows * cols * (dtype_size(in_dt) + dtype_size(op_dt) + (master ? 4 : 0));
+  const bool rowwise = !transpose && op_dt != DT_FP32 && cols % 8 == 0 && ld_op % 8 == 0 && (!master || ld_m % 8 == 0) &&
+                       (reinterpret_cast<uintptr_t>(in) % 16) == 0 && (reinterpret_cast<uintptr_t>(xop) % 16) == 0 &&
+                       (!master || (reinterpret_cast<uintptr_t>(master) % 16) == 0) && op_bs % 8 == 0 &&
+                       (!master || m_bs % 8 == 0);
+  if (rowwise) {
+    const long long nvec = rows * (cols / 8);
+    dim3 g(static_cast<unsigned>(std::min<long long>((nvec + 255) / 256, 8192)), static_cast<unsigned>(batch));
+    prof_begin(stream);
+#define MSB_INGEST(IN, OP)                                                                                        \
+  ingest_rows_kernel<IN, OP><<<g, 256, 0, stream>>>(in, rows, static_cast<int>(cols), scale, cast_dt, xop, ld_op, op_bs, \
+                                                    master, ld_m, m_bs)
+    if (op_dt == DT_BF16) {
+      if (in_dt == DT_BF16) MSB_INGEST(DT_BF16, DT_BF16);
+      else if (in_dt == DT_FP16) MSB_INGEST(DT_FP16, DT_BF16);
+      else MSB_INGEST(DT_FP32, DT_BF16);
+    } else {
+      if (in_dt == DT_BF16) MSB_INGEST(DT_BF16, DT_FP16);
+      else if (in_dt == DT_FP16) MSB_INGEST(DT_FP16, DT_FP16);
+      else MSB_INGEST(DT_FP32, DT_FP16);
+    }
+#undef MSB_INGEST
+    prof_end(2, stream, 0.0, bytes);
+    return launch_ok();
+  }
   dim3 g(static_cast<unsigned>((m + 31) / 32), static_cast<unsigned>((n + 31) / 32), static_cast<unsigned>(batch));
   prof_begin(stream);
   ingest_kernel<<<g, dim3(32, 8), 0, stream>>>(in, in_dt, static_cast<int>(rows), static_cast<int>(cols),
                                                transpose ? 1 : 0, scale, cast_dt, xop, op_dt, ld_op, op_bs, master,
                                                ld_m, m_bs);
-  prof_end(2, stream, 0.0,
-           static_cast<double>(batch) * rows * cols * (dtype_size(in_dt) + dtype_size(op_dt) + (master ? 4 : 0)));
+  prof_end(2, stream, 0.0, bytes);
   return launch_ok();
 }
 
