@@ -123,8 +123,16 @@ msign_status msign_profile_reset(void);
  *   io_dtype       MSIGN_BF16, MSIGN_FP16 or MSIGN_FP32
  *   compute_dtype  MSIGN_BF16: bf16 tensor-core operands, fp32 accumulation,
  *                  fp32 epilogue arithmetic and an fp32 copy of X between
- *                  steps.  (MSIGN_FP32 is reserved for the fp32-accurate
- *                  path and returns MSIGN_ERR_UNSUPPORTED when not built.)
+ *                  steps (the input is cast to bf16 first, as the routine of
+ *                  [P2] section 参考实现 does).
+ *                  MSIGN_FP16: the same with fp16 operands (the input is
+ *                  cast to fp16 first); 8x smaller rounding than bf16 at the
+ *                  same tensor-core rate ([P3] section 3.3 argues the same
+ *                  for Gram NS).
+ *                  MSIGN_FP32: fp32-accurate products: every operand is kept
+ *                  as two tf32 planes (hi, lo) and each product is
+ *                  hi*hi + hi*lo + lo*hi on the tf32 tensor cores with fp32
+ *                  accumulation (about 6x the bf16 time).
  *   coeffs         schedule (NULL: Jordan, T = 5, eps = 1e-20)
  *   workspace      device scratch of at least msign_ns_workspace_size() bytes
  * ------------------------------------------------------------------------ */

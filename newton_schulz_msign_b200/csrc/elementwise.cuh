@@ -13,6 +13,8 @@
 //                          transposed through a 32x32 shared-memory tile
 //                          when rows > cols, plus the fp32 copy of X0;
 //   ingest_rows_kernel     the same without transposition, 16-byte accesses.
+//                          With op_dt DT_TF32_HI both write the two tf32
+//                          planes (hi, lo) of the fp32-accurate operand.
 //   momentum_kernel        M <- mu M + G in fp32 (Muon, [P3] section 1.1).
 //   apply_update_kernel    W <- W - lr * scale * O^(T) with the oriented O.
 #pragma once
@@ -133,8 +135,8 @@ __global__ void __launch_bounds__(1024) norm_finalize_kernel(const float* partia
 // in[b] is rows x cols row-major with leading dimension `cols`.
 __global__ void __launch_bounds__(256) ingest_kernel(const void* in, int in_dt, int rows, int cols, int transpose,
                                                      const float* scale, int cast_dt, void* xop, int op_dt,
-                                                     long long ld_op, long long op_bs, float* master,
-                                                     long long ld_m, long long m_bs) {
+                                                     long long ld_op, long long op_bs, long long op_plane,
+                                                     float* master, long long ld_m, long long m_bs) {
   __shared__ float tile[32][33];
   const int b = blockIdx.z;
   const int n = transpose ? cols : rows;
@@ -174,9 +176,10 @@ __global__ void __launch_bounds__(256) ingest_kernel(const void* in, int in_dt, 
     const int i = i0 + ty + 8 * k, j = j0 + tx;
     if (i < n && j < m) {
       const float xs = v[k] * s;
-      store_elem(reinterpret_cast<char*>(xop) +
-                     (static_cast<long long>(b) * op_bs + static_cast<long long>(i) * ld_op + j) * dtype_size(op_dt),
-                 op_dt, xs);
+      char* dst = reinterpret_cast<char*>(xop) +
+                  (static_cast<long long>(b) * op_bs + static_cast<long long>(i) * ld_op + j) * dtype_size(op_dt);
+      store_elem(dst, op_dt, xs);
+      if (op_dt == DT_TF32_HI) store_elem(dst + op_plane * 4, DT_TF32_LO, xs);
       if (master) master[static_cast<long long>(b) * m_bs + static_cast<long long>(i) * ld_m + j] = xs;
     }
   }
@@ -189,8 +192,8 @@ __global__ void __launch_bounds__(256) ingest_kernel(const void* in, int in_dt, 
 template <int IN_DT, int OP_DT>
 __global__ void __launch_bounds__(256) ingest_rows_kernel(const void* in, long long rows, int cols,
                                                           const float* scale, int cast_dt, void* xop, long long ld_op,
-                                                          long long op_bs, float* master, long long ld_m,
-                                                          long long m_bs) {
+                                                          long long op_bs, long long op_plane, float* master,
+                                                          long long ld_m, long long m_bs) {
   const int b = blockIdx.y;
   const int vpr = cols / 8;  // vectors per row
   const long long nvec = rows * vpr;
@@ -220,6 +223,26 @@ __global__ void __launch_bounds__(256) ingest_rows_kernel(const void* in, long l
     }
 #pragma unroll
     for (int t = 0; t < 8; ++t) x[t] = round_to(x[t], cast_dt) * s;
+    if (OP_DT == DT_TF32_HI) {
+      // fp32-accurate operand: tf32 hi plane and tf32 lo plane
+      float* hp = reinterpret_cast<float*>(xop) + static_cast<long long>(b) * op_bs + i * ld_op + j;
+      float h[8], l[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        h[t] = to_tf32(x[t]);
+        l[t] = to_tf32(x[t] - h[t]);
+      }
+      reinterpret_cast<float4*>(hp)[0] = make_float4(h[0], h[1], h[2], h[3]);
+      reinterpret_cast<float4*>(hp)[1] = make_float4(h[4], h[5], h[6], h[7]);
+      reinterpret_cast<float4*>(hp + op_plane)[0] = make_float4(l[0], l[1], l[2], l[3]);
+      reinterpret_cast<float4*>(hp + op_plane)[1] = make_float4(l[4], l[5], l[6], l[7]);
+      if (master) {
+        float4* d = reinterpret_cast<float4*>(master + static_cast<long long>(b) * m_bs + i * ld_m + j);
+        d[0] = make_float4(x[0], x[1], x[2], x[3]);
+        d[1] = make_float4(x[4], x[5], x[6], x[7]);
+      }
+      continue;
+    }
     uint32_t o[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) {

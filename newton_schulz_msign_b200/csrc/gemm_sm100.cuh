@@ -76,11 +76,29 @@ constexpr int kBM = 256;      // output tile rows per CTA pair
 constexpr int kHalfM = 128;   // rows per CTA (= TMEM lanes)
 constexpr int kBN = 256;      // output tile columns
 constexpr int kHalfN = 128;   // B rows staged per CTA
-constexpr int kBK = 64;       // 64 16-bit elements = one 128-byte swizzle row
+constexpr int kRowBytes = 128;  // one 128-byte swizzle row of K per operand row and stage
 constexpr int kStages = 6;
 constexpr int kThreads = 192;
-constexpr int kATileBytes = kHalfM * kBK * 2;  // 16 KB
-constexpr int kBTileBytes = kHalfN * kBK * 2;  // 16 KB
+constexpr int kATileBytes = kHalfM * kRowBytes;  // 16 KB
+constexpr int kBTileBytes = kHalfN * kRowBytes;  // 16 KB
+
+// Operand kinds: 16-bit (bf16 / fp16, kind::f16) or tf32 (fp32 words,
+// kind::tf32).  A stage holds one 128-byte row of K per operand row either way.
+template <bool TF32>
+struct OpKind {
+  static constexpr int es = TF32 ? 4 : 2;              // operand element bytes
+  static constexpr int bke = kRowBytes / es;           // K elements per stage: 32 or 64
+  static constexpr int kmma = TF32 ? 8 : 16;           // K per MMA instruction
+  static constexpr int mn_chunk = kRowBytes / es;      // MN elements per chunk of an MN-major tile
+  static constexpr int chunks = 128 / mn_chunk;        // chunks per 128 MN rows: 4 or 2
+  static constexpr int chunk_bytes = bke * kRowBytes;  // 4 KB or 8 KB
+  static constexpr int mn_kstep = kmma * kRowBytes;    // MN-major descriptor advance per MMA: 1024 or 2048
+  // MN-major smem form: 16-bit types use the plain 128-byte swizzle (8-row
+  // atoms, 1024 B); 32-bit types need the 32-byte-chunk swizzle, whose atoms
+  // are 4 K rows (512 B) -- the tensor maps that feed them swizzle the same way.
+  static constexpr uint32_t mn_layout = TF32 ? 1u : 2u;
+  static constexpr uint32_t mn_sbo = TF32 ? 512u : 1024u;
+};
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kScratchStride = 33;  // padded row of the per-warp 32 x 32 fp32 transpose scratch
 constexpr int kStageOutBytes = 32 * kScratchStride * 4;
@@ -91,9 +109,12 @@ constexpr int kNumBarriers = 2 * kStages + 2 + 2 + 1;
 constexpr int kSmemBytes = 1024 /* alignment slack */ + kStages * kStageBytes + kEpiBytes + kNumBarriers * 8 + 16;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-enum : int { DT_BF16 = 0, DT_FP16 = 1, DT_FP32 = 2 };
+// Storage types.  DT_TF32_HI / DT_TF32_LO store fp32 words: the tf32 rounding
+// of v, and the tf32 rounding of the remainder v - hi (operand planes of the
+// fp32-accurate path, whose products hi*hi + hi*lo + lo*hi carry ~21 bits).
+enum : int { DT_BF16 = 0, DT_FP16 = 1, DT_FP32 = 2, DT_TF32_HI = 3, DT_TF32_LO = 4 };
 
-__host__ __device__ inline int dtype_size(int dt) { return dt == DT_FP32 ? 4 : 2; }
+__host__ __device__ inline int dtype_size(int dt) { return (dt == DT_BF16 || dt == DT_FP16) ? 2 : 4; }
 
 constexpr int kMaxOuts = 4;
 
@@ -118,7 +139,9 @@ struct ClassInfo {
   int a_sym;       // A operand is a symmetric matrix stored by upper 256-blocks
   int b_sym;       // same for the B operand (K-major)
   int b_mn_major;  // B operand stored K x N (MN-major)
-  int num_out, c_dtype, pad0;
+  int num_out, c_dtype;
+  int split;       // operands are hi/lo planes (batch coordinate 2b + plane): three K passes
+  long long c_plane;  // > 0: C is split too, its lo plane at C + c_plane elements
   float alpha, beta;
   const float* alpha_scale;  // optional per-batch factor on alpha
   const float* beta_scale;   // optional per-batch factor on beta
@@ -176,14 +199,20 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
 // ---------------------------------------------------------------- row I/O
 
 __device__ __forceinline__ float load_elem(const char* p, int dt) {
-  if (dt == DT_FP32) return *reinterpret_cast<const float*>(p);
+  if (dt == DT_FP32 || dt == DT_TF32_HI || dt == DT_TF32_LO) return *reinterpret_cast<const float*>(p);
   if (dt == DT_BF16) return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
   return __half2float(*reinterpret_cast<const __half*>(p));
 }
 
+__device__ __forceinline__ float split_value(int dt, float v) {
+  if (dt == DT_TF32_HI) return to_tf32(v);
+  if (dt == DT_TF32_LO) return to_tf32(v - to_tf32(v));
+  return v;
+}
+
 __device__ __forceinline__ void store_elem(char* p, int dt, float v) {
-  if (dt == DT_FP32)
-    *reinterpret_cast<float*>(p) = v;
+  if (dt == DT_FP32 || dt == DT_TF32_HI || dt == DT_TF32_LO)
+    *reinterpret_cast<float*>(p) = split_value(dt, v);
   else if (dt == DT_BF16)
     *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(v);
   else
@@ -194,7 +223,7 @@ __device__ __forceinline__ void store_elem(char* p, int dt, float v) {
 __device__ __forceinline__ void load_row32(const char* rowp, int dt, uint32_t mask, float (&v)[32]) {
   const int es = dtype_size(dt);
   if (mask == 0xFFFFFFFFu && (reinterpret_cast<uintptr_t>(rowp) & 15) == 0) {
-    if (dt == DT_FP32) {
+    if (dtype_size(dt) == 4) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float4 f = reinterpret_cast<const float4*>(rowp)[i];
@@ -234,10 +263,12 @@ __device__ __forceinline__ void load_row32(const char* rowp, int dt, uint32_t ma
 __device__ __forceinline__ void store_row32(char* rowp, int dt, uint32_t mask, const float (&v)[32]) {
   const int es = dtype_size(dt);
   if (mask == 0xFFFFFFFFu && (reinterpret_cast<uintptr_t>(rowp) & 15) == 0) {
-    if (dt == DT_FP32) {
+    if (dt == DT_FP32 || dt == DT_TF32_HI || dt == DT_TF32_LO) {
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        reinterpret_cast<float4*>(rowp)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        reinterpret_cast<float4*>(rowp)[i] =
+            make_float4(split_value(dt, v[4 * i]), split_value(dt, v[4 * i + 1]), split_value(dt, v[4 * i + 2]),
+                        split_value(dt, v[4 * i + 3]));
     } else {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -287,7 +318,14 @@ __device__ __forceinline__ uint32_t lane_mask(int n) { return n >= 32 ? 0xFFFFFF
 __device__ __forceinline__ void load_c(const ClassInfo& k, int b, int row0, int col0, int lane, float (&cv)[32]) {
   const int r = row0 + lane;
   const uint32_t m = (r < k.M) ? lane_mask(k.N - col0) : 0u;
-  load_row32(gaddr(k.C, k.c_dtype, k.ldc, k.c_bs, b, r, col0), k.c_dtype, m, cv);
+  const char* hp = gaddr(k.C, k.c_dtype, k.ldc, k.c_bs, b, r, col0);
+  load_row32(hp, k.c_dtype, m, cv);
+  if (k.c_plane > 0) {  // split C: value = hi + lo
+    float lo[32];
+    load_row32(hp + k.c_plane * 4, DT_FP32, m, lo);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) cv[i] += lo[i];
+  }
 }
 
 // One 32x32 block: this lane owns output row `row0 + lane`, columns
@@ -353,9 +391,12 @@ __device__ __forceinline__ void epilogue_block(const ClassInfo& k, int b, int ro
 
 // ---------------------------------------------------------------- kernel
 
-// Launched with clusters of 2 CTAs along x; gridDim.x is even.
+// Launched with clusters of 2 CTAs along x; gridDim.x is even.  TF32 selects
+// the operand kind (see OpKind).
+template <bool TF32>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_sm100_kernel(const __grid_constant__ GemmParams p) {
+  using OK = OpKind<TF32>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -420,19 +461,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const TileCoord tc = decode_tile(p, t);
         const ClassInfo& k = p.cls[tc.c].info;
         // per-tile state in registers
-        const int nk = (k.K + kBK - 1) / kBK;
+        const int nk = (k.K + OK::bke - 1) / OK::bke;
+        const int passes = k.split ? 3 : 1;  // split: hi*hi, hi*lo, lo*hi per K slice
         const int arow = tc.tm * kBM + static_cast<int>(rank) * kHalfM;
         const int bcol = tc.tn * kBN + static_cast<int>(rank) * kHalfN;
-        const int a_tr = k.a_sym ? (tc.tm * kBM) / kBK : 0;  // K slices below this read A transposed
-        const int b_tr = k.b_sym ? (tc.tn * kBN) / kBK : 0;
+        const int a_tr = k.a_sym ? (tc.tm * kBM) / OK::bke : 0;  // K slices below this read A transposed
+        const int b_tr = k.b_sym ? (tc.tn * kBN) / OK::bke : 0;
         const bool b_mn = k.b_mn_major != 0;
         const GemmClass& g = p.cls[tc.c];
         const void* tmA = &g.tmA;
         const void* tmA2 = &g.tmA2;
         const void* tmB = &g.tmB;
         const void* tmB2 = &g.tmB2;
-        const int bz = tc.b;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int step = 0; step < nk * passes; ++step) {
+          const int kb = step / passes, pass = step - kb * passes;
+          const int za = passes == 1 ? tc.b : 2 * tc.b + (pass == 2 ? 1 : 0);
+          const int zb = passes == 1 ? tc.b : 2 * tc.b + (pass == 1 ? 1 : 0);
           if (!wait_bounded(&empty[stage], phase ^ 1u, s_abort, p.err, limit)) {
             ok = false;
             break;
@@ -441,22 +485,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = sA + stage * kATileBytes;
           uint8_t* b_dst = sB + stage * kBTileBytes;
-          const int k0 = kb * kBK;
+          const int k0 = kb * OK::bke;
           if (kb < a_tr) {
             // stored transpose: rows k0.. of S, columns arow..arow+127 (MN-major)
-            tma_load_3d_pair(a_dst, tmA2, fbar, arow, k0, bz);
-            tma_load_3d_pair(a_dst + kBK * 64 * 2, tmA2, fbar, arow + 64, k0, bz);
+#pragma unroll
+            for (int c = 0; c < OK::chunks; ++c)
+              tma_load_3d_pair(a_dst + c * OK::chunk_bytes, tmA2, fbar, arow + c * OK::mn_chunk, k0, za);
           } else {
-            tma_load_3d_pair(a_dst, tmA, fbar, k0, arow, bz);
+            tma_load_3d_pair(a_dst, tmA, fbar, k0, arow, za);
           }
-          if (kb < b_tr) {
-            tma_load_3d_pair(b_dst, tmB2, fbar, bcol, k0, bz);
-            tma_load_3d_pair(b_dst + kBK * 64 * 2, tmB2, fbar, bcol + 64, k0, bz);
-          } else if (!b_mn) {
-            tma_load_3d_pair(b_dst, tmB, fbar, k0, bcol, bz);
+          if (kb < b_tr || b_mn) {
+            const void* tm = (kb < b_tr) ? tmB2 : tmB;
+#pragma unroll
+            for (int c = 0; c < OK::chunks; ++c)
+              tma_load_3d_pair(b_dst + c * OK::chunk_bytes, tm, fbar, bcol + c * OK::mn_chunk, k0, zb);
           } else {
-            tma_load_3d_pair(b_dst, tmB, fbar, bcol, k0, bz);
-            tma_load_3d_pair(b_dst + kBK * 64 * 2, tmB, fbar, bcol + 64, k0, bz);
+            tma_load_3d_pair(b_dst, tmB, fbar, k0, bcol, zb);
           }
           used |= 1u << stage;
           last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
@@ -488,18 +532,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // K-major and MN-major descriptors of stage 0; stage s adds s * tile
       // bytes and K step kk adds 32 (K-major) or 2048 (MN-major) bytes, all
       // in the 16-byte-unit start-address field.
-      const uint64_t dA_k = smem_desc_sw128(sA0, 16, 1024), dA_mn = smem_desc_sw128(sA0, kBK * 64 * 2, 1024);
-      const uint64_t dB_k = smem_desc_sw128(sB0, 16, 1024), dB_mn = smem_desc_sw128(sB0, kBK * 64 * 2, 1024);
+      const uint64_t dA_k = smem_desc_sw128(sA0, 16, 1024), dA_mn = smem_desc_sw128(sA0, OK::chunk_bytes, OK::mn_sbo, OK::mn_layout);
+      const uint64_t dB_k = smem_desc_sw128(sB0, 16, 1024), dB_mn = smem_desc_sw128(sB0, OK::chunk_bytes, OK::mn_sbo, OK::mn_layout);
       for (int t = pair; t < p.total_tiles && ok; t += num_pairs) {
         const TileCoord tc = decode_tile(p, t);
         const ClassInfo& k = p.cls[tc.c].info;
-        const int nk = (k.K + kBK - 1) / kBK;
-        const int a_tr = k.a_sym ? (tc.tm * kBM) / kBK : 0;
-        const int b_tr = k.b_sym ? (tc.tn * kBN) / kBK : (k.b_mn_major ? nk : 0);
+        const int nk = (k.K + OK::bke - 1) / OK::bke;
+        const int passes = k.split ? 3 : 1;
+        const int a_tr = k.a_sym ? (tc.tm * kBM) / OK::bke : 0;
+        const int b_tr = k.b_sym ? (tc.tn * kBN) / OK::bke : (k.b_mn_major ? nk : 0);
         if (!wait_bounded(&tempty[buf], bphase ^ 1u, s_abort, p.err, limit)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int step = 0; step < nk * passes; ++step) {
+          const int kb = step / passes;
           if (!wait_bounded(&full[stage], phase, s_abort, p.err, limit)) {
             ok = false;
             break;
@@ -510,11 +556,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t idesc = idesc0 | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16);
           const uint64_t da = (a_mn ? dA_mn : dA_k) + static_cast<uint64_t>((stage * kATileBytes) >> 4);
           const uint64_t db = (b_mn ? dB_mn : dB_k) + static_cast<uint64_t>((stage * kBTileBytes) >> 4);
-          const uint32_t sa = a_mn ? (2048 >> 4) : (32 >> 4);
-          const uint32_t sb = b_mn ? (2048 >> 4) : (32 >> 4);
+          const uint32_t sa = a_mn ? (OK::mn_kstep >> 4) : (32 >> 4);
+          const uint32_t sb = b_mn ? (OK::mn_kstep >> 4) : (32 >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_f16_pair(d_tmem, da + kk * sa, db + kk * sb, idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < OK::bke / OK::kmma; ++kk) {
+            const uint32_t acc = (step | kk) != 0 ? 1u : 0u;
+            if (TF32)
+              umma_tf32_pair(d_tmem, da + kk * sa, db + kk * sb, idesc, acc);
+            else
+              umma_f16_pair(d_tmem, da + kk * sa, db + kk * sb, idesc, acc);
+          }
           umma_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == kStages) {
             stage = 0;

@@ -56,8 +56,10 @@ msign_status device_state(DeviceState** out) {
     if (major != 10 || minor != 0) return MSIGN_ERR_UNSUPPORTED;  // built for sm_100a only
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MSIGN_ERR_CUDA;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_err_word) != cudaSuccess) return MSIGN_ERR_CUDA;
-    if (cudaFuncSetAttribute(gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_sm100_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(gemm_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+            cudaSuccess)
       return MSIGN_ERR_CUDA;
     {
       cudaLaunchConfig_t cfg = {};
@@ -72,7 +74,7 @@ msign_status device_state(DeviceState** out) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, gemm_sm100_kernel, &cfg) != cudaSuccess || clusters < 1) {
+      if (cudaOccupancyMaxActiveClusters(&clusters, gemm_sm100_kernel<false>, &cfg) != cudaSuccess || clusters < 1) {
         (void)cudaGetLastError();
         clusters = d.sms / 2;
       }
@@ -200,22 +202,29 @@ struct Mat {
 
 bool tma_ok(const Mat& m) {
   const int es = dtype_size(m.dt);
-  return m.dt != DT_FP32 && (reinterpret_cast<uintptr_t>(m.ptr) % 16) == 0 && (m.ld * es) % 16 == 0 &&
-         (m.bs * es) % 16 == 0;
+  return (reinterpret_cast<uintptr_t>(m.ptr) % 16) == 0 && (m.ld * es) % 16 == 0 && (m.bs * es) % 16 == 0;
 }
 
-bool encode(CUtensorMap* tm, const Mat& m, bool kmajor_rows_box, int box_rows, int64_t batch) {
-  // dims: (cols, rows, batch); box: (64, box_rows, 1)
+// 3-D tensor map (cols, rows, batch) with a box of one 128-byte swizzle row
+// (64 16-bit or 32 fp32 elements) by box_rows.  For split operands the
+// batch coordinate counts planes (2 per matrix) and m.bs is the plane stride.
+// mn_major: the box feeds an MN-major operand; fp32 words then take the
+// 32-byte-chunk form of the 128-byte swizzle, the only MN-major form the
+// tf32 MMA reads.
+bool encode(CUtensorMap* tm, const Mat& m, int box0, int box_rows, int64_t batch, bool mn_major = false) {
   const int es = dtype_size(m.dt);
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(m.cols), static_cast<cuuint64_t>(m.rows),
                         static_cast<cuuint64_t>(batch)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(m.ld * es), static_cast<cuuint64_t>(m.bs * es)};
-  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box0), static_cast<cuuint32_t>(box_rows), 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
-  (void)kmajor_rows_box;
-  CUresult r = g_encode(tm, m.dt == DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
-                        const_cast<void*>(m.ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  const CUtensorMapDataType dt = m.dt == DT_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : m.dt == DT_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const CUtensorMapSwizzle sw =
+      (mn_major && es == 4) ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+  CUresult r = g_encode(tm, dt, 3, const_cast<void*>(m.ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -242,6 +251,8 @@ struct ClassSpec {
   bool mirror = false;     // symmetric: write exact mirrors (else upper 256-blocks only)
   bool a_sym = false;      // A is a symmetric matrix stored by upper 256-blocks
   bool b_sym = false;      // B likewise
+  bool split = false;      // fp32-accurate: A and B are tf32 hi/lo planes (Mat.bs = plane stride)
+  int64_t c_plane = 0;     // > 0: C is split, lo plane at C + c_plane elements
   int64_t M = 0, N = 0, K = 0, batch = 0;
   float alpha = 1.0f, beta = 0.0f;
   const float* alpha_scale = nullptr;
@@ -285,27 +296,30 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     if (s.K <= 0 || s.outs.empty() || s.outs.size() > static_cast<size_t>(kMaxOuts)) return MSIGN_ERR_INVALID_ARG;
     if (s.symmetric && s.M != s.N) return MSIGN_ERR_INVALID_ARG;
     if (!tma_ok(s.A) || !tma_ok(s.B) || s.A.dt != ab_dt || s.B.dt != ab_dt) return MSIGN_ERR_UNSUPPORTED;
+    if ((ab_dt == DT_FP32) != s.split) return MSIGN_ERR_INVALID_ARG;
     if (s.M > INT32_MAX || s.N > INT32_MAX || s.K > INT32_MAX || s.batch > 65535) return MSIGN_ERR_UNSUPPORTED;
+    const int bke = kRowBytes / dtype_size(ab_dt);  // K elements per stage row
+    const int64_t zb = s.split ? 2 * s.batch : s.batch;
     Mat a = s.A;
     a.rows = s.M;
     a.cols = s.K;
-    if (!encode(&c.tmA, a, true, kHalfM, s.batch)) return MSIGN_ERR_CUDA;
-    if (s.a_sym && (s.M != s.K || !encode(&c.tmA2, a, false, kBK, s.batch))) return MSIGN_ERR_INVALID_ARG;
+    if (!encode(&c.tmA, a, bke, kHalfM, zb)) return MSIGN_ERR_CUDA;
+    if (s.a_sym && (s.M != s.K || !encode(&c.tmA2, a, bke, bke, zb, true))) return MSIGN_ERR_INVALID_ARG;
     Mat b = s.B;
     if (s.b_sym) {
       if (s.b_mn || s.N != s.K) return MSIGN_ERR_INVALID_ARG;
       b.rows = s.N;
       b.cols = s.K;
-      if (!encode(&c.tmB2, b, false, kBK, s.batch)) return MSIGN_ERR_CUDA;
+      if (!encode(&c.tmB2, b, bke, bke, zb, true)) return MSIGN_ERR_CUDA;
     }
     if (!s.b_mn) {
       b.rows = s.N;
       b.cols = s.K;
-      if (!encode(&c.tmB, b, true, kHalfN, s.batch)) return MSIGN_ERR_CUDA;
+      if (!encode(&c.tmB, b, bke, kHalfN, zb)) return MSIGN_ERR_CUDA;
     } else {
       b.rows = s.K;
       b.cols = s.N;
-      if (!encode(&c.tmB, b, false, kBK, s.batch)) return MSIGN_ERR_CUDA;
+      if (!encode(&c.tmB, b, bke, bke, zb, true)) return MSIGN_ERR_CUDA;
     }
     ClassInfo& ci = c.info;
     ci.M = static_cast<int>(s.M);
@@ -321,6 +335,8 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     ci.a_sym = s.a_sym ? 1 : 0;
     ci.b_sym = s.b_sym ? 1 : 0;
     ci.b_mn_major = s.b_mn ? 1 : 0;
+    ci.split = s.split ? 1 : 0;
+    ci.c_plane = s.c_plane;
     ci.num_out = static_cast<int>(s.outs.size());
     ci.alpha = s.alpha;
     ci.beta = s.beta;
@@ -336,7 +352,7 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
   if (total > INT32_MAX) return MSIGN_ERR_UNSUPPORTED;
   p.num_classes = static_cast<int>(specs.size());
   p.total_tiles = static_cast<int>(total);
-  const uint32_t fmt = (ab_dt == DT_BF16) ? 1u : 0u;
+  const uint32_t fmt = (ab_dt == DT_BF16) ? 1u : (ab_dt == DT_FP16 ? 0u : 2u);  // bf16, f16 or tf32
   p.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
             (static_cast<uint32_t>(kBM >> 4) << 24);
   p.err = dev->err;
@@ -355,8 +371,12 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     for (const EpiOut& e : s.outs)
       bytes += bt * dtype_size(e.dtype) * static_cast<double>(s.M) * s.N * (s.symmetric ? 0.5 : 1.0);
   }
+  if (ab_dt == DT_FP32) flops *= 3.0;  // three tf32 products per fp32-accurate product
   prof_begin(stream);
-  gemm_sm100_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
+  if (ab_dt == DT_FP32)
+    gemm_sm100_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(p);
+  else
+    gemm_sm100_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(p);
   prof_end(0, stream, flops, bytes);
   return cudaGetLastError() == cudaSuccess ? MSIGN_OK : MSIGN_ERR_CUDA;
 }
@@ -379,11 +399,12 @@ msign_status launch_norm(const void* in, int in_dt, int64_t per, int64_t batch, 
 
 msign_status launch_ingest(const void* in, int in_dt, int64_t rows, int64_t cols, bool transpose, const float* scale,
                            int cast_dt, void* xop, int op_dt, int64_t ld_op, int64_t op_bs, float* master,
-                           int64_t ld_m, int64_t m_bs, int64_t batch, cudaStream_t stream) {
+                           int64_t ld_m, int64_t m_bs, int64_t batch, cudaStream_t stream, int64_t op_plane = 0) {
   const int64_t n = transpose ? cols : rows, m = transpose ? rows : cols;
   const double bytes =
       static_cast<double>(batch) * rows * cols * (dtype_size(in_dt) + dtype_size(op_dt) + (master ? 4 : 0));
-  const bool rowwise = !transpose && op_dt != DT_FP32 && cols % 8 == 0 && ld_op % 8 == 0 && (!master || ld_m % 8 == 0) &&
+  const bool rowwise = !transpose && op_dt != DT_FP32 && op_dt != DT_TF32_LO && cols % 8 == 0 && ld_op % 8 == 0 &&
+                       (!master || ld_m % 8 == 0) && (op_dt != DT_TF32_HI || op_plane % 8 == 0) &&
                        (reinterpret_cast<uintptr_t>(in) % 16) == 0 && (reinterpret_cast<uintptr_t>(xop) % 16) == 0 &&
                        (!master || (reinterpret_cast<uintptr_t>(master) % 16) == 0) && op_bs % 8 == 0 &&
                        (!master || m_bs % 8 == 0);
@@ -393,8 +414,12 @@ msign_status launch_ingest(const void* in, int in_dt, int64_t rows, int64_t cols
     prof_begin(stream);
 #define MSB_INGEST(IN, OP)                                                                                        \
   ingest_rows_kernel<IN, OP><<<g, 256, 0, stream>>>(in, rows, static_cast<int>(cols), scale, cast_dt, xop, ld_op, op_bs, \
-                                                    master, ld_m, m_bs)
-    if (op_dt == DT_BF16) {
+                                                    op_plane, master, ld_m, m_bs)
+    if (op_dt == DT_TF32_HI) {
+      if (in_dt == DT_BF16) MSB_INGEST(DT_BF16, DT_TF32_HI);
+      else if (in_dt == DT_FP16) MSB_INGEST(DT_FP16, DT_TF32_HI);
+      else MSB_INGEST(DT_FP32, DT_TF32_HI);
+    } else if (op_dt == DT_BF16) {
       if (in_dt == DT_BF16) MSB_INGEST(DT_BF16, DT_BF16);
       else if (in_dt == DT_FP16) MSB_INGEST(DT_FP16, DT_BF16);
       else MSB_INGEST(DT_FP32, DT_BF16);
@@ -410,8 +435,8 @@ msign_status launch_ingest(const void* in, int in_dt, int64_t rows, int64_t cols
   dim3 g(static_cast<unsigned>((m + 31) / 32), static_cast<unsigned>((n + 31) / 32), static_cast<unsigned>(batch));
   prof_begin(stream);
   ingest_kernel<<<g, dim3(32, 8), 0, stream>>>(in, in_dt, static_cast<int>(rows), static_cast<int>(cols),
-                                               transpose ? 1 : 0, scale, cast_dt, xop, op_dt, ld_op, op_bs, master,
-                                               ld_m, m_bs);
+                                               transpose ? 1 : 0, scale, cast_dt, xop, op_dt, ld_op, op_bs, op_plane,
+                                               master, ld_m, m_bs);
   prof_end(2, stream, 0.0, bytes);
   return launch_ok();
 }
@@ -427,15 +452,18 @@ struct NsBuffers {
   void* B;        // bf16 n x ldn
 };
 
-void carve_ns(Carver& cv, int64_t batch, int64_t n, int64_t m, NsBuffers* b) {
+// fp32: the operand copies P, A and B hold two fp32 planes (tf32 hi, lo)
+// per matrix, [batch][plane][rows][ld].
+void carve_ns(Carver& cv, int64_t batch, int64_t n, int64_t m, NsBuffers* b, bool fp32 = false) {
   const int64_t ldm = round_up(m, 8), ldn = round_up(n, 8);
+  const uint64_t op = fp32 ? 8ull : 2ull;  // bytes per operand element (two fp32 planes, or bf16)
   b->partials = static_cast<float*>(cv.take(sizeof(float) * kNormParts * batch));
   b->scale = static_cast<float*>(cv.take(sizeof(float) * batch));
-  b->P[0] = cv.take(2ull * batch * n * ldm);
-  b->P[1] = cv.take(2ull * batch * n * ldm);
+  b->P[0] = cv.take(op * batch * n * ldm);
+  b->P[1] = cv.take(op * batch * n * ldm);
   b->master = static_cast<float*>(cv.take(4ull * batch * n * ldm));
-  b->A = cv.take(2ull * batch * n * ldn);
-  b->B = cv.take(2ull * batch * n * ldn);
+  b->A = cv.take(op * batch * n * ldn);
+  b->B = cv.take(op * batch * n * ldn);
 }
 
 // Launches a list of classes of one operand dtype, kMaxClasses at a time.
@@ -453,7 +481,15 @@ struct NsClass {
   NsBuffers w;
   int64_t batch, n, m;
   std::vector<EpiOut> final_outs;  // outputs of the last step's B X product
+  bool fp32 = false;               // fp32-accurate products (3xTF32 on split planes)
+  int op_dt = DT_BF16;             // 16-bit operand type otherwise (bf16 or fp16)
 };
+
+// Hi and lo plane outputs of a split matrix at `p` (planes of `plane` elements).
+std::vector<EpiOut> split_out(void* p, int64_t ld, int64_t plane) {
+  return {out_to(p, DT_TF32_HI, ld, 2 * plane, false),
+          out_to(static_cast<char*>(p) + 4 * plane, DT_TF32_LO, ld, 2 * plane, false)};
+}
 
 // The three products of one NS step ([P2] eq. 6, left form), each launched
 // once for all classes:
@@ -464,23 +500,56 @@ struct NsClass {
 msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b, float c, bool last,
                      cudaStream_t stream) {
   std::vector<ClassSpec> syrk, sqr, bx;
+  std::vector<ClassSpec> syrk32, sqr32, bx32;
   for (const NsClass& k : cls) {
     const int64_t n = k.n, m = k.m, ldm = round_up(m, 8), ldn = round_up(n, 8);
-    const Mat X{k.w.P[cur], DT_BF16, n, m, ldm, n * ldm};
-    const Mat A{k.w.A, DT_BF16, n, n, ldn, n * ldn};
-    const Mat B{k.w.B, DT_BF16, n, n, ldn, n * ldn};
+    if (k.fp32) {
+      // the same three products on tf32 hi/lo planes, each a three-pass split product
+      const int64_t pm = n * ldm, pn = n * ldn;  // plane strides
+      const Mat X{k.w.P[cur], DT_FP32, n, m, ldm, pm};
+      const Mat A{k.w.A, DT_FP32, n, n, ldn, pn};
+      const Mat B{k.w.B, DT_FP32, n, n, ldn, pn};
+      ClassSpec s;
+      s.A = X, s.B = X, s.symmetric = true, s.split = true;
+      s.M = n, s.N = n, s.K = m, s.batch = k.batch;
+      s.outs = split_out(k.w.A, ldn, pn);
+      syrk32.push_back(s);
+      ClassSpec q;
+      q.A = A, q.B = A, q.symmetric = true, q.a_sym = true, q.b_sym = true, q.split = true;
+      q.M = n, q.N = n, q.K = n, q.batch = k.batch;
+      q.alpha = c, q.beta = b;
+      q.C = k.w.A, q.c_dt = DT_FP32, q.ldc = ldn, q.c_bs = 2 * pn, q.c_plane = pn;
+      q.outs = split_out(k.w.B, ldn, pn);
+      sqr32.push_back(q);
+      ClassSpec x;
+      x.A = B, x.a_sym = true, x.B = X, x.b_mn = true, x.split = true;
+      x.M = n, x.N = m, x.K = n, x.batch = k.batch;
+      x.alpha = 1.0f, x.beta = a;
+      x.C = k.w.master, x.c_dt = DT_FP32, x.ldc = ldm, x.c_bs = pm;
+      if (!last) {
+        x.outs = split_out(k.w.P[cur ^ 1], ldm, pm);
+        x.outs.insert(x.outs.begin(), out_to(k.w.master, DT_FP32, ldm, pm, false));
+      } else {
+        x.outs = k.final_outs;
+      }
+      bx32.push_back(x);
+      continue;
+    }
+    const Mat X{k.w.P[cur], k.op_dt, n, m, ldm, n * ldm};
+    const Mat A{k.w.A, k.op_dt, n, n, ldn, n * ldn};
+    const Mat B{k.w.B, k.op_dt, n, n, ldn, n * ldn};
     ClassSpec s;  // A: upper 256-blocks of X X^T
     s.A = X, s.B = X, s.symmetric = true;
     s.M = n, s.N = n, s.K = m, s.batch = k.batch;
-    s.outs = {out_to(k.w.A, DT_BF16, ldn, n * ldn, false)};
+    s.outs = {out_to(k.w.A, k.op_dt, ldn, n * ldn, false)};
     syrk.push_back(s);
 
     ClassSpec q;  // B: upper 256-blocks of b A + c A A, both operands read from A's upper blocks
     q.A = A, q.B = A, q.symmetric = true, q.a_sym = true, q.b_sym = true;
     q.M = n, q.N = n, q.K = n, q.batch = k.batch;
     q.alpha = c, q.beta = b;
-    q.C = k.w.A, q.c_dt = DT_BF16, q.ldc = ldn, q.c_bs = n * ldn;
-    q.outs = {out_to(k.w.B, DT_BF16, ldn, n * ldn, false)};
+    q.C = k.w.A, q.c_dt = k.op_dt, q.ldc = ldn, q.c_bs = n * ldn;
+    q.outs = {out_to(k.w.B, k.op_dt, ldn, n * ldn, false)};
     sqr.push_back(q);
 
     ClassSpec x;  // X' = a X + B X with B read from its upper blocks
@@ -490,14 +559,19 @@ msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b,
     x.C = k.w.master, x.c_dt = DT_FP32, x.ldc = ldm, x.c_bs = n * ldm;
     if (!last)
       x.outs = {out_to(k.w.master, DT_FP32, ldm, n * ldm, false),
-                out_to(k.w.P[cur ^ 1], DT_BF16, ldm, n * ldm, false)};
+                out_to(k.w.P[cur ^ 1], k.op_dt, ldm, n * ldm, false)};
     else
       x.outs = k.final_outs;
     bx.push_back(x);
   }
-  msign_status st = launch_all(syrk, DT_BF16, stream);
-  if (st == MSIGN_OK) st = launch_all(sqr, DT_BF16, stream);
-  if (st == MSIGN_OK) st = launch_all(bx, DT_BF16, stream);
+  // one launch per phase and operand type (all 16-bit classes of a call share one type)
+  const int op16 = cls.empty() ? DT_BF16 : cls.front().op_dt;
+  msign_status st = launch_all(syrk, op16, stream);
+  if (st == MSIGN_OK) st = launch_all(syrk32, DT_FP32, stream);
+  if (st == MSIGN_OK) st = launch_all(sqr, op16, stream);
+  if (st == MSIGN_OK) st = launch_all(sqr32, DT_FP32, stream);
+  if (st == MSIGN_OK) st = launch_all(bx, op16, stream);
+  if (st == MSIGN_OK) st = launch_all(bx32, DT_FP32, stream);
   return st;
 }
 
@@ -635,12 +709,11 @@ msign_status msign_profile_reset(void) {
 }
 
 size_t msign_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute_dtype) {
-  (void)compute_dtype;
   if (batch <= 0 || rows <= 0 || cols <= 0) return 0;
   const int64_t n = std::min(rows, cols), m = std::max(rows, cols);
   Carver cv(nullptr);
   NsBuffers b;
-  carve_ns(cv, batch, n, m, &b);
+  carve_ns(cv, batch, n, m, &b, compute_dtype == MSIGN_FP32);
   return cv.off + 1024;
 }
 
@@ -654,7 +727,6 @@ msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dty
   if (st != MSIGN_OK) return st;
   if (batch == 0 || rows == 0 || cols == 0) return MSIGN_OK;
   if (in == nullptr || out == nullptr) return MSIGN_ERR_INVALID_ARG;
-  if (compute_dtype != MSIGN_BF16) return MSIGN_ERR_UNSUPPORTED;
   if (batch > 65535 || rows > (1 << 30) || cols > (1 << 30)) return MSIGN_ERR_UNSUPPORTED;
   const size_t need = msign_ns_workspace_size(batch, rows, cols, compute_dtype);
   if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
@@ -668,18 +740,26 @@ msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dty
   const int64_t n = tr ? cols : rows, m = tr ? rows : cols;
   const int64_t ldm = round_up(m, 8);
   const int io = to_dt(io_dtype);
+  const bool fp32 = compute_dtype == MSIGN_FP32;
+  const int cd = to_dt(compute_dtype);  // the input is cast to the compute dtype first
   Carver cv(workspace);
   NsBuffers w;
-  carve_ns(cv, batch, n, m, &w);
+  carve_ns(cv, batch, n, m, &w, fp32);
 
-  st = launch_norm(in, io, rows * cols, batch, DT_BF16, sch.eps, 0, w.partials, w.scale, stream);
+  st = launch_norm(in, io, rows * cols, batch, cd, sch.eps, 0, w.partials, w.scale, stream);
   if (st != MSIGN_OK) return st;
-  st = launch_ingest(in, io, rows, cols, tr, w.scale, DT_BF16, w.P[0], DT_BF16, ldm, n * ldm, w.master, ldm, n * ldm,
-                     batch, stream);
+  if (fp32)
+    st = launch_ingest(in, io, rows, cols, tr, w.scale, DT_FP32, w.P[0], DT_TF32_HI, ldm, 2 * n * ldm, w.master, ldm,
+                       n * ldm, batch, stream, n * ldm);
+  else
+    st = launch_ingest(in, io, rows, cols, tr, w.scale, cd, w.P[0], cd, ldm, n * ldm, w.master, ldm, n * ldm, batch,
+                       stream);
   if (st != MSIGN_OK) return st;
   std::vector<NsClass> cls(1);
   cls[0].w = w;
   cls[0].batch = batch, cls[0].n = n, cls[0].m = m;
+  cls[0].fp32 = fp32;
+  cls[0].op_dt = fp32 ? DT_BF16 : cd;
   cls[0].final_outs = {out_to(out, io, cols, rows * cols, tr)};
   return ns_iterate(cls, sch, stream);
 }

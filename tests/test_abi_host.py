@@ -88,7 +88,9 @@ def test_invalid_arguments_rejected_on_host(L):
         _lib.ERR_UNSUPPORTED
     # workspace missing for a real problem (pointer values are never dereferenced on this path)
     assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, None, None, 0, None) == _lib.ERR_WORKSPACE
-    assert L.msign_ns(16, 16, _lib.BF16, _lib.FP32, 1, 4, 4, None, None, 0, None) == _lib.ERR_UNSUPPORTED
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.FP32, 1, 4, 4, None, None, 0, None) == _lib.ERR_WORKSPACE
+    # the fp32-accurate path keeps two fp32 planes per operand: larger workspace
+    assert L.msign_ns_workspace_size(1, 512, 512, _lib.FP32) > L.msign_ns_workspace_size(1, 512, 512, _lib.BF16)
 
 
 def test_gram_ns_restart_validation(L):

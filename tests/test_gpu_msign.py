@@ -8,7 +8,7 @@ import newton_schulz_msign_b200 as msb
 from newton_schulz_msign_b200 import synth
 from oracle import ns_oracle as O
 
-from helpers import TOL_BF16, rel_fro, to_np
+from helpers import TOL_BF16, TOL_FP32, rel_fro, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -110,3 +110,49 @@ def test_momentum_like_full_size(rows, cols, batch):
         ref = O.msign_ns(to_np(x[i]), input_cast="bf16")
         assert rel_fro(to_np(y[i]), ref) < TOL_BF16
     assert torch.equal(y[0], y[1])
+
+
+# ---------------------------------------------------------------- fp16 and fp32 compute
+
+@pytest.mark.parametrize("shape", [(256, 512), (64, 128), (33, 257), (300, 100)])
+def test_compute_fp16(shape):
+    # fp16 operands: the input is cast to fp16 first; ~8x smaller error than bf16
+    x = torch.from_numpy(synth.gaussian(shape, seed=shape[0] + shape[1])).cuda()
+    y = msb.msign_ns(x, compute="fp16")
+    msb.sync_status()
+    ref = O.msign_ns(to_np(x), input_cast="fp16")
+    assert rel_fro(to_np(y), ref) < 5e-3
+
+
+@pytest.mark.parametrize("shape", [(256, 512), (64, 128), (33, 257), (300, 100), (520, 600), (7, 129)])
+def test_compute_fp32(shape):
+    # fp32-accurate path: 3xTF32 products, fp32 everywhere else; no input cast
+    x = torch.from_numpy(synth.gaussian(shape, seed=3 * shape[0] + shape[1])).cuda()
+    y = msb.msign_ns(x, compute="fp32")
+    msb.sync_status()
+    ref = O.msign_ns(to_np(x))
+    assert rel_fro(to_np(y), ref) < TOL_FP32
+
+
+def test_compute_fp32_batched_momentum_like():
+    xs = np.stack([synth.momentum_like(384, 1024, seed=s) for s in (1, 2)])
+    x = torch.from_numpy(xs).cuda()
+    y = msb.msign_ns(x, compute="fp32")
+    msb.sync_status()
+    assert rel_fro(to_np(y), O.msign_ns(to_np(x))) < TOL_FP32
+
+
+def test_compute_fp32_coefficient_table(coeff_tables):
+    x = torch.from_numpy(synth.gaussian((200, 600), seed=41)).cuda()
+    sched = coeff_tables["dion_5step"]
+    y = msb.msign_ns(x, compute="fp32", coeffs=sched)
+    msb.sync_status()
+    assert rel_fro(to_np(y), O.msign_ns(to_np(x), sched)) < TOL_FP32
+
+
+def test_compute_fp32_full_size():
+    # the 4096 x 4096 workload through the fp32-accurate path, checked whole
+    x = synth.momentum_like_torch(4096, 4096, seed=77, device="cuda")
+    y = msb.msign_ns(x, compute="fp32")
+    msb.sync_status()
+    assert rel_fro(to_np(y), O.msign_ns(to_np(x))) < TOL_FP32
