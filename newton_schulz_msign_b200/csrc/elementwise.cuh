@@ -131,7 +131,8 @@ __global__ void __launch_bounds__(1024) norm_finalize_kernel(const float* partia
 // Output space: n x m per matrix (n = rows, m = cols, or swapped when
 // `transpose`).  Block (32, 8) handles a 32 x 32 output tile.
 //   xop[i][j]    = round_op(cast(in) * s)      (operand copy, op_dt)
-//   master[i][j] = cast(in) * s                 (fp32 copy; nullable)
+//   master(i, j) = cast(in) * s                 (fp32 copy, blocked layout
+//                                                with padded width ld_m; nullable)
 // in[b] is rows x cols row-major with leading dimension `cols`.
 __global__ void __launch_bounds__(256) ingest_kernel(const void* in, int in_dt, int rows, int cols, int transpose,
                                                      const float* scale, int cast_dt, void* xop, int op_dt,
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(256) ingest_kernel(const void* in, int in_dt, 
                   (static_cast<long long>(b) * op_bs + static_cast<long long>(i) * ld_op + j) * dtype_size(op_dt);
       store_elem(dst, op_dt, xs);
       if (op_dt == DT_TF32_HI) store_elem(dst + op_plane * 4, DT_TF32_LO, xs);
-      if (master) master[static_cast<long long>(b) * m_bs + static_cast<long long>(i) * ld_m + j] = xs;
+      if (master) master[static_cast<long long>(b) * m_bs + blk_off(i, j, ld_m)] = xs;
     }
   }
 }
@@ -237,9 +238,9 @@ __global__ void __launch_bounds__(256) ingest_rows_kernel(const void* in, long l
       reinterpret_cast<float4*>(hp + op_plane)[0] = make_float4(l[0], l[1], l[2], l[3]);
       reinterpret_cast<float4*>(hp + op_plane)[1] = make_float4(l[4], l[5], l[6], l[7]);
       if (master) {
-        float4* d = reinterpret_cast<float4*>(master + static_cast<long long>(b) * m_bs + i * ld_m + j);
-        d[0] = make_float4(x[0], x[1], x[2], x[3]);
-        d[1] = make_float4(x[4], x[5], x[6], x[7]);
+        float* d = master + static_cast<long long>(b) * m_bs + blk_off(i, j, ld_m);
+        *reinterpret_cast<float4*>(d) = make_float4(x[0], x[1], x[2], x[3]);
+        *reinterpret_cast<float4*>(d + 128) = make_float4(x[4], x[5], x[6], x[7]);
       }
       continue;
     }
@@ -257,9 +258,9 @@ __global__ void __launch_bounds__(256) ingest_rows_kernel(const void* in, long l
     *reinterpret_cast<uint4*>(reinterpret_cast<char*>(xop) + (static_cast<long long>(b) * op_bs + i * ld_op + j) * 2) =
         make_uint4(o[0], o[1], o[2], o[3]);
     if (master) {
-      float4* d = reinterpret_cast<float4*>(master + static_cast<long long>(b) * m_bs + i * ld_m + j);
-      d[0] = make_float4(x[0], x[1], x[2], x[3]);
-      d[1] = make_float4(x[4], x[5], x[6], x[7]);
+      float* d = master + static_cast<long long>(b) * m_bs + blk_off(i, j, ld_m);
+      *reinterpret_cast<float4*>(d) = make_float4(x[0], x[1], x[2], x[3]);
+      *reinterpret_cast<float4*>(d + 128) = make_float4(x[4], x[5], x[6], x[7]);
     }
   }
 }
@@ -289,7 +290,8 @@ __global__ void __launch_bounds__(256) momentum_kernel(float* M, const void* G, 
 }
 
 // W (rows x cols, w_dt) <- W - coef * O where O is stored oriented:
-// n x m with leading dimension ld_o, transposed when `transpose`.
+// n x m in the blocked fp32 layout of padded width ld_o, transposed when
+// `transpose`.
 __global__ void __launch_bounds__(256) apply_update_kernel(void* W, int w_dt, int rows, int cols, const float* O,
                                                            long long ld_o, int transpose, float coef) {
   __shared__ float tile[32][33];
@@ -300,14 +302,14 @@ __global__ void __launch_bounds__(256) apply_update_kernel(void* W, int w_dt, in
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int i = i0 + ty + 8 * k, j = j0 + tx;
-      o[k] = (i < rows && j < cols) ? O[static_cast<long long>(i) * ld_o + j] : 0.0f;
+      o[k] = (i < rows && j < cols) ? O[blk_off(i, j, ld_o)] : 0.0f;
     }
   } else {
     // W(i, j) -= O(j, i): O is cols x rows
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int orow = j0 + ty + 8 * k, ocol = i0 + tx;
-      tile[ty + 8 * k][tx] = (orow < cols && ocol < rows) ? O[static_cast<long long>(orow) * ld_o + ocol] : 0.0f;
+      tile[ty + 8 * k][tx] = (orow < cols && ocol < rows) ? O[blk_off(orow, ocol, ld_o)] : 0.0f;
     }
     __syncthreads();
 #pragma unroll

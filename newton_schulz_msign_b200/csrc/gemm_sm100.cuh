@@ -104,7 +104,7 @@ constexpr int kScratchStride = 33;  // padded row of the per-warp 32 x 32 fp32 t
 constexpr int kStageOutBytes = 32 * kScratchStride * 4;
 constexpr int kEpiBytes = 4 * kStageOutBytes;  // one scratch block per epilogue warp
 constexpr int kTmemCols = 512;
-constexpr int kMaxClasses = 8;
+constexpr int kMaxClasses = 16;
 constexpr int kNumBarriers = 2 * kStages + 2 + 2 + 1;
 constexpr int kSmemBytes = 1024 /* alignment slack */ + kStages * kStageBytes + kEpiBytes + kNumBarriers * 8 + 16;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -126,7 +126,7 @@ struct EpiOut {
   int dtype;
   int transposed;
   float gamma;
-  int pad;
+  int blocked;  // fp32 in the 32 x 32 blocked layout (blk_off); direct stores only
 };
 
 // Per-class scalars: tile schedule and epilogue (read through the constant
@@ -147,7 +147,18 @@ struct ClassInfo {
   const float* beta_scale;   // optional per-batch factor on beta
   const void* C;             // optional epilogue input, C[row][col]
   long long ldc, c_bs;
+  int c_blocked;             // C is fp32 in the 32 x 32 blocked layout (blk_off)
   EpiOut out[kMaxOuts];
+  // Dependencies between classes of one launch, by 256-row block of each
+  // batch entry (index b * tiles_m + block; every class of a chain has the
+  // same row-block count).  A tile (tm, tn) starts once dep[tm] -- and
+  // dep[tn] when dep_both -- reach dep_target.  Each epilogue warp adds 1 to
+  // sig[tm] (and to sig[tn] for an off-diagonal tile of a symmetric class)
+  // after storing its rows, so a row block is complete at 8 x the number of
+  // tiles that touch it.
+  const int* dep;
+  int* sig;
+  int dep_target, dep_both;
 };
 
 struct alignas(64) GemmClass {
@@ -166,6 +177,8 @@ struct GemmParams {
   int* err;        // device error word (bit 0: a bounded wait ran out)
   unsigned long long timeout_ns;
 };
+
+static_assert(sizeof(GemmParams) <= 32764, "kernel parameter space");
 
 struct TileCoord {
   int c, b, tm, tn;
@@ -194,6 +207,19 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
     tn = tm + r;
   }
   return {c, b, tm, tn};
+}
+
+// ---------------------------------------------------------------- blocked fp32 layout
+//
+// The fp32 copy of X is private to the library, so it is laid out for the
+// epilogue's access pattern rather than row-major: 32 x 32 blocks, row-major
+// over blocks, and inside a block 8 column quads of 32 rows x 4 floats.  The
+// lane that owns row r of a block then finds its 4 consecutive columns next
+// to those of lanes r - 1 and r + 1, so one 16-byte access per lane covers
+// 512 contiguous bytes per warp.  `ldb` is the padded column count (a
+// multiple of 32); a matrix occupies round_up(rows, 32) x ldb floats.
+__host__ __device__ __forceinline__ long long blk_off(long long r, long long c, long long ldb) {
+  return (((r >> 5) * (ldb >> 5) + (c >> 5)) << 10) + (((c & 31) >> 2) << 7) + ((r & 31) << 2) + (c & 3);
 }
 
 // ---------------------------------------------------------------- row I/O
@@ -317,6 +343,22 @@ __device__ __forceinline__ uint32_t lane_mask(int n) { return n >= 32 ? 0xFFFFFF
 // Epilogue input of the block at (row0, col0) for this lane's row.
 __device__ __forceinline__ void load_c(const ClassInfo& k, int b, int row0, int col0, int lane, float (&cv)[32]) {
   const int r = row0 + lane;
+  if (k.c_blocked) {
+    // whole padded block, coalesced; elements outside C read as 0
+    const float* q = reinterpret_cast<const float*>(k.C) + static_cast<long long>(b) * k.c_bs +
+                     blk_off(row0, col0, k.ldc) + 4 * lane;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 f = *reinterpret_cast<const float4*>(q + 128 * j);
+      cv[4 * j + 0] = f.x, cv[4 * j + 1] = f.y, cv[4 * j + 2] = f.z, cv[4 * j + 3] = f.w;
+    }
+    if (r >= k.M || col0 + 32 > k.N) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (r >= k.M || col0 + i >= k.N) cv[i] = 0.0f;
+    }
+    return;
+  }
   const uint32_t m = (r < k.M) ? lane_mask(k.N - col0) : 0u;
   const char* hp = gaddr(k.C, k.c_dtype, k.ldc, k.c_bs, b, r, col0);
   load_row32(hp, k.c_dtype, m, cv);
@@ -361,6 +403,14 @@ __device__ __forceinline__ void epilogue_block(const ClassInfo& k, int b, int ro
     const float g = (col0 == row0) ? e.gamma : 0.0f;
 #pragma unroll
     for (int i = 0; i < 32; ++i) w[i] = (i == lane) ? acc[i] + g : acc[i];
+    if (e.blocked) {
+      // whole padded block, coalesced (elements outside the matrix are 0)
+      float* q = reinterpret_cast<float*>(e.ptr) + static_cast<long long>(b) * e.bs + blk_off(row0, col0, e.ld) + 4 * lane;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float4*>(q + 128 * j) = make_float4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+      continue;
+    }
     const bool direct = !e.transposed;
     const bool trans = e.transposed || mirror;
     if (direct && r < k.M) {
@@ -473,6 +523,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const void* tmA2 = &g.tmA2;
         const void* tmB = &g.tmB;
         const void* tmB2 = &g.tmB2;
+        if (k.dep != nullptr) {
+          // operands produced earlier in this launch: wait for their row blocks
+          const int* d = k.dep + tc.b * k.tiles_m;
+          if (!wait_counter(d + tc.tm, k.dep_target, s_abort, p.err, limit) ||
+              (k.dep_both && !wait_counter(d + tc.tn, k.dep_target, s_abort, p.err, limit))) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();
+        }
         for (int step = 0; step < nk * passes; ++step) {
           const int kb = step / passes, pass = step - kb * passes;
           const int za = passes == 1 ? tc.b : 2 * tc.b + (pass == 2 ? 1 : 0);
@@ -598,13 +658,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int jfirst = 0;
       if (mirror)
         while (jfirst < kBN / 32 && tc.tn * kBN + jfirst * 32 < row0) ++jfirst;
-      // the epilogue input of the first block is read before the
-      // accumulator is ready
       const bool has_c = k.C != nullptr;
+      int ok = 1;
+      if (has_c && k.dep != nullptr) {
+        // C was written earlier in this launch: acquire it for this warp
+        const int* d = k.dep + tc.b * k.tiles_m + tc.tm;
+        if (lane == 0) ok = wait_counter(d, k.dep_target, s_abort, p.err, limit) ? 1 : 0;
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) break;
+        // each lane's own acquire orders its C loads (plain, L1-cached)
+        // after the producers' release
+        (void)ld_acquire_gpu(d);
+      }
+      // the epilogue input of the first block is read before the
+      // accumulator is ready, that of each next block while one is stored
       float cv[32];
       if (has_c && row0 < k.M && jfirst < kBN / 32 && tc.tn * kBN + jfirst * 32 < k.N)
         load_c(k, tc.b, row0, tc.tn * kBN + jfirst * 32, lane, cv);
-      int ok = 1;
       if (lane == 0) ok = wait_bounded(&tfull[buf], bphase, s_abort, p.err, limit) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
@@ -613,6 +683,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int j = jfirst; j < kBN / 32; ++j) {
         const int col0 = tc.tn * kBN + j * 32;
         if (row0 >= k.M || col0 >= k.N) break;
+        float cn[32];
+        const bool pre = has_c && j + 1 < kBN / 32 && col0 + 32 < k.N;
+        if (pre) load_c(k, tc.b, row0, col0 + 32, lane, cn);
         uint32_t raw[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * kBN + j * 32),
                            raw);
@@ -620,12 +693,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float acc[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) acc[i] = __uint_as_float(raw[i]);
-        if (has_c && j != jfirst) load_c(k, tc.b, row0, col0, lane, cv);
         epilogue_block(k, tc.b, row0, col0, mirror, acc, cv, scratch, lane);
+        if (pre) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) cv[i] = cn[i];
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+      if (k.sig != nullptr) {
+        // publish this warp's rows of the tile to later classes of the launch
+        fence_proxy_async_global();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+          int* sg = k.sig + tc.b * k.tiles_m;
+          red_release_gpu_add(sg + tc.tm, 1);
+          if (k.symmetric && tc.tn != tc.tm) red_release_gpu_add(sg + tc.tn, 1);
+        }
+      }
       buf ^= 1;
       if (buf == 0) bphase ^= 1u;
     }

@@ -140,6 +140,11 @@ void prof_end(int kind, cudaStream_t s, double flops, double bytes) {
 // ---------------------------------------------------------------- helpers
 
 inline int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// NS steps per chained launch: 3 phases each, within kMaxClasses classes.
+constexpr int kChainSteps = 5;
+static_assert(3 * kChainSteps <= kMaxClasses, "a chain of kChainSteps steps fits one launch");
 
 int to_dt(msign_dtype d) { return d == MSIGN_BF16 ? DT_BF16 : d == MSIGN_FP16 ? DT_FP16 : DT_FP32; }
 
@@ -229,6 +234,10 @@ bool encode(CUtensorMap* tm, const Mat& m, int box0, int box_rows, int64_t batch
   return r == CUDA_SUCCESS;
 }
 
+// fp32 in the blocked layout of blk_off(): padded width and per-matrix size
+inline int64_t blk_ld(int64_t cols) { return round_up(cols, 32); }
+inline int64_t blk_size(int64_t rows, int64_t cols) { return round_up(rows, 32) * round_up(cols, 32); }
+
 EpiOut out_to(void* ptr, int dt, int64_t ld, int64_t bs, bool transposed, float gamma = 0.0f) {
   EpiOut e;
   std::memset(&e, 0, sizeof(e));
@@ -238,6 +247,13 @@ EpiOut out_to(void* ptr, int dt, int64_t ld, int64_t bs, bool transposed, float 
   e.bs = bs;
   e.transposed = transposed ? 1 : 0;
   e.gamma = gamma;
+  return e;
+}
+
+// A direct fp32 output in the blocked layout (ld = padded width, bs = matrix size).
+EpiOut out_blocked(float* ptr, int64_t ld, int64_t bs) {
+  EpiOut e = out_to(ptr, DT_FP32, ld, bs, false);
+  e.blocked = 1;
   return e;
 }
 
@@ -260,7 +276,13 @@ struct ClassSpec {
   const void* C = nullptr;
   int c_dt = DT_FP32;
   int64_t ldc = 0, c_bs = 0;
+  bool c_blocked = false;  // C is fp32 in the blocked layout
   std::vector<EpiOut> outs;
+  // in-launch dependencies (see ClassInfo): counters by batch entry and 256-row block
+  const int* dep = nullptr;
+  int* sig = nullptr;
+  int dep_target = 0;
+  bool dep_both = false;
 };
 
 // Square kBM x kBN tiles on or above the diagonal.
@@ -276,7 +298,10 @@ int64_t class_tiles(const ClassSpec& s) {
 }
 
 // Encodes and launches up to kMaxClasses classes of one operand dtype.
-msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_t stream) {
+// `ordered`: the classes form a chain (later classes read earlier outputs
+// through dep/sig counters) and keep their order; otherwise the longest
+// reductions go first.
+msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_t stream, bool ordered = false) {
   DeviceState* dev = nullptr;
   msign_status st = device_state(&dev);
   if (st != MSIGN_OK) return st;
@@ -285,7 +310,8 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
   if (specs.empty()) return MSIGN_OK;
   if (specs.size() > static_cast<size_t>(kMaxClasses)) return MSIGN_ERR_UNSUPPORTED;
   // longest reduction first: its tiles are the longest-running work items
-  std::stable_sort(specs.begin(), specs.end(), [](const ClassSpec& a, const ClassSpec& b) { return a.K > b.K; });
+  if (!ordered)
+    std::stable_sort(specs.begin(), specs.end(), [](const ClassSpec& a, const ClassSpec& b) { return a.K > b.K; });
 
   static thread_local GemmParams p;
   std::memset(&p, 0, sizeof(p));
@@ -346,7 +372,17 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     ci.c_dtype = s.c_dt;
     ci.ldc = s.ldc;
     ci.c_bs = s.c_bs;
+    ci.c_blocked = s.c_blocked ? 1 : 0;
+    if (s.c_blocked && (s.c_dt != DT_FP32 || s.c_plane != 0 || s.symmetric || s.ldc % 32 != 0))
+      return MSIGN_ERR_INVALID_ARG;
+    for (const EpiOut& e : s.outs)
+      if (e.blocked && (e.dtype != DT_FP32 || e.transposed || s.symmetric || e.ld % 32 != 0))
+        return MSIGN_ERR_INVALID_ARG;
     for (size_t o = 0; o < s.outs.size(); ++o) ci.out[o] = s.outs[o];
+    ci.dep = s.dep;
+    ci.sig = s.sig;
+    ci.dep_target = s.dep_target;
+    ci.dep_both = s.dep_both ? 1 : 0;
     total += class_tiles(s);
   }
   if (total > INT32_MAX) return MSIGN_ERR_UNSUPPORTED;
@@ -447,9 +483,10 @@ struct NsBuffers {
   float* partials;
   float* scale;
   void* P[2];     // bf16 operand copies of X (n x ldm)
-  float* master;  // fp32 X (n x ldm)
+  float* master;  // fp32 X, blocked layout (blk_ld(m) wide, blk_size(n, m) per matrix)
   void* A;        // bf16 n x ldn
   void* B;        // bf16 n x ldn
+  int* cnt;       // row-block counters of a chained launch: [kChainSteps][3 phases][batch][tiles]
 };
 
 // fp32: the operand copies P, A and B hold two fp32 planes (tf32 hi, lo)
@@ -461,9 +498,10 @@ void carve_ns(Carver& cv, int64_t batch, int64_t n, int64_t m, NsBuffers* b, boo
   b->scale = static_cast<float*>(cv.take(sizeof(float) * batch));
   b->P[0] = cv.take(op * batch * n * ldm);
   b->P[1] = cv.take(op * batch * n * ldm);
-  b->master = static_cast<float*>(cv.take(4ull * batch * n * ldm));
+  b->master = static_cast<float*>(cv.take(4ull * batch * blk_size(n, m)));
   b->A = cv.take(op * batch * n * ldn);
   b->B = cv.take(op * batch * n * ldn);
+  b->cnt = static_cast<int*>(cv.take(sizeof(int) * 3 * kChainSteps * batch * ceil_div(n, kBM)));
 }
 
 // Launches a list of classes of one operand dtype, kMaxClasses at a time.
@@ -491,98 +529,132 @@ std::vector<EpiOut> split_out(void* p, int64_t ld, int64_t plane) {
           out_to(static_cast<char*>(p) + 4 * plane, DT_TF32_LO, ld, 2 * plane, false)};
 }
 
-// The three products of one NS step ([P2] eq. 6, left form), each launched
-// once for all classes:
-//   SYRK   A = X X^T                  (symmetric, mirror store)
+// The three products of one NS step ([P2] eq. 6, left form) for one class:
+//   SYRK   A = X X^T                  (symmetric, upper 256-blocks)
 //   SQR    B = b A + c A A            (symmetric; A A = A A^T as A = A^T)
 //   BX     X' = a X + B X             (X read MN-major; the a X term uses
 //                                      the fp32 copy of X)
+// The fp32-accurate class runs the same products on tf32 hi/lo planes.
+void ns_specs(const NsClass& k, int cur, float a, float b, float c, bool last, ClassSpec* syrk, ClassSpec* sqr,
+              ClassSpec* bx) {
+  const int64_t n = k.n, m = k.m, ldm = round_up(m, 8), ldn = round_up(n, 8);
+  const int od = k.fp32 ? DT_FP32 : k.op_dt;
+  const bool sp = k.fp32;
+  const int64_t pm = n * ldm, pn = n * ldn;        // matrix (or plane) strides
+  const int64_t zn = sp ? 2 * pn : pn;             // batch stride of A and B
+  const Mat X{k.w.P[cur], od, n, m, ldm, pm};
+  const Mat A{k.w.A, od, n, n, ldn, pn};
+  const Mat B{k.w.B, od, n, n, ldn, pn};
+  auto outs = [&](void* p, int64_t ld, int64_t plane) {
+    return sp ? split_out(p, ld, plane) : std::vector<EpiOut>{out_to(p, od, ld, plane, false)};
+  };
+  ClassSpec& s = *syrk;
+  s = ClassSpec();
+  s.A = X, s.B = X, s.symmetric = true, s.split = sp;
+  s.M = n, s.N = n, s.K = m, s.batch = k.batch;
+  s.outs = outs(k.w.A, ldn, pn);
+
+  ClassSpec& q = *sqr;  // both operands read from A's upper blocks
+  q = ClassSpec();
+  q.A = A, q.B = A, q.symmetric = true, q.a_sym = true, q.b_sym = true, q.split = sp;
+  q.M = n, q.N = n, q.K = n, q.batch = k.batch;
+  q.alpha = c, q.beta = b;
+  q.C = k.w.A, q.c_dt = od, q.ldc = ldn, q.c_bs = zn, q.c_plane = sp ? pn : 0;
+  q.outs = outs(k.w.B, ldn, pn);
+
+  ClassSpec& x = *bx;  // B read from its upper blocks
+  x = ClassSpec();
+  x.A = B, x.a_sym = true, x.B = X, x.b_mn = true, x.split = sp;
+  x.M = n, x.N = m, x.K = n, x.batch = k.batch;
+  x.alpha = 1.0f, x.beta = a;
+  x.C = k.w.master, x.c_dt = DT_FP32, x.ldc = blk_ld(m), x.c_bs = blk_size(n, m), x.c_blocked = true;
+  if (!last) {
+    x.outs = outs(k.w.P[cur ^ 1], ldm, pm);
+    x.outs.insert(x.outs.begin(), out_blocked(k.w.master, blk_ld(m), blk_size(n, m)));
+  } else {
+    x.outs = k.final_outs;
+  }
+}
+
+// Operand dtype of a class's products.
+int ns_op_dt(const NsClass& k) { return k.fp32 ? DT_FP32 : k.op_dt; }
+
+// One NS step as three launches (one per phase), each over all classes.
 msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b, float c, bool last,
                      cudaStream_t stream) {
-  std::vector<ClassSpec> syrk, sqr, bx;
-  std::vector<ClassSpec> syrk32, sqr32, bx32;
-  for (const NsClass& k : cls) {
-    const int64_t n = k.n, m = k.m, ldm = round_up(m, 8), ldn = round_up(n, 8);
-    if (k.fp32) {
-      // the same three products on tf32 hi/lo planes, each a three-pass split product
-      const int64_t pm = n * ldm, pn = n * ldn;  // plane strides
-      const Mat X{k.w.P[cur], DT_FP32, n, m, ldm, pm};
-      const Mat A{k.w.A, DT_FP32, n, n, ldn, pn};
-      const Mat B{k.w.B, DT_FP32, n, n, ldn, pn};
-      ClassSpec s;
-      s.A = X, s.B = X, s.symmetric = true, s.split = true;
-      s.M = n, s.N = n, s.K = m, s.batch = k.batch;
-      s.outs = split_out(k.w.A, ldn, pn);
-      syrk32.push_back(s);
-      ClassSpec q;
-      q.A = A, q.B = A, q.symmetric = true, q.a_sym = true, q.b_sym = true, q.split = true;
-      q.M = n, q.N = n, q.K = n, q.batch = k.batch;
-      q.alpha = c, q.beta = b;
-      q.C = k.w.A, q.c_dt = DT_FP32, q.ldc = ldn, q.c_bs = 2 * pn, q.c_plane = pn;
-      q.outs = split_out(k.w.B, ldn, pn);
-      sqr32.push_back(q);
-      ClassSpec x;
-      x.A = B, x.a_sym = true, x.B = X, x.b_mn = true, x.split = true;
-      x.M = n, x.N = m, x.K = n, x.batch = k.batch;
-      x.alpha = 1.0f, x.beta = a;
-      x.C = k.w.master, x.c_dt = DT_FP32, x.ldc = ldm, x.c_bs = pm;
-      if (!last) {
-        x.outs = split_out(k.w.P[cur ^ 1], ldm, pm);
-        x.outs.insert(x.outs.begin(), out_to(k.w.master, DT_FP32, ldm, pm, false));
-      } else {
-        x.outs = k.final_outs;
+  std::vector<ClassSpec> ph[3];
+  std::vector<int> dts;
+  for (const NsClass& k : cls)
+    if (std::find(dts.begin(), dts.end(), ns_op_dt(k)) == dts.end()) dts.push_back(ns_op_dt(k));
+  for (int p = 0; p < 3; ++p)
+    for (int dt : dts) {
+      std::vector<ClassSpec> v;
+      for (const NsClass& k : cls) {
+        if (ns_op_dt(k) != dt) continue;
+        ClassSpec sp[3];
+        ns_specs(k, cur, a, b, c, last, &sp[0], &sp[1], &sp[2]);
+        v.push_back(sp[p]);
       }
-      bx32.push_back(x);
-      continue;
+      msign_status st = launch_all(v, dt, stream);
+      if (st != MSIGN_OK) return st;
     }
-    const Mat X{k.w.P[cur], k.op_dt, n, m, ldm, n * ldm};
-    const Mat A{k.w.A, k.op_dt, n, n, ldn, n * ldn};
-    const Mat B{k.w.B, k.op_dt, n, n, ldn, n * ldn};
-    ClassSpec s;  // A: upper 256-blocks of X X^T
-    s.A = X, s.B = X, s.symmetric = true;
-    s.M = n, s.N = n, s.K = m, s.batch = k.batch;
-    s.outs = {out_to(k.w.A, k.op_dt, ldn, n * ldn, false)};
-    syrk.push_back(s);
-
-    ClassSpec q;  // B: upper 256-blocks of b A + c A A, both operands read from A's upper blocks
-    q.A = A, q.B = A, q.symmetric = true, q.a_sym = true, q.b_sym = true;
-    q.M = n, q.N = n, q.K = n, q.batch = k.batch;
-    q.alpha = c, q.beta = b;
-    q.C = k.w.A, q.c_dt = k.op_dt, q.ldc = ldn, q.c_bs = n * ldn;
-    q.outs = {out_to(k.w.B, k.op_dt, ldn, n * ldn, false)};
-    sqr.push_back(q);
-
-    ClassSpec x;  // X' = a X + B X with B read from its upper blocks
-    x.A = B, x.a_sym = true, x.B = X, x.b_mn = true;
-    x.M = n, x.N = m, x.K = n, x.batch = k.batch;
-    x.alpha = 1.0f, x.beta = a;
-    x.C = k.w.master, x.c_dt = DT_FP32, x.ldc = ldm, x.c_bs = n * ldm;
-    if (!last)
-      x.outs = {out_to(k.w.master, DT_FP32, ldm, n * ldm, false),
-                out_to(k.w.P[cur ^ 1], k.op_dt, ldm, n * ldm, false)};
-    else
-      x.outs = k.final_outs;
-    bx.push_back(x);
-  }
-  // one launch per phase and operand type (all 16-bit classes of a call share one type)
-  const int op16 = cls.empty() ? DT_BF16 : cls.front().op_dt;
-  msign_status st = launch_all(syrk, op16, stream);
-  if (st == MSIGN_OK) st = launch_all(syrk32, DT_FP32, stream);
-  if (st == MSIGN_OK) st = launch_all(sqr, op16, stream);
-  if (st == MSIGN_OK) st = launch_all(sqr32, DT_FP32, stream);
-  if (st == MSIGN_OK) st = launch_all(bx, op16, stream);
-  if (st == MSIGN_OK) st = launch_all(bx32, DT_FP32, stream);
-  return st;
+  return MSIGN_OK;
 }
 
 // Runs all steps of the schedule on classes whose P[0] / master already hold X0.
+//
+// When every class shares one operand dtype and 3 x classes x steps fit in
+// one launch, up to kChainSteps steps run as ONE launch: the classes are the
+// phases in order, and each phase's tiles wait only for the row blocks they
+// read (SYRK on rows tm, tn of X; SQR on rows tm, tn of A; BX on row tm of
+// B) instead of for the whole previous phase.  This removes the launch gaps
+// and lets the last wave of one phase overlap the first tiles of the next.
+//   The write-after-read hazards of the reused buffers are covered by the
+// same counters: a tile that overwrites A, B or an X copy transitively waits
+// for every reader of the old contents (e.g. SYRK of step t+1 on A[i][j]
+// needs B rows i and j of step t, i.e. every SQR tile that read A rows i, j).
 msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cudaStream_t stream) {
   const int T = sch.steps();
+  bool uniform = !cls.empty();
+  for (const NsClass& k : cls) uniform = uniform && ns_op_dt(k) == ns_op_dt(cls.front());
+  const int per = uniform ? std::min<int>(kChainSteps, kMaxClasses / (3 * static_cast<int>(cls.size()))) : 0;
   int cur = 0;
-  for (int t = 0; t < T; ++t) {
-    msign_status st = ns_step(cls, cur, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == T - 1, stream);
+  if (per == 0) {
+    for (int t = 0; t < T; ++t) {
+      msign_status st = ns_step(cls, cur, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == T - 1, stream);
+      if (st != MSIGN_OK) return st;
+      cur ^= 1;
+    }
+    return MSIGN_OK;
+  }
+  for (int t0 = 0; t0 < T; t0 += per) {
+    const int t1 = std::min(T, t0 + per);
+    std::vector<ClassSpec> chain;
+    for (const NsClass& k : cls) {
+      const size_t bytes = sizeof(int) * 3 * (t1 - t0) * k.batch * ceil_div(k.n, kBM);
+      if (cudaMemsetAsync(k.w.cnt, 0, bytes, stream) != cudaSuccess) return MSIGN_ERR_CUDA;
+    }
+    for (int t = t0; t < t1; ++t, cur ^= 1) {
+      std::vector<ClassSpec> ph[3];
+      for (const NsClass& k : cls) {
+        ClassSpec sp[3];
+        ns_specs(k, cur, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == T - 1, &sp[0], &sp[1], &sp[2]);
+        const int64_t rb = ceil_div(k.n, kBM);  // 256-row blocks of X, A and B
+        auto ctr = [&](int step, int phase) { return k.w.cnt + (3 * (step - t0) + phase) * k.batch * rb; };
+        const int per_block_sym = static_cast<int>(8 * rb);                 // tiles touching a block of A or B
+        const int per_block_x = static_cast<int>(8 * ceil_div(k.m, kBN));  // tiles in a row block of X'
+        sp[0].sig = ctr(t, 0);
+        if (t > t0) sp[0].dep = ctr(t - 1, 2), sp[0].dep_target = per_block_x, sp[0].dep_both = true;
+        sp[1].sig = ctr(t, 1);
+        sp[1].dep = ctr(t, 0), sp[1].dep_target = per_block_sym, sp[1].dep_both = true;
+        if (t + 1 < t1) sp[2].sig = ctr(t, 2);
+        sp[2].dep = ctr(t, 1), sp[2].dep_target = per_block_sym, sp[2].dep_both = false;
+        for (int p = 0; p < 3; ++p) ph[p].push_back(sp[p]);
+      }
+      for (int p = 0; p < 3; ++p) chain.insert(chain.end(), ph[p].begin(), ph[p].end());
+    }
+    msign_status st = launch_grouped(chain, ns_op_dt(cls.front()), stream, /*ordered=*/true);
     if (st != MSIGN_OK) return st;
-    cur ^= 1;
   }
   return MSIGN_OK;
 }
@@ -749,11 +821,11 @@ msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dty
   st = launch_norm(in, io, rows * cols, batch, cd, sch.eps, 0, w.partials, w.scale, stream);
   if (st != MSIGN_OK) return st;
   if (fp32)
-    st = launch_ingest(in, io, rows, cols, tr, w.scale, DT_FP32, w.P[0], DT_TF32_HI, ldm, 2 * n * ldm, w.master, ldm,
-                       n * ldm, batch, stream, n * ldm);
+    st = launch_ingest(in, io, rows, cols, tr, w.scale, DT_FP32, w.P[0], DT_TF32_HI, ldm, 2 * n * ldm, w.master,
+                       blk_ld(m), blk_size(n, m), batch, stream, n * ldm);
   else
-    st = launch_ingest(in, io, rows, cols, tr, w.scale, cd, w.P[0], cd, ldm, n * ldm, w.master, ldm, n * ldm, batch,
-                       stream);
+    st = launch_ingest(in, io, rows, cols, tr, w.scale, cd, w.P[0], cd, ldm, n * ldm, w.master, blk_ld(m),
+                       blk_size(n, m), batch, stream);
   if (st != MSIGN_OK) return st;
   std::vector<NsClass> cls(1);
   cls[0].w = w;
@@ -1039,8 +1111,7 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
       ns[c].batch = counts[c];
       ns[c].n = shapes[c].first;
       ns[c].m = shapes[c].second;
-      const int64_t ldm = round_up(ns[c].m, 8);
-      ns[c].final_outs = {out_to(ns[c].w.master, DT_FP32, ldm, ns[c].n * ldm, false)};
+      ns[c].final_outs = {out_blocked(ns[c].w.master, blk_ld(ns[c].m), blk_size(ns[c].n, ns[c].m))};
     }
     // M <- mu M + G; X0 = bf16(M) / ||bf16(M)||_F into the class slot
     for (int i = begin; i < end; ++i) {
@@ -1059,10 +1130,10 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
                        k.w.scale + slot, stream);
       if (st != MSIGN_OK) return st;
       const bool tr = rows[i] > cols[i];
-      const int64_t ldm = round_up(k.m, 8), per = k.n * ldm;
+      const int64_t ldm = round_up(k.m, 8), per = k.n * ldm, mb = blk_size(k.n, k.m);
       st = launch_ingest(M[i], DT_FP32, rows[i], cols[i], tr, k.w.scale + slot, DT_BF16,
-                         static_cast<char*>(k.w.P[0]) + 2 * slot * per, DT_BF16, ldm, per, k.w.master + slot * per,
-                         ldm, per, 1, stream);
+                         static_cast<char*>(k.w.P[0]) + 2 * slot * per, DT_BF16, ldm, per, k.w.master + slot * mb,
+                         blk_ld(k.m), mb, 1, stream);
       if (st != MSIGN_OK) return st;
     }
     st = ns_iterate(ns, sch, stream);
@@ -1072,13 +1143,13 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
       const int c = cls[i - begin];
       if (c < 0) continue;
       const NsClass& k = ns[c];
-      const int64_t ldm = round_up(k.m, 8), per = k.n * ldm;
+      const int64_t mb = blk_size(k.n, k.m);
       const float coef = lr * std::sqrt(std::max(1.0f, static_cast<float>(rows[i]) / static_cast<float>(cols[i])));
       dim3 g(static_cast<unsigned>((cols[i] + 31) / 32), static_cast<unsigned>((rows[i] + 31) / 32));
       prof_begin(stream);
       apply_update_kernel<<<g, dim3(32, 8), 0, stream>>>(W[i], wd, static_cast<int>(rows[i]),
-                                                         static_cast<int>(cols[i]), k.w.master + slots[i - begin] * per,
-                                                         ldm, rows[i] > cols[i] ? 1 : 0, coef);
+                                                         static_cast<int>(cols[i]), k.w.master + slots[i - begin] * mb,
+                                                         blk_ld(k.m), rows[i] > cols[i] ? 1 : 0, coef);
       prof_end(3, stream, 0.0, static_cast<double>(rows[i]) * cols[i] * (4 + 2 * dtype_size(wd)));
       st = launch_ok();
       if (st != MSIGN_OK) return st;

@@ -78,6 +78,47 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
   }
 }
 
+// ---------------------------------------------------------------- tile counters
+//
+// Phases of one launch that feed each other (an output read as a later
+// operand) synchronise through int counters in global memory: the writer of
+// a tile adds to a counter with release semantics after its stores, the
+// reader waits with acquire loads until the counter reaches its target.
+// The reader's operands arrive by TMA (the async proxy), so both sides also
+// fence between the generic and the async proxy.
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Waits until *ctr >= target, with the same wall-clock bound and abort
+// protocol as wait_bounded().
+__device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatile int* abort_word, int* err,
+                                             uint64_t limit_ns) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(100);
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if (abort_word != nullptr && *abort_word) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      if (abort_word != nullptr) *abort_word = 1;
+      if (err != nullptr) atomicOr(err, 1);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
