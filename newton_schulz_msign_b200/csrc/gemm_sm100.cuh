@@ -169,6 +169,15 @@ struct alignas(64) GemmClass {
   ClassInfo info;
 };
 
+// Dynamic tile schedule (optional): the pairs claim tiles in increasing order
+// from one launch-wide counter, so a pair held up by a dependency never holds
+// back work that another pair could do.  Each pair's claims are published in
+// its ring of kRing entries (tag = sequence number + 1 in the high word, the
+// tile in the low word); the counter and the rings start at 0.
+constexpr int kRing = 16;
+constexpr int kMaxSchedPairs = 128;
+constexpr int kSchedBytes = 256 + kMaxSchedPairs * kRing * 8;
+
 struct GemmParams {
   GemmClass cls[kMaxClasses];
   int num_classes;
@@ -176,6 +185,8 @@ struct GemmParams {
   uint32_t idesc;  // instruction descriptor without the B-major bit
   int* err;        // device error word (bit 0: a bounded wait ran out)
   unsigned long long timeout_ns;
+  int* claim;                // dynamic schedule: next unclaimed tile (null: static round robin)
+  unsigned long long* ring;  // dynamic schedule: [pair][kRing] published claims
 };
 
 static_assert(sizeof(GemmParams) <= 32764, "kernel parameter space");
@@ -439,6 +450,53 @@ __device__ __forceinline__ void epilogue_block(const ClassInfo& k, int b, int ro
   }
 }
 
+// ---------------------------------------------------------------- tile sequence
+//
+// The seq-th tile of a pair.  Static: pair + seq * num_pairs.  Dynamic: the
+// claimer (the leader CTA's producer) takes the next tile from the counter
+// when it is ready to load it, and publishes it; every other role of the
+// pair (the peer's producer, the MMA issuer, both epilogues) reads the
+// publication.  A tile index >= total_tiles ends every role's loop.  Tiles
+// are claimed in increasing order and every dependency points to a lower
+// index, so the lowest unfinished tile always belongs to a pair that is
+// working on it.  The claimer runs at most a few tiles ahead of the pair's
+// last reader (the epilogue, held back by two TMEM buffers and the operand
+// stages), well inside the ring.  (Claiming one tile ahead was measured: it
+// hides the publication latency but holds ready tiles on busy pairs, which
+// costs more wherever dependencies gate the schedule.)
+__device__ __forceinline__ bool next_tile(const GemmParams& p, int pair, int num_pairs, bool claimer, int seq,
+                                          volatile int* abort_word, uint64_t limit_ns, int* t_out) {
+  if (p.claim == nullptr) {
+    *t_out = pair + seq * num_pairs;
+    return true;
+  }
+  unsigned long long* slot = p.ring + pair * kRing + (seq % kRing);
+  const unsigned long long tag = static_cast<unsigned long long>(seq + 1);
+  if (claimer) {
+    const int t = atomicAdd(p.claim, 1);
+    st_release_gpu_u64(slot, (tag << 32) | static_cast<unsigned int>(t));
+    *t_out = t;
+    return true;
+  }
+  unsigned long long v = ld_acquire_gpu_u64(slot);
+  if ((v >> 32) != tag) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      __nanosleep(32);
+      v = ld_acquire_gpu_u64(slot);
+      if ((v >> 32) == tag) break;
+      if (abort_word != nullptr && *abort_word) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        if (abort_word != nullptr) *abort_word = 1;
+        if (p.err != nullptr) atomicOr(p.err, 1);
+        return false;
+      }
+    }
+  }
+  *t_out = static_cast<int>(v & 0xFFFFFFFFu);
+  return true;
+}
+
 // ---------------------------------------------------------------- kernel
 
 // Launched with clusters of 2 CTAs along x; gridDim.x is even.  TF32 selects
@@ -507,7 +565,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t used = 0, last_phase = 0;  // per-stage bits (leader only)
       bool ok = true;
       const uint32_t sA0 = smem_u32(sA), sB0 = smem_u32(sB);
-      for (int t = pair; t < p.total_tiles && ok; t += num_pairs) {
+      for (int seq = 0; ok; ++seq) {
+        int t;
+        if (!next_tile(p, pair, num_pairs, leader, seq, s_abort, limit, &t)) {
+          ok = false;
+          break;
+        }
+        if (t >= p.total_tiles) break;
         const TileCoord tc = decode_tile(p, t);
         const ClassInfo& k = p.cls[tc.c].info;
         // per-tile state in registers
@@ -594,7 +658,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // in the 16-byte-unit start-address field.
       const uint64_t dA_k = smem_desc_sw128(sA0, 16, 1024), dA_mn = smem_desc_sw128(sA0, OK::chunk_bytes, OK::mn_sbo, OK::mn_layout);
       const uint64_t dB_k = smem_desc_sw128(sB0, 16, 1024), dB_mn = smem_desc_sw128(sB0, OK::chunk_bytes, OK::mn_sbo, OK::mn_layout);
-      for (int t = pair; t < p.total_tiles && ok; t += num_pairs) {
+      for (int seq = 0; ok; ++seq) {
+        int t;
+        if (!next_tile(p, pair, num_pairs, false, seq, s_abort, limit, &t)) break;
+        if (t >= p.total_tiles) break;
         const TileCoord tc = decode_tile(p, t);
         const ClassInfo& k = p.cls[tc.c].info;
         const int nk = (k.K + OK::bke - 1) / OK::bke;
@@ -649,7 +716,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
     int buf = 0;
     uint32_t bphase = 0;
-    for (int t = pair; t < p.total_tiles; t += num_pairs) {
+    for (int seq = 0;; ++seq) {
+      int t = 0, got = 1;
+      if (lane == 0) got = next_tile(p, pair, num_pairs, false, seq, s_abort, limit, &t) ? 1 : 0;
+      got = __shfl_sync(0xFFFFFFFFu, got, 0);
+      t = __shfl_sync(0xFFFFFFFFu, t, 0);
+      if (!got || t >= p.total_tiles) break;
       const TileCoord tc = decode_tile(p, t);
       const ClassInfo& k = p.cls[tc.c].info;
       const int row0 = tc.tm * kBM + static_cast<int>(rank) * kHalfM + q * 32;

@@ -301,7 +301,10 @@ int64_t class_tiles(const ClassSpec& s) {
 // `ordered`: the classes form a chain (later classes read earlier outputs
 // through dep/sig counters) and keep their order; otherwise the longest
 // reductions go first.
-msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_t stream, bool ordered = false) {
+// `sched`: kSchedBytes of zeroed device memory for a dynamic tile schedule
+// (null: static round robin).
+msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_t stream, bool ordered = false,
+                            void* sched = nullptr) {
   DeviceState* dev = nullptr;
   msign_status st = device_state(&dev);
   if (st != MSIGN_OK) return st;
@@ -393,6 +396,10 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
             (static_cast<uint32_t>(kBM >> 4) << 24);
   p.err = dev->err;
   p.timeout_ns = kWaitLimitNs;
+  if (sched != nullptr && dev->max_pairs <= kMaxSchedPairs) {
+    p.claim = static_cast<int*>(sched);
+    p.ring = reinterpret_cast<unsigned long long*>(static_cast<char*>(sched) + 256);
+  }
   // one CTA pair per co-resident cluster slot, never more pairs than tiles
   const int grid = 2 * static_cast<int>(std::min<int64_t>(total, dev->max_pairs));
   double flops = 0.0, bytes = 0.0;
@@ -486,7 +493,8 @@ struct NsBuffers {
   float* master;  // fp32 X, blocked layout (blk_ld(m) wide, blk_size(n, m) per matrix)
   void* A;        // bf16 n x ldn
   void* B;        // bf16 n x ldn
-  int* cnt;       // row-block counters of a chained launch: [kChainSteps][3 phases][batch][tiles]
+  int* cnt;       // chained launch: kSchedBytes of dynamic-schedule state, then the
+                  // row-block counters [kChainSteps][3 phases][batch][tiles]
 };
 
 // fp32: the operand copies P, A and B hold two fp32 planes (tf32 hi, lo)
@@ -501,7 +509,7 @@ void carve_ns(Carver& cv, int64_t batch, int64_t n, int64_t m, NsBuffers* b, boo
   b->master = static_cast<float*>(cv.take(4ull * batch * blk_size(n, m)));
   b->A = cv.take(op * batch * n * ldn);
   b->B = cv.take(op * batch * n * ldn);
-  b->cnt = static_cast<int*>(cv.take(sizeof(int) * 3 * kChainSteps * batch * ceil_div(n, kBM)));
+  b->cnt = static_cast<int*>(cv.take(kSchedBytes + sizeof(int) * 3 * kChainSteps * batch * ceil_div(n, kBM)));
 }
 
 // Launches a list of classes of one operand dtype, kMaxClasses at a time.
@@ -631,7 +639,7 @@ msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cu
     const int t1 = std::min(T, t0 + per);
     std::vector<ClassSpec> chain;
     for (const NsClass& k : cls) {
-      const size_t bytes = sizeof(int) * 3 * (t1 - t0) * k.batch * ceil_div(k.n, kBM);
+      const size_t bytes = kSchedBytes + sizeof(int) * 3 * (t1 - t0) * k.batch * ceil_div(k.n, kBM);
       if (cudaMemsetAsync(k.w.cnt, 0, bytes, stream) != cudaSuccess) return MSIGN_ERR_CUDA;
     }
     for (int t = t0; t < t1; ++t, cur ^= 1) {
@@ -640,7 +648,8 @@ msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cu
         ClassSpec sp[3];
         ns_specs(k, cur, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == T - 1, &sp[0], &sp[1], &sp[2]);
         const int64_t rb = ceil_div(k.n, kBM);  // 256-row blocks of X, A and B
-        auto ctr = [&](int step, int phase) { return k.w.cnt + (3 * (step - t0) + phase) * k.batch * rb; };
+        int* const base = k.w.cnt + kSchedBytes / sizeof(int);
+        auto ctr = [&](int step, int phase) { return base + (3 * (step - t0) + phase) * k.batch * rb; };
         const int per_block_sym = static_cast<int>(8 * rb);                 // tiles touching a block of A or B
         const int per_block_x = static_cast<int>(8 * ceil_div(k.m, kBN));  // tiles in a row block of X'
         sp[0].sig = ctr(t, 0);
@@ -653,7 +662,8 @@ msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cu
       }
       for (int p = 0; p < 3; ++p) chain.insert(chain.end(), ph[p].begin(), ph[p].end());
     }
-    msign_status st = launch_grouped(chain, ns_op_dt(cls.front()), stream, /*ordered=*/true);
+    // dynamic schedule state: the first class's area (zeroed with its counters)
+    msign_status st = launch_grouped(chain, ns_op_dt(cls.front()), stream, /*ordered=*/true, cls.front().w.cnt);
     if (st != MSIGN_OK) return st;
   }
   return MSIGN_OK;
