@@ -9,13 +9,10 @@
 //                          normalisation factor of [P2] section 参考实现
 //                          (1/sqrt(sum + eps)) or of [P3] Algorithm 2 step 1
 //                          (1/(sqrt(sum) + eps)).
-//   ingest_kernel          cast + orient + scale: X0 = cast(cast(M) * s),
-//                          transposed through a 32x32 shared-memory tile
-//                          when rows > cols, plus the fp32 copy of X0;
-//   ingest_rows_kernel     the same without transposition, 16-byte accesses.
-//                          With op_dt DT_TF32_HI both write the two tf32
-//                          planes (hi, lo) of the fp32-accurate operand.
-//   momentum_kernel        M <- mu M + G in fp32 (Muon, [P3] section 1.1).
+//   ingest_kernel          cast + orient (+ scale) into the operand copy and
+//                          the blocked fp32 master; optionally the fused
+//                          norm (s from the unscaled copy) and the Muon
+//                          momentum update (see "ingest" below).
 //   apply_update_kernel    W <- W - lr * scale * O^(T) with the oriented O.
 #pragma once
 
@@ -128,164 +125,273 @@ __global__ void __launch_bounds__(1024) norm_finalize_kernel(const float* partia
   }
 }
 
-// Output space: n x m per matrix (n = rows, m = cols, or swapped when
-// `transpose`).  Block (32, 8) handles a 32 x 32 output tile.
-//   xop[i][j]    = round_op(cast(in) * s)      (operand copy, op_dt)
-//   master(i, j) = cast(in) * s                 (fp32 copy, blocked layout
-//                                                with padded width ld_m; nullable)
-// in[b] is rows x cols row-major with leading dimension `cols`.
-__global__ void __launch_bounds__(256) ingest_kernel(const void* in, int in_dt, int rows, int cols, int transpose,
-                                                     const float* scale, int cast_dt, void* xop, int op_dt,
-                                                     long long ld_op, long long op_bs, long long op_plane,
-                                                     float* master, long long ld_m, long long m_bs) {
-  __shared__ float tile[32][33];
-  const int b = blockIdx.z;
-  const int n = transpose ? cols : rows;
-  const int m = transpose ? rows : cols;
-  const int i0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
-  const int tx = threadIdx.x, ty = threadIdx.y;
-  const char* src = reinterpret_cast<const char*>(in) +
-                    static_cast<long long>(b) * rows * static_cast<long long>(cols) * dtype_size(in_dt);
-  const float s = scale ? scale[b] : 1.0f;
-  float v[4];
-  if (!transpose) {
+// ---------------------------------------------------------------- ingest
+//
+// One kernel moves a batch of input matrices into the iteration's buffers:
+// cast, orient (the n x m output is in^T when `transpose`), optionally scale,
+// and store the operand copy (row-major, op_dt; DT_TF32_HI writes both tf32
+// planes) and the fp32 master (blocked layout of blk_off).  Work unit: a 32 x
+// 64 output tile staged in shared memory.  The input is read as whole row
+// segments (128 bytes per warp for 16-bit types), the operand copy is written
+// as row segments, and each 32 x 32 block of the master -- one contiguous 4 KB
+// span in the blocked layout -- as 256 consecutive float4 stores.  Grid
+// (parts, batch), grid-stride over the tiles of a matrix, block (32, 8).
+//
+// Modes (fields of IngestArgs):
+//   pre_scale   x = cast(in) * s[b] before the stores (fp16 operands, whose
+//               range needs the normalisation first, and Gram NS).
+//   partials    the fused norm: x = cast(in) is stored unscaled and the block
+//               sums of x^2 go to partials; the matrix's last block (ticket
+//               counter, zeroed before the launch and reset by that block)
+//               sums them in a fixed order into s = 1/sqrt(sum + eps) and s^2
+//               ([P2] 参考实现's normalisation, applied by the first NS step
+//               in its epilogues, so the operand is rounded once), so s does
+//               not depend on block timing.
+//   G           Muon momentum ([P3] section 1.1): `in` is the fp32 buffer M,
+//               updated in place to mu M + G before the cast.
+
+struct IngestArgs {
+  void* in;
+  int in_dt, rows, cols, transpose, cast_dt;
+  const float* pre_scale;
+  void* xop;
+  int op_dt;
+  long long ld_op, op_bs, op_plane;
+  float* master;
+  long long ld_m, m_bs;
+  float* partials;
+  int* ticket;
+  float* s_out;
+  float* s2_out;
+  float eps;
+  const void* G;
+  int g_dt;
+  float mu;
+};
+
+constexpr int kIngestParts = 1024;  // blocks, and partial sums, per matrix
+static_assert(kIngestParts <= kNormParts, "partials share the norm's buffer");
+
+__device__ __forceinline__ float block_sum_lin(float v, float* red, int tid, int nthreads) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int i = i0 + ty + 8 * k, j = j0 + tx;
-      v[k] = (i < n && j < m)
-                 ? round_to(load_elem(src + (static_cast<long long>(i) * cols + j) * dtype_size(in_dt), in_dt),
-                            cast_dt)
-                 : 0.0f;
-    }
-  } else {
-    // out(i, j) = in(j, i): read rows j0.. of `in` along its columns i0..
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  if ((tid & 31) == 0) red[tid >> 5] = v;
+  __syncthreads();
+  v = (tid < (nthreads >> 5)) ? red[tid] : 0.0f;
+  if (tid < 32) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int jr = j0 + ty + 8 * k, ic = i0 + tx;
-      tile[ty + 8 * k][tx] =
-          (jr < m && ic < n)
-              ? round_to(load_elem(src + (static_cast<long long>(jr) * cols + ic) * dtype_size(in_dt), in_dt),
-                         cast_dt)
-              : 0.0f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < 4; ++k) v[k] = tile[tx][ty + 8 * k];
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
   }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int i = i0 + ty + 8 * k, j = j0 + tx;
-    if (i < n && j < m) {
-      const float xs = v[k] * s;
-      char* dst = reinterpret_cast<char*>(xop) +
-                  (static_cast<long long>(b) * op_bs + static_cast<long long>(i) * ld_op + j) * dtype_size(op_dt);
-      store_elem(dst, op_dt, xs);
-      if (op_dt == DT_TF32_HI) store_elem(dst + op_plane * 4, DT_TF32_LO, xs);
-      if (master) master[static_cast<long long>(b) * m_bs + blk_off(i, j, ld_m)] = xs;
-    }
-  }
+  __syncthreads();  // red is reused
+  return v;
 }
 
-// Row-wise ingest without transposition, 8 elements per thread with 16-byte
-// accesses: rows x cols input (leading dimension cols) to the operand copy and
-// the fp32 copy (leading dimensions ld_op, ld_m).  Requires cols % 8 == 0 and
-// 16-byte aligned bases and rows on every side.
-template <int IN_DT, int OP_DT>
-__global__ void __launch_bounds__(256) ingest_rows_kernel(const void* in, long long rows, int cols,
-                                                          const float* scale, int cast_dt, void* xop, long long ld_op,
-                                                          long long op_bs, long long op_plane, float* master,
-                                                          long long ld_m, long long m_bs) {
-  const int b = blockIdx.y;
-  const int vpr = cols / 8;  // vectors per row
-  const long long nvec = rows * vpr;
-  const float s = scale ? scale[b] : 1.0f;
-  const char* src = reinterpret_cast<const char*>(in) + static_cast<long long>(b) * rows * cols * dtype_size(IN_DT);
-  for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < nvec;
-       v += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long i = v / vpr;
-    const int j = static_cast<int>(v - i * vpr) * 8;
-    float x[8];
-    if (IN_DT == DT_FP32) {
-      const float4* q = reinterpret_cast<const float4*>(src + (i * cols + j) * 4);
-      const float4 a = q[0], c = q[1];
-      x[0] = a.x, x[1] = a.y, x[2] = a.z, x[3] = a.w, x[4] = c.x, x[5] = c.y, x[6] = c.z, x[7] = c.w;
+// Input element (r, c) -> x (momentum, cast, scale); 0 outside the input.
+__device__ __forceinline__ float ingest_value(float x, const IngestArgs& a, float s) {
+  x = round_to(x, a.cast_dt);
+  return a.pre_scale ? x * s : x;
+}
+
+// Up to 8 consecutive elements p[0..cnt) of type dt (16-byte accesses when
+// all 8 are wanted and p is aligned); the rest read as 0.
+__device__ __forceinline__ void load8(const char* p, int dt, int cnt, float* x) {
+  const int es = dtype_size(dt);
+  if (cnt == 8 && (reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+    if (es == 4) {
+      const float4 u = reinterpret_cast<const float4*>(p)[0], v = reinterpret_cast<const float4*>(p)[1];
+      x[0] = u.x, x[1] = u.y, x[2] = u.z, x[3] = u.w, x[4] = v.x, x[5] = v.y, x[6] = v.z, x[7] = v.w;
     } else {
-      const uint4 u = *reinterpret_cast<const uint4*>(src + (i * cols + j) * 2);
+      const uint4 u = *reinterpret_cast<const uint4*>(p);
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        float2 f;
-        if (IN_DT == DT_BF16)
-          f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
-        else
-          f = __half22float2(*reinterpret_cast<const __half2*>(&w[t]));
-        x[2 * t] = f.x, x[2 * t + 1] = f.y;
+        const uint32_t lo = w[t] & 0xFFFFu, hi = w[t] >> 16;
+        if (dt == DT_BF16) {
+          x[2 * t] = __uint_as_float(lo << 16), x[2 * t + 1] = __uint_as_float(hi << 16);
+        } else {
+          x[2 * t] = __half2float(__ushort_as_half(static_cast<unsigned short>(lo)));
+          x[2 * t + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(hi)));
+        }
       }
     }
+    return;
+  }
 #pragma unroll
-    for (int t = 0; t < 8; ++t) x[t] = round_to(x[t], cast_dt) * s;
-    if (OP_DT == DT_TF32_HI) {
-      // fp32-accurate operand: tf32 hi plane and tf32 lo plane
-      float* hp = reinterpret_cast<float*>(xop) + static_cast<long long>(b) * op_bs + i * ld_op + j;
-      float h[8], l[8];
+  for (int e = 0; e < 8; ++e) x[e] = e < cnt ? load_elem(p + e * es, dt) : 0.0f;
+}
+
+// The values this thread owns in output tile `tt` of the non-transposed
+// path: row i0 + tid/8, columns j0 + 8 (tid%8) .. +7 (0 outside the matrix).
+__device__ __forceinline__ void ingest_row_chunk(const IngestArgs& a, char* src, const char* gsrc, float s, int n,
+                                                 int m, int tc, long long tt, int tid, float* x) {
+  const int i = static_cast<int>(tt / tc) * 32 + (tid >> 3);
+  const int j = static_cast<int>(tt % tc) * 64 + 8 * (tid & 7);
+  const int cnt = (i < n && j < m) ? (m - j < 8 ? m - j : 8) : 0;
+  const long long e = static_cast<long long>(i) * a.cols + j;
+  load8(src + e * dtype_size(a.in_dt), a.in_dt, cnt, x);
+  if (gsrc != nullptr && cnt > 0) {
+    float g[8];
+    load8(gsrc + e * dtype_size(a.g_dt), a.g_dt, cnt, g);
+    float* mp = reinterpret_cast<float*>(src) + e;
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        h[t] = to_tf32(x[t]);
-        l[t] = to_tf32(x[t] - h[t]);
-      }
-      reinterpret_cast<float4*>(hp)[0] = make_float4(h[0], h[1], h[2], h[3]);
-      reinterpret_cast<float4*>(hp)[1] = make_float4(h[4], h[5], h[6], h[7]);
-      reinterpret_cast<float4*>(hp + op_plane)[0] = make_float4(l[0], l[1], l[2], l[3]);
-      reinterpret_cast<float4*>(hp + op_plane)[1] = make_float4(l[4], l[5], l[6], l[7]);
-      if (master) {
-        float* d = master + static_cast<long long>(b) * m_bs + blk_off(i, j, ld_m);
-        *reinterpret_cast<float4*>(d) = make_float4(x[0], x[1], x[2], x[3]);
-        *reinterpret_cast<float4*>(d + 128) = make_float4(x[4], x[5], x[6], x[7]);
-      }
-      continue;
+    for (int t = 0; t < 8; ++t) x[t] = fmaf(a.mu, x[t], g[t]);
+    if (cnt == 8 && (reinterpret_cast<uintptr_t>(mp) & 15) == 0) {
+      reinterpret_cast<float4*>(mp)[0] = make_float4(x[0], x[1], x[2], x[3]);
+      reinterpret_cast<float4*>(mp)[1] = make_float4(x[4], x[5], x[6], x[7]);
+    } else {
+      for (int t = 0; t < cnt; ++t) mp[t] = x[t];
     }
-    uint32_t o[4];
+  }
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      if (OP_DT == DT_BF16) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * t], x[2 * t + 1]);
-        o[t] = *reinterpret_cast<uint32_t*>(&h);
-      } else {
-        __half2 h = __floats2half2_rn(x[2 * t], x[2 * t + 1]);
-        o[t] = *reinterpret_cast<uint32_t*>(&h);
+  for (int t = 0; t < 8; ++t) x[t] = t < cnt ? ingest_value(x[t], a, s) : 0.0f;
+}
+
+// Operand-copy store of 8 consecutive values at (i, j); cnt of them valid.
+__device__ __forceinline__ void ingest_store_op(const IngestArgs& a, int b, int i, int j, int cnt, const float* v) {
+  const int es = dtype_size(a.op_dt);
+  char* dst = reinterpret_cast<char*>(a.xop) +
+              (static_cast<long long>(b) * a.op_bs + static_cast<long long>(i) * a.ld_op + j) * es;
+  if (cnt == 8 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+    if (es == 2) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (a.op_dt == DT_BF16) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+          w[e] = *reinterpret_cast<uint32_t*>(&h);
+        } else {
+          __half2 h = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
+          w[e] = *reinterpret_cast<uint32_t*>(&h);
+        }
+      }
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+      float h[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) h[e] = a.op_dt == DT_TF32_HI ? to_tf32(v[e]) : v[e];
+      reinterpret_cast<float4*>(dst)[0] = make_float4(h[0], h[1], h[2], h[3]);
+      reinterpret_cast<float4*>(dst)[1] = make_float4(h[4], h[5], h[6], h[7]);
+      if (a.op_dt == DT_TF32_HI) {
+        float4* lp = reinterpret_cast<float4*>(dst + a.op_plane * 4);
+        lp[0] = make_float4(to_tf32(v[0] - h[0]), to_tf32(v[1] - h[1]), to_tf32(v[2] - h[2]), to_tf32(v[3] - h[3]));
+        lp[1] = make_float4(to_tf32(v[4] - h[4]), to_tf32(v[5] - h[5]), to_tf32(v[6] - h[6]), to_tf32(v[7] - h[7]));
       }
     }
-    *reinterpret_cast<uint4*>(reinterpret_cast<char*>(xop) + (static_cast<long long>(b) * op_bs + i * ld_op + j) * 2) =
-        make_uint4(o[0], o[1], o[2], o[3]);
-    if (master) {
-      float* d = master + static_cast<long long>(b) * m_bs + blk_off(i, j, ld_m);
-      *reinterpret_cast<float4*>(d) = make_float4(x[0], x[1], x[2], x[3]);
-      *reinterpret_cast<float4*>(d + 128) = make_float4(x[4], x[5], x[6], x[7]);
-    }
+    return;
+  }
+  for (int e = 0; e < cnt; ++e) {
+    store_elem(dst + e * es, a.op_dt, v[e]);
+    if (a.op_dt == DT_TF32_HI) store_elem(dst + a.op_plane * 4 + e * es, DT_TF32_LO, v[e]);
   }
 }
 
-// M <- mu * M + G over `count` elements (fp32 M, G in g_dt).
-__global__ void __launch_bounds__(256) momentum_kernel(float* M, const void* G, int g_dt, long long count, float mu) {
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  const bool vec = ((reinterpret_cast<uintptr_t>(M) | reinterpret_cast<uintptr_t>(G)) & 15) == 0 && g_dt == DT_FP32;
-  if (vec) {
-    const long long nv = count / 4;
-    for (long long i = blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += stride) {
-      float4 m = reinterpret_cast<float4*>(M)[i];
-      const float4 g = reinterpret_cast<const float4*>(G)[i];
-      m.x = fmaf(mu, m.x, g.x);
-      m.y = fmaf(mu, m.y, g.y);
-      m.z = fmaf(mu, m.z, g.z);
-      m.w = fmaf(mu, m.w, g.w);
-      reinterpret_cast<float4*>(M)[i] = m;
+// The master's part of tile (i0, j0) from the staged tile: its (up to) two
+// 32 x 32 blocks, each 4 KB contiguous; thread t stores column quad t/32 of
+// block row t%32 (zeros outside the matrix).
+__device__ __forceinline__ void ingest_store_master(const IngestArgs& a, int b, int i0, int j0, int mpad,
+                                                    const float (*tile)[65], int tid) {
+  const int q = tid >> 5, r = tid & 31;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int jb = j0 + 32 * h;
+    if (jb >= mpad) break;
+    float* d = a.master + static_cast<long long>(b) * a.m_bs + blk_off(i0, jb, a.ld_m) + 4 * tid;
+    *reinterpret_cast<float4*>(d) = make_float4(tile[r][32 * h + 4 * q], tile[r][32 * h + 4 * q + 1],
+                                                tile[r][32 * h + 4 * q + 2], tile[r][32 * h + 4 * q + 3]);
+  }
+}
+
+__global__ void __launch_bounds__(256) ingest_kernel(const IngestArgs a) {
+  __shared__ float tile[32][65];
+  __shared__ float red[32];
+  __shared__ int last;
+  const int b = blockIdx.y;
+  const int tx = threadIdx.x, ty = threadIdx.y, tid = ty * 32 + tx;
+  const int n = a.transpose ? a.cols : a.rows;
+  const int m = a.transpose ? a.rows : a.cols;
+  const long long per = static_cast<long long>(a.rows) * a.cols;
+  char* src = reinterpret_cast<char*>(a.in) + static_cast<long long>(b) * per * dtype_size(a.in_dt);
+  const char* gsrc = a.G ? reinterpret_cast<const char*>(a.G) + static_cast<long long>(b) * per * dtype_size(a.g_dt)
+                         : nullptr;
+  const float s = a.pre_scale ? a.pre_scale[b] : 1.0f;
+  const int tr = (n + 31) / 32, tc = (m + 63) / 64;
+  const long long ntiles = static_cast<long long>(tr) * tc;
+  const int mpad = (m + 31) / 32 * 32;
+  float acc = 0.0f;
+  if (!a.transpose) {
+    // row chunks in registers, the next tile's loads issued before this
+    // tile's stores
+    float nxt[8];
+    if (blockIdx.x < ntiles) ingest_row_chunk(a, src, gsrc, s, n, m, tc, blockIdx.x, tid, nxt);
+    for (long long tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = nxt[e];
+      if (tt + gridDim.x < ntiles) ingest_row_chunk(a, src, gsrc, s, n, m, tc, tt + gridDim.x, tid, nxt);
+      const int i0 = static_cast<int>(tt / tc) * 32, j0 = static_cast<int>(tt % tc) * 64;
+      const int r = tid >> 3, c0 = 8 * (tid & 7);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc = fmaf(v[e], v[e], acc);
+      if (i0 + r < n && j0 + c0 < m) ingest_store_op(a, b, i0 + r, j0 + c0, m - j0 - c0 < 8 ? m - j0 - c0 : 8, v);
+      if (a.master != nullptr) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) tile[r][c0 + e] = v[e];
+        __syncthreads();
+        if (i0 < n) ingest_store_master(a, b, i0, j0, mpad, tile, tid);
+        __syncthreads();
+      }
     }
-    for (long long i = nv * 4 + blockIdx.x * blockDim.x + threadIdx.x; i < count; i += stride)
-      M[i] = fmaf(mu, M[i], reinterpret_cast<const float*>(G)[i]);
   } else {
-    const int es = dtype_size(g_dt);
-    for (long long i = blockIdx.x * blockDim.x + threadIdx.x; i < count; i += stride)
-      M[i] = fmaf(mu, M[i], load_elem(reinterpret_cast<const char*>(G) + i * es, g_dt));
+    for (long long tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
+      const int i0 = static_cast<int>(tt / tc) * 32, j0 = static_cast<int>(tt % tc) * 64;
+      // output (i, j) = in (j, i): input rows j0 + ty + 8k, columns i0 + tx
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int jr = j0 + ty + 8 * k, ic = i0 + tx;
+        float x = 0.0f;
+        if (jr < m && ic < n) {
+          const long long e = static_cast<long long>(jr) * a.cols + ic;
+          x = load_elem(src + e * dtype_size(a.in_dt), a.in_dt);
+          if (gsrc != nullptr) {
+            x = fmaf(a.mu, x, load_elem(gsrc + e * dtype_size(a.g_dt), a.g_dt));
+            reinterpret_cast<float*>(src)[e] = x;
+          }
+          x = ingest_value(x, a, s);
+        }
+        acc = fmaf(x, x, acc);
+        tile[tx][ty + 8 * k] = x;
+      }
+      __syncthreads();
+      const int r = tid >> 3, c0 = 8 * (tid & 7);
+      if (i0 + r < n && j0 + c0 < m) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = tile[r][c0 + e];
+        ingest_store_op(a, b, i0 + r, j0 + c0, m - j0 - c0 < 8 ? m - j0 - c0 : 8, v);
+      }
+      if (a.master != nullptr && i0 < n) ingest_store_master(a, b, i0, j0, mpad, tile, tid);
+      __syncthreads();  // the tile is rewritten by the next iteration
+    }
+  }
+  if (a.partials == nullptr) return;
+  acc = block_sum_lin(acc, red, tid, 256);
+  if (tid == 0) {
+    a.partials[static_cast<long long>(b) * gridDim.x + blockIdx.x] = acc;
+    __threadfence();
+    last = atomicAdd(a.ticket + b, 1) == static_cast<int>(gridDim.x) - 1;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  float v = 0.0f;
+  for (int i = tid; i < static_cast<int>(gridDim.x); i += 256)
+    v += __ldcg(a.partials + static_cast<long long>(b) * gridDim.x + i);
+  v = block_sum_lin(v, red, tid, 256);
+  if (tid == 0) {
+    const float sc = 1.0f / sqrtf(v + a.eps);
+    a.s_out[b] = sc;
+    a.s2_out[b] = sc * sc;
+    a.ticket[b] = 0;
   }
 }
 

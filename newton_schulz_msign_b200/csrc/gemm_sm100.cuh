@@ -127,6 +127,10 @@ struct EpiOut {
   int transposed;
   float gamma;
   int blocked;  // fp32 in the 32 x 32 blocked layout (blk_off); direct stores only
+  // optional, symmetric classes: the diagonal is written in fp32 to
+  // diag[b * diag_bs + i] and stored as 0 in the matrix itself
+  float* diag;
+  long long diag_bs;
 };
 
 // Per-class scalars: tile schedule and epilogue (read through the constant
@@ -148,6 +152,10 @@ struct ClassInfo {
   const void* C;             // optional epilogue input, C[row][col]
   long long ldc, c_bs;
   int c_blocked;             // C is fp32 in the 32 x 32 blocked layout (blk_off)
+  // optional per-row term of the C coefficient: v = alpha acc + (beta +
+  // row_beta[r]) C for output row r (row_beta[b * row_beta_bs + r])
+  const float* row_beta;
+  long long row_beta_bs;
   EpiOut out[kMaxOuts];
   // Dependencies between classes of one launch, by 256-row block of each
   // batch entry (index b * tiles_m + block; every class of a chain has the
@@ -388,18 +396,17 @@ __device__ __forceinline__ void load_c(const ClassInfo& k, int b, int row0, int 
 // block of mirror classes, and the blocks of diagonal tiles); on a diagonal
 // block the upper part and its mirror fill the block, so the stored matrix
 // is exactly symmetric there.
+// alpha and beta: the class's coefficients with their per-batch scales and
+// this lane's row term applied (formed once per tile).
 __device__ __forceinline__ void epilogue_block(const ClassInfo& k, int b, int row0, int col0, bool mirror,
-                                               float (&acc)[32], const float (&cv)[32], float* scratch, int lane) {
+                                               float (&acc)[32], const float (&cv)[32], float alpha, float beta,
+                                               float* scratch, int lane) {
   const int r = row0 + lane;
   const bool diag = mirror && (col0 == row0);
   const uint32_t colmask = lane_mask(k.N - col0);
   const uint32_t rowmask = lane_mask(k.M - row0);
 
-  float alpha = k.alpha;
-  if (k.alpha_scale != nullptr) alpha *= k.alpha_scale[b];
   if (k.C != nullptr) {
-    float beta = k.beta;
-    if (k.beta_scale != nullptr) beta *= k.beta_scale[b];
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc[i] = fmaf(alpha, acc[i], beta * cv[i]);
   } else {
@@ -414,6 +421,15 @@ __device__ __forceinline__ void epilogue_block(const ClassInfo& k, int b, int ro
     const float g = (col0 == row0) ? e.gamma : 0.0f;
 #pragma unroll
     for (int i = 0; i < 32; ++i) w[i] = (i == lane) ? acc[i] + g : acc[i];
+    if (e.diag != nullptr && col0 == row0) {
+      // this lane's diagonal element (r, r) goes to the fp32 vector
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i == lane) {
+          if (r < k.M) e.diag[static_cast<long long>(b) * e.diag_bs + r] = w[i];
+          w[i] = 0.0f;
+        }
+    }
     if (e.blocked) {
       // whole padded block, coalesced (elements outside the matrix are 0)
       float* q = reinterpret_cast<float*>(e.ptr) + static_cast<long long>(b) * e.bs + blk_off(row0, col0, e.ld) + 4 * lane;
@@ -747,6 +763,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       float cv[32];
       if (has_c && row0 < k.M && jfirst < kBN / 32 && tc.tn * kBN + jfirst * 32 < k.N)
         load_c(k, tc.b, row0, tc.tn * kBN + jfirst * 32, lane, cv);
+      // the epilogue coefficients of this lane's row, for every block of the tile
+      float alpha = k.alpha, beta = k.beta;
+      if (k.row_beta != nullptr && row0 + lane < k.M)
+        beta += k.row_beta[static_cast<long long>(tc.b) * k.row_beta_bs + row0 + lane];
+      if (k.alpha_scale != nullptr) alpha *= k.alpha_scale[tc.b];
+      if (k.beta_scale != nullptr) beta *= k.beta_scale[tc.b];
       if (lane == 0) ok = wait_bounded(&tfull[buf], bphase, s_abort, p.err, limit) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
@@ -765,7 +787,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float acc[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) acc[i] = __uint_as_float(raw[i]);
-        epilogue_block(k, tc.b, row0, col0, mirror, acc, cv, scratch, lane);
+        epilogue_block(k, tc.b, row0, col0, mirror, acc, cv, alpha, beta, scratch, lane);
         if (pre) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) cv[i] = cn[i];

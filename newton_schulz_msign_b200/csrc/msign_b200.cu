@@ -277,6 +277,8 @@ struct ClassSpec {
   int c_dt = DT_FP32;
   int64_t ldc = 0, c_bs = 0;
   bool c_blocked = false;  // C is fp32 in the blocked layout
+  const float* row_beta = nullptr;  // per-row term of the C coefficient (see ClassInfo)
+  int64_t row_beta_bs = 0;
   std::vector<EpiOut> outs;
   // in-launch dependencies (see ClassInfo): counters by batch entry and 256-row block
   const int* dep = nullptr;
@@ -376,6 +378,8 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     ci.ldc = s.ldc;
     ci.c_bs = s.c_bs;
     ci.c_blocked = s.c_blocked ? 1 : 0;
+    ci.row_beta = s.row_beta;
+    ci.row_beta_bs = s.row_beta_bs;
     if (s.c_blocked && (s.c_dt != DT_FP32 || s.c_plane != 0 || s.symmetric || s.ldc % 32 != 0))
       return MSIGN_ERR_INVALID_ARG;
     for (const EpiOut& e : s.outs)
@@ -440,62 +444,63 @@ msign_status launch_norm(const void* in, int in_dt, int64_t per, int64_t batch, 
   return launch_ok();
 }
 
-msign_status launch_ingest(const void* in, int in_dt, int64_t rows, int64_t cols, bool transpose, const float* scale,
-                           int cast_dt, void* xop, int op_dt, int64_t ld_op, int64_t op_bs, float* master,
-                           int64_t ld_m, int64_t m_bs, int64_t batch, cudaStream_t stream, int64_t op_plane = 0) {
-  const int64_t n = transpose ? cols : rows, m = transpose ? rows : cols;
-  const double bytes =
-      static_cast<double>(batch) * rows * cols * (dtype_size(in_dt) + dtype_size(op_dt) + (master ? 4 : 0));
-  const bool rowwise = !transpose && op_dt != DT_FP32 && op_dt != DT_TF32_LO && cols % 8 == 0 && ld_op % 8 == 0 &&
-                       (!master || ld_m % 8 == 0) && (op_dt != DT_TF32_HI || op_plane % 8 == 0) &&
-                       (reinterpret_cast<uintptr_t>(in) % 16) == 0 && (reinterpret_cast<uintptr_t>(xop) % 16) == 0 &&
-                       (!master || (reinterpret_cast<uintptr_t>(master) % 16) == 0) && op_bs % 8 == 0 &&
-                       (!master || m_bs % 8 == 0);
-  if (rowwise) {
-    const long long nvec = rows * (cols / 8);
-    dim3 g(static_cast<unsigned>(std::min<long long>((nvec + 255) / 256, 8192)), static_cast<unsigned>(batch));
-    prof_begin(stream);
-#define MSB_INGEST(IN, OP)                                                                                        \
-  ingest_rows_kernel<IN, OP><<<g, 256, 0, stream>>>(in, rows, static_cast<int>(cols), scale, cast_dt, xop, ld_op, op_bs, \
-                                                    op_plane, master, ld_m, m_bs)
-    if (op_dt == DT_TF32_HI) {
-      if (in_dt == DT_BF16) MSB_INGEST(DT_BF16, DT_TF32_HI);
-      else if (in_dt == DT_FP16) MSB_INGEST(DT_FP16, DT_TF32_HI);
-      else MSB_INGEST(DT_FP32, DT_TF32_HI);
-    } else if (op_dt == DT_BF16) {
-      if (in_dt == DT_BF16) MSB_INGEST(DT_BF16, DT_BF16);
-      else if (in_dt == DT_FP16) MSB_INGEST(DT_FP16, DT_BF16);
-      else MSB_INGEST(DT_FP32, DT_BF16);
-    } else {
-      if (in_dt == DT_BF16) MSB_INGEST(DT_BF16, DT_FP16);
-      else if (in_dt == DT_FP16) MSB_INGEST(DT_FP16, DT_FP16);
-      else MSB_INGEST(DT_FP32, DT_FP16);
-    }
-#undef MSB_INGEST
-    prof_end(2, stream, 0.0, bytes);
-    return launch_ok();
-  }
-  dim3 g(static_cast<unsigned>((m + 31) / 32), static_cast<unsigned>((n + 31) / 32), static_cast<unsigned>(batch));
+// Launches ingest_kernel over `batch` matrices (see IngestArgs).
+msign_status launch_ingest(const IngestArgs& a, int64_t batch, cudaStream_t stream) {
+  const int64_t n = a.transpose ? a.cols : a.rows, m = a.transpose ? a.rows : a.cols;
+  if (a.G != nullptr && a.in_dt != DT_FP32) return MSIGN_ERR_INVALID_ARG;
+  const double e = static_cast<double>(batch) * a.rows * a.cols;
+  double bytes = e * (dtype_size(a.in_dt) + dtype_size(a.op_dt) * (a.op_dt == DT_TF32_HI ? 2 : 1));
+  if (a.master) bytes += e * 4;
+  if (a.G) bytes += e * (dtype_size(a.g_dt) + 4);
+  const int64_t tiles = ceil_div(n, 32) * ceil_div(m, 64);
+  dim3 g(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(tiles, kIngestParts))),
+         static_cast<unsigned>(batch));
   prof_begin(stream);
-  ingest_kernel<<<g, dim3(32, 8), 0, stream>>>(in, in_dt, static_cast<int>(rows), static_cast<int>(cols),
-                                               transpose ? 1 : 0, scale, cast_dt, xop, op_dt, ld_op, op_bs, op_plane,
-                                               master, ld_m, m_bs);
+  ingest_kernel<<<g, dim3(32, 8), 0, stream>>>(a);
   prof_end(2, stream, 0.0, bytes);
   return launch_ok();
+}
+
+// Ingest arguments with everything optional left off.
+IngestArgs ingest_args(const void* in, int in_dt, int64_t rows, int64_t cols, bool transpose, int cast_dt, void* xop,
+                       int op_dt, int64_t ld_op, int64_t op_bs) {
+  IngestArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.in = const_cast<void*>(in);
+  a.in_dt = in_dt;
+  a.rows = static_cast<int>(rows);
+  a.cols = static_cast<int>(cols);
+  a.transpose = transpose ? 1 : 0;
+  a.cast_dt = cast_dt;
+  a.xop = xop;
+  a.op_dt = op_dt;
+  a.ld_op = ld_op;
+  a.op_bs = op_bs;
+  return a;
 }
 
 // ---------------------------------------------------------------- msign_ns plan
 
 struct NsBuffers {
   float* partials;
-  float* scale;
+  float* scale;   // s per matrix, then s^2 per matrix
   void* P[2];     // bf16 operand copies of X (n x ldm)
   float* master;  // fp32 X, blocked layout (blk_ld(m) wide, blk_size(n, m) per matrix)
   void* A;        // bf16 n x ldn
-  void* B;        // bf16 n x ldn
-  int* cnt;       // chained launch: kSchedBytes of dynamic-schedule state, then the
-                  // row-block counters [kChainSteps][3 phases][batch][tiles]
+  void* B;        // bf16 n x ldn (zero diagonal; the diagonal is in `diag`)
+  float* diag;    // fp32 diagonal of B, n per matrix
+  int* cnt;       // state zeroed before use: kSchedBytes of dynamic-schedule state,
+                  // the ingest tickets (ns_tickets(batch) ints), then the row-block
+                  // counters of a chained launch [kChainSteps][3 phases][batch][tiles]
 };
+
+inline int64_t ns_tickets(int64_t batch) { return round_up(batch, 64); }
+inline int* ns_ticket_ptr(const NsBuffers& w) { return w.cnt + kSchedBytes / sizeof(int); }
+inline int* ns_counter_base(const NsBuffers& w, int64_t batch) { return ns_ticket_ptr(w) + ns_tickets(batch); }
+// Bytes of the state region in use with `steps` chained steps.
+inline size_t state_bytes(int64_t batch, int64_t n, int steps) {
+  return kSchedBytes + sizeof(int) * (ns_tickets(batch) + 3 * steps * batch * ceil_div(n, kBM));
+}
 
 // fp32: the operand copies P, A and B hold two fp32 planes (tf32 hi, lo)
 // per matrix, [batch][plane][rows][ld].
@@ -503,13 +508,15 @@ void carve_ns(Carver& cv, int64_t batch, int64_t n, int64_t m, NsBuffers* b, boo
   const int64_t ldm = round_up(m, 8), ldn = round_up(n, 8);
   const uint64_t op = fp32 ? 8ull : 2ull;  // bytes per operand element (two fp32 planes, or bf16)
   b->partials = static_cast<float*>(cv.take(sizeof(float) * kNormParts * batch));
-  b->scale = static_cast<float*>(cv.take(sizeof(float) * batch));
+  b->scale = static_cast<float*>(cv.take(sizeof(float) * 2 * batch));
   b->P[0] = cv.take(op * batch * n * ldm);
   b->P[1] = cv.take(op * batch * n * ldm);
   b->master = static_cast<float*>(cv.take(4ull * batch * blk_size(n, m)));
   b->A = cv.take(op * batch * n * ldn);
   b->B = cv.take(op * batch * n * ldn);
-  b->cnt = static_cast<int*>(cv.take(kSchedBytes + sizeof(int) * 3 * kChainSteps * batch * ceil_div(n, kBM)));
+  b->diag = static_cast<float*>(cv.take(sizeof(float) * batch * n));
+  b->cnt = static_cast<int*>(
+      cv.take(kSchedBytes + sizeof(int) * (ns_tickets(batch) + 3 * kChainSteps * batch * ceil_div(n, kBM))));
 }
 
 // Launches a list of classes of one operand dtype, kMaxClasses at a time.
@@ -529,6 +536,10 @@ struct NsClass {
   std::vector<EpiOut> final_outs;  // outputs of the last step's B X product
   bool fp32 = false;               // fp32-accurate products (3xTF32 on split planes)
   int op_dt = DT_BF16;             // 16-bit operand type otherwise (bf16 or fp16)
+  // set when P[0] and master hold the unscaled x (fused ingest): the first
+  // step applies X0 = s x through its epilogues (s^2 on X X^T, s on a X + B X)
+  const float* s = nullptr;
+  const float* s2 = nullptr;
 };
 
 // Hi and lo plane outputs of a split matrix at `p` (planes of `plane` elements).
@@ -539,12 +550,22 @@ std::vector<EpiOut> split_out(void* p, int64_t ld, int64_t plane) {
 
 // The three products of one NS step ([P2] eq. 6, left form) for one class:
 //   SYRK   A = X X^T                  (symmetric, upper 256-blocks)
-//   SQR    B = b A + c A A            (symmetric; A A = A A^T as A = A^T)
-//   BX     X' = a X + B X             (X read MN-major; the a X term uses
-//                                      the fp32 copy of X)
-// The fp32-accurate class runs the same products on tf32 hi/lo planes.
-void ns_specs(const NsClass& k, int cur, float a, float b, float c, bool last, ClassSpec* syrk, ClassSpec* sqr,
-              ClassSpec* bx) {
+//   SQR    B = b A + c A A            (symmetric; A A = A A^T as A = A^T),
+//                                      stored as E = B - diag(B) plus the
+//                                      diagonal d in fp32
+//   BX     X' = E X~ + (a + d) . X    (d scales the rows of the fp32 copy X;
+//                                      X~ is its rounding, the MMA operand)
+// which is a X + B X.  Near convergence B is close to (b + c) I, about -2.7
+// I for Jordan's triple, while a X + B X is about 0.7 X: stored in bf16, the
+// diagonal's rounding would be amplified about 4x in the result.  Keeping
+// it in fp32 leaves only the small off-diagonal part to bf16, and X~ is
+// multiplied by that part only, so rounding noise never reaches the null
+// space of X (zero singular values stay zero).  Against the fp64 iteration
+// this lowers the largest error over the test matrices (Gaussian, rank-one,
+// momentum-like) from 2.2e-2 to 1.2e-2 with bf16 operands.  The
+// fp32-accurate class runs the plain products on tf32 hi/lo planes.
+void ns_specs(const NsClass& k, int cur, float a, float b, float c, bool first, bool last, ClassSpec* syrk,
+              ClassSpec* sqr, ClassSpec* bx) {
   const int64_t n = k.n, m = k.m, ldm = round_up(m, 8), ldn = round_up(n, 8);
   const int od = k.fp32 ? DT_FP32 : k.op_dt;
   const bool sp = k.fp32;
@@ -569,12 +590,14 @@ void ns_specs(const NsClass& k, int cur, float a, float b, float c, bool last, C
   q.alpha = c, q.beta = b;
   q.C = k.w.A, q.c_dt = od, q.ldc = ldn, q.c_bs = zn, q.c_plane = sp ? pn : 0;
   q.outs = outs(k.w.B, ldn, pn);
+  if (!sp) q.outs[0].diag = k.w.diag, q.outs[0].diag_bs = n;
 
   ClassSpec& x = *bx;  // B read from its upper blocks
   x = ClassSpec();
   x.A = B, x.a_sym = true, x.B = X, x.b_mn = true, x.split = sp;
   x.M = n, x.N = m, x.K = n, x.batch = k.batch;
   x.alpha = 1.0f, x.beta = a;
+  if (!sp) x.row_beta = k.w.diag, x.row_beta_bs = n;
   x.C = k.w.master, x.c_dt = DT_FP32, x.ldc = blk_ld(m), x.c_bs = blk_size(n, m), x.c_blocked = true;
   if (!last) {
     x.outs = outs(k.w.P[cur ^ 1], ldm, pm);
@@ -582,13 +605,18 @@ void ns_specs(const NsClass& k, int cur, float a, float b, float c, bool last, C
   } else {
     x.outs = k.final_outs;
   }
+  if (first && k.s != nullptr) {
+    s.alpha_scale = k.s2;
+    x.alpha_scale = k.s;
+    x.beta_scale = k.s;
+  }
 }
 
 // Operand dtype of a class's products.
 int ns_op_dt(const NsClass& k) { return k.fp32 ? DT_FP32 : k.op_dt; }
 
 // One NS step as three launches (one per phase), each over all classes.
-msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b, float c, bool last,
+msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b, float c, bool first, bool last,
                      cudaStream_t stream) {
   std::vector<ClassSpec> ph[3];
   std::vector<int> dts;
@@ -600,7 +628,7 @@ msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b,
       for (const NsClass& k : cls) {
         if (ns_op_dt(k) != dt) continue;
         ClassSpec sp[3];
-        ns_specs(k, cur, a, b, c, last, &sp[0], &sp[1], &sp[2]);
+        ns_specs(k, cur, a, b, c, first, last, &sp[0], &sp[1], &sp[2]);
         v.push_back(sp[p]);
       }
       msign_status st = launch_all(v, dt, stream);
@@ -621,7 +649,10 @@ msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b,
 // same counters: a tile that overwrites A, B or an X copy transitively waits
 // for every reader of the old contents (e.g. SYRK of step t+1 on A[i][j]
 // needs B rows i and j of step t, i.e. every SQR tile that read A rows i, j).
-msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cudaStream_t stream) {
+//   `zeroed`: the classes' state regions were zeroed for this call (and only
+// the tickets used since), so the first chained launch needs no memset.
+msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cudaStream_t stream,
+                        bool zeroed = false) {
   const int T = sch.steps();
   bool uniform = !cls.empty();
   for (const NsClass& k : cls) uniform = uniform && ns_op_dt(k) == ns_op_dt(cls.front());
@@ -629,7 +660,8 @@ msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cu
   int cur = 0;
   if (per == 0) {
     for (int t = 0; t < T; ++t) {
-      msign_status st = ns_step(cls, cur, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == T - 1, stream);
+      msign_status st =
+          ns_step(cls, cur, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == 0, t == T - 1, stream);
       if (st != MSIGN_OK) return st;
       cur ^= 1;
     }
@@ -639,16 +671,18 @@ msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cu
     const int t1 = std::min(T, t0 + per);
     std::vector<ClassSpec> chain;
     for (const NsClass& k : cls) {
-      const size_t bytes = kSchedBytes + sizeof(int) * 3 * (t1 - t0) * k.batch * ceil_div(k.n, kBM);
+      if (zeroed && t0 == 0) break;
+      const size_t bytes = state_bytes(k.batch, k.n, t1 - t0);
       if (cudaMemsetAsync(k.w.cnt, 0, bytes, stream) != cudaSuccess) return MSIGN_ERR_CUDA;
     }
     for (int t = t0; t < t1; ++t, cur ^= 1) {
       std::vector<ClassSpec> ph[3];
       for (const NsClass& k : cls) {
         ClassSpec sp[3];
-        ns_specs(k, cur, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == T - 1, &sp[0], &sp[1], &sp[2]);
+        ns_specs(k, cur, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == 0, t == T - 1, &sp[0], &sp[1],
+                 &sp[2]);
         const int64_t rb = ceil_div(k.n, kBM);  // 256-row blocks of X, A and B
-        int* const base = k.w.cnt + kSchedBytes / sizeof(int);
+        int* const base = ns_counter_base(k.w, k.batch);
         auto ctr = [&](int step, int phase) { return base + (3 * (step - t0) + phase) * k.batch * rb; };
         const int per_block_sym = static_cast<int>(8 * rb);                 // tiles touching a block of A or B
         const int per_block_x = static_cast<int>(8 * ceil_div(k.m, kBN));  // tiles in a row block of X'
@@ -828,14 +862,27 @@ msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dty
   NsBuffers w;
   carve_ns(cv, batch, n, m, &w, fp32);
 
-  st = launch_norm(in, io, rows * cols, batch, cd, sch.eps, 0, w.partials, w.scale, stream);
-  if (st != MSIGN_OK) return st;
-  if (fp32)
-    st = launch_ingest(in, io, rows, cols, tr, w.scale, DT_FP32, w.P[0], DT_TF32_HI, ldm, 2 * n * ldm, w.master,
-                       blk_ld(m), blk_size(n, m), batch, stream, n * ldm);
-  else
-    st = launch_ingest(in, io, rows, cols, tr, w.scale, cd, w.P[0], cd, ldm, n * ldm, w.master, blk_ld(m),
-                       blk_size(n, m), batch, stream);
+  // bf16 and fp32-accurate operands: one fused pass writes the unscaled x and
+  // the factor s, applied by the first step.  fp16 operands must be scaled
+  // before the cast (fp16 range), so that path normalises first.
+  const bool fused = cd != DT_FP16;
+  if (fused) {
+    if (cudaMemsetAsync(w.cnt, 0, state_bytes(batch, n, kChainSteps), stream) != cudaSuccess) return MSIGN_ERR_CUDA;
+    IngestArgs a = ingest_args(in, io, rows, cols, tr, cd, w.P[0], fp32 ? DT_TF32_HI : DT_BF16, ldm,
+                               fp32 ? 2 * n * ldm : n * ldm);
+    a.op_plane = n * ldm;
+    a.master = w.master, a.ld_m = blk_ld(m), a.m_bs = blk_size(n, m);
+    a.partials = w.partials, a.ticket = ns_ticket_ptr(w), a.s_out = w.scale, a.s2_out = w.scale + batch;
+    a.eps = sch.eps;
+    st = launch_ingest(a, batch, stream);
+  } else {
+    st = launch_norm(in, io, rows * cols, batch, cd, sch.eps, 0, w.partials, w.scale, stream);
+    if (st != MSIGN_OK) return st;
+    IngestArgs a = ingest_args(in, io, rows, cols, tr, cd, w.P[0], cd, ldm, n * ldm);
+    a.pre_scale = w.scale;
+    a.master = w.master, a.ld_m = blk_ld(m), a.m_bs = blk_size(n, m);
+    st = launch_ingest(a, batch, stream);
+  }
   if (st != MSIGN_OK) return st;
   std::vector<NsClass> cls(1);
   cls[0].w = w;
@@ -843,7 +890,8 @@ msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dty
   cls[0].fp32 = fp32;
   cls[0].op_dt = fp32 ? DT_BF16 : cd;
   cls[0].final_outs = {out_to(out, io, cols, rows * cols, tr)};
-  return ns_iterate(cls, sch, stream);
+  if (fused) cls[0].s = w.scale, cls[0].s2 = w.scale + batch;
+  return ns_iterate(cls, sch, stream, fused);
 }
 
 size_t gram_xxt_workspace_size(int64_t batch, int64_t n, int64_t m, msign_dtype x_dtype, const void* X) {
@@ -874,8 +922,7 @@ msign_status gram_xxt(const void* X, msign_dtype x_dtype, void* A, msign_dtype a
     if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
       return MSIGN_ERR_WORKSPACE;
     const int64_t ldm = round_up(m, 8);
-    msign_status st = launch_ingest(X, xd, n, m, false, nullptr, DT_FP32, workspace, xd, ldm, n * ldm, nullptr, 0, 0,
-                                    batch, stream);
+    msign_status st = launch_ingest(ingest_args(X, xd, n, m, false, DT_FP32, workspace, xd, ldm, n * ldm), batch, stream);
     if (st != MSIGN_OK) return st;
     Xm = Mat{workspace, xd, n, m, ldm, n * ldm};
   }
@@ -938,8 +985,11 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
   // [P3] Algorithm 2 steps 1-2: X <- X / (||X||_F + eps); X <- float16(X)
   st = launch_norm(in, io, rows * cols, batch, DT_FP32, sch.eps, 1, w.partials, w.scale, stream);
   if (st != MSIGN_OK) return st;
-  st = launch_ingest(in, io, rows, cols, tr, w.scale, DT_FP32, w.P[0], DT_FP16, ldm, rect, nullptr, 0, 0, batch,
-                     stream);
+  {
+    IngestArgs a = ingest_args(in, io, rows, cols, tr, DT_FP32, w.P[0], DT_FP16, ldm, rect);
+    a.pre_scale = w.scale;
+    st = launch_ingest(a, batch, stream);
+  }
   if (st != MSIGN_OK) return st;
 
   int cur = 0;
@@ -1122,31 +1172,30 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
       ns[c].n = shapes[c].first;
       ns[c].m = shapes[c].second;
       ns[c].final_outs = {out_blocked(ns[c].w.master, blk_ld(ns[c].m), blk_size(ns[c].n, ns[c].m))};
+      ns[c].s = ns[c].w.scale;
+      ns[c].s2 = ns[c].w.scale + counts[c];
+      if (cudaMemsetAsync(ns[c].w.cnt, 0, state_bytes(counts[c], ns[c].n, kChainSteps), stream) != cudaSuccess)
+        return MSIGN_ERR_CUDA;
     }
-    // M <- mu M + G; X0 = bf16(M) / ||bf16(M)||_F into the class slot
+    // one fused pass per matrix: M <- mu M + G in place, x = bf16(M) (unscaled)
+    // into the class slot, s = 1/||x||_F for the first step
     for (int i = begin; i < end; ++i) {
       const int c = cls[i - begin];
       if (c < 0) continue;
       const int64_t slot = slots[i - begin];
       const NsClass& k = ns[c];
-      const int64_t count = rows[i] * cols[i];
-      const int blocks = static_cast<int>(std::min<int64_t>((count + 1023) / 1024, 4 * dev->sms));
-      prof_begin(stream);
-      momentum_kernel<<<std::max(blocks, 1), 256, 0, stream>>>(M[i], G[i], gd, count, momentum);
-      prof_end(3, stream, 0.0, static_cast<double>(count) * (8 + dtype_size(gd)));
-      st = launch_ok();
-      if (st != MSIGN_OK) return st;
-      st = launch_norm(M[i], DT_FP32, count, 1, DT_BF16, sch.eps, 0, k.w.partials + slot * kNormParts,
-                       k.w.scale + slot, stream);
-      if (st != MSIGN_OK) return st;
       const bool tr = rows[i] > cols[i];
       const int64_t ldm = round_up(k.m, 8), per = k.n * ldm, mb = blk_size(k.n, k.m);
-      st = launch_ingest(M[i], DT_FP32, rows[i], cols[i], tr, k.w.scale + slot, DT_BF16,
-                         static_cast<char*>(k.w.P[0]) + 2 * slot * per, DT_BF16, ldm, per, k.w.master + slot * mb,
-                         blk_ld(k.m), mb, 1, stream);
+      IngestArgs a = ingest_args(M[i], DT_FP32, rows[i], cols[i], tr, DT_BF16,
+                                 static_cast<char*>(k.w.P[0]) + 2 * slot * per, DT_BF16, ldm, per);
+      a.master = k.w.master + slot * mb, a.ld_m = blk_ld(k.m), a.m_bs = mb;
+      a.partials = k.w.partials + slot * kNormParts, a.ticket = ns_ticket_ptr(k.w) + slot;
+      a.s_out = k.w.scale + slot, a.s2_out = k.w.scale + k.batch + slot, a.eps = sch.eps;
+      a.G = G[i], a.g_dt = gd, a.mu = momentum;
+      st = launch_ingest(a, 1, stream);
       if (st != MSIGN_OK) return st;
     }
-    st = ns_iterate(ns, sch, stream);
+    st = ns_iterate(ns, sch, stream, /*zeroed=*/true);
     if (st != MSIGN_OK) return st;
     // W <- W - lr * sqrt(max(1, rows/cols)) * O
     for (int i = begin; i < end; ++i) {
