@@ -37,6 +37,7 @@ struct DeviceState {
   bool ready = false;
   int sms = 0;
   int max_pairs = 0;  // CTA pairs of the GEMM kernel that fit on the GPU at once
+  int ingest_blocks = 0;  // ingest_kernel blocks resident at once on the whole GPU
   int* err = nullptr;
 };
 
@@ -79,6 +80,12 @@ msign_status device_state(DeviceState** out) {
         clusters = d.sms / 2;
       }
       d.max_pairs = clusters;
+      int per_sm = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ingest_kernel, 256, 0) != cudaSuccess || per_sm < 1) {
+        (void)cudaGetLastError();
+        per_sm = 4;
+      }
+      d.ingest_blocks = per_sm * d.sms;
     }
     if (g_encode == nullptr) {
       void* fn = nullptr;
@@ -452,8 +459,14 @@ msign_status launch_ingest(const IngestArgs& a, int64_t batch, cudaStream_t stre
   double bytes = e * (dtype_size(a.in_dt) + dtype_size(a.op_dt) * (a.op_dt == DT_TF32_HI ? 2 : 1));
   if (a.master) bytes += e * 4;
   if (a.G) bytes += e * (dtype_size(a.g_dt) + 4);
+  DeviceState* dev = nullptr;
+  msign_status st = device_state(&dev);
+  if (st != MSIGN_OK) return st;
+  // one full wave of resident blocks over the whole batch, grid-striding
+  // over the tiles: no partial last wave
   const int64_t tiles = ceil_div(n, 32) * ceil_div(m, 64);
-  dim3 g(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(tiles, kIngestParts))),
+  const int64_t wave = std::max<int64_t>(1, dev->ingest_blocks / std::max<int64_t>(batch, 1));
+  dim3 g(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>({tiles, wave, int64_t(kIngestParts)}))),
          static_cast<unsigned>(batch));
   prof_begin(stream);
   ingest_kernel<<<g, dim3(32, 8), 0, stream>>>(a);
