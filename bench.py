@@ -352,6 +352,125 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
+# ---------------------------------------------------------------- other workloads
+#
+# `--workload NAME` times one of the other configurations the tests cover,
+# with the same rules as the headline (warm-up, L2 flush before each timed
+# call, CUDA events on the launching stream, clocks sampled meanwhile).
+# Useful FLOPs come from the library's own launch records (triangle-counted
+# per product), so they match the headline's bookkeeping.  These lines are
+# measurements for the record, not the driver's metric.
+
+WORKLOADS = {
+    "msign_8x4096": ("msign", dict(batch=8, rows=4096, cols=4096)),
+    "msign_4x4096x11008": ("msign", dict(batch=4, rows=4096, cols=11008)),
+    "msign_2048": ("msign", dict(batch=1, rows=2048, cols=2048)),
+    "msign_1024x4096": ("msign", dict(batch=1, rows=1024, cols=4096)),
+    "msign_4096_fp32": ("msign", dict(batch=1, rows=4096, cols=4096, compute="fp32")),
+    "gram_xxt_4096": ("gram_xxt", dict(n=4096)),
+    "gram_xxt_8192": ("gram_xxt", dict(n=8192)),
+    "gram_ns_1024x4096": ("gram_ns", dict(rows=1024, cols=4096)),
+    "gram_ns_2048x16384": ("gram_ns", dict(rows=2048, cols=16384)),
+    "muon_llama3_8b_layer": ("muon", dict()),
+}
+
+
+def run_workload(args):
+    import torch
+
+    import newton_schulz_msign_b200 as msb
+    from newton_schulz_msign_b200 import synth
+
+    kind, cfg = WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    desc = {"workload": args.workload}
+    if kind == "msign":
+        b, r, c = cfg["batch"], cfg["rows"], cfg["cols"]
+        comp = cfg.get("compute", "bf16")
+        x = torch.stack([synth.momentum_like_torch(r, c, seed=2000 + i, device=dev) for i in range(b)])
+        x = x.to(torch.bfloat16).contiguous()
+        out = torch.empty_like(x)
+        ws = torch.empty(msb.msign_ns_workspace_size(b, r, c, comp), dtype=torch.uint8, device=dev)
+        call = lambda: msb.msign_ns(x, out, compute=comp, workspace=ws)
+        desc.update(batch=b, rows=r, cols=c, compute=comp, input="momentum-like, bf16")
+    elif kind == "gram_xxt":
+        n = cfg["n"]
+        x = synth.gaussian_torch((n, n), seed=3000, device=dev, std=1.0 / n ** 0.5, dtype=torch.bfloat16)
+        a = torch.empty(n, n, dtype=torch.bfloat16, device=dev)
+        call = lambda: msb.gram_xxt(x, a)
+        desc.update(n=n, m=n, input="N(0, 1/m) bf16", output="full n x n bf16, exactly symmetric")
+    elif kind == "gram_ns":
+        r, c = cfg["rows"], cfg["cols"]
+        x = synth.gaussian_torch((r, c), seed=4000, device=dev, dtype=torch.bfloat16)
+        out = torch.empty_like(x)
+        ws = torch.empty(msb.gram_ns_workspace_size(1, r, c), dtype=torch.uint8, device=dev)
+        call = lambda: msb.gram_ns(x, out, workspace=ws)
+        desc.update(rows=r, cols=c, input="N(0,1) bf16", inner="fp16", restart_after=[2])
+    else:
+        shapes = [(r, c) for _, r, c in synth.llama3_8b_layer_shapes()]
+        W = [synth.gaussian_torch(s_, seed=5000 + i, device=dev, std=0.02, dtype=torch.bfloat16)
+             for i, s_ in enumerate(shapes)]
+        M = [torch.zeros(s_, dtype=torch.float32, device=dev) for s_ in shapes]
+        G = [synth.gaussian_torch(s_, seed=6000 + i, device=dev, std=1e-4, dtype=torch.bfloat16)
+             for i, s_ in enumerate(shapes)]
+        ws = torch.empty(msb.muon_step_workspace_size(shapes), dtype=torch.uint8, device=dev)
+        call = lambda: msb.muon_step(W, M, G, momentum=0.95, lr=0.02, workspace=ws)
+        desc.update(matrices=[list(s_) for s_ in shapes], w="bf16", m="fp32", g="N(0, 1e-4^2) bf16",
+                    momentum=0.95, lr=0.02, note="one Llama-3-8B decoder layer; every call is a further step")
+    for _ in range(args.warmup):
+        call()
+    msb.sync_status()
+
+    def timed(instrumented):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        msb.profile_reset()
+        msb.profile_enable(instrumented)
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            ev[k][0].record(stream)
+            call()
+            ev[k][1].record(stream)
+        wait_idle(ev[-1][1])
+        msb.profile_enable(False)
+        msb.sync_status()
+        return [a_.elapsed_time(b_) for a_, b_ in ev]
+
+    clocks = ClockSampler(0)
+    clocks.start()
+    per_call = timed(False)
+    clk = clocks.stop()
+    timed(True)
+    kinds = {k: msb.profile_read(k) for k in ("gemm", "norm", "ingest", "elementwise")}
+    msb.profile_reset()
+    ms = statistics.median(per_call)
+    g = kinds["gemm"]
+    fp32 = cfg.get("compute", "bf16") == "fp32"
+    # the launch records count the fp32-accurate path's three tf32 passes
+    flops = g["flops"] / args.steps / (3.0 if fp32 else 1.0)
+    peaks = measured_peaks()
+    pk = peaks["bf16_tflops"] * (0.5 if fp32 else 1.0)  # tf32 runs at half the bf16 rate
+    achieved = g["flops"] / (g["ms"] / 1e3) / 1e12 if g["ms"] > 0 else None
+    print(json.dumps({
+        "workload": args.workload, "metric": "ms per call and useful TFLOP/s", "value": ms, "unit": "ms/call",
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": False,
+        "per_call_ms": {"min": min(per_call), "median": ms, "max": max(per_call)},
+        "useful_flops_per_call": flops, "useful_tflops": flops / (ms / 1e3) / 1e12,
+        "frac_of_peak": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+        "roofline": {"bound": "tensor", "kernel": "gemm_sm100_kernel", "achieved": achieved, "peak": pk,
+                     "unit": "TFLOP/s", "frac": achieved / pk if achieved else None,
+                     "launches_per_call": g["launches"] / args.steps,
+                     "peak_source": peaks["source"] + (" bf16 burst" if pk == peaks["bf16_tflops"] else
+                                                       " bf16 burst x 1/2 (tf32 rate)")},
+        "gpu_launches_per_call": sum(v["launches"] for v in kinds.values()) / args.steps,
+        "other_kernels": {k: {"launches": v["launches"], "ms": v["ms"]} for k, v in kinds.items() if k != "gemm"},
+        "clocks": clk, "config": desc, "l2": "flushed (256 MiB write) before every timed call", "data": "synthetic",
+    }), flush=True)
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -412,11 +531,15 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the host oracle timing")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
+                    help="time another configuration instead of the headline (1 GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload is not None:
+        run_workload(args)
     else:
         run_ours(args)
 
