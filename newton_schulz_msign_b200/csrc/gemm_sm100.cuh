@@ -133,6 +133,17 @@ struct EpiOut {
   long long diag_bs;
 };
 
+// One dependency of a class on an earlier class of the launch (its row-block
+// counters): rows tm and/or tn of the consumer tile, or all `rows` rows,
+// must have reached `target`.
+constexpr int kMaxDeps = 6;
+constexpr int kTileSignals = 8;  // arrivals per finished tile on each row it touches: a pair's 8 epilogue warps
+enum : int { DEP_TM = 1, DEP_TN = 2, DEP_ALL = 4 };
+struct RowDep {
+  const int* ptr;  // counters of batch entry 0; entry b at ptr + b * rows
+  int rows, target, mode;
+};
+
 // Per-class scalars: tile schedule and epilogue (read through the constant
 // cache of the kernel parameters).
 struct ClassInfo {
@@ -158,15 +169,15 @@ struct ClassInfo {
   long long row_beta_bs;
   EpiOut out[kMaxOuts];
   // Dependencies between classes of one launch, by 256-row block of each
-  // batch entry (index b * tiles_m + block; every class of a chain has the
-  // same row-block count).  A tile (tm, tn) starts once dep[tm] -- and
-  // dep[tn] when dep_both -- reach dep_target.  Each epilogue warp adds 1 to
-  // sig[tm] (and to sig[tn] for an off-diagonal tile of a symmetric class)
-  // after storing its rows, so a row block is complete at 8 x the number of
-  // tiles that touch it.
-  const int* dep;
+  // batch entry: each epilogue warp adds 1 to sig[b * tiles_m + tm] (and to
+  // sig[... + tn] for an off-diagonal tile of a symmetric class) after
+  // storing its rows, so a row block of a class is complete at 8 x the
+  // number of its tiles that touch it.  A tile (tm, tn) starts once every
+  // entry of deps[] is met (see RowDep); the epilogue acquires deps[c_dep]
+  // (the producer of C) before reading C.
+  RowDep deps[kMaxDeps];
+  int num_deps, c_dep;
   int* sig;
-  int dep_target, dep_both;
 };
 
 struct alignas(64) GemmClass {
@@ -603,14 +614,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const void* tmA2 = &g.tmA2;
         const void* tmB = &g.tmB;
         const void* tmB2 = &g.tmB2;
-        if (k.dep != nullptr) {
-          // operands produced earlier in this launch: wait for their row blocks
-          const int* d = k.dep + tc.b * k.tiles_m;
-          if (!wait_counter(d + tc.tm, k.dep_target, s_abort, p.err, limit) ||
-              (k.dep_both && !wait_counter(d + tc.tn, k.dep_target, s_abort, p.err, limit))) {
-            ok = false;
-            break;
+        if (k.num_deps > 0) {
+          // operands produced earlier in this launch (and earlier readers of
+          // the buffers this tile overwrites): wait for their row blocks
+          for (int e = 0; e < k.num_deps && ok; ++e) {
+            const RowDep& d = k.deps[e];
+            const int* base = d.ptr + static_cast<long long>(tc.b) * d.rows;
+            if (d.mode & DEP_ALL) {
+              for (int r = 0; r < d.rows && ok; ++r) ok = wait_counter(base + r, d.target, s_abort, p.err, limit);
+            } else {
+              if (d.mode & DEP_TM) ok = ok && wait_counter(base + tc.tm, d.target, s_abort, p.err, limit);
+              if (d.mode & DEP_TN) ok = ok && wait_counter(base + tc.tn, d.target, s_abort, p.err, limit);
+            }
           }
+          if (!ok) break;
           fence_proxy_async_global();
         }
         for (int step = 0; step < nk * passes; ++step) {
@@ -748,10 +765,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         while (jfirst < kBN / 32 && tc.tn * kBN + jfirst * 32 < row0) ++jfirst;
       const bool has_c = k.C != nullptr;
       int ok = 1;
-      if (has_c && k.dep != nullptr) {
+      if (has_c && k.c_dep >= 0) {
         // C was written earlier in this launch: acquire it for this warp
-        const int* d = k.dep + tc.b * k.tiles_m + tc.tm;
-        if (lane == 0) ok = wait_counter(d, k.dep_target, s_abort, p.err, limit) ? 1 : 0;
+        const RowDep& dd = k.deps[k.c_dep];
+        const int* d = dd.ptr + static_cast<long long>(tc.b) * dd.rows + tc.tm;
+        if (lane == 0) ok = wait_counter(d, dd.target, s_abort, p.err, limit) ? 1 : 0;
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (!ok) break;
         // each lane's own acquire orders its C loads (plain, L1-cached)
@@ -802,7 +820,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __threadfence();
         __syncwarp();
         if (lane == 0) {
-          int* sg = k.sig + tc.b * k.tiles_m;
+          int* sg = k.sig + static_cast<long long>(tc.b) * k.tiles_m;
           red_release_gpu_add(sg + tc.tm, 1);
           if (k.symmetric && tc.tn != tc.tm) red_release_gpu_add(sg + tc.tn, 1);
         }

@@ -287,11 +287,10 @@ struct ClassSpec {
   const float* row_beta = nullptr;  // per-row term of the C coefficient (see ClassInfo)
   int64_t row_beta_bs = 0;
   std::vector<EpiOut> outs;
-  // in-launch dependencies (see ClassInfo): counters by batch entry and 256-row block
-  const int* dep = nullptr;
+  // in-launch dependencies (see ClassInfo): row-block counters of earlier classes
+  std::vector<RowDep> deps;
+  int c_dep = -1;  // the entry of deps that produced C
   int* sig = nullptr;
-  int dep_target = 0;
-  bool dep_both = false;
 };
 
 // Square kBM x kBN tiles on or above the diagonal.
@@ -393,10 +392,12 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
       if (e.blocked && (e.dtype != DT_FP32 || e.transposed || s.symmetric || e.ld % 32 != 0))
         return MSIGN_ERR_INVALID_ARG;
     for (size_t o = 0; o < s.outs.size(); ++o) ci.out[o] = s.outs[o];
-    ci.dep = s.dep;
+    if (s.deps.size() > static_cast<size_t>(kMaxDeps) || s.c_dep >= static_cast<int>(s.deps.size()))
+      return MSIGN_ERR_INVALID_ARG;
+    for (size_t e = 0; e < s.deps.size(); ++e) ci.deps[e] = s.deps[e];
+    ci.num_deps = static_cast<int>(s.deps.size());
+    ci.c_dep = s.c_dep;
     ci.sig = s.sig;
-    ci.dep_target = s.dep_target;
-    ci.dep_both = s.dep_both ? 1 : 0;
     total += class_tiles(s);
   }
   if (total > INT32_MAX) return MSIGN_ERR_UNSUPPORTED;
@@ -699,12 +700,13 @@ msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cu
         auto ctr = [&](int step, int phase) { return base + (3 * (step - t0) + phase) * k.batch * rb; };
         const int per_block_sym = static_cast<int>(8 * rb);                 // tiles touching a block of A or B
         const int per_block_x = static_cast<int>(8 * ceil_div(k.m, kBN));  // tiles in a row block of X'
+        const int rows = static_cast<int>(rb);
         sp[0].sig = ctr(t, 0);
-        if (t > t0) sp[0].dep = ctr(t - 1, 2), sp[0].dep_target = per_block_x, sp[0].dep_both = true;
+        if (t > t0) sp[0].deps = {RowDep{ctr(t - 1, 2), rows, per_block_x, DEP_TM | DEP_TN}};
         sp[1].sig = ctr(t, 1);
-        sp[1].dep = ctr(t, 0), sp[1].dep_target = per_block_sym, sp[1].dep_both = true;
+        sp[1].deps = {RowDep{ctr(t, 0), rows, per_block_sym, DEP_TM | DEP_TN}}, sp[1].c_dep = 0;
         if (t + 1 < t1) sp[2].sig = ctr(t, 2);
-        sp[2].dep = ctr(t, 1), sp[2].dep_target = per_block_sym, sp[2].dep_both = false;
+        sp[2].deps = {RowDep{ctr(t, 1), rows, per_block_sym, DEP_TM}}, sp[2].c_dep = 0;
         for (int p = 0; p < 3; ++p) ph[p].push_back(sp[p]);
       }
       for (int p = 0; p < 3; ++p) chain.insert(chain.end(), ph[p].begin(), ph[p].end());
@@ -726,6 +728,8 @@ struct GramBuffers {
   void* Z;
   void* Q[2];
   void* RZ;
+  int* cnt;  // zeroed before each chained launch: kSchedBytes of schedule state, then the
+             // row-block counters of up to kMaxClasses classes [class][batch][tiles]
 };
 
 void carve_gram(Carver& cv, int64_t batch, int64_t n, int64_t m, GramBuffers* b) {
@@ -739,7 +743,107 @@ void carve_gram(Carver& cv, int64_t batch, int64_t n, int64_t m, GramBuffers* b)
   b->Q[0] = cv.take(2ull * batch * n * ldn);
   b->Q[1] = cv.take(2ull * batch * n * ldn);
   b->RZ = cv.take(2ull * batch * n * ldn);
+  b->cnt = static_cast<int*>(cv.take(kSchedBytes + sizeof(int) * kMaxClasses * batch * ceil_div(n, kBM)));
 }
+
+// Classes of one chained launch whose dependencies are derived from the
+// buffers they read and write, by 256-row block (see RowDep):
+//   read after write  -- the producer's rows the consumer tile reads: row tm
+//                        of an A operand, row tn of a K-major B operand, all
+//                        rows of an MN-major one (X in Q X), row tm for C;
+//   write after read  -- every earlier reader of the buffer being
+//                        overwritten, on the rows of the written tile (tm,
+//                        and tn for a symmetric output), or on all its rows
+//                        when that reader read the buffer MN-major;
+//   write after write -- the buffer's previous writer, on the same rows.
+// A class waits only for classes before it, so the launch cannot deadlock.
+// When a launch would exceed kMaxClasses, the chain is launched and
+// restarted: stream order covers everything across launches.
+struct Chain {
+  struct Use {
+    int cls, mode;
+  };
+  struct Buf {
+    int writer = -1;
+    std::vector<Use> readers;
+  };
+  int* state;  // kSchedBytes + counters
+  int64_t batch, rows;
+  int ab_dt;
+  cudaStream_t stream;
+  std::vector<ClassSpec> cls;
+  std::vector<int> target;  // per class: 8 x tiles touching a row block
+  std::vector<std::pair<const void*, Buf>> bufs;
+
+  Buf& buf(const void* p) {
+    for (auto& b : bufs)
+      if (b.first == p) return b.second;
+    bufs.push_back({p, Buf{}});
+    return bufs.back().second;
+  }
+  int* counters(int c) { return state + kSchedBytes / sizeof(int) + static_cast<int64_t>(c) * batch * rows; }
+
+  msign_status flush() {
+    if (cls.empty()) return MSIGN_OK;
+    const size_t bytes = kSchedBytes + sizeof(int) * cls.size() * batch * rows;
+    if (cudaMemsetAsync(state, 0, bytes, stream) != cudaSuccess) return MSIGN_ERR_CUDA;
+    msign_status st = launch_grouped(cls, ab_dt, stream, /*ordered=*/true, state);
+    cls.clear();
+    target.clear();
+    bufs.clear();
+    return st;
+  }
+
+  // reads: (buffer, DEP_TM / DEP_TN / DEP_ALL); c_buf: the buffer read as C
+  msign_status add(ClassSpec s, const std::vector<std::pair<const void*, int>>& reads, const void* c_buf,
+                   const std::vector<const void*>& writes) {
+    if (cls.size() == static_cast<size_t>(kMaxClasses)) {
+      msign_status st = flush();
+      if (st != MSIGN_OK) return st;
+    }
+    const int me = static_cast<int>(cls.size());
+    std::vector<std::pair<int, int>> need;  // (class, mode)
+    auto want = [&](int c, int mode) {
+      for (auto& n : need)
+        if (n.first == c) {
+          n.second |= mode;
+          return;
+        }
+      need.push_back({c, mode});
+    };
+    const int out_rows = s.symmetric ? (DEP_TM | DEP_TN) : DEP_TM;
+    for (const auto& r : reads) {
+      const Buf& b = buf(r.first);
+      if (b.writer >= 0) want(b.writer, r.second);
+    }
+    if (c_buf != nullptr && buf(c_buf).writer >= 0) want(buf(c_buf).writer, DEP_TM);  // C tile (tm, tn)
+    for (const void* w : writes) {
+      const Buf& b = buf(w);
+      for (const Use& u : b.readers) want(u.cls, (u.mode & DEP_ALL) ? DEP_ALL : out_rows);
+      if (b.writer >= 0) want(b.writer, out_rows);
+    }
+    s.deps.clear();
+    s.c_dep = -1;
+    for (const auto& n : need) {
+      const int mode = (n.second & DEP_ALL) ? DEP_ALL : n.second;
+      s.deps.push_back(RowDep{counters(n.first), static_cast<int>(rows), target[n.first], mode});
+      if (c_buf != nullptr && buf(c_buf).writer == n.first) s.c_dep = static_cast<int>(s.deps.size()) - 1;
+    }
+    if (s.deps.size() > static_cast<size_t>(kMaxDeps)) return MSIGN_ERR_UNSUPPORTED;
+    s.sig = counters(me);
+    const int64_t tiles_n = ceil_div(s.N, kBN);
+    target.push_back(static_cast<int>(kTileSignals * (s.symmetric ? rows : tiles_n)));
+    cls.push_back(s);
+    for (const void* w : writes) {
+      Buf& b = buf(w);
+      b.writer = me;
+      b.readers.clear();
+    }
+    for (const auto& r : reads) buf(r.first).readers.push_back({me, r.second});
+    if (c_buf != nullptr) buf(c_buf).readers.push_back({me, DEP_TM});
+    return MSIGN_OK;
+  }
+};
 
 // Restart schedule -> segment bounds [0, r1, r2, ..., T].
 msign_status gram_segments(int T, const int* restart_after, int n_restart, std::vector<int>* bounds) {
@@ -1005,6 +1109,11 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
   }
   if (st != MSIGN_OK) return st;
 
+  // every product of the iteration, chained (see Chain); a tile of a later
+  // product starts as soon as the row blocks it touches are final
+  Chain ch;
+  ch.state = w.cnt, ch.batch = batch, ch.rows = ceil_div(n, kBM), ch.ab_dt = DT_FP16, ch.stream = stream;
+  const int DEP_TMN = DEP_TM | DEP_TN;
   int cur = 0;
   for (size_t seg = 0; seg + 1 < bounds.size(); ++seg) {
     const int s0 = bounds[seg], s1 = bounds[seg + 1];
@@ -1014,7 +1123,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
       s.A = X, s.B = X, s.symmetric = true;
       s.M = n, s.N = n, s.K = m, s.batch = batch;
       s.outs = sym_out(w.R, 0.0f);
-      st = launch_grouped({s}, DT_FP16, stream);
+      st = ch.add(s, {{w.P[cur], DEP_TMN}}, nullptr, {w.R});
       if (st != MSIGN_OK) return st;
     }
     int q = -1;  // Q = I until the first step of the segment sets it
@@ -1028,15 +1137,16 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
         s.alpha = c, s.beta = b;
         s.C = w.R, s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
         s.outs = sym_out(w.Z, 0.0f);
+        std::vector<const void*> writes{w.Z};
         if (first) {
           std::vector<EpiOut> qo = sym_out(w.Q[0], a);
           s.outs.insert(s.outs.end(), qo.begin(), qo.end());
+          writes.push_back(w.Q[0]);
         }
-        st = launch_grouped({s}, DT_FP16, stream);
+        st = ch.add(s, {{w.R, DEP_TMN}}, w.R, writes);
         if (st != MSIGN_OK) return st;
         if (first) q = 0;
       }
-      std::vector<ClassSpec> pair;
       if (!first) {  // Q <- Q Z + a Q
         ClassSpec s;
         s.A = sqm(w.Q[q]), s.B = sqm(w.Z), s.symmetric = true, s.a_sym = true, s.b_sym = true;
@@ -1044,7 +1154,8 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
         s.alpha = 1.0f, s.beta = a;
         s.C = w.Q[q], s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
         s.outs = sym_out(w.Q[q ^ 1], 0.0f);
-        pair.push_back(s);
+        st = ch.add(s, {{w.Q[q], DEP_TM}, {w.Z, DEP_TN}}, w.Q[q], {w.Q[q ^ 1]});
+        if (st != MSIGN_OK) return st;
       }
       if (!last) {  // RZ <- R Z + a R
         ClassSpec s;
@@ -1053,10 +1164,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
         s.alpha = 1.0f, s.beta = a;
         s.C = w.R, s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
         s.outs = sym_out(w.RZ, 0.0f);
-        pair.push_back(s);
-      }
-      if (!pair.empty()) {
-        st = launch_grouped(pair, DT_FP16, stream);
+        st = ch.add(s, {{w.R, DEP_TM}, {w.Z, DEP_TN}}, w.R, {w.RZ});
         if (st != MSIGN_OK) return st;
       }
       if (!first) q ^= 1;
@@ -1067,7 +1175,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
         s.alpha = 1.0f, s.beta = a;
         s.C = w.RZ, s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
         s.outs = sym_out(w.R, 0.0f);
-        st = launch_grouped({s}, DT_FP16, stream);
+        st = ch.add(s, {{w.Z, DEP_TM}, {w.RZ, DEP_TN}}, w.RZ, {w.R});
         if (st != MSIGN_OK) return st;
       }
     }
@@ -1075,16 +1183,17 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
       ClassSpec s;
       s.A = sqm(w.Q[q]), s.a_sym = true, s.B = X, s.b_mn = true;
       s.M = n, s.N = m, s.K = n, s.batch = batch;
+      void* dst = (seg + 2 == bounds.size()) ? out : w.P[cur ^ 1];
       if (seg + 2 == bounds.size())
         s.outs = {out_to(out, io, cols, rows * cols, tr)};
       else
         s.outs = {out_to(w.P[cur ^ 1], DT_FP16, ldm, rect, false)};
-      st = launch_grouped({s}, DT_FP16, stream);
+      st = ch.add(s, {{w.Q[q], DEP_TM}, {w.P[cur], DEP_ALL}}, nullptr, {dst});
       if (st != MSIGN_OK) return st;
     }
     cur ^= 1;
   }
-  return MSIGN_OK;
+  return ch.flush();
 }
 
 // Workspace of one group of Muon matrices: one NsBuffers set per distinct
