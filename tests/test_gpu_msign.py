@@ -66,6 +66,14 @@ def test_coefficient_tables(coeff_tables, table):
     assert rel_fro(got, ref) < TOL_BF16
 
 
+def test_long_schedule_batched():
+    # seven steps over a batch of three: the steps span two chained launches
+    x = synth.gaussian((3, 96, 200), seed=12)
+    coeffs = [(3.4445, -4.7750, 2.0315)] * 7
+    got, ref = run_case(x, coeffs=coeffs)
+    assert rel_fro(got, ref) < TOL_BF16
+
+
 def test_momentum_like_spectrum():
     x = synth.momentum_like(512, 1024, seed=6)
     got, ref = run_case(x)

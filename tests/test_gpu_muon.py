@@ -60,6 +60,19 @@ def test_muon_small_mixed_shapes(wdt, gdt):
         check_matrix(W0[i], M0[i], G[i], W[i], M[i], 0.02)
 
 
+def test_muon_many_shape_classes():
+    # seven distinct oriented shapes: more classes than one chained launch
+    # holds, so every step runs phase by phase
+    shapes = [(64, 128), (96, 96), (200, 72), (80, 240), (48, 160), (32, 96), (120, 130)]
+    W, M, G = make(shapes, torch.float32, torch.float32, seed=500)
+    W0 = [w.clone() for w in W]
+    M0 = [m.clone() for m in M]
+    msb.muon_step(W, M, G, momentum=0.95, lr=0.02)
+    msb.sync_status()
+    for i in range(len(shapes)):
+        check_matrix(W0[i], M0[i], G[i], W[i], M[i], 0.02)
+
+
 def test_muon_equals_msign_composition():
     # the fused step equals momentum + msign_ns + scaled update done by hand
     shapes = [(256, 128), (128, 384)]

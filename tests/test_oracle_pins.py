@@ -292,3 +292,53 @@ def test_muon_step_closed_form(shape):
     np.testing.assert_allclose(M1, 0.95 * M + G, atol=0)
     scale = math.sqrt(max(1.0, shape[0] / shape[1]))
     np.testing.assert_allclose(W1, W - 0.02 * scale * O.msign_ns_closed_form(0.95 * M + G), atol=1e-12)
+
+
+# ---------------------------------------------------------------- improved initial normalisation
+
+@pytest.mark.parametrize("shape", [(40, 90), (90, 40), (64, 64)])
+def test_improved_init_closed_form(shape):
+    # [P2] section 改进初值: rescaling X0 (and its Gram powers) by
+    # n = ||(X0 X0^T)^2||_F^(1/4) at step 0 is the plain iteration on the
+    # singular values sigma_i / (||M||_F n), with n^8 = sum (sigma_i/||M||_F)^8;
+    # written here through the SVD, independently of the oracle's matrix steps
+    M = np.random.default_rng(sum(shape)).standard_normal(shape)
+    U, s, Vt = np.linalg.svd(M, full_matrices=False)
+    x = s / np.sqrt(np.sum(s ** 2) + 1e-20)
+    n = (np.sum(x ** 8) + 1e-20) ** 0.125
+    expect = (U * O.ns_scalar(x / n)) @ Vt
+    got = O.msign_ns_improved_init(M)
+    assert np.allclose(got, expect, rtol=1e-10, atol=1e-12)
+    # and it is not the plain iteration
+    assert not np.allclose(got, O.msign_ns(M), atol=1e-3)
+
+
+def test_improved_init_raises_small_singular_values():
+    # the page's measurement: on 100 x 100 Gaussian matrices the smallest
+    # output singular value mostly more than doubles, and the mean singular
+    # value moves closer to 1
+    ratios, closer = [], 0
+    for seed in range(20):
+        M = np.random.default_rng(1000 + seed).standard_normal((100, 100))
+        s0 = np.linalg.svd(O.msign_ns(M), compute_uv=False)
+        s1 = np.linalg.svd(O.msign_ns_improved_init(M), compute_uv=False)
+        ratios.append(s1.min() / s0.min())
+        closer += abs(s1.mean() - 1) < abs(s0.mean() - 1)
+    assert np.median(ratios) >= 2.0
+    assert closer >= 18
+
+
+def test_improved_init_is_a_rescale_of_the_input():
+    # the improved iteration on M equals the plain iteration started from
+    # X0 / n -- i.e. msign_ns on M scaled so that its Frobenius normalisation
+    # lands on X0 / n -- checked on the batch axis as well
+    Ms = np.random.default_rng(7).standard_normal((3, 30, 50))
+    got = O.msign_ns_improved_init(Ms)
+    for i in range(3):
+        X0 = Ms[i] / np.sqrt(np.sum(Ms[i] ** 2) + 1e-20)
+        A = X0 @ X0.T
+        n = (np.sum((A @ A) ** 2) + 1e-20) ** 0.125
+        Y = X0 / n
+        for a, b, c in [(3.4445, -4.7750, 2.0315)] * 5:
+            Y = a * Y + b * (Y @ Y.T) @ Y + c * (Y @ Y.T) @ (Y @ Y.T) @ Y
+        assert np.allclose(got[i], Y, rtol=1e-10, atol=1e-12)
