@@ -367,6 +367,7 @@ WORKLOADS = {
     "msign_2048": ("msign", dict(batch=1, rows=2048, cols=2048)),
     "msign_1024x4096": ("msign", dict(batch=1, rows=1024, cols=4096)),
     "msign_4096_fp32": ("msign", dict(batch=1, rows=4096, cols=4096, compute="fp32")),
+    "msign_4096_improved_init": ("msign", dict(batch=1, rows=4096, cols=4096, improved=True)),
     "gram_xxt_4096": ("gram_xxt", dict(n=4096)),
     "gram_xxt_8192": ("gram_xxt", dict(n=8192)),
     "gram_ns_1024x4096": ("gram_ns", dict(rows=1024, cols=4096)),
@@ -394,8 +395,9 @@ def run_workload(args):
         x = x.to(torch.bfloat16).contiguous()
         out = torch.empty_like(x)
         ws = torch.empty(msb.msign_ns_workspace_size(b, r, c, comp), dtype=torch.uint8, device=dev)
-        call = lambda: msb.msign_ns(x, out, compute=comp, workspace=ws)
-        desc.update(batch=b, rows=r, cols=c, compute=comp, input="momentum-like, bf16")
+        imp = cfg.get("improved", False)
+        call = lambda: msb.msign_ns(x, out, compute=comp, improved_init=imp, workspace=ws)
+        desc.update(batch=b, rows=r, cols=c, compute=comp, input="momentum-like, bf16", improved_init=imp)
     elif kind == "gram_xxt":
         n = cfg["n"]
         x = synth.gaussian_torch((n, n), seed=3000, device=dev, std=1.0 / n ** 0.5, dtype=torch.bfloat16)

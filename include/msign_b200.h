@@ -72,11 +72,21 @@ typedef enum {
  * laid out a_1 b_1 c_1 a_2 b_2 c_2 ... in a HOST array.  abc == NULL means
  * Jordan's triple repeated `steps` times (steps <= 0 then means 5).
  * eps < 0 selects the default of the routine (1e-20 for msign_ns, 1e-7 for
- * gram_ns). */
+ * gram_ns).
+ * init selects the initial normalisation of msign_ns and muon_step:
+ *   0  X0 = X / sqrt(sum X^2 + eps) (the msign page's reference routine);
+ *   1  additionally, at step 0, rescale X0, X0 X0^T and (X0 X0^T)^2 by n,
+ *      n^2 and n^4 with n = (||(X0 X0^T)^2||_F^2 + eps)^(1/8) -- the
+ *      sharper bound on the largest singular value from the msign page's
+ *      section on improving the initial value (改进初值).  bf16 and fp16
+ *      compute only (MSIGN_ERR_UNSUPPORTED with the fp32-accurate path and
+ *      with gram_ns).
+ * Added in ABI 101; a caller built against ABI 100 has no `init` field. */
 typedef struct {
   int steps;
   const float *abc;
   float eps;
+  int init;
 } msign_coeffs;
 
 /* Library ABI version (major * 100 + minor). */

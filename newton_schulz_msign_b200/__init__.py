@@ -81,8 +81,11 @@ def msign_ns_workspace_size(batch: int, rows: int, cols: int, compute: str = "bf
     return int(_lib.lib().msign_ns_workspace_size(batch, rows, cols, _compute_code(compute)))
 
 
-def msign_ns(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, workspace=None, stream=None):
-    """Newton-Schulz msign of the last two dims of ``x`` (bf16/fp16/fp32 CUDA tensor)."""
+def msign_ns(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, improved_init=False, workspace=None,
+             stream=None):
+    """Newton-Schulz msign of the last two dims of ``x`` (bf16/fp16/fp32 CUDA tensor).
+
+    ``improved_init``: the sharper step-0 normalisation (msign_coeffs.init = 1)."""
     torch = _torch()
     _need_cuda(x, "x")
     if x.dim() < 2:
@@ -95,7 +98,7 @@ def msign_ns(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, works
     if out.shape != x.shape or out.dtype != x.dtype:
         raise ValueError("out must match x in shape and dtype")
     ws, wsb = _workspace(msign_ns_workspace_size(batch, rows, cols, compute), x.device, workspace)
-    c, keep = make_coeffs(coeffs, eps)
+    c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0)
     st = _lib.lib().msign_ns(x.data_ptr(), out.data_ptr(), _dtype_code(x), _compute_code(compute), batch, rows,
                              cols, ctypes.byref(c) if c is not None else None, _ptr(ws), wsb, _stream(stream))
     del keep
@@ -173,7 +176,7 @@ def muon_step_workspace_size(shapes) -> int:
 
 
 def muon_step(weights, momenta, grads, *, momentum: float = 0.95, lr: float = 0.02, coeffs=None, eps=None,
-              workspace=None, stream=None):
+              improved_init=False, workspace=None, stream=None):
     """In-place Muon update of lists of weights (bf16/fp32), fp32 momenta and grads (bf16/fp32)."""
     torch = _torch()
     num = len(weights)
@@ -199,7 +202,7 @@ def muon_step(weights, momenta, grads, *, momentum: float = 0.95, lr: float = 0.
     G = (ctypes.c_void_p * num)(*[g.data_ptr() for g in grads])
     rows = _i64_array([s[0] for s in shapes])
     cols = _i64_array([s[1] for s in shapes])
-    c, keep = make_coeffs(coeffs, eps)
+    c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0)
     st = _lib.lib().muon_step(num, W, M, G, rows, cols, wdt.pop(), gdt.pop(), float(momentum), float(lr),
                               ctypes.byref(c) if c is not None else None, _ptr(ws), wsb, _stream(stream))
     del keep

@@ -29,7 +29,8 @@ EXPORTS = (
 
 
 class MsignCoeffs(ctypes.Structure):
-    _fields_ = [("steps", ctypes.c_int), ("abc", ctypes.POINTER(ctypes.c_float)), ("eps", ctypes.c_float)]
+    _fields_ = [("steps", ctypes.c_int), ("abc", ctypes.POINTER(ctypes.c_float)), ("eps", ctypes.c_float),
+                ("init", ctypes.c_int)]
 
 
 class MsignError(RuntimeError):
@@ -107,12 +108,13 @@ def check(status: int, what: str) -> None:
         raise MsignError(status, what)
 
 
-def make_coeffs(schedule=None, eps=None):
+def make_coeffs(schedule=None, eps=None, init=0):
     """(MsignCoeffs, keep-alive buffer) for a list of (a, b, c) triples."""
-    if schedule is None and eps is None:
+    if schedule is None and eps is None and not init:
         return None, None
     c = MsignCoeffs()
     c.eps = -1.0 if eps is None else float(eps)
+    c.init = int(init)
     if schedule is None:
         c.steps = 0
         c.abc = None

@@ -167,6 +167,12 @@ struct ClassInfo {
   // row_beta[r]) C for output row r (row_beta[b * row_beta_bs + r])
   const float* row_beta;
   long long row_beta_bs;
+  // optional, symmetric classes: each epilogue warp stores the sum of v^2
+  // over the tile elements it stores, the full symmetric matrix counted (an
+  // element above the diagonal twice, for its unstored mirror), at
+  // sumsq[b * sumsq_bs + (tm * tiles_n + tn) * 8 + warp slot]
+  float* sumsq;
+  long long sumsq_bs;
   EpiOut out[kMaxOuts];
   // Dependencies between classes of one launch, by 256-row block of each
   // batch entry: each epilogue warp adds 1 to sig[b * tiles_m + tm] (and to
@@ -411,7 +417,7 @@ __device__ __forceinline__ void load_c(const ClassInfo& k, int b, int row0, int 
 // this lane's row term applied (formed once per tile).
 __device__ __forceinline__ void epilogue_block(const ClassInfo& k, int b, int row0, int col0, bool mirror,
                                                float (&acc)[32], const float (&cv)[32], float alpha, float beta,
-                                               float* scratch, int lane) {
+                                               float* scratch, int lane, float& sq) {
   const int r = row0 + lane;
   const bool diag = mirror && (col0 == row0);
   const uint32_t colmask = lane_mask(k.N - col0);
@@ -423,6 +429,14 @@ __device__ __forceinline__ void epilogue_block(const ClassInfo& k, int b, int ro
   } else {
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc[i] *= alpha;
+  }
+  if (k.sumsq != nullptr && r < k.M) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int c = col0 + i;
+      const float wgt = c > r ? 2.0f : (c == r ? 1.0f : 0.0f);
+      if (c < k.N) sq = fmaf(wgt * acc[i], acc[i], sq);
+    }
   }
 
 #pragma unroll 1
@@ -779,6 +793,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // the epilogue input of the first block is read before the
       // accumulator is ready, that of each next block while one is stored
       float cv[32];
+      float sq = 0.0f;  // this lane's part of the tile's sum of squares (sumsq classes)
       if (has_c && row0 < k.M && jfirst < kBN / 32 && tc.tn * kBN + jfirst * 32 < k.N)
         load_c(k, tc.b, row0, tc.tn * kBN + jfirst * 32, lane, cv);
       // the epilogue coefficients of this lane's row, for every block of the tile
@@ -805,11 +820,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float acc[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) acc[i] = __uint_as_float(raw[i]);
-        epilogue_block(k, tc.b, row0, col0, mirror, acc, cv, alpha, beta, scratch, lane);
+        epilogue_block(k, tc.b, row0, col0, mirror, acc, cv, alpha, beta, scratch, lane, sq);
         if (pre) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) cv[i] = cn[i];
         }
+      }
+      if (k.sumsq != nullptr) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xFFFFFFFFu, sq, o);
+        if (lane == 0)
+          k.sumsq[static_cast<long long>(tc.b) * k.sumsq_bs + (static_cast<long long>(tc.tm) * k.tiles_n + tc.tn) * 8 +
+                  rank * 4 + q] = sq;
       }
       tc_fence_before();
       __syncwarp();

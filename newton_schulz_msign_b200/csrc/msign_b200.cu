@@ -173,6 +173,7 @@ struct Carver {
 struct Schedule {
   std::vector<float> abc;
   float eps;
+  int init = 0;  // 1: sharper step-0 normalisation (msign_coeffs.init)
   int steps() const { return static_cast<int>(abc.size() / 3); }
 };
 
@@ -190,6 +191,8 @@ msign_status read_schedule(const msign_coeffs* c, float default_eps, Schedule* s
     }
     if (c->eps >= 0.0f) eps = c->eps;
     if (!std::isfinite(eps)) return MSIGN_ERR_INVALID_ARG;
+    if (c->init != 0 && c->init != 1) return MSIGN_ERR_INVALID_ARG;
+    s->init = c->init;
   }
   if (T > kMaxSteps) return MSIGN_ERR_UNSUPPORTED;
   s->abc.resize(3 * T);
@@ -291,6 +294,8 @@ struct ClassSpec {
   std::vector<RowDep> deps;
   int c_dep = -1;  // the entry of deps that produced C
   int* sig = nullptr;
+  float* sumsq = nullptr;  // see ClassInfo
+  int64_t sumsq_bs = 0;
 };
 
 // Square kBM x kBN tiles on or above the diagonal.
@@ -398,6 +403,9 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     ci.num_deps = static_cast<int>(s.deps.size());
     ci.c_dep = s.c_dep;
     ci.sig = s.sig;
+    ci.sumsq = s.sumsq;
+    ci.sumsq_bs = s.sumsq_bs;
+    if (s.sumsq != nullptr && !s.symmetric) return MSIGN_ERR_INVALID_ARG;
     total += class_tiles(s);
   }
   if (total > INT32_MAX) return MSIGN_ERR_UNSUPPORTED;
@@ -503,6 +511,8 @@ struct NsBuffers {
   void* A;        // bf16 n x ldn
   void* B;        // bf16 n x ldn (zero diagonal; the diagonal is in `diag`)
   float* diag;    // fp32 diagonal of B, n per matrix
+  float* sumsq;   // sharper initial normalisation: ||A^2||_F^2 partials, [batch][tiles^2][8]
+  float* scale_n; // and the step-0 factor s / n per matrix
   int* cnt;       // state zeroed before use: kSchedBytes of dynamic-schedule state,
                   // the ingest tickets (ns_tickets(batch) ints), then the row-block
                   // counters of a chained launch [kChainSteps][3 phases][batch][tiles]
@@ -511,9 +521,9 @@ struct NsBuffers {
 inline int64_t ns_tickets(int64_t batch) { return round_up(batch, 64); }
 inline int* ns_ticket_ptr(const NsBuffers& w) { return w.cnt + kSchedBytes / sizeof(int); }
 inline int* ns_counter_base(const NsBuffers& w, int64_t batch) { return ns_ticket_ptr(w) + ns_tickets(batch); }
-// Bytes of the state region in use with `steps` chained steps.
-inline size_t state_bytes(int64_t batch, int64_t n, int steps) {
-  return kSchedBytes + sizeof(int) * (ns_tickets(batch) + 3 * steps * batch * ceil_div(n, kBM));
+// Bytes of the state region in use with `items` chained phases.
+inline size_t state_bytes(int64_t batch, int64_t n, int items) {
+  return kSchedBytes + sizeof(int) * (ns_tickets(batch) + items * batch * ceil_div(n, kBM));
 }
 
 // fp32: the operand copies P, A and B hold two fp32 planes (tf32 hi, lo)
@@ -529,8 +539,9 @@ void carve_ns(Carver& cv, int64_t batch, int64_t n, int64_t m, NsBuffers* b, boo
   b->A = cv.take(op * batch * n * ldn);
   b->B = cv.take(op * batch * n * ldn);
   b->diag = static_cast<float*>(cv.take(sizeof(float) * batch * n));
-  b->cnt = static_cast<int*>(
-      cv.take(kSchedBytes + sizeof(int) * (ns_tickets(batch) + 3 * kChainSteps * batch * ceil_div(n, kBM))));
+  b->sumsq = static_cast<float*>(cv.take(sizeof(float) * batch * ceil_div(n, kBM) * ceil_div(n, kBM) * 8));
+  b->scale_n = static_cast<float*>(cv.take(sizeof(float) * batch));
+  b->cnt = static_cast<int*>(cv.take(state_bytes(batch, n, kMaxClasses)));
 }
 
 // Launches a list of classes of one operand dtype, kMaxClasses at a time.
@@ -554,6 +565,7 @@ struct NsClass {
   // step applies X0 = s x through its epilogues (s^2 on X X^T, s on a X + B X)
   const float* s = nullptr;
   const float* s2 = nullptr;
+  bool improved = false;  // sharper step-0 normalisation (Schedule::init)
 };
 
 // Hi and lo plane outputs of a split matrix at `p` (planes of `plane` elements).
@@ -624,14 +636,36 @@ void ns_specs(const NsClass& k, int cur, float a, float b, float c, bool first, 
     x.alpha_scale = k.s;
     x.beta_scale = k.s;
   }
+  if (first && k.improved) {
+    // step 0 of the sharper normalisation: the SQR product stores A^2 itself
+    // (and the partials of ||A^2||_F^2); improved_init_kernel then forms B,
+    // and B X runs with X0 / n, i.e. with s / n on both of its terms
+    q.alpha = 1.0f, q.beta = 0.0f, q.C = nullptr;
+    q.sumsq = k.w.sumsq, q.sumsq_bs = ceil_div(n, kBM) * ceil_div(n, kBM) * 8;
+    x.alpha_scale = k.w.scale_n;
+    x.beta_scale = k.w.scale_n;
+  }
 }
 
 // Operand dtype of a class's products.
 int ns_op_dt(const NsClass& k) { return k.fp32 ? DT_FP32 : k.op_dt; }
 
+// Between step 0's SQR (which stored A^2) and its B X product: the sharper
+// normalisation's B and s / n (improved_init_kernel).
+msign_status launch_improved_init(const NsClass& k, const Schedule& sch, cudaStream_t stream) {
+  const int64_t nb = ceil_div(k.n, kBM), ldn = round_up(k.n, 8);
+  dim3 g(static_cast<unsigned>(nb * nb), static_cast<unsigned>(k.batch), 8);
+  prof_begin(stream);
+  improved_init_kernel<<<g, 256, 0, stream>>>(k.w.A, k.w.B, k.op_dt, k.w.diag, ldn, k.n * ldn, static_cast<int>(k.n),
+                                              static_cast<int>(nb), k.w.sumsq, nb * nb * 8, sch.abc[1], sch.abc[2],
+                                              sch.eps, k.s, k.w.scale_n);
+  prof_end(3, stream, 0.0, static_cast<double>(k.batch) * k.n * k.n * 3.0);
+  return launch_ok();
+}
+
 // One NS step as three launches (one per phase), each over all classes.
-msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b, float c, bool first, bool last,
-                     cudaStream_t stream) {
+msign_status ns_step(const std::vector<NsClass>& cls, const Schedule& sch, int cur, float a, float b, float c,
+                     bool first, bool last, cudaStream_t stream) {
   std::vector<ClassSpec> ph[3];
   std::vector<int> dts;
   for (const NsClass& k : cls)
@@ -647,6 +681,12 @@ msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b,
       }
       msign_status st = launch_all(v, dt, stream);
       if (st != MSIGN_OK) return st;
+      if (p == 1 && first)
+        for (const NsClass& k : cls)
+          if (k.improved && ns_op_dt(k) == dt) {
+            st = launch_improved_init(k, sch, stream);
+            if (st != MSIGN_OK) return st;
+          }
     }
   return MSIGN_OK;
 }
@@ -668,52 +708,68 @@ msign_status ns_step(const std::vector<NsClass>& cls, int cur, float a, float b,
 msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cudaStream_t stream,
                         bool zeroed = false) {
   const int T = sch.steps();
-  bool uniform = !cls.empty();
-  for (const NsClass& k : cls) uniform = uniform && ns_op_dt(k) == ns_op_dt(cls.front());
-  const int per = uniform ? std::min<int>(kChainSteps, kMaxClasses / (3 * static_cast<int>(cls.size()))) : 0;
-  int cur = 0;
-  if (per == 0) {
+  const int ncls = static_cast<int>(cls.size());
+  bool uniform = !cls.empty(), improved = false;
+  for (const NsClass& k : cls) uniform = uniform && ns_op_dt(k) == ns_op_dt(cls.front()), improved |= k.improved;
+  const int per_launch = uniform ? kMaxClasses / (3 * ncls) * 3 : 0;  // phases per chained launch
+  if (per_launch == 0) {
     for (int t = 0; t < T; ++t) {
-      msign_status st =
-          ns_step(cls, cur, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == 0, t == T - 1, stream);
+      msign_status st = ns_step(cls, sch, t & 1, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == 0,
+                                t == T - 1, stream);
       if (st != MSIGN_OK) return st;
-      cur ^= 1;
     }
     return MSIGN_OK;
   }
-  for (int t0 = 0; t0 < T; t0 += per) {
-    const int t1 = std::min(T, t0 + per);
-    std::vector<ClassSpec> chain;
-    for (const NsClass& k : cls) {
-      if (zeroed && t0 == 0) break;
-      const size_t bytes = state_bytes(k.batch, k.n, t1 - t0);
-      if (cudaMemsetAsync(k.w.cnt, 0, bytes, stream) != cudaSuccess) return MSIGN_ERR_CUDA;
+  // The phases (t, p) in order, p = 0 SYRK, 1 SQR, 2 BX, packed into chained
+  // launches of at most per_launch phases.  With the sharper normalisation
+  // the first launch ends after step 0's SQR, and improved_init_kernel runs
+  // before the launch that starts with step 0's B X.
+  const int total = 3 * T;
+  for (int i = 0; i < total;) {
+    int j = i;
+    while (j < total && j - i < per_launch) {
+      ++j;
+      if (improved && j - 1 == 1) break;  // just placed step 0's SQR
     }
-    for (int t = t0; t < t1; ++t, cur ^= 1) {
-      std::vector<ClassSpec> ph[3];
+    if (!(zeroed && i == 0))
+      for (const NsClass& k : cls)
+        if (cudaMemsetAsync(k.w.cnt, 0, state_bytes(k.batch, k.n, j - i), stream) != cudaSuccess)
+          return MSIGN_ERR_CUDA;
+    std::vector<ClassSpec> chain;
+    for (int it = i; it < j; ++it) {
+      const int t = it / 3, p = it % 3;
       for (const NsClass& k : cls) {
         ClassSpec sp[3];
-        ns_specs(k, cur, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == 0, t == T - 1, &sp[0], &sp[1],
+        ns_specs(k, t & 1, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == 0, t == T - 1, &sp[0], &sp[1],
                  &sp[2]);
+        ClassSpec q = sp[p];
         const int64_t rb = ceil_div(k.n, kBM);  // 256-row blocks of X, A and B
         int* const base = ns_counter_base(k.w, k.batch);
-        auto ctr = [&](int step, int phase) { return base + (3 * (step - t0) + phase) * k.batch * rb; };
-        const int per_block_sym = static_cast<int>(8 * rb);                 // tiles touching a block of A or B
-        const int per_block_x = static_cast<int>(8 * ceil_div(k.m, kBN));  // tiles in a row block of X'
+        auto ctr = [&](int item) { return base + (item - i) * k.batch * rb; };
         const int rows = static_cast<int>(rb);
-        sp[0].sig = ctr(t, 0);
-        if (t > t0) sp[0].deps = {RowDep{ctr(t - 1, 2), rows, per_block_x, DEP_TM | DEP_TN}};
-        sp[1].sig = ctr(t, 1);
-        sp[1].deps = {RowDep{ctr(t, 0), rows, per_block_sym, DEP_TM | DEP_TN}}, sp[1].c_dep = 0;
-        if (t + 1 < t1) sp[2].sig = ctr(t, 2);
-        sp[2].deps = {RowDep{ctr(t, 1), rows, per_block_sym, DEP_TM}}, sp[2].c_dep = 0;
-        for (int p = 0; p < 3; ++p) ph[p].push_back(sp[p]);
+        const int per_block_sym = static_cast<int>(kTileSignals * rb);                 // tiles touching a block of A or B
+        const int per_block_x = static_cast<int>(kTileSignals * ceil_div(k.m, kBN));  // tiles in a row block of X'
+        const int prod = it - 1;  // the phase this one reads: the previous one in the order
+        q.sig = ctr(it);
+        if (prod >= i) {
+          if (p == 0) q.deps = {RowDep{ctr(prod), rows, per_block_x, DEP_TM | DEP_TN}};
+          if (p == 1) q.deps = {RowDep{ctr(prod), rows, per_block_sym, DEP_TM | DEP_TN}};
+          if (p == 2) q.deps = {RowDep{ctr(prod), rows, per_block_sym, DEP_TM}};
+          q.c_dep = q.C != nullptr && p != 0 ? 0 : -1;
+        }
+        chain.push_back(q);
       }
-      for (int p = 0; p < 3; ++p) chain.insert(chain.end(), ph[p].begin(), ph[p].end());
     }
     // dynamic schedule state: the first class's area (zeroed with its counters)
     msign_status st = launch_grouped(chain, ns_op_dt(cls.front()), stream, /*ordered=*/true, cls.front().w.cnt);
     if (st != MSIGN_OK) return st;
+    if (improved && j == 2)
+      for (const NsClass& k : cls)
+        if (k.improved) {
+          st = launch_improved_init(k, sch, stream);
+          if (st != MSIGN_OK) return st;
+        }
+    i = j;
   }
   return MSIGN_OK;
 }
@@ -875,7 +931,7 @@ using namespace msb;
 
 extern "C" {
 
-int msign_abi_version(void) { return 100; }
+int msign_abi_version(void) { return 101; }
 
 const char* msign_status_string(msign_status s) {
   switch (s) {
@@ -958,6 +1014,7 @@ msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dty
   Schedule sch;
   msign_status st = read_schedule(coeffs, kNsEps, &sch);
   if (st != MSIGN_OK) return st;
+  if (sch.init != 0 && compute_dtype == MSIGN_FP32) return MSIGN_ERR_UNSUPPORTED;
   if (batch == 0 || rows == 0 || cols == 0) return MSIGN_OK;
   if (in == nullptr || out == nullptr) return MSIGN_ERR_INVALID_ARG;
   if (batch > 65535 || rows > (1 << 30) || cols > (1 << 30)) return MSIGN_ERR_UNSUPPORTED;
@@ -984,7 +1041,7 @@ msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dty
   // before the cast (fp16 range), so that path normalises first.
   const bool fused = cd != DT_FP16;
   if (fused) {
-    if (cudaMemsetAsync(w.cnt, 0, state_bytes(batch, n, kChainSteps), stream) != cudaSuccess) return MSIGN_ERR_CUDA;
+    if (cudaMemsetAsync(w.cnt, 0, state_bytes(batch, n, kMaxClasses), stream) != cudaSuccess) return MSIGN_ERR_CUDA;
     IngestArgs a = ingest_args(in, io, rows, cols, tr, cd, w.P[0], fp32 ? DT_TF32_HI : DT_BF16, ldm,
                                fp32 ? 2 * n * ldm : n * ldm);
     a.op_plane = n * ldm;
@@ -1008,6 +1065,7 @@ msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dty
   cls[0].op_dt = fp32 ? DT_BF16 : cd;
   cls[0].final_outs = {out_to(out, io, cols, rows * cols, tr)};
   if (fused) cls[0].s = w.scale, cls[0].s2 = w.scale + batch;
+  cls[0].improved = sch.init == 1;
   return ns_iterate(cls, sch, stream, fused);
 }
 
@@ -1072,6 +1130,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
   Schedule sch;
   msign_status st = read_schedule(coeffs, kGramEps, &sch);
   if (st != MSIGN_OK) return st;
+  if (sch.init != 0) return MSIGN_ERR_UNSUPPORTED;  // the sharper normalisation is a standard-NS option
   const int T = sch.steps();
   std::vector<int> bounds;
   st = gram_segments(T, restart_after, n_restart, &bounds);
@@ -1296,7 +1355,8 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
       ns[c].final_outs = {out_blocked(ns[c].w.master, blk_ld(ns[c].m), blk_size(ns[c].n, ns[c].m))};
       ns[c].s = ns[c].w.scale;
       ns[c].s2 = ns[c].w.scale + counts[c];
-      if (cudaMemsetAsync(ns[c].w.cnt, 0, state_bytes(counts[c], ns[c].n, kChainSteps), stream) != cudaSuccess)
+      ns[c].improved = sch.init == 1;
+      if (cudaMemsetAsync(ns[c].w.cnt, 0, state_bytes(counts[c], ns[c].n, kMaxClasses), stream) != cudaSuccess)
         return MSIGN_ERR_CUDA;
     }
     // one fused pass per matrix: M <- mu M + G in place, x = bf16(M) (unscaled)

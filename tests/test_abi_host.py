@@ -45,7 +45,7 @@ def test_exported_symbols_match_nm(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.msign_abi_version() == 100
+    assert L.msign_abi_version() == 101
     assert L.msign_status_string(_lib.OK) == b"ok"
     assert b"timed out" in L.msign_status_string(_lib.ERR_TIMEOUT)
     assert L.msign_status_string(99) == b"unknown status"
@@ -91,6 +91,19 @@ def test_invalid_arguments_rejected_on_host(L):
     assert L.msign_ns(16, 16, _lib.BF16, _lib.FP32, 1, 4, 4, None, None, 0, None) == _lib.ERR_WORKSPACE
     # the fp32-accurate path keeps two fp32 planes per operand: larger workspace
     assert L.msign_ns_workspace_size(1, 512, 512, _lib.FP32) > L.msign_ns_workspace_size(1, 512, 512, _lib.BF16)
+
+
+def test_init_option_validation(L):
+    # msign_coeffs.init: 0 or 1; the sharper normalisation needs 16-bit
+    # operands and is a standard-NS option
+    c = _lib.MsignCoeffs()
+    c.steps, c.abc, c.eps, c.init = 0, None, -1.0, 2
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == _lib.ERR_INVALID_ARG
+    c.init = 1
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.FP32, 1, 4, 4, ctypes.byref(c), None, 0, None) == _lib.ERR_UNSUPPORTED
+    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, ctypes.byref(c), None, 0, None, 0, None) == _lib.ERR_UNSUPPORTED
+    # bf16 with init = 1 passes the argument checks (fails only on the missing workspace)
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == _lib.ERR_WORKSPACE
 
 
 def test_gram_ns_restart_validation(L):

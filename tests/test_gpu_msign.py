@@ -164,3 +164,34 @@ def test_compute_fp32_full_size():
     y = msb.msign_ns(x, compute="fp32")
     msb.sync_status()
     assert rel_fro(to_np(y), O.msign_ns(to_np(x))) < TOL_FP32
+
+
+# ---------------------------------------------------------------- sharper initial normalisation
+
+@pytest.mark.parametrize("shape,compute", [((256, 512), "bf16"), ((300, 100), "bf16"), ((3, 96, 200), "bf16"),
+                                           ((520, 600), "bf16"), ((256, 512), "fp16")])
+def test_improved_init(shape, compute):
+    # the msign page's sharper step-0 normalisation against its fp64 oracle
+    x = torch.from_numpy(synth.gaussian(shape, seed=shape[-1] + 17)).cuda().to(torch.bfloat16)
+    y = msb.msign_ns(x, compute=compute, improved_init=True)
+    msb.sync_status()
+    ref = O.msign_ns_improved_init(to_np(x), input_cast=compute)
+    assert rel_fro(to_np(y), ref) < TOL_BF16
+    # and it is not the plain iteration
+    assert rel_fro(to_np(y), O.msign_ns(to_np(x), input_cast=compute)) > 5 * TOL_BF16
+
+
+def test_improved_init_long_schedule_and_momentum_like():
+    x = torch.from_numpy(synth.momentum_like(384, 1024, seed=21)).cuda().to(torch.bfloat16)
+    coeffs = [(3.4445, -4.7750, 2.0315)] * 7
+    y = msb.msign_ns(x, coeffs=coeffs, improved_init=True)
+    msb.sync_status()
+    ref = O.msign_ns_improved_init(to_np(x), coeffs, input_cast="bf16")
+    assert rel_fro(to_np(y), ref) < TOL_BF16
+
+
+def test_improved_init_full_size():
+    x = synth.momentum_like_torch(4096, 4096, seed=78, device="cuda").to(torch.bfloat16)
+    y = msb.msign_ns(x, improved_init=True)
+    msb.sync_status()
+    assert rel_fro(to_np(y), O.msign_ns_improved_init(to_np(x), input_cast="bf16")) < TOL_BF16

@@ -121,3 +121,18 @@ def test_muon_llama_layer_full_size():
         assert torch.isfinite(w).all()
     for i in (0, 1, 6):
         check_matrix(W0[i], M0[i], G[i], W[i], M[i], 0.02)
+
+
+def test_muon_improved_init():
+    # the sharper step-0 normalisation inside the Muon update
+    shapes = [(128, 256), (256, 128), (96, 96)]
+    W, M, G = make(shapes, torch.float32, torch.float32, seed=600)
+    W0 = [w.clone() for w in W]
+    M0 = [m.clone() for m in M]
+    msb.muon_step(W, M, G, momentum=0.95, lr=0.02, improved_init=True)
+    msb.sync_status()
+    for i, (r, c) in enumerate(shapes):
+        Mr = 0.95 * to_np(M0[i]) + to_np(G[i])
+        O_ref = O.msign_ns_improved_init(Mr, input_cast="bf16")
+        dW_ref = -0.02 * math.sqrt(max(1.0, r / c)) * O_ref
+        assert rel_fro(to_np(W[i]) - to_np(W0[i]), dW_ref) < TOL_BF16
