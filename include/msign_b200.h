@@ -92,6 +92,15 @@ typedef struct {
 /* Library ABI version (major * 100 + minor). */
 int msign_abi_version(void);
 
+/* Fires the failure path of the library's bounded waits, for tests: one
+ * kernel thread waits on an mbarrier that nothing completes and on a device
+ * counter that nothing increments, each for limit_ns (0 < limit_ns <= 1e9),
+ * then returns.  Each expiry sets the device error word, so the next
+ * msign_sync_status(stream) returns MSIGN_ERR_TIMEOUT (and clears the word);
+ * the context stays usable.  Asynchronous on `stream`.  No counterpart on
+ * the pages. */
+msign_status msign_selftest_timeout(uint64_t limit_ns, msign_stream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *msign_status_string(msign_status status);
 

@@ -17,7 +17,8 @@ from ._lib import BF16, FP16, FP32, MsignError, check, make_coeffs
 
 __all__ = [
     "MsignError", "msign_ns", "msign_ns_workspace_size", "gram_xxt", "gram_xxt_workspace_size", "gram_ns",
-    "gram_ns_workspace_size", "muon_step", "muon_step_workspace_size", "sync_status", "library_path",
+    "gram_ns_workspace_size", "muon_step", "muon_step_workspace_size", "sync_status", "selftest_timeout",
+    "library_path",
 ]
 
 
@@ -212,6 +213,13 @@ def muon_step(weights, momenta, grads, *, momentum: float = 0.95, lr: float = 0.
 # ---------------------------------------------------------------- launch records
 
 PROFILE_KINDS = {"gemm": 0, "norm": 1, "ingest": 2, "elementwise": 3}
+
+
+def selftest_timeout(limit_ns: int = 50_000_000, stream=None) -> None:
+    """Makes the library's bounded waits expire on purpose (see
+    msign_selftest_timeout): the next sync_status() raises MsignError with
+    status ERR_TIMEOUT, and the GPU context stays usable."""
+    check(_lib.lib().msign_selftest_timeout(int(limit_ns), _stream(stream)), "msign_selftest_timeout")
 
 
 def profile_enable(enable: bool = True) -> None:

@@ -25,6 +25,7 @@ EXPORTS = (
     "muon_step_workspace_size", "muon_step",
     "msign_profile_enable", "msign_profile_read", "msign_profile_reset",
     "msign_ns_noalloc_max_bytes", "msign_ns_noalloc",
+    "msign_selftest_timeout",
 )
 
 
@@ -90,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.msign_profile_reset.argtypes = []
         L.msign_ns_noalloc_max_bytes.restype = SZ
         L.msign_ns_noalloc_max_bytes.argtypes = []
+        L.msign_selftest_timeout.restype = I32
+        L.msign_selftest_timeout.argtypes = [ctypes.c_uint64, P]
         L.msign_ns_noalloc.restype = I32
         L.msign_ns_noalloc.argtypes = [P, P, I32, I64, I64, I64, ctypes.POINTER(MsignCoeffs), P]
         _lib = L

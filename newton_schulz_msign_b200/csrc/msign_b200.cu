@@ -446,6 +446,21 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
 
 msign_status launch_ok() { return cudaGetLastError() == cudaSuccess ? MSIGN_OK : MSIGN_ERR_CUDA; }
 
+// The failure path of every bounded wait, made to fire on purpose: one
+// thread waits on an mbarrier that no one arrives on and on a counter that
+// no one increments.  Each wait gives up after limit_ns, sets the device
+// error word and returns; the kernel then ends normally.
+__device__ int g_never_signalled = 0;
+
+__global__ void selftest_timeout_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  (void)wait_bounded(&bar, 0, nullptr, err, limit_ns);
+  (void)wait_counter(&g_never_signalled, 1, nullptr, err, limit_ns);
+}
+
 // Frobenius normalisation factor of every matrix of a batch into scale[].
 msign_status launch_norm(const void* in, int in_dt, int64_t per, int64_t batch, int cast_dt, float eps, int mode,
                          float* partials, float* scale, cudaStream_t stream) {
@@ -943,6 +958,15 @@ const char* msign_status_string(msign_status s) {
     case MSIGN_ERR_TIMEOUT: return "a bounded device wait timed out";
   }
   return "unknown status";
+}
+
+msign_status msign_selftest_timeout(uint64_t limit_ns, msign_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return MSIGN_ERR_INVALID_ARG;
+  DeviceState* dev = nullptr;
+  msign_status st = device_state(&dev);
+  if (st != MSIGN_OK) return st;
+  selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(dev->err, limit_ns);
+  return launch_ok();
 }
 
 msign_status msign_sync_status(msign_stream_t stream) {

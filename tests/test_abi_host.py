@@ -106,6 +106,11 @@ def test_init_option_validation(L):
     assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == _lib.ERR_WORKSPACE
 
 
+def test_selftest_timeout_validation(L):
+    assert L.msign_selftest_timeout(0, None) == _lib.ERR_INVALID_ARG
+    assert L.msign_selftest_timeout(2_000_000_000, None) == _lib.ERR_INVALID_ARG
+
+
 def test_gram_ns_restart_validation(L):
     r = (ctypes.c_int * 1)(5)  # must lie in 1..T-1
     assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, None, ctypes.cast(r, ctypes.POINTER(ctypes.c_int)), 1, None, 0,
