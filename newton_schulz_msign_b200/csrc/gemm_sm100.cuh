@@ -136,9 +136,12 @@ struct EpiOut {
 // One dependency of a class on an earlier class of the launch (its row-block
 // counters): rows tm and/or tn of the consumer tile, or all `rows` rows,
 // must have reached `target`.
-constexpr int kMaxDeps = 6;
+constexpr int kMaxDeps = 10;
+constexpr int kMaxAddends = 3;
 constexpr int kTileSignals = 8;  // arrivals per finished tile on each row it touches: a pair's 8 epilogue warps
-enum : int { DEP_TM = 1, DEP_TN = 2, DEP_ALL = 4 };
+// DEP_EPI: waited for by the epilogue only, before it reads or stores
+// anything (write-after-read orders, and the other parts of a split K)
+enum : int { DEP_TM = 1, DEP_TN = 2, DEP_ALL = 4, DEP_EPI = 8 };
 struct RowDep {
   const int* ptr;  // counters of batch entry 0; entry b at ptr + b * rows
   int rows, target, mode;
@@ -173,6 +176,14 @@ struct ClassInfo {
   // sumsq[b * sumsq_bs + (tm * tiles_n + tn) * 8 + warp slot]
   float* sumsq;
   long long sumsq_bs;
+  // split K: this class covers K slices [k_begin, k_begin + K) of the
+  // product (the tensor maps span the whole K); its epilogue first adds the
+  // other parts' fp32 partial tiles addend[0..num_addends) (blocked layout,
+  // add_ld wide, add_bs per batch entry), in that order
+  int k_begin;
+  int num_addends;
+  const float* addend[kMaxAddends];
+  long long add_ld, add_bs;
   EpiOut out[kMaxOuts];
   // Dependencies between classes of one launch, by 256-row block of each
   // batch entry: each epilogue warp adds 1 to sig[b * tiles_m + tm] (and to
@@ -620,8 +631,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int passes = k.split ? 3 : 1;  // split: hi*hi, hi*lo, lo*hi per K slice
         const int arow = tc.tm * kBM + static_cast<int>(rank) * kHalfM;
         const int bcol = tc.tn * kBN + static_cast<int>(rank) * kHalfN;
-        const int a_tr = k.a_sym ? (tc.tm * kBM) / OK::bke : 0;  // K slices below this read A transposed
-        const int b_tr = k.b_sym ? (tc.tn * kBN) / OK::bke : 0;
+        const int ko = k.k_begin / OK::bke;  // first K slice of this class (split K)
+        const int a_tr = k.a_sym ? (tc.tm * kBM) / OK::bke - ko : 0;  // K slices below this read A transposed
+        const int b_tr = k.b_sym ? (tc.tn * kBN) / OK::bke - ko : 0;
         const bool b_mn = k.b_mn_major != 0;
         const GemmClass& g = p.cls[tc.c];
         const void* tmA = &g.tmA;
@@ -633,6 +645,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // the buffers this tile overwrites): wait for their row blocks
           for (int e = 0; e < k.num_deps && ok; ++e) {
             const RowDep& d = k.deps[e];
+            if (d.mode & DEP_EPI) continue;
             const int* base = d.ptr + static_cast<long long>(tc.b) * d.rows;
             if (d.mode & DEP_ALL) {
               for (int r = 0; r < d.rows && ok; ++r) ok = wait_counter(base + r, d.target, s_abort, p.err, limit);
@@ -656,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = sA + stage * kATileBytes;
           uint8_t* b_dst = sB + stage * kBTileBytes;
-          const int k0 = kb * OK::bke;
+          const int k0 = (kb + ko) * OK::bke;
           if (kb < a_tr) {
             // stored transpose: rows k0.. of S, columns arow..arow+127 (MN-major)
 #pragma unroll
@@ -713,8 +726,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const ClassInfo& k = p.cls[tc.c].info;
         const int nk = (k.K + OK::bke - 1) / OK::bke;
         const int passes = k.split ? 3 : 1;
-        const int a_tr = k.a_sym ? (tc.tm * kBM) / OK::bke : 0;
-        const int b_tr = k.b_sym ? (tc.tn * kBN) / OK::bke : (k.b_mn_major ? nk : 0);
+        const int ko = k.k_begin / OK::bke;
+        const int a_tr = k.a_sym ? (tc.tm * kBM) / OK::bke - ko : 0;
+        const int b_tr = k.b_sym ? (tc.tn * kBN) / OK::bke - ko : (k.b_mn_major ? nk : 0);
         if (!wait_bounded(&tempty[buf], bphase ^ 1u, s_abort, p.err, limit)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
@@ -790,6 +804,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // after the producers' release
         (void)ld_acquire_gpu(d);
       }
+      {
+        // epilogue-only dependencies (the other parts of a split K, whose
+        // partials are added below, and write-after-read orders: nothing is
+        // stored before they are met); every lane waits, so every lane has
+        // its own acquire
+        bool eok = true;
+        for (int e = 0; e < k.num_deps && eok; ++e) {
+          const RowDep& d = k.deps[e];
+          if (!(d.mode & DEP_EPI)) continue;
+          const int* base = d.ptr + static_cast<long long>(tc.b) * d.rows;
+          if (d.mode & DEP_ALL) {
+            for (int r = 0; r < d.rows && eok; ++r) eok = wait_counter(base + r, d.target, s_abort, p.err, limit);
+          } else {
+            if (d.mode & DEP_TM) eok = eok && wait_counter(base + tc.tm, d.target, s_abort, p.err, limit);
+            if (d.mode & DEP_TN) eok = eok && wait_counter(base + tc.tn, d.target, s_abort, p.err, limit);
+          }
+        }
+        if (!__all_sync(0xFFFFFFFFu, eok)) break;
+      }
       // the epilogue input of the first block is read before the
       // accumulator is ready, that of each next block while one is stored
       float cv[32];
@@ -820,6 +853,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float acc[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) acc[i] = __uint_as_float(raw[i]);
+        for (int a = 0; a < k.num_addends; ++a) {
+          // split K: this block of another part's fp32 partial (coalesced)
+          const float* ap = k.addend[a] + static_cast<long long>(tc.b) * k.add_bs + blk_off(row0, col0, k.add_ld) + 4 * lane;
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 f = *reinterpret_cast<const float4*>(ap + 128 * j4);
+            acc[4 * j4 + 0] += f.x;
+            acc[4 * j4 + 1] += f.y;
+            acc[4 * j4 + 2] += f.z;
+            acc[4 * j4 + 3] += f.w;
+          }
+        }
         epilogue_block(k, tc.b, row0, col0, mirror, acc, cv, alpha, beta, scratch, lane, sq);
         if (pre) {
 #pragma unroll

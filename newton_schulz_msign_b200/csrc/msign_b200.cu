@@ -296,6 +296,11 @@ struct ClassSpec {
   int* sig = nullptr;
   float* sumsq = nullptr;  // see ClassInfo
   int64_t sumsq_bs = 0;
+  // split K (see ClassInfo): K slices [k_begin, k_begin + K) of a product of
+  // inner dimension k_total (0: K), plus the other parts' partials to add
+  int64_t k_begin = 0, k_total = 0;
+  std::vector<const float*> addends;
+  int64_t add_ld = 0, add_bs = 0;
 };
 
 // Square kBM x kBN tiles on or above the diagonal.
@@ -342,24 +347,27 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     if (s.M > INT32_MAX || s.N > INT32_MAX || s.K > INT32_MAX || s.batch > 65535) return MSIGN_ERR_UNSUPPORTED;
     const int bke = kRowBytes / dtype_size(ab_dt);  // K elements per stage row
     const int64_t zb = s.split ? 2 * s.batch : s.batch;
+    const int64_t kt = s.k_total > 0 ? s.k_total : s.K;  // the product's whole inner dimension
+    if (s.k_begin < 0 || s.k_begin % kBM != 0 || s.k_begin + s.K > kt || s.addends.size() > kMaxAddends)
+      return MSIGN_ERR_INVALID_ARG;
     Mat a = s.A;
     a.rows = s.M;
-    a.cols = s.K;
+    a.cols = kt;
     if (!encode(&c.tmA, a, bke, kHalfM, zb)) return MSIGN_ERR_CUDA;
-    if (s.a_sym && (s.M != s.K || !encode(&c.tmA2, a, bke, bke, zb, true))) return MSIGN_ERR_INVALID_ARG;
+    if (s.a_sym && (s.M != kt || !encode(&c.tmA2, a, bke, bke, zb, true))) return MSIGN_ERR_INVALID_ARG;
     Mat b = s.B;
     if (s.b_sym) {
-      if (s.b_mn || s.N != s.K) return MSIGN_ERR_INVALID_ARG;
+      if (s.b_mn || s.N != kt) return MSIGN_ERR_INVALID_ARG;
       b.rows = s.N;
-      b.cols = s.K;
+      b.cols = kt;
       if (!encode(&c.tmB2, b, bke, bke, zb, true)) return MSIGN_ERR_CUDA;
     }
     if (!s.b_mn) {
       b.rows = s.N;
-      b.cols = s.K;
+      b.cols = kt;
       if (!encode(&c.tmB, b, bke, kHalfN, zb)) return MSIGN_ERR_CUDA;
     } else {
-      b.rows = s.K;
+      b.rows = kt;
       b.cols = s.N;
       if (!encode(&c.tmB, b, bke, bke, zb, true)) return MSIGN_ERR_CUDA;
     }
@@ -394,8 +402,7 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     if (s.c_blocked && (s.c_dt != DT_FP32 || s.c_plane != 0 || s.symmetric || s.ldc % 32 != 0))
       return MSIGN_ERR_INVALID_ARG;
     for (const EpiOut& e : s.outs)
-      if (e.blocked && (e.dtype != DT_FP32 || e.transposed || s.symmetric || e.ld % 32 != 0))
-        return MSIGN_ERR_INVALID_ARG;
+      if (e.blocked && (e.dtype != DT_FP32 || e.transposed || e.ld % 32 != 0)) return MSIGN_ERR_INVALID_ARG;
     for (size_t o = 0; o < s.outs.size(); ++o) ci.out[o] = s.outs[o];
     if (s.deps.size() > static_cast<size_t>(kMaxDeps) || s.c_dep >= static_cast<int>(s.deps.size()))
       return MSIGN_ERR_INVALID_ARG;
@@ -405,6 +412,11 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     ci.sig = s.sig;
     ci.sumsq = s.sumsq;
     ci.sumsq_bs = s.sumsq_bs;
+    ci.k_begin = static_cast<int>(s.k_begin);
+    ci.num_addends = static_cast<int>(s.addends.size());
+    for (size_t e = 0; e < s.addends.size(); ++e) ci.addend[e] = s.addends[e];
+    ci.add_ld = s.add_ld;
+    ci.add_bs = s.add_bs;
     if (s.sumsq != nullptr && !s.symmetric) return MSIGN_ERR_INVALID_ARG;
     total += class_tiles(s);
   }
@@ -801,6 +813,7 @@ struct GramBuffers {
   void* RZ;
   int* cnt;  // zeroed before each chained launch: kSchedBytes of schedule state, then the
              // row-block counters of up to kMaxClasses classes [class][batch][tiles]
+  float* part[kMaxAddends];  // split-K partials of n x n products (blocked fp32)
 };
 
 void carve_gram(Carver& cv, int64_t batch, int64_t n, int64_t m, GramBuffers* b) {
@@ -815,6 +828,7 @@ void carve_gram(Carver& cv, int64_t batch, int64_t n, int64_t m, GramBuffers* b)
   b->Q[1] = cv.take(2ull * batch * n * ldn);
   b->RZ = cv.take(2ull * batch * n * ldn);
   b->cnt = static_cast<int*>(cv.take(kSchedBytes + sizeof(int) * kMaxClasses * batch * ceil_div(n, kBM)));
+  for (int q = 0; q < kMaxAddends; ++q) b->part[q] = static_cast<float*>(cv.take(4ull * batch * blk_size(n, n)));
 }
 
 // Classes of one chained launch whose dependencies are derived from the
@@ -865,7 +879,10 @@ struct Chain {
     return st;
   }
 
-  // reads: (buffer, DEP_TM / DEP_TN / DEP_ALL); c_buf: the buffer read as C
+  // reads: (buffer, DEP_TM / DEP_TN / DEP_ALL, plus DEP_EPI when only the
+  // epilogue reads it); c_buf: the buffer read as C.  Reads are waited for
+  // before the mainloop; write-after-read and write-after-write orders only
+  // before the epilogue stores (DEP_EPI), so the mainloop starts early.
   msign_status add(ClassSpec s, const std::vector<std::pair<const void*, int>>& reads, const void* c_buf,
                    const std::vector<const void*>& writes) {
     if (cls.size() == static_cast<size_t>(kMaxClasses)) {
@@ -873,10 +890,10 @@ struct Chain {
       if (st != MSIGN_OK) return st;
     }
     const int me = static_cast<int>(cls.size());
-    std::vector<std::pair<int, int>> need;  // (class, mode)
+    std::vector<std::pair<int, int>> need;  // (class, mode): one entry per class and DEP_EPI kind
     auto want = [&](int c, int mode) {
       for (auto& n : need)
-        if (n.first == c) {
+        if (n.first == c && (n.second & DEP_EPI) == (mode & DEP_EPI)) {
           n.second |= mode;
           return;
         }
@@ -890,15 +907,25 @@ struct Chain {
     if (c_buf != nullptr && buf(c_buf).writer >= 0) want(buf(c_buf).writer, DEP_TM);  // C tile (tm, tn)
     for (const void* w : writes) {
       const Buf& b = buf(w);
-      for (const Use& u : b.readers) want(u.cls, (u.mode & DEP_ALL) ? DEP_ALL : out_rows);
-      if (b.writer >= 0) want(b.writer, out_rows);
+      for (const Use& u : b.readers) want(u.cls, DEP_EPI | ((u.mode & DEP_ALL) ? DEP_ALL : out_rows));
+      if (b.writer >= 0) want(b.writer, DEP_EPI | out_rows);
     }
     s.deps.clear();
     s.c_dep = -1;
     for (const auto& n : need) {
-      const int mode = (n.second & DEP_ALL) ? DEP_ALL : n.second;
+      int mode = (n.second & DEP_ALL) ? (DEP_ALL | (n.second & DEP_EPI)) : n.second;
+      if (mode & DEP_EPI) {
+        // already covered by a wait on the same class before the mainloop?
+        bool covered = false;
+        for (const auto& o : need)
+          if (o.first == n.first && !(o.second & DEP_EPI) &&
+              ((o.second & DEP_ALL) || ((mode & ~o.second & (DEP_TM | DEP_TN | DEP_ALL)) == 0)))
+            covered = true;
+        if (covered) continue;
+      }
       s.deps.push_back(RowDep{counters(n.first), static_cast<int>(rows), target[n.first], mode});
-      if (c_buf != nullptr && buf(c_buf).writer == n.first) s.c_dep = static_cast<int>(s.deps.size()) - 1;
+      if (c_buf != nullptr && buf(c_buf).writer == n.first && !(mode & DEP_EPI))
+        s.c_dep = static_cast<int>(s.deps.size()) - 1;
     }
     if (s.deps.size() > static_cast<size_t>(kMaxDeps)) return MSIGN_ERR_UNSUPPORTED;
     s.sig = counters(me);
@@ -913,6 +940,39 @@ struct Chain {
     for (const auto& r : reads) buf(r.first).readers.push_back({me, r.second});
     if (c_buf != nullptr) buf(c_buf).readers.push_back({me, DEP_TM});
     return MSIGN_OK;
+  }
+
+  // The same product with its inner dimension split into `parts` ranges of
+  // whole 256-blocks: every part but the last stores its fp32 partial tiles
+  // into part_buf[p] (blocked layout, part_ld wide, part_bs per matrix);
+  // the last part adds them, in order, to its own accumulator before the
+  // product's real epilogue, waiting for them in its epilogue only.  All
+  // parts run their mainloops side by side: a product of few tiles and a
+  // long K fills more of the GPU.  The sum is taken in a fixed order.
+  msign_status add_split(const ClassSpec& s, int parts, const std::vector<std::pair<const void*, int>>& reads,
+                         const void* c_buf, const std::vector<const void*>& writes, float* const* part_buf,
+                         int64_t part_ld, int64_t part_bs) {
+    const int64_t K = s.K, len = round_up(ceil_div(K, std::max(parts, 1)), kBM);
+    parts = static_cast<int>(std::min<int64_t>(ceil_div(K, len), kMaxAddends + 1));
+    if (parts <= 1) return add(s, reads, c_buf, writes);
+    const int out_rows = s.symmetric ? (DEP_TM | DEP_TN) : DEP_TM;
+    std::vector<std::pair<const void*, int>> last_reads = reads;
+    for (int q = 0; q + 1 < parts; ++q) {
+      ClassSpec c;
+      c.A = s.A, c.B = s.B, c.b_mn = s.b_mn, c.symmetric = s.symmetric, c.mirror = s.mirror;
+      c.a_sym = s.a_sym, c.b_sym = s.b_sym, c.split = s.split;
+      c.M = s.M, c.N = s.N, c.batch = s.batch;
+      c.K = len, c.k_begin = q * len, c.k_total = K;
+      c.outs = {out_blocked(part_buf[q], part_ld, part_bs)};
+      msign_status st = add(c, reads, nullptr, {part_buf[q]});
+      if (st != MSIGN_OK) return st;
+      last_reads.push_back({part_buf[q], DEP_EPI | out_rows});
+    }
+    ClassSpec c = s;
+    c.k_begin = (parts - 1) * len, c.K = K - c.k_begin, c.k_total = K;
+    for (int q = 0; q + 1 < parts; ++q) c.addends.push_back(part_buf[q]);
+    c.add_ld = part_ld, c.add_bs = part_bs;
+    return add(c, last_reads, c_buf, writes);
   }
 };
 
@@ -1197,6 +1257,20 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
   Chain ch;
   ch.state = w.cnt, ch.batch = batch, ch.rows = ceil_div(n, kBM), ch.ab_dt = DT_FP16, ch.stream = stream;
   const int DEP_TMN = DEP_TM | DEP_TN;
+  // split K for the symmetric products when their tiles leave CTA pairs idle
+  // and K is long: each part keeps at least 2048 of K (measured: with shorter
+  // parts the extra partial-store epilogue costs more than the mainloop saves;
+  // 2048 x 16384 gains 6%, the n x n products of K = n <= 2048 stay whole)
+  const int64_t sym_tiles = triangle_tiles(n) * batch;
+  auto parts_for = [&](int64_t K) {
+    return static_cast<int>(std::min<int64_t>(
+        {kMaxAddends + 1, std::max<int64_t>(1, dev->max_pairs / std::max<int64_t>(sym_tiles, 1)),
+         std::max<int64_t>(1, K / 2048)}));
+  };
+  auto add_sym = [&](const ClassSpec& s, const std::vector<std::pair<const void*, int>>& reads, const void* c_buf,
+                     const std::vector<const void*>& writes) {
+    return ch.add_split(s, parts_for(s.K), reads, c_buf, writes, w.part, blk_ld(n), blk_size(n, n));
+  };
   int cur = 0;
   for (size_t seg = 0; seg + 1 < bounds.size(); ++seg) {
     const int s0 = bounds[seg], s1 = bounds[seg + 1];
@@ -1206,7 +1280,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
       s.A = X, s.B = X, s.symmetric = true;
       s.M = n, s.N = n, s.K = m, s.batch = batch;
       s.outs = sym_out(w.R, 0.0f);
-      st = ch.add(s, {{w.P[cur], DEP_TMN}}, nullptr, {w.R});
+      st = add_sym(s, {{w.P[cur], DEP_TMN}}, nullptr, {w.R});
       if (st != MSIGN_OK) return st;
     }
     int q = -1;  // Q = I until the first step of the segment sets it
@@ -1226,7 +1300,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
           s.outs.insert(s.outs.end(), qo.begin(), qo.end());
           writes.push_back(w.Q[0]);
         }
-        st = ch.add(s, {{w.R, DEP_TMN}}, w.R, writes);
+        st = add_sym(s, {{w.R, DEP_TMN}}, w.R, writes);
         if (st != MSIGN_OK) return st;
         if (first) q = 0;
       }
@@ -1237,7 +1311,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
         s.alpha = 1.0f, s.beta = a;
         s.C = w.Q[q], s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
         s.outs = sym_out(w.Q[q ^ 1], 0.0f);
-        st = ch.add(s, {{w.Q[q], DEP_TM}, {w.Z, DEP_TN}}, w.Q[q], {w.Q[q ^ 1]});
+        st = add_sym(s, {{w.Q[q], DEP_TM}, {w.Z, DEP_TN}}, w.Q[q], {w.Q[q ^ 1]});
         if (st != MSIGN_OK) return st;
       }
       if (!last) {  // RZ <- R Z + a R
@@ -1247,7 +1321,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
         s.alpha = 1.0f, s.beta = a;
         s.C = w.R, s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
         s.outs = sym_out(w.RZ, 0.0f);
-        st = ch.add(s, {{w.R, DEP_TM}, {w.Z, DEP_TN}}, w.R, {w.RZ});
+        st = add_sym(s, {{w.R, DEP_TM}, {w.Z, DEP_TN}}, w.R, {w.RZ});
         if (st != MSIGN_OK) return st;
       }
       if (!first) q ^= 1;
@@ -1258,7 +1332,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
         s.alpha = 1.0f, s.beta = a;
         s.C = w.RZ, s.c_dt = DT_FP16, s.ldc = ldn, s.c_bs = sq;
         s.outs = sym_out(w.R, 0.0f);
-        st = ch.add(s, {{w.Z, DEP_TM}, {w.RZ, DEP_TN}}, w.RZ, {w.R});
+        st = add_sym(s, {{w.Z, DEP_TM}, {w.RZ, DEP_TN}}, w.RZ, {w.R});
         if (st != MSIGN_OK) return st;
       }
     }

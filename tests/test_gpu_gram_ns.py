@@ -30,6 +30,14 @@ def test_gram_ns_shapes(shape):
     assert rel_fro(got, O.msign_ns(X)) < TOL_BF16
 
 
+@pytest.mark.parametrize("shape", [(300, 6000), (520, 9000), (6000, 300)])
+def test_gram_ns_split_k(shape):
+    # few tiles and a long inner dimension: X X^T runs as several K parts
+    # (the last one ragged) whose fp32 partials are summed in a fixed order
+    got, X = run(synth.gaussian(shape, seed=shape[0] + shape[1]))
+    assert rel_fro(got, O.gram_ns(X)) < TOL_BF16
+
+
 @pytest.mark.parametrize("restarts", [(), (1,), (2,), (3,), (1, 3), (1, 2, 3, 4)])
 def test_gram_ns_restart_schedules(restarts):
     got, X = run(synth.gaussian((192, 768), seed=11), restarts=restarts)

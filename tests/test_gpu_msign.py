@@ -74,6 +74,15 @@ def test_long_schedule_batched():
     assert rel_fro(got, ref) < TOL_BF16
 
 
+def test_many_small_matrices():
+    # a large batch of small matrices: hundreds of tiles per phase, one set
+    # of row-block counters per matrix, tiles claimed through the ring
+    x = synth.gaussian((300, 64, 96), seed=13)
+    got, ref = run_case(x)
+    err = max(rel_fro(got[i], ref[i]) for i in range(300))
+    assert err < TOL_BF16, err
+
+
 def test_momentum_like_spectrum():
     x = synth.momentum_like(512, 1024, seed=6)
     got, ref = run_case(x)
