@@ -371,7 +371,13 @@ WORKLOADS = {
     "gram_xxt_4096": ("gram_xxt", dict(n=4096)),
     "gram_xxt_8192": ("gram_xxt", dict(n=8192)),
     "gram_ns_1024x4096": ("gram_ns", dict(rows=1024, cols=4096)),
+    "gram_ns_1024x16384": ("gram_ns", dict(rows=1024, cols=16384)),
+    "gram_ns_2048x4096": ("gram_ns", dict(rows=2048, cols=4096)),
     "gram_ns_2048x16384": ("gram_ns", dict(rows=2048, cols=16384)),
+    # the same wide shapes through standard NS, for the Gram-NS comparison
+    "msign_1024x16384": ("msign", dict(batch=1, rows=1024, cols=16384)),
+    "msign_2048x4096": ("msign", dict(batch=1, rows=2048, cols=4096)),
+    "msign_2048x16384": ("msign", dict(batch=1, rows=2048, cols=16384)),
     "muon_llama3_8b_layer": ("muon", dict()),
 }
 

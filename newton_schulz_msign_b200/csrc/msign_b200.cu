@@ -540,6 +540,8 @@ struct NsBuffers {
   float* diag;    // fp32 diagonal of B, n per matrix
   float* sumsq;   // sharper initial normalisation: ||A^2||_F^2 partials, [batch][tiles^2][8]
   float* scale_n; // and the step-0 factor s / n per matrix
+  int syrk_parts;  // K parts of the X X^T product (see syrk_parts()), 1 = whole
+  float* part[kMaxAddends];  // their fp32 partials (blocked), parts - 1 of them
   int* cnt;       // state zeroed before use: kSchedBytes of dynamic-schedule state,
                   // the ingest tickets (ns_tickets(batch) ints), then the row-block
                   // counters of a chained launch [kChainSteps][3 phases][batch][tiles]
@@ -552,6 +554,23 @@ inline int* ns_counter_base(const NsBuffers& w, int64_t batch) { return ns_ticke
 inline size_t state_bytes(int64_t batch, int64_t n, int items) {
   return kSchedBytes + sizeof(int) * (ns_tickets(batch) + items * batch * ceil_div(n, kBM));
 }
+
+// CTA pairs the split-K plan assumes (a B200: 148 SMs).  The plan must not
+// depend on the device, because the workspace size is a host-only query.
+constexpr int kPlanPairs = 74;
+
+// K parts of the X X^T product (K = m) of a class whose triangle tiles
+// leave CTA pairs idle: whole 256-blocks, each at least 4096 long.  In the
+// chained iteration the split pays only there: measured on 1 x 2048 x 4096
+// (two parts of 2048) it was 9% slower, on 1 x 1024 x 16384 (four parts of
+// 4096) 16% faster.
+inline int syrk_parts(int64_t batch, int64_t n, int64_t m) {
+  const int64_t want = std::min<int64_t>({kMaxAddends + 1,
+                                          std::max<int64_t>(1, kPlanPairs / std::max<int64_t>(1, triangle_tiles(n) * batch)),
+                                          std::max<int64_t>(1, m / 4096)});
+  return static_cast<int>(ceil_div(m, round_up(ceil_div(m, want), kBM)));
+}
+inline int64_t syrk_part_len(int64_t m, int parts) { return round_up(ceil_div(m, parts), kBM); }
 
 // fp32: the operand copies P, A and B hold two fp32 planes (tf32 hi, lo)
 // per matrix, [batch][plane][rows][ld].
@@ -568,6 +587,9 @@ void carve_ns(Carver& cv, int64_t batch, int64_t n, int64_t m, NsBuffers* b, boo
   b->diag = static_cast<float*>(cv.take(sizeof(float) * batch * n));
   b->sumsq = static_cast<float*>(cv.take(sizeof(float) * batch * ceil_div(n, kBM) * ceil_div(n, kBM) * 8));
   b->scale_n = static_cast<float*>(cv.take(sizeof(float) * batch));
+  b->syrk_parts = fp32 ? 1 : syrk_parts(batch, n, m);
+  for (int q = 0; q < kMaxAddends; ++q)
+    b->part[q] = q + 1 < b->syrk_parts ? static_cast<float*>(cv.take(4ull * batch * blk_size(n, n))) : nullptr;
   b->cnt = static_cast<int*>(cv.take(state_bytes(batch, n, kMaxClasses)));
 }
 
@@ -738,8 +760,15 @@ msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cu
   const int ncls = static_cast<int>(cls.size());
   bool uniform = !cls.empty(), improved = false;
   for (const NsClass& k : cls) uniform = uniform && ns_op_dt(k) == ns_op_dt(cls.front()), improved |= k.improved;
-  const int per_launch = uniform ? kMaxClasses / (3 * ncls) * 3 : 0;  // phases per chained launch
-  if (per_launch == 0) {
+  // classes a phase takes in a launch: X X^T may run as several K parts
+  auto phase_classes = [&](int p) {
+    int c = 0;
+    for (const NsClass& k : cls) c += p == 0 ? k.w.syrk_parts : 1;
+    return c;
+  };
+  const bool chained = uniform && std::max({phase_classes(0), phase_classes(1), phase_classes(2)}) <= kMaxClasses &&
+                       3 * ncls <= kMaxClasses;
+  if (!chained) {
     for (int t = 0; t < T; ++t) {
       msign_status st = ns_step(cls, sch, t & 1, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == 0,
                                 t == T - 1, stream);
@@ -748,42 +777,72 @@ msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cu
     return MSIGN_OK;
   }
   // The phases (t, p) in order, p = 0 SYRK, 1 SQR, 2 BX, packed into chained
-  // launches of at most per_launch phases.  With the sharper normalisation
+  // launches of at most kMaxClasses classes.  With the sharper normalisation
   // the first launch ends after step 0's SQR, and improved_init_kernel runs
   // before the launch that starts with step 0's B X.
   const int total = 3 * T;
   for (int i = 0; i < total;) {
-    int j = i;
-    while (j < total && j - i < per_launch) {
+    int j = i, used = 0;
+    while (j < total && used + phase_classes(j % 3) <= kMaxClasses) {
+      used += phase_classes(j % 3);
       ++j;
       if (improved && j - 1 == 1) break;  // just placed step 0's SQR
     }
     if (!(zeroed && i == 0))
       for (const NsClass& k : cls)
-        if (cudaMemsetAsync(k.w.cnt, 0, state_bytes(k.batch, k.n, j - i), stream) != cudaSuccess)
-          return MSIGN_ERR_CUDA;
+        if (cudaMemsetAsync(k.w.cnt, 0, state_bytes(k.batch, k.n, used), stream) != cudaSuccess) return MSIGN_ERR_CUDA;
     std::vector<ClassSpec> chain;
+    std::vector<int> slots(cls.size(), 0);                // next counter slot of each class
+    std::vector<std::vector<int>> done(cls.size());       // counter slot of each phase's final class
     for (int it = i; it < j; ++it) {
       const int t = it / 3, p = it % 3;
-      for (const NsClass& k : cls) {
+      for (size_t ci = 0; ci < cls.size(); ++ci) {
+        const NsClass& k = cls[ci];
         ClassSpec sp[3];
         ns_specs(k, t & 1, sch.abc[3 * t], sch.abc[3 * t + 1], sch.abc[3 * t + 2], t == 0, t == T - 1, &sp[0], &sp[1],
                  &sp[2]);
         ClassSpec q = sp[p];
         const int64_t rb = ceil_div(k.n, kBM);  // 256-row blocks of X, A and B
         int* const base = ns_counter_base(k.w, k.batch);
-        auto ctr = [&](int item) { return base + (item - i) * k.batch * rb; };
+        auto ctr = [&](int slot) { return base + static_cast<int64_t>(slot) * k.batch * rb; };
         const int rows = static_cast<int>(rb);
         const int per_block_sym = static_cast<int>(kTileSignals * rb);                 // tiles touching a block of A or B
         const int per_block_x = static_cast<int>(kTileSignals * ceil_div(k.m, kBN));  // tiles in a row block of X'
-        const int prod = it - 1;  // the phase this one reads: the previous one in the order
-        q.sig = ctr(it);
-        if (prod >= i) {
-          if (p == 0) q.deps = {RowDep{ctr(prod), rows, per_block_x, DEP_TM | DEP_TN}};
-          if (p == 1) q.deps = {RowDep{ctr(prod), rows, per_block_sym, DEP_TM | DEP_TN}};
-          if (p == 2) q.deps = {RowDep{ctr(prod), rows, per_block_sym, DEP_TM}};
-          q.c_dep = q.C != nullptr && p != 0 ? 0 : -1;
+        // the phase this one reads: the previous one in the order
+        std::vector<RowDep> reads;
+        if (it - 1 >= i) {
+          const int ps = done[ci][it - 1 - i];
+          if (p == 0) reads = {RowDep{ctr(ps), rows, per_block_x, DEP_TM | DEP_TN}};
+          if (p == 1) reads = {RowDep{ctr(ps), rows, per_block_sym, DEP_TM | DEP_TN}};
+          if (p == 2) reads = {RowDep{ctr(ps), rows, per_block_sym, DEP_TM}};
         }
+        if (p == 0 && k.w.syrk_parts > 1) {
+          // split K (see Chain::add_split): parts 0 .. P-2 store fp32
+          // partials, the final part adds them in its epilogue
+          const int P = k.w.syrk_parts;
+          const int64_t len = syrk_part_len(k.m, P);
+          std::vector<RowDep> epi;
+          for (int qq = 0; qq + 1 < P; ++qq) {
+            ClassSpec c;
+            c.A = q.A, c.B = q.B, c.symmetric = true, c.split = q.split;
+            c.M = q.M, c.N = q.N, c.batch = q.batch;
+            c.K = len, c.k_begin = qq * len, c.k_total = k.m;
+            c.outs = {out_blocked(k.w.part[qq], blk_ld(k.n), blk_size(k.n, k.n))};
+            c.deps = reads;
+            c.sig = ctr(slots[ci]);
+            epi.push_back(RowDep{ctr(slots[ci]), rows, per_block_sym, DEP_EPI | DEP_TM | DEP_TN});
+            ++slots[ci];
+            chain.push_back(c);
+          }
+          q.k_begin = (P - 1) * len, q.K = k.m - q.k_begin, q.k_total = k.m;
+          for (int qq = 0; qq + 1 < P; ++qq) q.addends.push_back(k.w.part[qq]);
+          q.add_ld = blk_ld(k.n), q.add_bs = blk_size(k.n, k.n);
+          reads.insert(reads.end(), epi.begin(), epi.end());
+        }
+        q.deps = reads;
+        q.c_dep = (q.C != nullptr && p != 0 && it - 1 >= i) ? 0 : -1;
+        q.sig = ctr(slots[ci]);
+        done[ci].push_back(slots[ci]++);
         chain.push_back(q);
       }
     }

@@ -83,6 +83,16 @@ def test_many_small_matrices():
     assert err < TOL_BF16, err
 
 
+@pytest.mark.parametrize("shape", [(300, 9000), (520, 17000), (9000, 300), (2, 300, 8500)])
+def test_syrk_split_k(shape):
+    # few X X^T tiles over a long K (at least 4096 per part): the product
+    # runs as 2 to 4 K parts whose fp32 partials the last part adds, the
+    # last part ragged
+    x = synth.gaussian(shape, seed=shape[-1] + shape[-2])
+    got, ref = run_case(x)
+    assert rel_fro(got, ref) < TOL_BF16
+
+
 def test_momentum_like_spectrum():
     x = synth.momentum_like(512, 1024, seed=6)
     got, ref = run_case(x)
@@ -178,7 +188,7 @@ def test_compute_fp32_full_size():
 # ---------------------------------------------------------------- sharper initial normalisation
 
 @pytest.mark.parametrize("shape,compute", [((256, 512), "bf16"), ((300, 100), "bf16"), ((3, 96, 200), "bf16"),
-                                           ((520, 600), "bf16"), ((256, 512), "fp16")])
+                                           ((520, 600), "bf16"), ((256, 512), "fp16"), ((300, 9000), "bf16")])
 def test_improved_init(shape, compute):
     # the msign page's sharper step-0 normalisation against its fp64 oracle
     x = torch.from_numpy(synth.gaussian(shape, seed=shape[-1] + 17)).cuda().to(torch.bfloat16)
