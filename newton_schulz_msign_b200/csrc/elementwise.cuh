@@ -410,8 +410,8 @@ __global__ void __launch_bounds__(256) ingest_kernel(const IngestArgs a) {
 // the tile; 256 threads.
 __global__ void __launch_bounds__(256) improved_init_kernel(const void* A, void* B, int op_dt, float* d, long long ld,
                                                             long long bs, int n, int nb, const float* partials,
-                                                            long long parts_bs, float bcoef, float ccoef, float eps,
-                                                            const float* scale_in, float* scale_out) {
+                                                            long long parts_bs, int slots, float bcoef, float ccoef,
+                                                            float eps, const float* scale_in, float* scale_out) {
   __shared__ float red[32];
   const int b = blockIdx.y;
   const int tm = blockIdx.x / nb, tn = blockIdx.x % nb;
@@ -420,8 +420,8 @@ __global__ void __launch_bounds__(256) improved_init_kernel(const void* A, void*
   // ||A2||_F^2: the partials of the upper tiles, in a fixed order
   float v = 0.0f;
   const float* pp = partials + static_cast<long long>(b) * parts_bs;
-  for (int i = tid; i < nb * nb * 8; i += 256) {
-    const int t = i / 8;
+  for (int i = tid; i < nb * nb * slots; i += 256) {
+    const int t = i / slots;
     if (t / nb <= t % nb) v += pp[i];
   }
   v = block_sum_lin(v, red, tid, 256);

@@ -78,7 +78,12 @@ constexpr int kBN = 256;      // output tile columns
 constexpr int kHalfN = 128;   // B rows staged per CTA
 constexpr int kRowBytes = 128;  // one 128-byte swizzle row of K per operand row and stage
 constexpr int kStages = 6;
-constexpr int kThreads = 192;
+// Epilogue warps per CTA: two per TMEM lane quarter, each taking half of the
+// tile's columns, so that a tile's accumulator drains in half the time
+// (where tiles are few, the drain of a phase's last tiles gates the next
+// phase).
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA issuer, epilogue
 constexpr int kATileBytes = kHalfM * kRowBytes;  // 16 KB
 constexpr int kBTileBytes = kHalfN * kRowBytes;  // 16 KB
 
@@ -102,7 +107,7 @@ struct OpKind {
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kScratchStride = 33;  // padded row of the per-warp 32 x 32 fp32 transpose scratch
 constexpr int kStageOutBytes = 32 * kScratchStride * 4;
-constexpr int kEpiBytes = 4 * kStageOutBytes;  // one scratch block per epilogue warp
+constexpr int kEpiBytes = kEpiWarps * kStageOutBytes;  // one scratch block per epilogue warp
 constexpr int kTmemCols = 512;
 constexpr int kMaxClasses = 16;
 constexpr int kNumBarriers = 2 * kStages + 2 + 2 + 1;
@@ -138,7 +143,7 @@ struct EpiOut {
 // must have reached `target`.
 constexpr int kMaxDeps = 10;
 constexpr int kMaxAddends = 3;
-constexpr int kTileSignals = 8;  // arrivals per finished tile on each row it touches: a pair's 8 epilogue warps
+constexpr int kTileSignals = 2 * kEpiWarps;  // arrivals per finished tile on each row it touches: a pair's epilogue warps
 // DEP_EPI: waited for by the epilogue only, before it reads or stores
 // anything (write-after-read orders, and the other parts of a split K)
 enum : int { DEP_TM = 1, DEP_TN = 2, DEP_ALL = 4, DEP_EPI = 8 };
@@ -173,7 +178,7 @@ struct ClassInfo {
   // optional, symmetric classes: each epilogue warp stores the sum of v^2
   // over the tile elements it stores, the full symmetric matrix counted (an
   // element above the diagonal twice, for its unstored mirror), at
-  // sumsq[b * sumsq_bs + (tm * tiles_n + tn) * 8 + warp slot]
+  // sumsq[b * sumsq_bs + (tm * tiles_n + tn) * kTileSignals + warp slot]
   float* sumsq;
   long long sumsq_bs;
   // split K: this class covers K slices [k_begin, k_begin + K) of the
@@ -417,6 +422,39 @@ __device__ __forceinline__ void load_c(const ClassInfo& k, int b, int row0, int 
   }
 }
 
+// Brings a warp's epilogue inputs for columns [c0, c1) of rows row0 ..
+// row0 + 31 into L2 while the accumulator is still being computed, so that
+// the per-block loads (load_c, the split-K addends) hit L2.  Only lines
+// inside the matrices are touched.
+__device__ __forceinline__ void prefetch_blocked_l2(const float* base, long long ldb, int row0, int c0, int c1,
+                                                    int lane) {
+  // the blocks of one 32-row band are contiguous along the columns
+  const float* q = base + blk_off(row0, c0, ldb);
+  const int lines = ((c1 - c0 + 31) >> 5) * 32;  // 4 KB blocks of 32 lines
+  for (int i = lane; i < lines; i += 32) prefetch_l2(q + 32 * i);
+}
+
+__device__ __forceinline__ void prefetch_epilogue_l2(const ClassInfo& k, int b, int row0, int c0, int c1, int lane) {
+  if (k.C != nullptr) {
+    if (k.c_blocked) {
+      prefetch_blocked_l2(reinterpret_cast<const float*>(k.C) + static_cast<long long>(b) * k.c_bs, k.ldc, row0, c0,
+                          c1, lane);
+    } else if (row0 + lane < k.M) {
+      const int es = dtype_size(k.c_dtype);
+      const char* p0 = gaddr(k.C, k.c_dtype, k.ldc, k.c_bs, b, row0 + lane, c0);
+      const char* p1 = p0 + static_cast<long long>(c1 - c0 - 1) * es;  // last element
+      for (int plane = 0; plane < (k.c_plane > 0 ? 2 : 1); ++plane) {
+        const long long off = plane ? k.c_plane * 4 : 0;
+        for (uintptr_t a = reinterpret_cast<uintptr_t>(p0 + off) & ~uintptr_t(127);
+             a <= reinterpret_cast<uintptr_t>(p1 + off); a += 128)
+          prefetch_l2(reinterpret_cast<const void*>(a));
+      }
+    }
+  }
+  for (int a = 0; a < k.num_addends; ++a)
+    prefetch_blocked_l2(k.addend[a] + static_cast<long long>(b) * k.add_bs, k.add_ld, row0, c0, c1, lane);
+}
+
 // One 32x32 block: this lane owns output row `row0 + lane`, columns
 // col0..col0+31, whose fp32 accumulators are in `acc` and epilogue input in
 // `cv` (when the class has one).  `mirror`: the block is stored together
@@ -488,15 +526,15 @@ __device__ __forceinline__ void epilogue_block(const ClassInfo& k, int b, int ro
 #pragma unroll
       for (int i = 0; i < 32; ++i) scratch[i * kScratchStride + lane] = w[i];
       __syncwarp();
-      float t[32];
+      // w now takes the transposed block's row
 #pragma unroll
-      for (int j = 0; j < 32; ++j) t[j] = scratch[lane * kScratchStride + j];
+      for (int j = 0; j < 32; ++j) w[j] = scratch[lane * kScratchStride + j];
       __syncwarp();
       const int tr = col0 + lane;  // row of the transposed block
       if (tr < k.N) {
         uint32_t m = rowmask;
         if (diag) m &= (lane == 0) ? 0u : (0xFFFFFFFFu >> (32 - lane));  // rows r < c (strict)
-        store_row32(gaddr(e.ptr, e.dtype, e.ld, e.bs, b, tr, row0), e.dtype, m, t);
+        store_row32(gaddr(e.ptr, e.dtype, e.ld, e.bs, b, tr, row0), e.dtype, m, w);
       }
     }
   }
@@ -586,7 +624,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 2 * 4);  // one arrival per epilogue warp of each CTA
+      mbar_init(&tempty[i], 2 * kEpiWarps);  // one arrival per epilogue warp of each CTA
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -772,7 +810,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;  // TMEM lane quarter this warp may read
-    float* scratch = reinterpret_cast<float*>(sOut + (warp - 2) * kStageOutBytes);
+    const int ew = warp - 2;  // epilogue warp index
+    // this warp's 32-column blocks of every tile: [jbeg, jend)
+    constexpr int kBlocksPerWarp = (kBN / 32) / (kEpiWarps / 4);
+    const int jbeg = (ew >> 2) * kBlocksPerWarp, jend = jbeg + kBlocksPerWarp;
+    float* scratch = reinterpret_cast<float*>(sOut + ew * kStageOutBytes);
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
     int buf = 0;
@@ -788,9 +830,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int row0 = tc.tm * kBM + static_cast<int>(rank) * kHalfM + q * 32;
       // mirrored tiles visit only blocks on or above the diagonal
       const bool mirror = k.symmetric && (k.mirror || tc.tm == tc.tn);
-      int jfirst = 0;
+      int jfirst = jbeg;
       if (mirror)
-        while (jfirst < kBN / 32 && tc.tn * kBN + jfirst * 32 < row0) ++jfirst;
+        while (jfirst < jend && tc.tn * kBN + jfirst * 32 < row0) ++jfirst;
       const bool has_c = k.C != nullptr;
       int ok = 1;
       if (has_c && k.c_dep >= 0) {
@@ -823,12 +865,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (!__all_sync(0xFFFFFFFFu, eok)) break;
       }
-      // the epilogue input of the first block is read before the
-      // accumulator is ready, that of each next block while one is stored
+      // the epilogue inputs of this warp's blocks go to L2 now, and the
+      // first block's are read before the accumulator is ready
       float cv[32];
       float sq = 0.0f;  // this lane's part of the tile's sum of squares (sumsq classes)
-      if (has_c && row0 < k.M && jfirst < kBN / 32 && tc.tn * kBN + jfirst * 32 < k.N)
-        load_c(k, tc.b, row0, tc.tn * kBN + jfirst * 32, lane, cv);
+      if (row0 < k.M && jfirst < jend && tc.tn * kBN + jfirst * 32 < k.N) {
+        const int c0 = tc.tn * kBN + jfirst * 32;
+        prefetch_epilogue_l2(k, tc.b, row0, c0, min(k.N, tc.tn * kBN + jend * 32), lane);
+        if (has_c) load_c(k, tc.b, row0, c0, lane, cv);
+      }
       // the epilogue coefficients of this lane's row, for every block of the tile
       float alpha = k.alpha, beta = k.beta;
       if (k.row_beta != nullptr && row0 + lane < k.M)
@@ -840,12 +885,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int j = jfirst; j < kBN / 32; ++j) {
+      for (int j = jfirst; j < jend; ++j) {
         const int col0 = tc.tn * kBN + j * 32;
         if (row0 >= k.M || col0 >= k.N) break;
-        float cn[32];
-        const bool pre = has_c && j + 1 < kBN / 32 && col0 + 32 < k.N;
-        if (pre) load_c(k, tc.b, row0, col0 + 32, lane, cn);
+        // (issued before the accumulator load, so that the two overlap)
+        if (has_c && j > jfirst) load_c(k, tc.b, row0, col0, lane, cv);
         uint32_t raw[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * kBN + j * 32),
                            raw);
@@ -866,17 +910,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         epilogue_block(k, tc.b, row0, col0, mirror, acc, cv, alpha, beta, scratch, lane, sq);
-        if (pre) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) cv[i] = cn[i];
-        }
       }
       if (k.sumsq != nullptr) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xFFFFFFFFu, sq, o);
         if (lane == 0)
-          k.sumsq[static_cast<long long>(tc.b) * k.sumsq_bs + (static_cast<long long>(tc.tm) * k.tiles_n + tc.tn) * 8 +
-                  rank * 4 + q] = sq;
+          k.sumsq[static_cast<long long>(tc.b) * k.sumsq_bs + (static_cast<long long>(tc.tm) * k.tiles_n + tc.tn) * kTileSignals +
+                  rank * kEpiWarps + ew] = sq;
       }
       tc_fence_before();
       __syncwarp();

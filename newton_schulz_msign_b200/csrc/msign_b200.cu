@@ -538,7 +538,7 @@ struct NsBuffers {
   void* A;        // bf16 n x ldn
   void* B;        // bf16 n x ldn (zero diagonal; the diagonal is in `diag`)
   float* diag;    // fp32 diagonal of B, n per matrix
-  float* sumsq;   // sharper initial normalisation: ||A^2||_F^2 partials, [batch][tiles^2][8]
+  float* sumsq;   // sharper initial normalisation: ||A^2||_F^2 partials, [batch][tiles^2][kTileSignals]
   float* scale_n; // and the step-0 factor s / n per matrix
   int syrk_parts;  // K parts of the X X^T product (see syrk_parts()), 1 = whole
   float* part[kMaxAddends];  // their fp32 partials (blocked), parts - 1 of them
@@ -585,7 +585,7 @@ void carve_ns(Carver& cv, int64_t batch, int64_t n, int64_t m, NsBuffers* b, boo
   b->A = cv.take(op * batch * n * ldn);
   b->B = cv.take(op * batch * n * ldn);
   b->diag = static_cast<float*>(cv.take(sizeof(float) * batch * n));
-  b->sumsq = static_cast<float*>(cv.take(sizeof(float) * batch * ceil_div(n, kBM) * ceil_div(n, kBM) * 8));
+  b->sumsq = static_cast<float*>(cv.take(sizeof(float) * batch * ceil_div(n, kBM) * ceil_div(n, kBM) * kTileSignals));
   b->scale_n = static_cast<float*>(cv.take(sizeof(float) * batch));
   b->syrk_parts = fp32 ? 1 : syrk_parts(batch, n, m);
   for (int q = 0; q < kMaxAddends; ++q)
@@ -690,7 +690,7 @@ void ns_specs(const NsClass& k, int cur, float a, float b, float c, bool first, 
     // (and the partials of ||A^2||_F^2); improved_init_kernel then forms B,
     // and B X runs with X0 / n, i.e. with s / n on both of its terms
     q.alpha = 1.0f, q.beta = 0.0f, q.C = nullptr;
-    q.sumsq = k.w.sumsq, q.sumsq_bs = ceil_div(n, kBM) * ceil_div(n, kBM) * 8;
+    q.sumsq = k.w.sumsq, q.sumsq_bs = ceil_div(n, kBM) * ceil_div(n, kBM) * kTileSignals;
     x.alpha_scale = k.w.scale_n;
     x.beta_scale = k.w.scale_n;
   }
@@ -706,7 +706,7 @@ msign_status launch_improved_init(const NsClass& k, const Schedule& sch, cudaStr
   dim3 g(static_cast<unsigned>(nb * nb), static_cast<unsigned>(k.batch), 8);
   prof_begin(stream);
   improved_init_kernel<<<g, 256, 0, stream>>>(k.w.A, k.w.B, k.op_dt, k.w.diag, ldn, k.n * ldn, static_cast<int>(k.n),
-                                              static_cast<int>(nb), k.w.sumsq, nb * nb * 8, sch.abc[1], sch.abc[2],
+                                              static_cast<int>(nb), k.w.sumsq, nb * nb * kTileSignals, kTileSignals, sch.abc[1], sch.abc[2],
                                               sch.eps, k.s, k.w.scale_n);
   prof_end(3, stream, 0.0, static_cast<double>(k.batch) * k.n * k.n * 3.0);
   return launch_ok();
