@@ -422,39 +422,6 @@ __device__ __forceinline__ void load_c(const ClassInfo& k, int b, int row0, int 
   }
 }
 
-// Brings a warp's epilogue inputs for columns [c0, c1) of rows row0 ..
-// row0 + 31 into L2 while the accumulator is still being computed, so that
-// the per-block loads (load_c, the split-K addends) hit L2.  Only lines
-// inside the matrices are touched.
-__device__ __forceinline__ void prefetch_blocked_l2(const float* base, long long ldb, int row0, int c0, int c1,
-                                                    int lane) {
-  // the blocks of one 32-row band are contiguous along the columns
-  const float* q = base + blk_off(row0, c0, ldb);
-  const int lines = ((c1 - c0 + 31) >> 5) * 32;  // 4 KB blocks of 32 lines
-  for (int i = lane; i < lines; i += 32) prefetch_l2(q + 32 * i);
-}
-
-__device__ __forceinline__ void prefetch_epilogue_l2(const ClassInfo& k, int b, int row0, int c0, int c1, int lane) {
-  if (k.C != nullptr) {
-    if (k.c_blocked) {
-      prefetch_blocked_l2(reinterpret_cast<const float*>(k.C) + static_cast<long long>(b) * k.c_bs, k.ldc, row0, c0,
-                          c1, lane);
-    } else if (row0 + lane < k.M) {
-      const int es = dtype_size(k.c_dtype);
-      const char* p0 = gaddr(k.C, k.c_dtype, k.ldc, k.c_bs, b, row0 + lane, c0);
-      const char* p1 = p0 + static_cast<long long>(c1 - c0 - 1) * es;  // last element
-      for (int plane = 0; plane < (k.c_plane > 0 ? 2 : 1); ++plane) {
-        const long long off = plane ? k.c_plane * 4 : 0;
-        for (uintptr_t a = reinterpret_cast<uintptr_t>(p0 + off) & ~uintptr_t(127);
-             a <= reinterpret_cast<uintptr_t>(p1 + off); a += 128)
-          prefetch_l2(reinterpret_cast<const void*>(a));
-      }
-    }
-  }
-  for (int a = 0; a < k.num_addends; ++a)
-    prefetch_blocked_l2(k.addend[a] + static_cast<long long>(b) * k.add_bs, k.add_ld, row0, c0, c1, lane);
-}
-
 // One 32x32 block: this lane owns output row `row0 + lane`, columns
 // col0..col0+31, whose fp32 accumulators are in `acc` and epilogue input in
 // `cv` (when the class has one).  `mirror`: the block is stored together
@@ -865,15 +832,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (!__all_sync(0xFFFFFFFFu, eok)) break;
       }
-      // the epilogue inputs of this warp's blocks go to L2 now, and the
-      // first block's are read before the accumulator is ready
+      // the first block's epilogue input is read before the accumulator is
+      // ready, each next block's just before its accumulator load
       float cv[32];
       float sq = 0.0f;  // this lane's part of the tile's sum of squares (sumsq classes)
-      if (row0 < k.M && jfirst < jend && tc.tn * kBN + jfirst * 32 < k.N) {
-        const int c0 = tc.tn * kBN + jfirst * 32;
-        prefetch_epilogue_l2(k, tc.b, row0, c0, min(k.N, tc.tn * kBN + jend * 32), lane);
-        if (has_c) load_c(k, tc.b, row0, c0, lane, cv);
-      }
+      if (has_c && row0 < k.M && jfirst < jend && tc.tn * kBN + jfirst * 32 < k.N)
+        load_c(k, tc.b, row0, tc.tn * kBN + jfirst * 32, lane, cv);
       // the epilogue coefficients of this lane's row, for every block of the tile
       float alpha = k.alpha, beta = k.beta;
       if (k.row_beta != nullptr && row0 + lane < k.M)

@@ -131,10 +131,6 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatil
 
 // ---------------------------------------------------------------- TMA
 
-// Asks for the 128-byte line holding `p` to be brought into L2 (a hint: no
-// register is written and nothing waits for it).
-__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
-
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
