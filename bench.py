@@ -45,7 +45,7 @@ FLUSH_BYTES = 256 << 20
 # launch (all 15 products, chained) of a 4096^2 msign call, from the ncu
 # capture summarised in profiles/gemm_sm100_msign4096.md; valid only for the
 # kernel source whose hash is recorded with it.
-NCU_TRAFFIC = {"bytes_per_launch": 1356.996e6, "kernel_sha": "8909252fcb4cced8"}
+NCU_TRAFFIC = {"bytes_per_launch": 1225.08e6, "kernel_sha": "69cfabdded31a602"}
 
 
 def useful_flops(n: int, m: int, steps: int) -> float:
