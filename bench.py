@@ -379,6 +379,10 @@ WORKLOADS = {
     "msign_2048x4096": ("msign", dict(batch=1, rows=2048, cols=4096)),
     "msign_2048x16384": ("msign", dict(batch=1, rows=2048, cols=16384)),
     "muon_llama3_8b_layer": ("muon", dict()),
+    # the automatic route (Gram NS where msign_ns_route picks it)
+    "msign_4x4096x11008_auto": ("msign", dict(batch=4, rows=4096, cols=11008, method="auto")),
+    "msign_1024x16384_auto": ("msign", dict(batch=1, rows=1024, cols=16384, method="auto")),
+    "muon_llama3_8b_layer_auto": ("muon", dict(method="auto")),
 }
 
 
@@ -402,8 +406,10 @@ def run_workload(args):
         out = torch.empty_like(x)
         ws = torch.empty(msb.msign_ns_workspace_size(b, r, c, comp), dtype=torch.uint8, device=dev)
         imp = cfg.get("improved", False)
-        call = lambda: msb.msign_ns(x, out, compute=comp, improved_init=imp, workspace=ws)
-        desc.update(batch=b, rows=r, cols=c, compute=comp, input="momentum-like, bf16", improved_init=imp)
+        meth = cfg.get("method", "standard")
+        call = lambda: msb.msign_ns(x, out, compute=comp, improved_init=imp, method=meth, workspace=ws)
+        desc.update(batch=b, rows=r, cols=c, compute=comp, input="momentum-like, bf16", improved_init=imp,
+                    method=meth, route=msb.msign_ns_route(b, r, c, comp, method=meth, improved_init=imp))
     elif kind == "gram_xxt":
         n = cfg["n"]
         x = synth.gaussian_torch((n, n), seed=3000, device=dev, std=1.0 / n ** 0.5, dtype=torch.bfloat16)
@@ -425,9 +431,11 @@ def run_workload(args):
         G = [synth.gaussian_torch(s_, seed=6000 + i, device=dev, std=1e-4, dtype=torch.bfloat16)
              for i, s_ in enumerate(shapes)]
         ws = torch.empty(msb.muon_step_workspace_size(shapes), dtype=torch.uint8, device=dev)
-        call = lambda: msb.muon_step(W, M, G, momentum=0.95, lr=0.02, workspace=ws)
+        meth = cfg.get("method", "standard")
+        call = lambda: msb.muon_step(W, M, G, momentum=0.95, lr=0.02, method=meth, workspace=ws)
         desc.update(matrices=[list(s_) for s_ in shapes], w="bf16", m="fp32", g="N(0, 1e-4^2) bf16",
-                    momentum=0.95, lr=0.02, note="one Llama-3-8B decoder layer; every call is a further step")
+                    momentum=0.95, lr=0.02, method=meth,
+                    note="one Llama-3-8B decoder layer; every call is a further step")
     for _ in range(args.warmup):
         call()
     msb.sync_status()
@@ -462,6 +470,7 @@ def run_workload(args):
     peaks = measured_peaks()
     pk = peaks["bf16_tflops"] * (0.5 if fp32 else 1.0)  # tf32 runs at half the bf16 rate
     achieved = g["flops"] / (g["ms"] / 1e3) / 1e12 if g["ms"] > 0 else None
+    # useful FLOPs: those of the products that ran (Gram NS's on its route)
     print(json.dumps({
         "workload": args.workload, "metric": "ms per call and useful TFLOP/s", "value": ms, "unit": "ms/call",
         "steps": args.steps, "warmup": args.warmup, "higher_is_better": False,

@@ -81,12 +81,21 @@ typedef enum {
  *      section on improving the initial value (改进初值).  bf16 and fp16
  *      compute only (MSIGN_ERR_UNSUPPORTED with the fp32-accurate path and
  *      with gram_ns).
- * Added in ABI 101; a caller built against ABI 100 has no `init` field. */
+ * method selects the iteration msign_ns and muon_step run (gram_ns takes 0
+ * only):
+ *   0  standard Newton-Schulz, always;
+ *   1  automatic: Gram Newton-Schulz ([P3] Algorithm 2, the page's restart
+ *      after step 2 when T >= 3, fp16 inside, eps as for gram_ns) where it is
+ *      expected to be faster, standard Newton-Schulz elsewhere.
+ *      msign_ns_route() reports the choice for a shape.
+ * Added in ABI 101 (init) and 102 (method); a caller built against an
+ * older ABI lacks the later fields. */
 typedef struct {
   int steps;
   const float *abc;
   float eps;
   int init;
+  int method;
 } msign_coeffs;
 
 /* Library ABI version (major * 100 + minor). */
@@ -152,10 +161,31 @@ msign_status msign_profile_reset(void);
  *                  as two tf32 planes (hi, lo) and each product is
  *                  hi*hi + hi*lo + lo*hi on the tf32 tensor cores with fp32
  *                  accumulation (about 6x the bf16 time).
- *   coeffs         schedule (NULL: Jordan, T = 5, eps = 1e-20)
+ *   coeffs         schedule (NULL: Jordan, T = 5, eps = 1e-20, standard NS);
+ *                  coeffs->method = 1 lets the call run Gram NS instead (see
+ *                  msign_ns_route)
  *   workspace      device scratch of at least msign_ns_workspace_size() bytes
+ *                  (enough for either iteration wherever the route picks it)
  * ------------------------------------------------------------------------ */
 size_t msign_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute_dtype);
+
+/* The iteration msign_ns runs for these arguments: 0 standard NS, 1 Gram NS,
+ * or a negated status for a schedule or dtype msign_ns would reject
+ * (-MSIGN_ERR_INVALID_ARG, -MSIGN_ERR_UNSUPPORTED).  Host only.
+ *
+ * With coeffs->method = 1 the call takes Gram NS when all of these hold:
+ * 16-bit compute (Gram NS iterates in fp16; the fp32-accurate path stays
+ * standard), init = 0 (the sharper normalisation is a standard-NS option),
+ * m - n >= 4096 and n >= 512 after orientation (n <= m), and Gram NS's
+ * workspace is no larger than msign_ns_workspace_size().  [P3] section 2
+ * counts (17 + 3 alpha) n^3 FLOPs for Gram NS against T (3 alpha + 1) n^3
+ * for standard NS with symmetric products, alpha = m / n, so Gram NS does
+ * less work whenever alpha > 1; measured on a B200, its chain of n x n fp16
+ * products pays once m - n reaches about 4096 (e.g. 4096 x 8192, 2048 x 6144,
+ * 1024 x 6144), and below n = 512 both are latency-bound.  The two results
+ * agree within 2e-2 (relative Frobenius). */
+int msign_ns_route(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute_dtype,
+                   const msign_coeffs *coeffs);
 
 msign_status msign_ns(const void *in, void *out, msign_dtype io_dtype, msign_dtype compute_dtype,
                       int64_t batch, int64_t rows, int64_t cols, const msign_coeffs *coeffs,
@@ -246,6 +276,13 @@ msign_status gram_ns(const void *in, void *out, msign_dtype io_dtype,
  *   W_i <- W_i - lr * sqrt(max(1, rows_i / cols_i)) * O_i
  * Matrices of equal (oriented) shape share grouped launches; all shapes in
  * one call are scheduled together.
+ * With coeffs->method = 1, a matrix for which msign_ns_route(1, rows_i,
+ * cols_i, MSIGN_BF16, coeffs) is 1 runs Gram NS instead, when Gram NS's
+ * workspace plus a bf16 copy of O_i fits in this matrix's standard-route
+ * workspace (4096 x 14336 does, 4096 x 11008 does not): M_i is updated by
+ * its own elementwise pass, O_i = gram_ns(M_i) (restart after step 2 when
+ * T >= 3) is stored in bf16, and W_i is updated from it.  Such matrices run
+ * one at a time after the standard-route groups.
  *
  *   W, M, G     HOST arrays of `num` DEVICE pointers.  W_i in w_dtype
  *               (BF16 or FP32) is updated in place; M_i is fp32 and updated

@@ -82,11 +82,27 @@ def msign_ns_workspace_size(batch: int, rows: int, cols: int, compute: str = "bf
     return int(_lib.lib().msign_ns_workspace_size(batch, rows, cols, _compute_code(compute)))
 
 
-def msign_ns(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, improved_init=False, workspace=None,
-             stream=None):
+_METHODS = {"standard": 0, "auto": 1}
+
+
+def msign_ns_route(batch: int, rows: int, cols: int, compute: str = "bf16", *, method: str = "auto", coeffs=None,
+                   improved_init=False) -> str:
+    """The iteration ``msign_ns`` runs for these arguments: "standard" or "gram" (host only)."""
+    c, keep = make_coeffs(coeffs, None, 1 if improved_init else 0, _METHODS[method])
+    r = _lib.lib().msign_ns_route(batch, rows, cols, _compute_code(compute), ctypes.byref(c) if c is not None else None)
+    del keep
+    if r < 0:
+        check(-r, "msign_ns_route")
+    return "gram" if r == 1 else "standard"
+
+
+def msign_ns(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, improved_init=False, method="standard",
+             workspace=None, stream=None):
     """Newton-Schulz msign of the last two dims of ``x`` (bf16/fp16/fp32 CUDA tensor).
 
-    ``improved_init``: the sharper step-0 normalisation (msign_coeffs.init = 1)."""
+    ``improved_init``: the sharper step-0 normalisation (msign_coeffs.init = 1).
+    ``method``: "standard" (standard NS) or "auto" (Gram NS where ``msign_ns_route``
+    picks it, msign_coeffs.method = 1)."""
     torch = _torch()
     _need_cuda(x, "x")
     if x.dim() < 2:
@@ -99,7 +115,7 @@ def msign_ns(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, impro
     if out.shape != x.shape or out.dtype != x.dtype:
         raise ValueError("out must match x in shape and dtype")
     ws, wsb = _workspace(msign_ns_workspace_size(batch, rows, cols, compute), x.device, workspace)
-    c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0)
+    c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0, _METHODS[method])
     st = _lib.lib().msign_ns(x.data_ptr(), out.data_ptr(), _dtype_code(x), _compute_code(compute), batch, rows,
                              cols, ctypes.byref(c) if c is not None else None, _ptr(ws), wsb, _stream(stream))
     del keep
@@ -177,8 +193,11 @@ def muon_step_workspace_size(shapes) -> int:
 
 
 def muon_step(weights, momenta, grads, *, momentum: float = 0.95, lr: float = 0.02, coeffs=None, eps=None,
-              improved_init=False, workspace=None, stream=None):
-    """In-place Muon update of lists of weights (bf16/fp32), fp32 momenta and grads (bf16/fp32)."""
+              improved_init=False, method="standard", workspace=None, stream=None):
+    """In-place Muon update of lists of weights (bf16/fp32), fp32 momenta and grads (bf16/fp32).
+
+    ``method="auto"``: matrices the msign route gives to Gram NS take it here too
+    (msign_coeffs.method = 1; see ``msign_ns_route``)."""
     torch = _torch()
     num = len(weights)
     if not (len(momenta) == num and len(grads) == num):
@@ -203,7 +222,7 @@ def muon_step(weights, momenta, grads, *, momentum: float = 0.95, lr: float = 0.
     G = (ctypes.c_void_p * num)(*[g.data_ptr() for g in grads])
     rows = _i64_array([s[0] for s in shapes])
     cols = _i64_array([s[1] for s in shapes])
-    c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0)
+    c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0, _METHODS[method])
     st = _lib.lib().muon_step(num, W, M, G, rows, cols, wdt.pop(), gdt.pop(), float(momentum), float(lr),
                               ctypes.byref(c) if c is not None else None, _ptr(ws), wsb, _stream(stream))
     del keep

@@ -19,7 +19,7 @@ BF16, FP16, FP32 = 0, 1, 2
 
 EXPORTS = (
     "msign_abi_version", "msign_status_string", "msign_sync_status",
-    "msign_ns_workspace_size", "msign_ns",
+    "msign_ns_workspace_size", "msign_ns", "msign_ns_route",
     "gram_xxt_workspace_size", "gram_xxt",
     "gram_ns_workspace_size", "gram_ns",
     "muon_step_workspace_size", "muon_step",
@@ -31,7 +31,7 @@ EXPORTS = (
 
 class MsignCoeffs(ctypes.Structure):
     _fields_ = [("steps", ctypes.c_int), ("abc", ctypes.POINTER(ctypes.c_float)), ("eps", ctypes.c_float),
-                ("init", ctypes.c_int)]
+                ("init", ctypes.c_int), ("method", ctypes.c_int)]
 
 
 class MsignError(RuntimeError):
@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
         L.msign_ns_workspace_size.argtypes = [I64, I64, I64, I32]
         L.msign_ns.restype = I32
         L.msign_ns.argtypes = [P, P, I32, I32, I64, I64, I64, ctypes.POINTER(MsignCoeffs), P, SZ, P]
+        L.msign_ns_route.restype = I32
+        L.msign_ns_route.argtypes = [I64, I64, I64, I32, ctypes.POINTER(MsignCoeffs)]
         L.gram_xxt_workspace_size.restype = SZ
         L.gram_xxt_workspace_size.argtypes = [I64, I64, I64, I32, P]
         L.gram_xxt.restype = I32
@@ -111,13 +113,14 @@ def check(status: int, what: str) -> None:
         raise MsignError(status, what)
 
 
-def make_coeffs(schedule=None, eps=None, init=0):
+def make_coeffs(schedule=None, eps=None, init=0, method=0):
     """(MsignCoeffs, keep-alive buffer) for a list of (a, b, c) triples."""
-    if schedule is None and eps is None and not init:
+    if schedule is None and eps is None and not init and not method:
         return None, None
     c = MsignCoeffs()
     c.eps = -1.0 if eps is None else float(eps)
     c.init = int(init)
+    c.method = int(method)
     if schedule is None:
         c.steps = 0
         c.abc = None

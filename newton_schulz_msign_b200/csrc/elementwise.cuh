@@ -14,6 +14,8 @@
 //                          norm (s from the unscaled copy) and the Muon
 //                          momentum update (see "ingest" below).
 //   apply_update_kernel    W <- W - lr * scale * O^(T) with the oriented O.
+//   momentum_kernel,       the Muon momentum and update for a matrix whose
+//   update_rows_kernel     msign runs as Gram NS (O stored like W).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -483,6 +485,29 @@ __global__ void __launch_bounds__(256) apply_update_kernel(void* W, int w_dt, in
       store_elem(p, w_dt, load_elem(p, w_dt) - coef * o[k]);
     }
   }
+}
+
+// M <- mu M + G, elementwise over n fp32 values (G in g_dt): the Muon
+// momentum of a matrix whose msign runs as Gram NS.  The same fused
+// multiply-add as the standard route's ingest.
+__global__ void __launch_bounds__(256) momentum_kernel(float* M, const void* G, int g_dt, float mu, long long n) {
+  const char* g = static_cast<const char*>(G);
+  const int es = dtype_size(g_dt);
+  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * 256)
+    M[i] = fmaf(mu, M[i], load_elem(g + i * es, g_dt));
+}
+
+// W <- W - coef * O, elementwise over n values, O (o_dt) stored like W
+// (w_dt); the same arithmetic as apply_update_kernel.
+__global__ void __launch_bounds__(256) update_rows_kernel(void* W, int w_dt, const void* O, int o_dt, float coef,
+                                                          long long n) {
+  char* w = static_cast<char*>(W);
+  const char* o = static_cast<const char*>(O);
+  const int ew = dtype_size(w_dt), eo = dtype_size(o_dt);
+  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * 256)
+    store_elem(w + i * ew, w_dt, load_elem(w + i * ew, w_dt) - coef * load_elem(o + i * eo, o_dt));
 }
 
 }  // namespace msb

@@ -173,7 +173,8 @@ struct Carver {
 struct Schedule {
   std::vector<float> abc;
   float eps;
-  int init = 0;  // 1: sharper step-0 normalisation (msign_coeffs.init)
+  int init = 0;    // 1: sharper step-0 normalisation (msign_coeffs.init)
+  int method = 0;  // 1: msign_ns may run Gram NS (msign_coeffs.method)
   int steps() const { return static_cast<int>(abc.size() / 3); }
 };
 
@@ -193,6 +194,8 @@ msign_status read_schedule(const msign_coeffs* c, float default_eps, Schedule* s
     if (!std::isfinite(eps)) return MSIGN_ERR_INVALID_ARG;
     if (c->init != 0 && c->init != 1) return MSIGN_ERR_INVALID_ARG;
     s->init = c->init;
+    if (c->method != 0 && c->method != 1) return MSIGN_ERR_INVALID_ARG;
+    s->method = c->method;
   }
   if (T > kMaxSteps) return MSIGN_ERR_UNSUPPORTED;
   s->abc.resize(3 * T);
@@ -875,6 +878,20 @@ struct GramBuffers {
   float* part[kMaxAddends];  // split-K partials of n x n products (blocked fp32)
 };
 
+// K parts of a Gram-NS symmetric product of inner dimension K (see
+// Chain::add_split): only where the triangle tiles leave CTA pairs idle, each
+// part at least 2048 of K (measured: with shorter parts the extra
+// partial-store epilogue costs more than the mainloop saves; 2048 x 16384
+// gains 6%, the n x n products of K = n <= 2048 stay whole).  Planned from
+// the shape alone, like syrk_parts, so the workspace query stays host-only.
+inline int gram_parts(int64_t batch, int64_t n, int64_t K) {
+  const int64_t want = std::min<int64_t>({kMaxAddends + 1,
+                                          std::max<int64_t>(1, kPlanPairs / std::max<int64_t>(1, triangle_tiles(n) * batch)),
+                                          std::max<int64_t>(1, K / 2048)});
+  const int64_t len = round_up(ceil_div(K, want), kBM);
+  return static_cast<int>(std::min<int64_t>(ceil_div(K, len), kMaxAddends + 1));
+}
+
 void carve_gram(Carver& cv, int64_t batch, int64_t n, int64_t m, GramBuffers* b) {
   const int64_t ldm = round_up(m, 8), ldn = round_up(n, 8);
   b->partials = static_cast<float*>(cv.take(sizeof(float) * kNormParts * batch));
@@ -887,7 +904,10 @@ void carve_gram(Carver& cv, int64_t batch, int64_t n, int64_t m, GramBuffers* b)
   b->Q[1] = cv.take(2ull * batch * n * ldn);
   b->RZ = cv.take(2ull * batch * n * ldn);
   b->cnt = static_cast<int*>(cv.take(kSchedBytes + sizeof(int) * kMaxClasses * batch * ceil_div(n, kBM)));
-  for (int q = 0; q < kMaxAddends; ++q) b->part[q] = static_cast<float*>(cv.take(4ull * batch * blk_size(n, n)));
+  // fp32 partials for the split products: K is m (X X^T) or n (n x n)
+  const int parts = std::max(gram_parts(batch, n, m), gram_parts(batch, n, n));
+  for (int q = 0; q < kMaxAddends; ++q)
+    b->part[q] = q + 1 < parts ? static_cast<float*>(cv.take(4ull * batch * blk_size(n, n))) : nullptr;
 }
 
 // Classes of one chained launch whose dependencies are derived from the
@@ -1063,9 +1083,31 @@ using namespace msb;
 
 // ================================================================ C ABI
 
+// msign_ns's automatic route (msign_coeffs.method = 1): Gram NS where it is
+// expected to beat standard NS.  Measured on a B200 (default schedules, time
+// of Gram NS over standard NS): 0.86 at 4096 x 8192, 0.71 at 4096 x 14336,
+// 0.91 at 2048 x 6144, 0.92 at 1024 x 6144, 0.75 at 1024 x 16384, 0.92 at
+// 512 x 8192, all with m - n >= 4096; 1.04 at 1024 x 4096, 1.05 at
+// 2048 x 4096, 0.98 at 512 x 4096, 0.99 at 256 x 4096, 1.13 at 256 x 2048,
+// all below it.  Gram NS saves FLOPs in proportion to m - n (it touches the
+// n x m operand only in its first and last products), while its n x n chain
+// costs latency that only large problems hide.  Only shapes whose Gram-NS
+// workspace fits in msign_ns's qualify, so the workspace query stays the
+// same for both routes.
+constexpr int64_t kGramMinExcess = 4096;  // m - n
+constexpr int64_t kGramMinRows = 512;     // n
+
+bool gram_route(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute, const Schedule& sch) {
+  if (sch.method != 1 || compute == MSIGN_FP32 || sch.init != 0) return false;
+  if (batch <= 0 || rows <= 0 || cols <= 0) return false;
+  const int64_t n = std::min(rows, cols), m = std::max(rows, cols);
+  if (n < kGramMinRows || m - n < kGramMinExcess) return false;
+  return gram_ns_workspace_size(batch, rows, cols) <= msign_ns_workspace_size(batch, rows, cols, compute);
+}
+
 extern "C" {
 
-int msign_abi_version(void) { return 101; }
+int msign_abi_version(void) { return 102; }
 
 const char* msign_status_string(msign_status s) {
   switch (s) {
@@ -1149,6 +1191,15 @@ size_t msign_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols, msign_
   return cv.off + 1024;
 }
 
+int msign_ns_route(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute_dtype, const msign_coeffs* coeffs) {
+  if (!valid_dtype(compute_dtype) || batch < 0 || rows < 0 || cols < 0) return -MSIGN_ERR_INVALID_ARG;
+  Schedule sch;
+  const msign_status st = read_schedule(coeffs, kNsEps, &sch);
+  if (st != MSIGN_OK) return -static_cast<int>(st);
+  if (sch.init != 0 && compute_dtype == MSIGN_FP32) return -MSIGN_ERR_UNSUPPORTED;
+  return gram_route(batch, rows, cols, compute_dtype, sch) ? 1 : 0;
+}
+
 msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dtype compute_dtype, int64_t batch,
                       int64_t rows, int64_t cols, const msign_coeffs* coeffs, void* workspace,
                       size_t workspace_bytes, msign_stream_t stream_) {
@@ -1164,6 +1215,16 @@ msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dty
   const size_t need = msign_ns_workspace_size(batch, rows, cols, compute_dtype);
   if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
     return MSIGN_ERR_WORKSPACE;
+  if (gram_route(batch, rows, cols, compute_dtype, sch)) {
+    // Gram NS with the same schedule, Gram NS's eps unless one was given,
+    // and the page's restart after step 2 where the schedule has one
+    msign_coeffs g = {};
+    g.steps = sch.steps();
+    g.abc = sch.abc.data();
+    g.eps = (coeffs != nullptr && coeffs->eps >= 0.0f) ? coeffs->eps : -1.0f;
+    return gram_ns(in, out, io_dtype, batch, rows, cols, &g, nullptr, sch.steps() >= 3 ? -1 : 0, workspace,
+                   workspace_bytes, stream_);
+  }
   DeviceState* dev = nullptr;
   st = device_state(&dev);
   if (st != MSIGN_OK) return st;
@@ -1265,34 +1326,17 @@ size_t gram_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols) {
   return cv.off + 1024;
 }
 
-msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t batch, int64_t rows, int64_t cols,
-                     const msign_coeffs* coeffs, const int* restart_after, int n_restart, void* workspace,
-                     size_t workspace_bytes, msign_stream_t stream_) {
-  if (!valid_dtype(io_dtype)) return MSIGN_ERR_INVALID_ARG;
-  if (batch < 0 || rows < 0 || cols < 0) return MSIGN_ERR_INVALID_ARG;
-  Schedule sch;
-  msign_status st = read_schedule(coeffs, kGramEps, &sch);
-  if (st != MSIGN_OK) return st;
-  if (sch.init != 0) return MSIGN_ERR_UNSUPPORTED;  // the sharper normalisation is a standard-NS option
-  const int T = sch.steps();
-  std::vector<int> bounds;
-  st = gram_segments(T, restart_after, n_restart, &bounds);
-  if (st != MSIGN_OK) return st;
-  if (batch == 0 || rows == 0 || cols == 0) return MSIGN_OK;
-  if (in == nullptr || out == nullptr) return MSIGN_ERR_INVALID_ARG;
-  if (batch > 65535 || rows > (1 << 30) || cols > (1 << 30)) return MSIGN_ERR_UNSUPPORTED;
-  const size_t need = gram_ns_workspace_size(batch, rows, cols);
-  if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
-    return MSIGN_ERR_WORKSPACE;
-  DeviceState* dev = nullptr;
-  st = device_state(&dev);
-  if (st != MSIGN_OK) return st;
+}  // extern "C"
 
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+// Gram NS on validated arguments: `in` (in_dt) -> `out` (out_dt), the
+// segment bounds of the restart schedule, a workspace of at least
+// gram_ns_workspace_size() bytes.  [P3] Algorithm 2.
+msign_status gram_run(const void* in, int in_dt, void* out, int out_dt, int64_t batch, int64_t rows, int64_t cols,
+                      const Schedule& sch, const std::vector<int>& bounds, void* workspace, cudaStream_t stream) {
+  msign_status st = MSIGN_OK;
   const bool tr = rows > cols;
   const int64_t n = tr ? cols : rows, m = tr ? rows : cols;
   const int64_t ldm = round_up(m, 8), ldn = round_up(n, 8);
-  const int io = to_dt(io_dtype);
   Carver cv(workspace);
   GramBuffers w;
   carve_gram(cv, batch, n, m, &w);
@@ -1302,10 +1346,10 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
   auto sqm = [&](void* p) { return Mat{p, DT_FP16, n, n, ldn, sq}; };
 
   // [P3] Algorithm 2 steps 1-2: X <- X / (||X||_F + eps); X <- float16(X)
-  st = launch_norm(in, io, rows * cols, batch, DT_FP32, sch.eps, 1, w.partials, w.scale, stream);
+  st = launch_norm(in, in_dt, rows * cols, batch, DT_FP32, sch.eps, 1, w.partials, w.scale, stream);
   if (st != MSIGN_OK) return st;
   {
-    IngestArgs a = ingest_args(in, io, rows, cols, tr, DT_FP32, w.P[0], DT_FP16, ldm, rect);
+    IngestArgs a = ingest_args(in, in_dt, rows, cols, tr, DT_FP32, w.P[0], DT_FP16, ldm, rect);
     a.pre_scale = w.scale;
     st = launch_ingest(a, batch, stream);
   }
@@ -1316,16 +1360,8 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
   Chain ch;
   ch.state = w.cnt, ch.batch = batch, ch.rows = ceil_div(n, kBM), ch.ab_dt = DT_FP16, ch.stream = stream;
   const int DEP_TMN = DEP_TM | DEP_TN;
-  // split K for the symmetric products when their tiles leave CTA pairs idle
-  // and K is long: each part keeps at least 2048 of K (measured: with shorter
-  // parts the extra partial-store epilogue costs more than the mainloop saves;
-  // 2048 x 16384 gains 6%, the n x n products of K = n <= 2048 stay whole)
-  const int64_t sym_tiles = triangle_tiles(n) * batch;
-  auto parts_for = [&](int64_t K) {
-    return static_cast<int>(std::min<int64_t>(
-        {kMaxAddends + 1, std::max<int64_t>(1, dev->max_pairs / std::max<int64_t>(sym_tiles, 1)),
-         std::max<int64_t>(1, K / 2048)}));
-  };
+  // split K for the symmetric products with few tiles and a long K
+  auto parts_for = [&](int64_t K) { return gram_parts(batch, n, K); };
   auto add_sym = [&](const ClassSpec& s, const std::vector<std::pair<const void*, int>>& reads, const void* c_buf,
                      const std::vector<const void*>& writes) {
     return ch.add_split(s, parts_for(s.K), reads, c_buf, writes, w.part, blk_ld(n), blk_size(n, n));
@@ -1401,7 +1437,7 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
       s.M = n, s.N = m, s.K = n, s.batch = batch;
       void* dst = (seg + 2 == bounds.size()) ? out : w.P[cur ^ 1];
       if (seg + 2 == bounds.size())
-        s.outs = {out_to(out, io, cols, rows * cols, tr)};
+        s.outs = {out_to(out, out_dt, cols, rows * cols, tr)};
       else
         s.outs = {out_to(w.P[cur ^ 1], DT_FP16, ldm, rect, false)};
       st = ch.add(s, {{w.Q[q], DEP_TM}, {w.P[cur], DEP_ALL}}, nullptr, {dst});
@@ -1410,6 +1446,37 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
     cur ^= 1;
   }
   return ch.flush();
+}
+
+extern "C" {
+
+msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t batch, int64_t rows, int64_t cols,
+                     const msign_coeffs* coeffs, const int* restart_after, int n_restart, void* workspace,
+                     size_t workspace_bytes, msign_stream_t stream_) {
+  if (!valid_dtype(io_dtype)) return MSIGN_ERR_INVALID_ARG;
+  if (batch < 0 || rows < 0 || cols < 0) return MSIGN_ERR_INVALID_ARG;
+  Schedule sch;
+  msign_status st = read_schedule(coeffs, kGramEps, &sch);
+  if (st != MSIGN_OK) return st;
+  if (sch.init != 0) return MSIGN_ERR_UNSUPPORTED;  // the sharper normalisation is a standard-NS option
+  if (sch.method != 0) return MSIGN_ERR_INVALID_ARG;  // a route choice is msign_ns's
+  const int T = sch.steps();
+  std::vector<int> bounds;
+  st = gram_segments(T, restart_after, n_restart, &bounds);
+  if (st != MSIGN_OK) return st;
+  if (batch == 0 || rows == 0 || cols == 0) return MSIGN_OK;
+  if (in == nullptr || out == nullptr) return MSIGN_ERR_INVALID_ARG;
+  if (batch > 65535 || rows > (1 << 30) || cols > (1 << 30)) return MSIGN_ERR_UNSUPPORTED;
+  const size_t need = gram_ns_workspace_size(batch, rows, cols);
+  if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
+    return MSIGN_ERR_WORKSPACE;
+  DeviceState* dev = nullptr;
+  st = device_state(&dev);
+  if (st != MSIGN_OK) return st;
+
+  const int io = to_dt(io_dtype);
+  return gram_run(in, io, out, io, batch, rows, cols, sch, bounds, workspace,
+                  reinterpret_cast<cudaStream_t>(stream_));
 }
 
 // Workspace of one group of Muon matrices: one NsBuffers set per distinct
@@ -1424,15 +1491,20 @@ static size_t muon_group_bytes(const std::vector<std::pair<int64_t, int64_t>>& s
   return cv.off + 1024;
 }
 
+// The standard-NS classes of matrices begin .. end - 1: one per distinct
+// oriented shape; empty matrices and those marked in `gram` (the Gram-NS
+// route) belong to none.
 static void muon_group_shapes(const int64_t* rows, const int64_t* cols, int begin, int end,
                               std::vector<std::pair<int64_t, int64_t>>* shapes, std::vector<int64_t>* counts,
-                              std::vector<int>* cls_of, std::vector<int64_t>* slot_of) {
+                              std::vector<int>* cls_of, std::vector<int64_t>* slot_of,
+                              const std::vector<char>* gram = nullptr) {
   shapes->clear();
   counts->clear();
   cls_of->assign(end - begin, -1);
   slot_of->assign(end - begin, -1);
   for (int i = begin; i < end; ++i) {
     if (rows[i] == 0 || cols[i] == 0) continue;
+    if (gram != nullptr && (*gram)[i]) continue;
     const std::pair<int64_t, int64_t> sh{std::min(rows[i], cols[i]), std::max(rows[i], cols[i])};
     size_t c = 0;
     while (c < shapes->size() && (*shapes)[c] != sh) ++c;
@@ -1443,6 +1515,15 @@ static void muon_group_shapes(const int64_t* rows, const int64_t* cols, int begi
     (*cls_of)[i - begin] = static_cast<int>(c);
     (*slot_of)[i - begin] = (*counts)[c]++;
   }
+}
+
+// Workspace of one Muon matrix on the Gram-NS route: Gram NS's own, then O
+// in bf16, stored like W.
+static size_t muon_gram_o_offset(int64_t rows, int64_t cols) {
+  return static_cast<size_t>(round_up(static_cast<int64_t>(gram_ns_workspace_size(1, rows, cols)), 256));
+}
+static size_t muon_gram_bytes(int64_t rows, int64_t cols) {
+  return muon_gram_o_offset(rows, cols) + static_cast<size_t>(2 * rows * cols);
 }
 
 size_t muon_step_workspace_size(int num, const int64_t* rows, const int64_t* cols) {
@@ -1485,6 +1566,26 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   const int wd = to_dt(w_dtype), gd = to_dt(g_dtype);
 
+  // msign_coeffs.method = 1: matrices that msign_ns's route would give to
+  // Gram NS take it here too, when Gram NS's workspace and a bf16 O fit in
+  // the standard route's workspace for the same matrix (so the workspace
+  // query is the same for both routes)
+  std::vector<char> gram(num, 0);
+  Schedule gsch;
+  std::vector<int> gbounds;
+  if (sch.method == 1) {
+    for (int i = 0; i < num; ++i) {
+      if (rows[i] == 0 || cols[i] == 0 || !gram_route(1, rows[i], cols[i], MSIGN_BF16, sch)) continue;
+      const std::pair<int64_t, int64_t> sh{std::min(rows[i], cols[i]), std::max(rows[i], cols[i])};
+      gram[i] = muon_gram_bytes(rows[i], cols[i]) <= muon_group_bytes({sh}, {1}) ? 1 : 0;
+    }
+    gsch.abc = sch.abc;
+    gsch.eps = (coeffs != nullptr && coeffs->eps >= 0.0f) ? coeffs->eps : kGramEps;
+    st = gram_segments(gsch.steps(), nullptr, gsch.steps() >= 3 ? -1 : 0, &gbounds);
+    if (st != MSIGN_OK) return st;
+  }
+  const unsigned ew_grid = static_cast<unsigned>(std::max(1, dev->sms) * 8);
+
   int begin = 0;
   while (begin < num) {
     // the longest prefix of the remaining list whose workspace fits
@@ -1493,12 +1594,37 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
     std::vector<int64_t> counts, slots;
     std::vector<int> cls;
     while (end < num) {
-      muon_group_shapes(rows, cols, begin, end + 1, &shapes, &counts, &cls, &slots);
+      muon_group_shapes(rows, cols, begin, end + 1, &shapes, &counts, &cls, &slots, &gram);
       if (muon_group_bytes(shapes, counts) > workspace_bytes) break;
       ++end;
     }
-    muon_group_shapes(rows, cols, begin, end, &shapes, &counts, &cls, &slots);
+    muon_group_shapes(rows, cols, begin, end, &shapes, &counts, &cls, &slots, &gram);
+    // the Gram-NS matrices of this range, one at a time, after the group
+    auto run_gram = [&]() -> msign_status {
+      for (int i = begin; i < end; ++i) {
+        if (!gram[i]) continue;
+        const int64_t ne = rows[i] * cols[i];
+        const unsigned g = static_cast<unsigned>(std::min<int64_t>(ceil_div(ne, 256), ew_grid));
+        prof_begin(stream);
+        momentum_kernel<<<g, 256, 0, stream>>>(M[i], G[i], gd, momentum, ne);
+        prof_end(3, stream, 0.0, static_cast<double>(ne) * (8 + dtype_size(gd)));
+        msign_status r = launch_ok();
+        if (r != MSIGN_OK) return r;
+        void* o = static_cast<char*>(workspace) + muon_gram_o_offset(rows[i], cols[i]);
+        r = gram_run(M[i], DT_FP32, o, DT_BF16, 1, rows[i], cols[i], gsch, gbounds, workspace, stream);
+        if (r != MSIGN_OK) return r;
+        const float coef = lr * std::sqrt(std::max(1.0f, static_cast<float>(rows[i]) / static_cast<float>(cols[i])));
+        prof_begin(stream);
+        update_rows_kernel<<<g, 256, 0, stream>>>(W[i], wd, o, DT_BF16, coef, ne);
+        prof_end(3, stream, 0.0, static_cast<double>(ne) * (2 + 2 * dtype_size(wd)));
+        r = launch_ok();
+        if (r != MSIGN_OK) return r;
+      }
+      return MSIGN_OK;
+    };
     if (shapes.empty()) {
+      st = run_gram();
+      if (st != MSIGN_OK) return st;
       begin = end;
       continue;
     }
@@ -1552,6 +1678,8 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
       st = launch_ok();
       if (st != MSIGN_OK) return st;
     }
+    st = run_gram();
+    if (st != MSIGN_OK) return st;
     begin = end;
   }
   return MSIGN_OK;

@@ -45,7 +45,7 @@ def test_exported_symbols_match_nm(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.msign_abi_version() == 101
+    assert L.msign_abi_version() == 102
     assert L.msign_status_string(_lib.OK) == b"ok"
     assert b"timed out" in L.msign_status_string(_lib.ERR_TIMEOUT)
     assert L.msign_status_string(99) == b"unknown status"
@@ -104,6 +104,71 @@ def test_init_option_validation(L):
     assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, ctypes.byref(c), None, 0, None, 0, None) == _lib.ERR_UNSUPPORTED
     # bf16 with init = 1 passes the argument checks (fails only on the missing workspace)
     assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == _lib.ERR_WORKSPACE
+
+
+def _route(L, batch, rows, cols, compute=_lib.BF16, method=1, init=0, steps=0):
+    c = _lib.MsignCoeffs()
+    c.steps, c.abc, c.eps, c.init, c.method = steps, None, -1.0, init, method
+    return L.msign_ns_route(batch, rows, cols, compute, ctypes.byref(c))
+
+
+def test_route_rule(L):
+    # the automatic route takes Gram NS only for 16-bit problems with
+    # n >= 512 and m - n >= 4096, in either orientation, whose Gram-NS
+    # workspace fits in msign_ns's
+    assert _route(L, 1, 1024, 16384) == 1
+    assert _route(L, 1, 16384, 1024) == 1
+    assert _route(L, 3, 512, 4608) == 1
+    assert _route(L, 1, 4096, 8192) == 1
+    assert _route(L, 4, 4096, 11008) == 1
+    assert _route(L, 1, 14336, 4096) == 1
+    assert _route(L, 1, 1024, 16384, compute=_lib.FP16) == 1
+    assert _route(L, 1, 1024, 5119) == 0    # m - n < 4096
+    assert _route(L, 1, 1024, 4096) == 0
+    assert _route(L, 1, 2048, 4096) == 0
+    assert _route(L, 1, 511, 8192) == 0     # n < 512
+    assert _route(L, 1, 4096, 4096) == 0
+    assert _route(L, 1, 1024, 16384, compute=_lib.FP32) == 0   # fp32-accurate stays standard
+    assert _route(L, 1, 1024, 16384, init=1) == 0              # sharper init is standard-only
+    assert _route(L, 1, 1024, 16384, method=0) == 0
+    assert L.msign_ns_route(1, 1024, 16384, _lib.BF16, None) == 0  # NULL coeffs: standard
+    # arguments msign_ns rejects come back negated
+    assert _route(L, 1, 1024, 16384, method=2) == -_lib.ERR_INVALID_ARG
+    assert _route(L, 1, 1024, 16384, compute=_lib.FP32, init=1) == -_lib.ERR_UNSUPPORTED
+    assert _route(L, 1, 1024, 16384, steps=100) == -_lib.ERR_UNSUPPORTED
+    assert L.msign_ns_route(-1, 4, 4, _lib.BF16, None) == -_lib.ERR_INVALID_ARG
+
+
+def test_route_workspace_fits(L):
+    # wherever the route picks Gram NS, its workspace fits in msign_ns's
+    # (the one query a caller makes)
+    routed = 0
+    for batch in (1, 2, 8):
+        for n in (512, 640, 1024, 1536, 2048, 3072, 4096, 8192, 16384):
+            for m in (n + 4096, n + 5000, 2 * n, 3 * n, 4 * n, 8 * n, 16 * n):
+                if _route(L, batch, n, m) == 1:
+                    routed += 1
+                    assert L.gram_ns_workspace_size(batch, n, m) <= L.msign_ns_workspace_size(batch, n, m, _lib.BF16)
+    assert routed > 100
+
+
+def test_method_field_validation(L):
+    c = _lib.MsignCoeffs()
+    c.steps, c.abc, c.eps, c.init, c.method = 0, None, -1.0, 0, 1
+    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, ctypes.byref(c), None, -1, 16, 1 << 20, None) == \
+        _lib.ERR_INVALID_ARG
+    one = (ctypes.c_void_p * 1)(16)
+    rows = (ctypes.c_int64 * 1)(8)
+    cols = (ctypes.c_int64 * 1)(8)
+    # muon_step takes the route too: these arguments pass the checks and
+    # fail only on the missing workspace
+    assert L.muon_step(1, one, one, one, rows, cols, _lib.BF16, _lib.BF16, 0.95, 0.02, ctypes.byref(c), None, 0,
+                       None) == _lib.ERR_WORKSPACE
+    c.method = 3
+    assert L.muon_step(1, one, one, one, rows, cols, _lib.BF16, _lib.BF16, 0.95, 0.02, ctypes.byref(c), None, 0,
+                       None) == _lib.ERR_INVALID_ARG
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == \
+        _lib.ERR_INVALID_ARG
 
 
 def test_selftest_timeout_validation(L):

@@ -136,3 +136,35 @@ def test_muon_improved_init():
         O_ref = O.msign_ns_improved_init(Mr, input_cast="bf16")
         dW_ref = -0.02 * math.sqrt(max(1.0, r / c)) * O_ref
         assert rel_fro(to_np(W[i]) - to_np(W0[i]), dW_ref) < TOL_BF16
+
+
+def test_muon_auto_route_mixed():
+    # method="auto": the wide matrices (m - n >= 4096, n >= 512) run Gram NS,
+    # the others standard NS, in one call; each against its fp64 oracle
+    shapes = [(600, 5000), (256, 384), (5000, 600), (512, 512)]
+    gram_shapes = {(600, 5000), (5000, 600)}
+    for r, c in shapes:
+        want = "gram" if (r, c) in gram_shapes else "standard"
+        assert msb.msign_ns_route(1, r, c, method="auto") == want
+    W, M, G = make(shapes, torch.bfloat16, torch.bfloat16, seed=900)
+    W0 = [w.clone() for w in W]
+    M0 = [m.clone() for m in M]
+    msb.muon_step(W, M, G, momentum=0.95, lr=0.02, method="auto")
+    msb.sync_status()
+    for i, (r, c) in enumerate(shapes):
+        if (r, c) not in gram_shapes:
+            check_matrix(W0[i], M0[i], G[i], W[i], M[i], 0.02)
+            continue
+        m_ref = 0.95 * to_np(M0[i]).astype(np.float64) + to_np(G[i]).astype(np.float64)
+        assert rel_fro(to_np(M[i]), m_ref) < 1e-6
+        # O from Gram NS of the fp32 momentum (fp16 inside), as the GPU gets it
+        o_ref = O.gram_ns(to_np(M[i]))
+        w_ref = to_np(W0[i]) - 0.02 * math.sqrt(max(1.0, r / c)) * o_ref
+        dW_ref = w_ref - to_np(W0[i])
+        w1 = to_np(W[i])
+        half_ulp = np.ldexp(1.0, np.frexp(np.abs(w1))[1] - 9)
+        excess = np.maximum(np.abs(w1 - w_ref) - half_ulp, 0.0)
+        assert np.linalg.norm(excess) <= TOL_BF16 * np.linalg.norm(dW_ref)
+        # and the standard-NS update agrees within the same tolerance
+        w_std, _, _ = O.muon_step(to_np(W0[i]), to_np(M0[i]), to_np(G[i]), momentum=0.95, lr=0.02, input_cast="bf16")
+        assert rel_fro(w_ref - to_np(W0[i]), w_std - to_np(W0[i])) < TOL_BF16
