@@ -218,9 +218,9 @@ def test_improved_init_full_size():
 
 # ---------------------------------------------------------------- automatic route (msign_coeffs.method = 1)
 
-@pytest.mark.parametrize("shape", [(600, 5000), (5000, 600), (2, 512, 4096)])
+@pytest.mark.parametrize("shape", [(600, 5000), (5000, 600), (2, 512, 4608)])
 def test_auto_route_runs_gram_ns(shape):
-    # wide enough for the route: the call is Gram NS with its defaults
+    # wide enough for the route (m - n >= 4096): the call is Gram NS with its defaults
     x = torch.from_numpy(synth.gaussian(shape, seed=shape[-1] + 3 * shape[-2])).to(torch.bfloat16).cuda()
     batch = x.numel() // (shape[-2] * shape[-1])
     assert msb.msign_ns_route(batch, shape[-2], shape[-1], method="auto") == "gram"
@@ -235,7 +235,7 @@ def test_auto_route_runs_gram_ns(shape):
 
 def test_auto_route_short_schedule_has_no_restart():
     # two steps leave no room for the restart after step 2
-    x = torch.from_numpy(synth.gaussian((512, 4096), seed=31)).to(torch.bfloat16).cuda()
+    x = torch.from_numpy(synth.gaussian((512, 4608), seed=31)).to(torch.bfloat16).cuda()
     coeffs = [(3.4445, -4.7750, 2.0315)] * 2
     y = msb.msign_ns(x, coeffs=coeffs, method="auto")
     g = msb.gram_ns(x, coeffs=coeffs, restart_after=())
@@ -244,7 +244,7 @@ def test_auto_route_short_schedule_has_no_restart():
     assert rel_fro(to_np(y), O.gram_ns(to_np(x), coeffs, restart_after=())) < TOL_BF16
 
 
-@pytest.mark.parametrize("shape,compute", [((512, 1024), "bf16"), ((1024, 16384), "fp32")])
+@pytest.mark.parametrize("shape,compute", [((512, 1024), "bf16"), ((512, 4096), "bf16"), ((1024, 16384), "fp32")])
 def test_auto_route_keeps_standard_ns(shape, compute):
     # not wide enough, or the fp32-accurate path: the call is standard NS
     x = torch.from_numpy(synth.gaussian(shape, seed=41)).to(torch.bfloat16).cuda()

@@ -66,13 +66,14 @@ def test_noalloc_rejects_problems_beyond_the_builtin_scratch():
 def test_noalloc_follows_the_automatic_route():
     # msign_coeffs.method = 1 through the no-allocation entry point: a shape
     # the route sends to Gram NS fits the built-in scratch too
-    x = torch.from_numpy(synth.gaussian((512, 4096), seed=73)).to(torch.bfloat16).cuda()
+    x = torch.from_numpy(synth.gaussian((512, 4608), seed=73)).to(torch.bfloat16).cuda()
+    assert msb.msign_ns_route(1, 512, 4608, method="auto") == "gram"
     ref = msb.msign_ns(x, method="auto")
     out = torch.empty_like(x)
     c = _lib.MsignCoeffs()
     c.steps, c.abc, c.eps, c.init, c.method = 0, None, -1.0, 0, 1
     L = _lib.lib()
     stream = torch.cuda.current_stream().cuda_stream
-    assert L.msign_ns_noalloc(x.data_ptr(), out.data_ptr(), _lib.BF16, 1, 512, 4096, c, stream) == _lib.OK
+    assert L.msign_ns_noalloc(x.data_ptr(), out.data_ptr(), _lib.BF16, 1, 512, 4608, c, stream) == _lib.OK
     msb.sync_status()
     assert torch.equal(out, ref)
