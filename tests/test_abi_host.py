@@ -203,3 +203,17 @@ def test_binding_refuses_cpu_tensors():
     import newton_schulz_msign_b200 as msb
     with pytest.raises(ValueError, match="CUDA"):
         msb.msign_ns(torch.zeros(4, 4))
+
+
+def test_binding_route_query():
+    # the Python binding's route query is host-only as well
+    import newton_schulz_msign_b200 as msb
+    build.build()
+    assert msb.msign_ns_route(1, 1024, 16384) == "gram"
+    assert msb.msign_ns_route(1, 1024, 16384, method="standard") == "standard"
+    assert msb.msign_ns_route(1, 1024, 16384, "fp32") == "standard"
+    assert msb.msign_ns_route(1, 1024, 16384, improved_init=True) == "standard"
+    assert msb.msign_ns_route(4, 4096, 11008) == "gram"
+    assert msb.msign_ns_route(8, 4096, 4096) == "standard"
+    with pytest.raises(msb.MsignError):
+        msb.msign_ns_route(1, 1024, 16384, coeffs=[(1.0, 0.0, 0.0)] * 100)
