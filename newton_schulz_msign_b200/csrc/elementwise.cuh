@@ -487,27 +487,71 @@ __global__ void __launch_bounds__(256) apply_update_kernel(void* W, int w_dt, in
   }
 }
 
+// Stores cnt <= 8 consecutive values in dt (16-byte stores when whole and
+// aligned), rounding to nearest even like store_elem.
+__device__ __forceinline__ void store8(char* p, int dt, int cnt, const float* v) {
+  if (cnt == 8 && (reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+    if (dt == DT_FP32) {
+      reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+      reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+      uint32_t w[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint32_t lo = dt == DT_BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(v[2 * t]))
+                                          : __half_as_ushort(__float2half_rn(v[2 * t]));
+        const uint32_t hi = dt == DT_BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(v[2 * t + 1]))
+                                          : __half_as_ushort(__float2half_rn(v[2 * t + 1]));
+        w[t] = lo | (hi << 16);
+      }
+      *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return;
+  }
+  const int es = dtype_size(dt);
+  for (int e = 0; e < cnt; ++e) store_elem(p + e * es, dt, v[e]);
+}
+
 // M <- mu M + G, elementwise over n fp32 values (G in g_dt): the Muon
 // momentum of a matrix whose msign runs as Gram NS.  The same fused
-// multiply-add as the standard route's ingest.
+// multiply-add as the standard route's ingest; 8 values per thread step.
 __global__ void __launch_bounds__(256) momentum_kernel(float* M, const void* G, int g_dt, float mu, long long n) {
   const char* g = static_cast<const char*>(G);
   const int es = dtype_size(g_dt);
-  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * 256)
-    M[i] = fmaf(mu, M[i], load_elem(g + i * es, g_dt));
+  const long long chunks = (n + 7) / 8;
+  for (long long c = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; c < chunks;
+       c += static_cast<long long>(gridDim.x) * 256) {
+    const long long e = 8 * c;
+    const int cnt = static_cast<int>(n - e < 8 ? n - e : 8);
+    float m[8], gv[8];
+    load8(reinterpret_cast<const char*>(M + e), DT_FP32, cnt, m);
+    load8(g + e * es, g_dt, cnt, gv);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) m[t] = fmaf(mu, m[t], gv[t]);
+    store8(reinterpret_cast<char*>(M + e), DT_FP32, cnt, m);
+  }
 }
 
 // W <- W - coef * O, elementwise over n values, O (o_dt) stored like W
-// (w_dt); the same arithmetic as apply_update_kernel.
+// (w_dt); the same arithmetic as apply_update_kernel; 8 values per thread
+// step.
 __global__ void __launch_bounds__(256) update_rows_kernel(void* W, int w_dt, const void* O, int o_dt, float coef,
                                                           long long n) {
   char* w = static_cast<char*>(W);
   const char* o = static_cast<const char*>(O);
   const int ew = dtype_size(w_dt), eo = dtype_size(o_dt);
-  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * 256)
-    store_elem(w + i * ew, w_dt, load_elem(w + i * ew, w_dt) - coef * load_elem(o + i * eo, o_dt));
+  const long long chunks = (n + 7) / 8;
+  for (long long c = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; c < chunks;
+       c += static_cast<long long>(gridDim.x) * 256) {
+    const long long e = 8 * c;
+    const int cnt = static_cast<int>(n - e < 8 ? n - e : 8);
+    float wv[8], ov[8];
+    load8(w + e * ew, w_dt, cnt, wv);
+    load8(o + e * eo, o_dt, cnt, ov);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) wv[t] = wv[t] - coef * ov[t];
+    store8(w + e * ew, w_dt, cnt, wv);
+  }
 }
 
 }  // namespace msb

@@ -1604,7 +1604,7 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
       for (int i = begin; i < end; ++i) {
         if (!gram[i]) continue;
         const int64_t ne = rows[i] * cols[i];
-        const unsigned g = static_cast<unsigned>(std::min<int64_t>(ceil_div(ne, 256), ew_grid));
+        const unsigned g = static_cast<unsigned>(std::min<int64_t>(ceil_div(ne, 8 * 256), ew_grid));
         prof_begin(stream);
         momentum_kernel<<<g, 256, 0, stream>>>(M[i], G[i], gd, momentum, ne);
         prof_end(3, stream, 0.0, static_cast<double>(ne) * (8 + dtype_size(gd)));
