@@ -21,7 +21,7 @@ Sources (cited by page title and section/equation):
   Algorithm 1 (Naive Gram Newton-Schulz, section 2.3), Algorithm 2
   (Stabilized Gram Newton-Schulz, section 3.4), Theorem 1 (section 2.2).
 
-Conventions (readings of the pages, each listed in the design doc):
+Conventions (readings of the pages where they leave a step open):
 
 * Arithmetic is fp64 throughout.  The only roundings are the explicit
   casts the pages prescribe: the input cast to the compute dtype of [P2]
