@@ -359,7 +359,7 @@ def run_ours(args):
 # call, CUDA events on the launching stream, clocks sampled meanwhile).
 # Useful FLOPs come from the library's own launch records (triangle-counted
 # per product), so they match the headline's bookkeeping.  These lines are
-# measurements for the record, not the driver's metric.
+# measurements for the record beside the headline metric.
 
 WORKLOADS = {
     "msign_8x4096": ("msign", dict(batch=8, rows=4096, cols=4096)),
