@@ -147,7 +147,9 @@ msign_status msign_profile_reset(void);
  * t = 1..T:  A = X X^T;  B = b_t A + c_t A A;  X = a_t X + B X;  finally
  * transpose back and write X in io_dtype.
  *
- *   in, out        device pointers, batch x rows x cols in io_dtype
+ *   in, out        device pointers, batch x rows x cols in io_dtype; out may
+ *                  be in (the input is read whole into the workspace before
+ *                  the first store to out)
  *   io_dtype       MSIGN_BF16, MSIGN_FP16 or MSIGN_FP32
  *   compute_dtype  MSIGN_BF16: bf16 tensor-core operands, fp32 accumulation,
  *                  fp32 epilogue arithmetic and an fp32 copy of X between
@@ -255,6 +257,8 @@ msign_status gram_xxt(const void *X, msign_dtype x_dtype, void *A, msign_dtype a
  * triangle schedule; the a_t terms are added in fp32 epilogues.  Operands
  * are fp16, accumulation fp32.
  *
+ *   in, out        device pointers, batch x rows x cols in io_dtype; out may
+ *                  be in, as for msign_ns
  *   restart_after  HOST array of step numbers after which to restart
  *                  (values in 1..T-1); NULL with n_restart < 0 selects the
  *                  page's schedule {2}; n_restart == 0 means no restart.

@@ -82,3 +82,12 @@ def test_gram_ns_wide_full_size(n, m):
     assert np.all(np.isfinite(got))
     assert rel_fro(got, O.gram_ns(X)) < TOL_BF16
     assert rel_fro(got, O.msign_ns(X)) < TOL_BF16
+
+
+def test_gram_ns_in_place():
+    x = torch.from_numpy(synth.gaussian((384, 2048), seed=91)).to(torch.bfloat16).cuda()
+    ref = msb.gram_ns(x)
+    y = x.clone()
+    msb.gram_ns(y, y)
+    msb.sync_status()
+    assert torch.equal(y, ref)

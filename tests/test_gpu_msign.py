@@ -253,3 +253,15 @@ def test_auto_route_keeps_standard_ns(shape, compute):
     b = msb.msign_ns(x, compute=compute)
     msb.sync_status()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("shape,compute,method", [((256, 768), "bf16", "standard"), ((300, 100), "fp16", "standard"),
+                                                  ((200, 600), "fp32", "standard"), ((600, 5000), "bf16", "auto")])
+def test_in_place(shape, compute, method):
+    # out may be in: the input is read whole before the first store to out
+    x = torch.from_numpy(synth.gaussian(shape, seed=shape[0] + 5 * shape[1])).to(torch.bfloat16).cuda()
+    ref = msb.msign_ns(x, compute=compute, method=method)
+    y = x.clone()
+    msb.msign_ns(y, y, compute=compute, method=method)
+    msb.sync_status()
+    assert torch.equal(y, ref)
