@@ -159,11 +159,15 @@ def gram_ns(x, out=None, *, coeffs=None, eps=None, restart_after=(2,), workspace
     """Stabilized Gram Newton-Schulz (fp16 inner iteration) of the last two dims of ``x``."""
     torch = _torch()
     _need_cuda(x, "x")
+    if x.dim() < 2:
+        raise ValueError("x needs at least two dims")
     rows, cols = x.shape[-2], x.shape[-1]
     batch = math.prod(x.shape[:-2])
     if out is None:
         out = torch.empty_like(x)
     _need_cuda(out, "out")
+    if out.shape != x.shape or out.dtype != x.dtype:
+        raise ValueError("out must match x in shape and dtype")
     ws, wsb = _workspace(gram_ns_workspace_size(batch, rows, cols), x.device, workspace)
     c, keep = make_coeffs(coeffs, eps)
     if restart_after is None:
