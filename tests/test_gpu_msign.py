@@ -139,6 +139,19 @@ def test_momentum_like_full_size(rows, cols, batch):
     assert torch.equal(y[0], y[1])
 
 
+def test_headline_configuration():
+    # the timed workload exactly: one 4096 x 4096 momentum-like bf16 matrix
+    # (seed 1000, rank 0), default schedule, caller output and workspace,
+    # checked whole against the fp64 oracle
+    x = synth.momentum_like_torch(4096, 4096, seed=1000, device="cuda").to(torch.bfloat16).contiguous()
+    out = torch.empty_like(x)
+    ws = torch.empty(msb.msign_ns_workspace_size(1, 4096, 4096), dtype=torch.uint8, device="cuda")
+    msb.msign_ns(x, out, workspace=ws)
+    msb.msign_ns(x, out, workspace=ws)  # a second call on the same workspace
+    msb.sync_status()
+    assert rel_fro(to_np(out), O.msign_ns(to_np(x), input_cast="bf16")) < TOL_BF16
+
+
 # ---------------------------------------------------------------- fp16 and fp32 compute
 
 @pytest.mark.parametrize("shape", [(256, 512), (64, 128), (33, 257), (300, 100)])
