@@ -246,6 +246,16 @@ def test_auto_route_runs_gram_ns(shape):
     assert rel_fro(to_np(y), O.msign_ns(X)) < TOL_BF16
 
 
+def test_auto_route_full_size():
+    # n = 4096 on the Gram-NS route (no split products at this size): the
+    # fp16 iteration against fp64 standard NS, the route's acceptance bound
+    x = synth.momentum_like_torch(4096, 8192, seed=81, device="cuda").to(torch.bfloat16)
+    assert msb.msign_ns_route(1, 4096, 8192, method="auto") == "gram"
+    y = msb.msign_ns(x, method="auto")
+    msb.sync_status()
+    assert rel_fro(to_np(y), O.msign_ns(to_np(x))) < TOL_BF16
+
+
 def test_auto_route_short_schedule_has_no_restart():
     # two steps leave no room for the restart after step 2
     x = torch.from_numpy(synth.gaussian((512, 4608), seed=31)).to(torch.bfloat16).cuda()
