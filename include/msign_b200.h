@@ -28,7 +28,8 @@
  * - The caller owns every buffer.  The library allocates nothing: it works
  *   in the caller's workspace, whose size the *_workspace_size() query gives
  *   (a workspace must be 256-byte aligned).  Inputs are never written
- *   unless stated.  Outputs must not overlap inputs or the workspace.
+ *   unless stated.  Outputs must not overlap the workspace, nor an input
+ *   unless the entry point says so (msign_ns and gram_ns accept out == in).
  * - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
  *   the legacy default stream).  Argument checks happen on the host before
  *   anything is enqueued; on any error status nothing has been enqueued,
