@@ -40,6 +40,11 @@
  * - Coefficient schedules are HOST arrays.  NULL selects Jordan's triple
  *   for T = 5 steps ([P2] eq. 7).
  * - Empty problems (batch, rows or cols = 0) are valid and do nothing.
+ * - Entry points run on the CURRENT device (cudaGetDevice) and every pointer
+ *   of a call must belong to it.  The library keeps per-device addresses
+ *   (its device error word, the msign_ns_noalloc scratch) for the life of
+ *   the process: do not use it across a cudaDeviceReset() or any other
+ *   destruction of the device's primary context.
  */
 #ifndef MSIGN_B200_H
 #define MSIGN_B200_H
@@ -198,15 +203,16 @@ msign_status msign_ns(const void *in, void *out, msign_dtype io_dtype, msign_dty
  * msign_ns_noalloc: msign_ns for callers that cannot allocate device memory.
  * The pages have no counterpart of this entry point.
  *
- * Some callers may not call cudaMalloc where they need msign: code being
- * captured into a CUDA graph (an allocation there can synchronise the device
- * and is not captured), plugins hosted by a framework that reserves all GPU
- * memory for its own pool, and loops that forbid allocation after start-up.
- * This variant takes no workspace: it computes exactly what msign_ns does
- * with compute_dtype MSIGN_BF16, in a scratch array built into the library
- * (a file-scope __device__ array of msign_ns_noalloc_max_bytes() = 32 MiB,
- * held on every GPU that loads the library until the process exits).  It
- * makes no device allocation of its own; inputs and outputs are the caller's.
+ * Some callers may not call cudaMalloc where they need msign: plugins hosted
+ * by a framework that reserves all GPU memory for its own pool (an
+ * allocation outside that pool fails or steals from it), and real-time
+ * loops that forbid allocation after start-up (cudaMalloc can synchronise
+ * the device and takes an unbounded time).  This variant takes no
+ * workspace: it computes exactly what msign_ns does with compute_dtype
+ * MSIGN_BF16, in a scratch array built into the library (a file-scope
+ * __device__ array of msign_ns_noalloc_max_bytes() = 32 MiB, held on every
+ * GPU that loads the library until the process exits).  It makes no device
+ * allocation of its own; inputs and outputs are the caller's.
  *
  * - A problem whose msign_ns_workspace_size(batch, rows, cols, MSIGN_BF16)
  *   exceeds the built-in scratch is rejected with MSIGN_ERR_WORKSPACE before
@@ -215,10 +221,11 @@ msign_status msign_ns(const void *in, void *out, msign_dtype io_dtype, msign_dty
  *   (cudaGetSymbolAddress) with the device current; make that first call
  *   before any stream capture that contains later calls.
  * - All calls on a device share the one array and leave their intermediate
- *   results in it; nothing in it needs to start at zero.  Calls whose
- *   executions overlap on the GPU (different streams, or different host
- *   threads without ordering) race on the array and give wrong results:
- *   order them on one stream.
+ *   results in it.  Each call clears the part that must start at zero (its
+ *   schedule and dependency counters) on its stream before use; every other
+ *   part is written before it is read.  Calls whose executions overlap on
+ *   the GPU (different streams, or different host threads without ordering)
+ *   race on the array and give wrong results: order them on one stream.
  * ------------------------------------------------------------------------ */
 size_t msign_ns_noalloc_max_bytes(void);
 

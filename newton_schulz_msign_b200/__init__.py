@@ -44,10 +44,12 @@ def _compute_code(name) -> int:
     return {"bf16": BF16, "fp16": FP16, "fp32": FP32}[name]
 
 
-def _stream(stream) -> int:
+def _stream(stream, device=None) -> int:
+    """The raw cudaStream_t: the given stream, else the current stream of
+    ``device`` (of the current device when None)."""
     torch = _torch()
     if stream is None:
-        return torch.cuda.current_stream().cuda_stream
+        return torch.cuda.current_stream(device).cuda_stream
     return getattr(stream, "cuda_stream", stream)
 
 
@@ -58,8 +60,17 @@ def _need_cuda(t, name):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _same_device(t, device, name):
+    """The C side works on the current device: every tensor of a call must
+    live on the device the call runs on."""
+    if t is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call runs on {device}")
+
+
 def _workspace(nbytes, device, workspace):
     torch = _torch()
+    if workspace is not None:
+        _same_device(workspace, device, "workspace")
     if nbytes == 0:
         return workspace, (0 if workspace is None else workspace.numel() * workspace.element_size())
     if workspace is None:
@@ -71,9 +82,13 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
-def sync_status(stream=None) -> None:
-    """Waits for the stream and raises MsignError if a kernel's bounded wait ran out."""
-    check(_lib.lib().msign_sync_status(_stream(stream)), "msign_sync_status")
+def sync_status(stream=None, device=None) -> None:
+    """Waits for the stream (default: the current stream of ``device``, or of
+    the current device) and raises MsignError if a kernel's bounded wait on
+    that device ran out."""
+    torch = _torch()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        check(_lib.lib().msign_sync_status(_stream(stream, device)), "msign_sync_status")
 
 
 # ---------------------------------------------------------------- msign_ns
@@ -112,13 +127,16 @@ def msign_ns(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, impro
     if out is None:
         out = torch.empty_like(x)
     _need_cuda(out, "out")
+    _same_device(out, x.device, "out")
     if out.shape != x.shape or out.dtype != x.dtype:
         raise ValueError("out must match x in shape and dtype")
-    ws, wsb = _workspace(msign_ns_workspace_size(batch, rows, cols, compute), x.device, workspace)
-    c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0, _METHODS[method])
-    st = _lib.lib().msign_ns(x.data_ptr(), out.data_ptr(), _dtype_code(x), _compute_code(compute), batch, rows,
-                             cols, ctypes.byref(c) if c is not None else None, _ptr(ws), wsb, _stream(stream))
-    del keep
+    with torch.cuda.device(x.device):
+        ws, wsb = _workspace(msign_ns_workspace_size(batch, rows, cols, compute), x.device, workspace)
+        c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0, _METHODS[method])
+        st = _lib.lib().msign_ns(x.data_ptr(), out.data_ptr(), _dtype_code(x), _compute_code(compute), batch, rows,
+                                 cols, ctypes.byref(c) if c is not None else None, _ptr(ws), wsb,
+                                 _stream(stream, x.device))
+        del keep
     check(st, "msign_ns")
     return out
 
@@ -140,11 +158,13 @@ def gram_xxt(x, out=None, *, out_dtype=None, workspace=None, stream=None):
     if out is None:
         out = torch.empty(*x.shape[:-2], n, n, dtype=out_dtype or x.dtype, device=x.device)
     _need_cuda(out, "out")
+    _same_device(out, x.device, "out")
     if tuple(out.shape) != tuple(x.shape[:-2]) + (n, n):
         raise ValueError("out must be (..., n, n)")
-    ws, wsb = _workspace(gram_xxt_workspace_size(x), x.device, workspace)
-    st = _lib.lib().gram_xxt(x.data_ptr(), _dtype_code(x), out.data_ptr(), _dtype_code(out), batch, n, m, _ptr(ws),
-                             wsb, _stream(stream))
+    with torch.cuda.device(x.device):
+        ws, wsb = _workspace(gram_xxt_workspace_size(x), x.device, workspace)
+        st = _lib.lib().gram_xxt(x.data_ptr(), _dtype_code(x), out.data_ptr(), _dtype_code(out), batch, n, m,
+                                 _ptr(ws), wsb, _stream(stream, x.device))
     check(st, "gram_xxt")
     return out
 
@@ -166,19 +186,21 @@ def gram_ns(x, out=None, *, coeffs=None, eps=None, restart_after=(2,), workspace
     if out is None:
         out = torch.empty_like(x)
     _need_cuda(out, "out")
+    _same_device(out, x.device, "out")
     if out.shape != x.shape or out.dtype != x.dtype:
         raise ValueError("out must match x in shape and dtype")
-    ws, wsb = _workspace(gram_ns_workspace_size(batch, rows, cols), x.device, workspace)
     c, keep = make_coeffs(coeffs, eps)
     if restart_after is None:
         rbuf, nr = None, -1
     else:
         r = [int(v) for v in restart_after]
         rbuf, nr = (ctypes.c_int * max(1, len(r)))(*r), len(r)
-    st = _lib.lib().gram_ns(x.data_ptr(), out.data_ptr(), _dtype_code(x), batch, rows, cols,
-                            ctypes.byref(c) if c is not None else None,
-                            ctypes.cast(rbuf, ctypes.POINTER(ctypes.c_int)) if rbuf is not None else None, nr,
-                            _ptr(ws), wsb, _stream(stream))
+    with torch.cuda.device(x.device):
+        ws, wsb = _workspace(gram_ns_workspace_size(batch, rows, cols), x.device, workspace)
+        st = _lib.lib().gram_ns(x.data_ptr(), out.data_ptr(), _dtype_code(x), batch, rows, cols,
+                                ctypes.byref(c) if c is not None else None,
+                                ctypes.cast(rbuf, ctypes.POINTER(ctypes.c_int)) if rbuf is not None else None, nr,
+                                _ptr(ws), wsb, _stream(stream, x.device))
     del keep
     check(st, "gram_ns")
     return out
@@ -208,9 +230,11 @@ def muon_step(weights, momenta, grads, *, momentum: float = 0.95, lr: float = 0.
         raise ValueError("weights, momenta and grads must have the same length")
     if num == 0:
         return
+    device = weights[0].device
     for w, m, g in zip(weights, momenta, grads):
         for t, nm in ((w, "weight"), (m, "momentum"), (g, "grad")):
             _need_cuda(t, nm)
+            _same_device(t, device, nm)
         if w.dim() != 2 or w.shape != m.shape or w.shape != g.shape:
             raise ValueError("each weight, momentum and grad must be the same 2-D shape")
         if m.dtype != torch.float32:
@@ -220,15 +244,17 @@ def muon_step(weights, momenta, grads, *, momentum: float = 0.95, lr: float = 0.
     if len(wdt) != 1 or len(gdt) != 1:
         raise TypeError("all weights (and all grads) must share one dtype")
     shapes = [tuple(w.shape) for w in weights]
-    ws, wsb = _workspace(muon_step_workspace_size(shapes), weights[0].device, workspace)
     W = (ctypes.c_void_p * num)(*[w.data_ptr() for w in weights])
     M = (ctypes.c_void_p * num)(*[m.data_ptr() for m in momenta])
     G = (ctypes.c_void_p * num)(*[g.data_ptr() for g in grads])
     rows = _i64_array([s[0] for s in shapes])
     cols = _i64_array([s[1] for s in shapes])
     c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0, _METHODS[method])
-    st = _lib.lib().muon_step(num, W, M, G, rows, cols, wdt.pop(), gdt.pop(), float(momentum), float(lr),
-                              ctypes.byref(c) if c is not None else None, _ptr(ws), wsb, _stream(stream))
+    with torch.cuda.device(device):
+        ws, wsb = _workspace(muon_step_workspace_size(shapes), device, workspace)
+        st = _lib.lib().muon_step(num, W, M, G, rows, cols, wdt.pop(), gdt.pop(), float(momentum), float(lr),
+                                  ctypes.byref(c) if c is not None else None, _ptr(ws), wsb,
+                                  _stream(stream, device))
     del keep
     check(st, "muon_step")
 

@@ -1691,11 +1691,11 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
 // ---------------------------------------------------------------- no-allocation variant
 //
 // Some callers cannot allocate device memory at the point where they need
-// msign: code inside a stream capture that must not call cudaMalloc (which
-// may synchronise the device), plugins hosted by a framework that owns all of
-// the GPU's memory through its own pool, or real-time loops that forbid any
-// allocation after start-up.  msign_ns_noalloc() serves them from a fixed
-// scratch array that lives in the library's own device image.
+// msign: plugins hosted by a framework that owns all of the GPU's memory
+// through its own pool, or real-time loops that forbid any allocation after
+// start-up (cudaMalloc may synchronise the device).  msign_ns_noalloc()
+// serves them from a fixed scratch array that lives in the library's own
+// device image.
 
 namespace msb {
 
@@ -1733,8 +1733,10 @@ msign_status msign_ns_noalloc(const void* in, void* out, msign_dtype io_dtype, i
     }
     scratch = g_noalloc_ptr[dev];
   }
-  // Every buffer msign_ns carves from its workspace is written before it is
-  // read, so the contents left by an earlier call need no clearing.
+  // msign_ns clears the state it needs at zero (tile claims, ingest tickets,
+  // row-block counters) with a cudaMemsetAsync on `stream` before use, and
+  // writes every other buffer it carves before reading it, so what an
+  // earlier call left in the array does not matter.
   return msign_ns(in, out, io_dtype, MSIGN_BF16, batch, rows, cols, coeffs, scratch, kNoAllocScratchBytes, stream);
 }
 

@@ -27,9 +27,11 @@ Conventions (readings of the pages where they leave a step open):
   casts the pages prescribe: the input cast to the compute dtype of [P2]
   "参考实现" (``input_cast='bf16'``) and the fp16 cast of step 2 of
   Algorithm 2 in [P3] section 3.4 (``cast_fp16=True``).
-* Orientation: the iteration runs on the side with fewer rows; a matrix
-  with rows > cols is transposed first and transposed back at the end
-  (square matrices are not transposed) ([P2] "参考实现").
+* Orientation: standard NS forms its Gram matrix on the smaller side of X
+  (X X^T for rows <= cols, X^T X otherwise), which is why [P2] "参考实现"
+  transposes tall inputs; Gram NS works on the wide orientation (n <= m,
+  tall inputs transposed and the result transposed back) as [P3]
+  Algorithms 1-2 are written for X in R^{n x m} with n <= m.
 * Standard NS normalises with sqrt(sum(x^2) + eps), eps = 1e-20 ([P2]
   "参考实现"); Gram NS with ||X||_F + eps, eps = 1e-7 ([P3] Alg. 1 step 1,
   Alg. 2 step 1).
@@ -69,8 +71,8 @@ def round_to_bf16(x) -> np.ndarray:
     bfloat16 keeps the top 16 bits of an IEEE float32.  The input is first
     taken as float32 (the inputs the method receives are float32 or already
     bfloat16-valued), then the low 16 bits are rounded away: add 0x7FFF plus
-    the lowest kept bit, and clear the low half.  This is the cast of
-    ``x.astype('bfloat16')`` in [P2] "参考实现".
+    the lowest kept bit, and clear the low half.  This is the input rounding
+    the routine of [P2] section 参考实现 applies before normalising.
     """
     f = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
     u = f.view(np.uint32).astype(np.uint64)
@@ -158,36 +160,60 @@ def msign_ns_closed_form(M, coeffs=None, eps: float = 1e-20) -> np.ndarray:
 # Standard Newton-Schulz msign
 # ----------------------------------------------------------------------------
 
+def _gram_side(X):
+    """(G, left): the smaller Gram matrix of X and which side it sits on.
+
+    For rows <= cols, G = X X^T (rows x rows) and left = True; otherwise
+    G = X^T X (cols x cols) and left = False.  Square matrices take the
+    left form."""
+    Xt = np.swapaxes(X, -1, -2)
+    if X.shape[-2] <= X.shape[-1]:
+        return X @ Xt, True
+    return Xt @ X, False
+
+
+def _quintic(X, a, b, c):
+    """One step of [P2] eq. 6: X <- a X + b X (X^T X) + c X (X^T X)^2, the
+    odd quintic applied to every singular value of X.
+
+    The three terms are formed one by one through the smaller Gram matrix G
+    (eq. 6 on the right of X, or the same polynomial written on the left,
+    a X + b (X X^T) X + c (X X^T)^2 X, when X is wide): with P1 = G X and
+    P2 = G P1 (or X G and P1 G) the step is a X + b P1 + c P2."""
+    G, left = _gram_side(X)
+    if left:
+        P1 = G @ X
+        P2 = G @ P1
+    else:
+        P1 = X @ G
+        P2 = P1 @ G
+    return a * X + b * P1 + c * P2
+
+
+def _frobenius_start(X, eps):
+    """X0 = X / ||X||_F ([P2] eq. 4), with the routine's guard eps added to
+    the sum of squares under the square root."""
+    return X / np.sqrt(np.sum(X * X, axis=(-2, -1), keepdims=True) + eps)
+
+
 def msign_ns(M, coeffs=None, eps: float = 1e-20, input_cast=None) -> np.ndarray:
     """Quintic Newton-Schulz msign, batched over leading dims, in fp64.
 
-    Steps ([P2] eq. 4 and 6, section 参考实现):
-      1. cast the input to the compute dtype (``input_cast``; None = none);
-      2. if rows > cols work on the transpose (the side with the smaller
-         Gram matrix);
-      3. X = X / sqrt(sum(X^2) + eps);
-      4. for each (a, b, c):  A = X X^T;  B = b A + c A A;  X = a X + B X
-         (the left form of the quintic, as in the flash-muon post of
-         nil9.net, which is the same polynomial as [P2] eq. 6 written on
-         the other side);
-      5. transpose back.
+    [P2] eq. 4 starts from X0 = M / ||M||_F, which puts every singular value
+    in [0, 1]; eq. 6 then applies x -> a x + b x^3 + c x^5 to the singular
+    values once per step (one (a, b, c) per step, Jordan's triple by default,
+    eq. 7).  The page's routine first rounds the input to the compute dtype
+    (``input_cast``; None = no rounding) and guards the norm with eps = 1e-20
+    under the square root.  Everything here is fp64; each step is
+    ``_quintic`` (which forms the Gram matrix on the smaller side, the
+    reason the routine transposes tall inputs).
     """
     X = _apply_input_cast(M, input_cast)
     if X.ndim < 2:
         raise ValueError("msign needs at least a matrix")
-    flip = X.shape[-2] > X.shape[-1]
-    if flip:
-        X = np.swapaxes(X, -1, -2)
-    X = np.array(X, dtype=np.float64, copy=True)
-    norm = np.sqrt(np.sum(X * X, axis=(-2, -1), keepdims=True) + eps)
-    X = X / norm
-    XT = lambda Y: np.swapaxes(Y, -1, -2)  # noqa: E731
+    X = _frobenius_start(X, eps)
     for a, b, c in _as_schedule(coeffs):
-        A = X @ XT(X)
-        B = b * A + c * (A @ A)
-        X = a * X + B @ X
-    if flip:
-        X = XT(X)
+        X = _quintic(X, a, b, c)
     return np.ascontiguousarray(X)
 
 
@@ -195,32 +221,26 @@ def msign_ns_improved_init(M, coeffs=None, eps: float = 1e-20, input_cast=None) 
     """Standard NS with the sharper initial normalisation of [P2] section
     改进初值, in fp64.
 
-    The Frobenius norm over-shrinks: sigma_1 <= (sum sigma^8)^(1/8) =
-    ||(X X^T)^2||_F^(1/4) <= ||X||_F.  The first step already forms
-    A = X0 X0^T and A^2, so it rescales from them:
-      1-3. as ``msign_ns`` (cast, orient, X0 = X / sqrt(sum(X^2) + eps));
-      4. step 0: A = X0 X0^T, A2 = A A, n = (sum(A2^2) + eps)^(1/8);
-         X0 <- X0 / n, A <- A / n^2, A2 <- A2 / n^4;  X1 = a X0 + (b A + c A2) X0;
-      5. later steps as ``msign_ns``; transpose back.
+    The Frobenius norm shrinks X0 more than needed.  With G the Gram matrix
+    of X0 and sigma its singular values, ||G^2||_F^2 = sum sigma^8, so
+    sigma_1 <= (sum sigma^8)^(1/8) = ||G^2||_F^(1/4) <= ||X0||_F = 1.  The
+    section therefore divides X0 by nu = ||G^2||_F^(1/4) (eps guards the
+    zero matrix: nu = (||G^2||_F^2 + eps)^(1/8)), which keeps sigma_1 <= 1
+    while enlarging the small singular values, and then runs the same steps.
+    The page reuses the step-0 products (dividing G by nu^2 and G^2 by
+    nu^4) to save work; this oracle forms the rescaled X0 and starts over,
+    which is the same iteration in exact arithmetic.
     """
     X = _apply_input_cast(M, input_cast)
     if X.ndim < 2:
         raise ValueError("msign needs at least a matrix")
-    flip = X.shape[-2] > X.shape[-1]
-    if flip:
-        X = np.swapaxes(X, -1, -2)
-    X = np.array(X, dtype=np.float64, copy=True)
-    X = X / np.sqrt(np.sum(X * X, axis=(-2, -1), keepdims=True) + eps)
-    XT = lambda Y: np.swapaxes(Y, -1, -2)  # noqa: E731
-    for t, (a, b, c) in enumerate(_as_schedule(coeffs)):
-        A = X @ XT(X)
-        A2 = A @ A
-        if t == 0:
-            n = (np.sum(A2 * A2, axis=(-2, -1), keepdims=True) + eps) ** 0.125
-            X, A, A2 = X / n, A / n ** 2, A2 / n ** 4
-        X = a * X + (b * A + c * A2) @ X
-    if flip:
-        X = XT(X)
+    X = _frobenius_start(X, eps)
+    G, _ = _gram_side(X)
+    G2 = G @ G
+    nu = (np.sum(G2 * G2, axis=(-2, -1), keepdims=True) + eps) ** 0.125
+    X = X / nu
+    for a, b, c in _as_schedule(coeffs):
+        X = _quintic(X, a, b, c)
     return np.ascontiguousarray(X)
 
 

@@ -217,3 +217,15 @@ def test_binding_route_query():
     assert msb.msign_ns_route(8, 4096, 4096) == "standard"
     with pytest.raises(msb.MsignError):
         msb.msign_ns_route(1, 1024, 16384, coeffs=[(1.0, 0.0, 0.0)] * 100)
+
+
+def test_binding_rejects_tensors_on_another_device():
+    # every tensor of a call must live on the device the call runs on
+    import torch
+
+    import newton_schulz_msign_b200 as msb
+
+    with pytest.raises(ValueError):
+        msb._same_device(torch.empty(1), torch.device("cuda", 0), "out")
+    msb._same_device(torch.empty(1), torch.device("cpu"), "out")
+    msb._same_device(None, torch.device("cuda", 0), "workspace")

@@ -31,26 +31,31 @@ def check_matrix(W0, M0, G, W1, M1, lr, mu=0.95):
     assert rel_fro(to_np(M1), Mr) < 1e-6
     scale = math.sqrt(max(1.0, r / c))
     dW_ref = Wr - to_np(W0)
-    dW = to_np(W1) - to_np(W0)
+    w1 = to_np(W1)
     if W1.dtype == torch.float32:
-        assert rel_fro(dW, dW_ref) < TOL_BF16
+        excess = np.abs(w1 - Wr)
     else:
-        # bf16 weights: W1 is the bf16 rounding of W0 + dW_gpu.  Remove half a
-        # bf16 ulp of W1 per element (the rounding); what is left is the
-        # update's own error and must be within the bf16-path tolerance of the
-        # exact update, in Frobenius norm.
-        w1 = to_np(W1)
+        # bf16 weights: W1 is the bf16 rounding of W0 + dW_gpu, so
+        # |W1 - Wr| <= half a bf16 ulp of W1 + |dW_gpu - dW_ref| per element.
+        # Removing the half ulp leaves (at most) the update's own error.
         half_ulp = np.ldexp(1.0, np.frexp(np.abs(w1))[1] - 9)
         excess = np.maximum(np.abs(w1 - Wr) - half_ulp, 0.0)
-        assert np.linalg.norm(excess) <= TOL_BF16 * np.linalg.norm(dW_ref)
+    # the update's error within the bf16-path tolerance of the exact update,
+    # in Frobenius norm ...
+    assert np.linalg.norm(excess) <= TOL_BF16 * np.linalg.norm(dW_ref)
+    # ... and element by element within a fifth of the update's RMS entry:
+    # rounding noise of relative size ~1e-2 stays far below that, while one
+    # wrong element (a mask or index slip) is of the size of the entry itself
+    rms = lr * scale * np.sqrt(np.mean(Or * Or))
+    assert float(excess.max()) <= 0.2 * rms
 
 
 @pytest.mark.parametrize("wdt,gdt", [(torch.float32, torch.float32), (torch.float32, torch.bfloat16),
                                      (torch.bfloat16, torch.bfloat16)])
 def test_muon_small_mixed_shapes(wdt, gdt):
-    # Gaussian momenta of small, very wide matrices sit near the bf16 error
-    # envelope (see the error table of the design notes); these stay inside it
-    shapes = [(64, 128), (128, 64), (96, 96), (200, 72), (64, 128), (80, 240)]
+    # ragged shapes of both orientations; 33 x 257 (a small, flat, very wide
+    # Gaussian spectrum) is the hardest case for bf16 operands
+    shapes = [(64, 128), (128, 64), (96, 96), (200, 72), (64, 128), (33, 257), (80, 240)]
     W, M, G = make(shapes, wdt, gdt, seed=100)
     W0 = [w.clone() for w in W]
     M0 = [m.clone() for m in M]
@@ -106,9 +111,9 @@ def test_muon_small_workspace_processes_in_groups():
 
 def test_muon_llama_layer_full_size():
     # one Llama-3-8B decoder layer (q, k, v, o, gate, up, down) at full size,
-    # bf16 weights, fp32 momentum, G ~ N(0, 1e-4^2); the q, k and down
-    # matrices (one per distinct oriented shape class) are checked against
-    # the oracle, the rest for finiteness.
+    # bf16 weights, fp32 momentum, G ~ N(0, 1e-4^2); all seven matrices are
+    # checked against the oracle (gate and up are the tall ones, which run
+    # transposed on ingest and are stored back transposed)
     shapes = [(r, c) for _, r, c in synth.llama3_8b_layer_shapes()]
     W, M, G = make(shapes, torch.bfloat16, torch.bfloat16, seed=400)
     for m in M:
@@ -119,7 +124,7 @@ def test_muon_llama_layer_full_size():
     msb.sync_status()
     for w in W:
         assert torch.isfinite(w).all()
-    for i in (0, 1, 6):
+    for i in range(len(shapes)):
         check_matrix(W0[i], M0[i], G[i], W[i], M[i], 0.02)
 
 
@@ -165,6 +170,7 @@ def test_muon_auto_route_mixed():
         half_ulp = np.ldexp(1.0, np.frexp(np.abs(w1))[1] - 9)
         excess = np.maximum(np.abs(w1 - w_ref) - half_ulp, 0.0)
         assert np.linalg.norm(excess) <= TOL_BF16 * np.linalg.norm(dW_ref)
+        assert float(excess.max()) <= 0.2 * 0.02 * math.sqrt(max(1.0, r / c)) * np.sqrt(np.mean(o_ref * o_ref))
         # and the standard-NS update agrees within the same tolerance
         w_std, _, _ = O.muon_step(to_np(W0[i]), to_np(M0[i]), to_np(G[i]), momentum=0.95, lr=0.02, input_cast="bf16")
         assert rel_fro(w_ref - to_np(W0[i]), w_std - to_np(W0[i])) < TOL_BF16
