@@ -390,6 +390,66 @@ def muon_step(W, M, G, momentum: float = 0.95, lr: float = 0.02, coeffs=None,
 
 
 # ----------------------------------------------------------------------------
+# Mousse: msign in a space whitened by Shampoo-style Kronecker factors
+# (the Mousse post, anti-entrophic.github.io/posts/10054, section "Mousse")
+# ----------------------------------------------------------------------------
+
+def spd_inv_root(A, p: int = 4, eps: float = 0.0) -> np.ndarray:
+    """(A + eps I)^(-1/p) of a symmetric positive (semi)definite matrix,
+    batched over leading dims, from its eigendecomposition in fp64.
+
+    The Mousse post writes its preconditioners as P = L^(1/4) and
+    Q = R^(1/4) and uses their inverses; eps is the usual damping that
+    keeps a rank-deficient statistic invertible.  Raises ValueError if a
+    damped eigenvalue is not positive.
+    """
+    A = np.asarray(A, dtype=np.float64)
+    A = 0.5 * (A + np.swapaxes(A, -1, -2))
+    w, V = np.linalg.eigh(A)
+    w = w + eps
+    if np.any(w <= 0.0):
+        raise ValueError("spd_inv_root needs positive damped eigenvalues")
+    return (V * w[..., None, :] ** (-1.0 / p)) @ np.swapaxes(V, -1, -2)
+
+
+def mousse_statistics(G, L=None, R=None, beta: float = 1.0):
+    """Shampoo-style Kronecker statistics of a gradient G (rows x cols):
+    L <- beta L + G G^T (rows x rows) and R <- beta R + G^T G (cols x cols).
+
+    The post approximates the Hessian by (R kron L)^(1/2) "Shampoo-style"
+    and gives no update rule for the two factors; the plainest reading is
+    Shampoo's accumulated Gram matrices of the gradient, with beta = 1 a
+    running sum and beta < 1 an exponential average.  Returns (L, R)."""
+    G = np.asarray(G, dtype=np.float64)
+    Gt = np.swapaxes(G, -1, -2)
+    GG, GtG = G @ Gt, Gt @ G
+    L = GG if L is None else beta * np.asarray(L, dtype=np.float64) + GG
+    R = GtG if R is None else beta * np.asarray(R, dtype=np.float64) + GtG
+    return L, R
+
+
+def mousse_direction(G, L, R, coeffs=None, eps: float = 0.0, exact: bool = False) -> np.ndarray:
+    """The Mousse direction D = L^(-1/4) msign(L^(-1/4) G R^(-1/4)) R^(-1/4);
+    the update is Delta W = -D (times a learning rate).
+
+    From the post: with P = L^(1/4), Q = R^(1/4) the constraint
+    ||P Delta W Q||_op <= 1 and Y = P Delta W Q turn min Tr(G^T Delta W)
+    into min Tr(G~^T Y) over ||Y||_op <= 1 with G~ = P^-1 G Q^-1, whose
+    minimiser is Y = -msign(G~); mapping back gives Delta W =
+    -P^-1 msign(G~) Q^-1.  ``exact`` takes msign from the SVD (the
+    constrained optimum); otherwise msign is the Newton-Schulz iteration of
+    ``msign_ns`` with ``coeffs`` (what an optimizer runs).  L and R are
+    damped by eps before their roots are taken.
+    """
+    G = np.asarray(G, dtype=np.float64)
+    Pi = spd_inv_root(L, 4, eps)
+    Qi = spd_inv_root(R, 4, eps)
+    Gt = Pi @ G @ Qi
+    O = msign_svd(Gt) if exact else msign_ns(Gt, coeffs)
+    return Pi @ O @ Qi
+
+
+# ----------------------------------------------------------------------------
 # FLOP bookkeeping ([P3] sections 1.2, 2.4, 3.4)
 # ----------------------------------------------------------------------------
 

@@ -342,3 +342,92 @@ def test_improved_init_is_a_rescale_of_the_input():
         for a, b, c in [(3.4445, -4.7750, 2.0315)] * 5:
             Y = a * Y + b * (Y @ Y.T) @ Y + c * (Y @ Y.T) @ (Y @ Y.T) @ Y
         assert np.allclose(got[i], Y, rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------- Mousse
+
+def _spd(n, seed, cond=1e3):
+    """Random symmetric positive definite matrix with eigenvalues spread over
+    [1/cond, 1] and its eigendecomposition."""
+    g = np.random.default_rng(seed)
+    q, _ = np.linalg.qr(g.standard_normal((n, n)))
+    w = np.logspace(-math.log10(cond), 0, n)
+    return (q * w) @ q.T, w, q
+
+
+@pytest.mark.parametrize("p", [1, 2, 4])
+def test_spd_inv_root_inverts_the_power(p):
+    A, _, _ = _spd(24, seed=p)
+    X = O.spd_inv_root(A, p, eps=1e-3)
+    Ad = A + 1e-3 * np.eye(24)
+    # X^p (A + eps I) = I, and X is symmetric positive definite
+    np.testing.assert_allclose(np.linalg.matrix_power(X, p) @ Ad, np.eye(24), atol=1e-9)
+    np.testing.assert_allclose(X, X.T, atol=1e-12)
+    assert np.linalg.eigvalsh(X).min() > 0
+    if p == 1:
+        np.testing.assert_allclose(X, np.linalg.inv(Ad), rtol=1e-9, atol=1e-9)
+    if p == 2:
+        np.testing.assert_allclose(X, scipy.linalg.inv(scipy.linalg.sqrtm(Ad)).real, rtol=1e-8, atol=1e-9)
+
+
+def test_spd_inv_root_of_a_diagonal_is_elementwise():
+    d = np.array([4.0, 1.0, 0.0625, 16.0])
+    np.testing.assert_allclose(O.spd_inv_root(np.diag(d), 4), np.diag([2 ** -0.5, 1.0, 2.0, 0.5]), rtol=1e-14)
+    with pytest.raises(ValueError):
+        O.spd_inv_root(np.diag([1.0, 0.0]), 4)
+
+
+def test_mousse_statistics_are_shampoo_gram_sums():
+    g1 = synth.gaussian((5, 7), seed=1).astype(np.float64)
+    g2 = synth.gaussian((5, 7), seed=2).astype(np.float64)
+    L, R = O.mousse_statistics(g1)
+    L, R = O.mousse_statistics(g2, L, R, beta=0.5)
+    np.testing.assert_allclose(L, 0.5 * np.einsum("ik,jk->ij", g1, g1) + np.einsum("ik,jk->ij", g2, g2))
+    np.testing.assert_allclose(R, 0.5 * np.einsum("ki,kj->ij", g1, g1) + np.einsum("ki,kj->ij", g2, g2))
+
+
+@pytest.mark.parametrize("shape", [(16, 40), (40, 16), (24, 24)])
+def test_mousse_with_identity_factors_is_muon(shape):
+    G = synth.gaussian(shape, seed=sum(shape)).astype(np.float64)
+    r, c = shape
+    np.testing.assert_allclose(O.mousse_direction(G, np.eye(r), np.eye(c)), O.msign_ns(G), atol=1e-12)
+    np.testing.assert_allclose(O.mousse_direction(G, np.eye(r), np.eye(c), exact=True), O.msign_svd(G), atol=1e-12)
+
+
+@pytest.mark.parametrize("shape", [(12, 30), (30, 12)])
+def test_mousse_exact_direction_solves_the_constrained_problem(shape):
+    # the post's problem: min Tr(G^T dW) s.t. ||P dW Q||_op <= 1 with
+    # P = L^(1/4), Q = R^(1/4); its minimum is -||P^-1 G Q^-1||_* (nuclear
+    # norm), reached at dW = -D, and P D Q has every singular value 1
+    r, c = shape
+    G = synth.gaussian(shape, seed=r * c).astype(np.float64)
+    L, _, _ = _spd(r, seed=r, cond=50.0)
+    R, _, _ = _spd(c, seed=c + 1, cond=20.0)
+    D = O.mousse_direction(G, L, R, exact=True)
+    P = scipy.linalg.fractional_matrix_power(L, 0.25).real
+    Q = scipy.linalg.fractional_matrix_power(R, 0.25).real
+    np.testing.assert_allclose(np.linalg.svd(P @ D @ Q, compute_uv=False), 1.0, atol=1e-9)
+    Gt = np.linalg.solve(P, G) @ np.linalg.inv(Q)
+    nuclear = np.linalg.svd(Gt, compute_uv=False).sum()
+    assert abs(np.trace(G.T @ (-D)) + nuclear) < 1e-9 * nuclear
+    # no other feasible step does better: random directions scaled onto the
+    # constraint's boundary
+    g = np.random.default_rng(3)
+    for _ in range(20):
+        Y = g.standard_normal(shape)
+        Y /= np.linalg.norm(Y, 2)
+        dW = np.linalg.solve(P, Y) @ np.linalg.inv(Q)
+        assert np.trace(G.T @ dW) >= -nuclear - 1e-9
+
+
+def test_mousse_diagonal_factors_scale_rows_and_columns():
+    G = synth.gaussian((10, 14), seed=5).astype(np.float64)
+    lr_ = np.linspace(0.5, 4.0, 10)
+    lc = np.linspace(0.2, 3.0, 14)
+    D = O.mousse_direction(G, np.diag(lr_), np.diag(lc), exact=True)
+    pr, pc = lr_ ** -0.25, lc ** -0.25
+    ref = pr[:, None] * O.msign_svd(pr[:, None] * G * pc[None, :]) * pc[None, :]
+    np.testing.assert_allclose(D, ref, atol=1e-12)
+    # and the factors' scale only rescales the direction
+    D2 = O.mousse_direction(G, 16.0 * np.diag(lr_), 81.0 * np.diag(lc), exact=True)
+    np.testing.assert_allclose(D2, D / (2.0 * 3.0), atol=1e-12)
