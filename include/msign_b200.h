@@ -22,9 +22,11 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- * - Matrices are dense, row-major, batched back to back: matrix i of a batch
- *   of rows x cols starts at element i*rows*cols.  All pointers passed as
- *   matrices are DEVICE pointers unless stated otherwise.
+ * - Matrices are dense and row-major.  A batch of rows x cols matrices lies
+ *   back to back (matrix i starts at element i*rows*cols) unless the entry
+ *   point takes a batch stride (msign_ns and gram_ns: matrix i starts at
+ *   element i*stride).  All pointers passed as matrices are DEVICE pointers
+ *   unless stated otherwise.
  * - The caller owns every buffer.  The library allocates nothing: it works
  *   in the caller's workspace, whose size the *_workspace_size() query gives
  *   (a workspace must be 256-byte aligned).  Inputs are never written
@@ -95,7 +97,8 @@ typedef enum {
  *      expected to be faster, standard Newton-Schulz elsewhere.
  *      msign_ns_route() reports the choice for a shape.
  * Added in ABI 101 (init) and 102 (method); a caller built against an
- * older ABI lacks the later fields. */
+ * older ABI lacks the later fields.  ABI 103 added the batch strides of
+ * msign_ns and gram_ns. */
 typedef struct {
   int steps;
   const float *abc;
@@ -156,6 +159,13 @@ msign_status msign_profile_reset(void);
  *   in, out        device pointers, batch x rows x cols in io_dtype; out may
  *                  be in (the input is read whole into the workspace before
  *                  the first store to out)
+ *   in_stride,     elements from the start of one matrix of `in` (`out`) to
+ *   out_stride     the next: 0 means rows*cols (back to back), otherwise at
+ *                  least rows*cols (MSIGN_ERR_INVALID_ARG else), e.g. every
+ *                  other matrix of a larger batch.  Each matrix itself is
+ *                  dense row-major.  The pages' routine acts on the last two
+ *                  dims of a batch (section 参考实现); a stride lets a caller
+ *                  pass a batch that is a view into a larger tensor.
  *   io_dtype       MSIGN_BF16, MSIGN_FP16 or MSIGN_FP32
  *   compute_dtype  MSIGN_BF16: bf16 tensor-core operands, fp32 accumulation,
  *                  fp32 epilogue arithmetic and an fp32 copy of X between
@@ -196,8 +206,9 @@ int msign_ns_route(int64_t batch, int64_t rows, int64_t cols, msign_dtype comput
                    const msign_coeffs *coeffs);
 
 msign_status msign_ns(const void *in, void *out, msign_dtype io_dtype, msign_dtype compute_dtype,
-                      int64_t batch, int64_t rows, int64_t cols, const msign_coeffs *coeffs,
-                      void *workspace, size_t workspace_bytes, msign_stream_t stream);
+                      int64_t batch, int64_t rows, int64_t cols, int64_t in_stride, int64_t out_stride,
+                      const msign_coeffs *coeffs, void *workspace, size_t workspace_bytes,
+                      msign_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * msign_ns_noalloc: msign_ns for callers that cannot allocate device memory.
@@ -267,6 +278,8 @@ msign_status gram_xxt(const void *X, msign_dtype x_dtype, void *A, msign_dtype a
  *
  *   in, out        device pointers, batch x rows x cols in io_dtype; out may
  *                  be in, as for msign_ns
+ *   in_stride,     batch strides in elements, as for msign_ns (0: back to
+ *   out_stride     back)
  *   restart_after  HOST array of step numbers after which to restart
  *                  (values in 1..T-1); NULL with n_restart < 0 selects the
  *                  page's schedule {2}; n_restart == 0 means no restart.
@@ -274,8 +287,8 @@ msign_status gram_xxt(const void *X, msign_dtype x_dtype, void *A, msign_dtype a
 size_t gram_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols);
 
 msign_status gram_ns(const void *in, void *out, msign_dtype io_dtype,
-                     int64_t batch, int64_t rows, int64_t cols, const msign_coeffs *coeffs,
-                     const int *restart_after, int n_restart,
+                     int64_t batch, int64_t rows, int64_t cols, int64_t in_stride, int64_t out_stride,
+                     const msign_coeffs *coeffs, const int *restart_after, int n_restart,
                      void *workspace, size_t workspace_bytes, msign_stream_t stream);
 
 /* ------------------------------------------------------------------------
@@ -311,6 +324,57 @@ msign_status muon_step(int num, void *const *W, float *const *M, const void *con
                        msign_dtype w_dtype, msign_dtype g_dtype,
                        float momentum, float lr, const msign_coeffs *coeffs,
                        void *workspace, size_t workspace_bytes, msign_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Mousse: msign in a space whitened by Shampoo-style Kronecker factors (the
+ * Mousse post, anti-entrophic.github.io/posts/10054, section "Mousse"):
+ *
+ *   Delta W = -L^(-1/4) msign(L^(-1/4) G R^(-1/4)) R^(-1/4)
+ *
+ * for a gradient G (rows x cols), L (rows x rows) and R (cols x cols)
+ * symmetric positive semidefinite statistics (Shampoo's accumulated G G^T
+ * and G^T G are the plain choice; the post leaves their update open).
+ * mousse_inv_root computes the roots, which an optimizer refreshes every few
+ * steps; mousse_direction is the per-step hot path and returns
+ * D = L^(-1/4) msign(L^(-1/4) G R^(-1/4)) R^(-1/4), the update being -lr D.
+ * ------------------------------------------------------------------------ */
+
+/* out = (A + eps I)^(-1/4) for each of `batch` symmetric positive
+ * semidefinite n x n fp32 matrices A (device, back to back; only the upper
+ * triangle of each A is read).  Coupled Newton iteration for inverse p-th
+ * roots with p = 4, X_{j+1} = X_j T_j, M_{j+1} = T_j^4 M_j,
+ * T_j = (5 I - M_j) / 4, from X_0 = s^(1/4) I, M_0 = s (A + eps I),
+ * s = 1 / (||A||_F + eps); every product runs on the tensor cores in
+ * fp32-accurate arithmetic (3xTF32, as msign_ns's MSIGN_FP32).
+ *
+ *   eps    damping >= 0 (a rank-deficient statistic needs eps > 0)
+ *   iters  Newton steps (0: 20).  An eigenvalue lambda of A converges once
+ *          s (lambda + eps) has been driven to 1: it grows by a factor of
+ *          about 2.4 per step while small, then converges quadratically,
+ *          so iters ~ log(kappa) / log(2.44) + 4 with kappa =
+ *          (||A||_F + eps) / (lambda_min + eps).  2 <= iters <= 1000.
+ *   out    device, batch x n x n fp32, exactly symmetric
+ *   workspace  at least mousse_inv_root_workspace_size() bytes
+ * ------------------------------------------------------------------------ */
+size_t mousse_inv_root_workspace_size(int64_t batch, int64_t n);
+
+msign_status mousse_inv_root(const float *A, float *out, int64_t batch, int64_t n, float eps, int iters,
+                             void *workspace, size_t workspace_bytes, msign_stream_t stream);
+
+/* out = L_root msign(L_root G R_root) R_root for each of `batch` matrices G
+ * (rows x cols, io_dtype, back to back), with L_root = L^(-1/4)
+ * (batch x rows x rows fp32) and R_root = R^(-1/4) (batch x cols x cols
+ * fp32), e.g. from mousse_inv_root.  The four projection products run with
+ * bf16 operands and fp32 accumulation; msign is msign_ns with bf16 compute
+ * and the `coeffs` schedule (method must be 0; init 0 or 1).  out is
+ * batch x rows x cols in io_dtype and must not overlap G.
+ *   workspace  at least mousse_direction_workspace_size() bytes
+ * ------------------------------------------------------------------------ */
+size_t mousse_direction_workspace_size(int64_t batch, int64_t rows, int64_t cols);
+
+msign_status mousse_direction(const void *G, void *out, msign_dtype io_dtype, int64_t batch, int64_t rows,
+                              int64_t cols, const float *L_root, const float *R_root, const msign_coeffs *coeffs,
+                              void *workspace, size_t workspace_bytes, msign_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -17,8 +17,8 @@ from ._lib import BF16, FP16, FP32, MsignError, check, make_coeffs
 
 __all__ = [
     "MsignError", "msign_ns", "msign_ns_workspace_size", "gram_xxt", "gram_xxt_workspace_size", "gram_ns",
-    "gram_ns_workspace_size", "muon_step", "muon_step_workspace_size", "sync_status", "selftest_timeout",
-    "library_path",
+    "gram_ns_workspace_size", "muon_step", "muon_step_workspace_size", "mousse_inv_root", "mousse_direction",
+    "sync_status", "selftest_timeout", "library_path",
 ]
 
 
@@ -58,6 +58,31 @@ def _need_cuda(t, name):
         raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _batch_layout(t, name):
+    """(batch, rows, cols, stride) of a CUDA tensor whose last two dims are a
+    dense row-major matrix and whose leading dims step through memory with
+    one stride (any view of that form, e.g. ``big[:, 0]``); stride 0 means
+    back to back."""
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dim() < 2:
+        raise ValueError(f"{name} needs at least two dims")
+    rows, cols = t.shape[-2], t.shape[-1]
+    if (cols > 1 and t.stride(-1) != 1) or (rows > 1 and t.stride(-2) != cols):
+        raise ValueError(f"{name}: each matrix (the last two dims) must be dense row-major")
+    lead = [(t.shape[d], t.stride(d)) for d in range(t.dim() - 2) if t.shape[d] != 1]
+    batch = math.prod(sz for sz, _ in lead)
+    if batch <= 1 or rows * cols == 0:
+        return batch, rows, cols, 0
+    stride = lead[-1][1]
+    for (sz_o, st_o), (sz_i, st_i) in zip(lead[:-1], lead[1:]):
+        if st_o != st_i * sz_i:
+            raise ValueError(f"{name}: the batch dims must step through memory with one stride")
+    if stride < rows * cols:
+        raise ValueError(f"{name}: matrices of the batch overlap (stride {stride} < {rows * cols})")
+    return batch, rows, cols, (0 if stride == rows * cols else stride)
 
 
 def _same_device(t, device, name):
@@ -115,27 +140,25 @@ def msign_ns(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, impro
              workspace=None, stream=None):
     """Newton-Schulz msign of the last two dims of ``x`` (bf16/fp16/fp32 CUDA tensor).
 
+    ``x`` and ``out`` may be batched views whose matrices are dense but not
+    back to back (e.g. ``big[:, 0]``): their batch strides are passed on.
     ``improved_init``: the sharper step-0 normalisation (msign_coeffs.init = 1).
     ``method``: "standard" (standard NS) or "auto" (Gram NS where ``msign_ns_route``
     picks it, msign_coeffs.method = 1)."""
     torch = _torch()
-    _need_cuda(x, "x")
-    if x.dim() < 2:
-        raise ValueError("x needs at least two dims")
-    rows, cols = x.shape[-2], x.shape[-1]
-    batch = math.prod(x.shape[:-2])
+    batch, rows, cols, in_stride = _batch_layout(x, "x")
     if out is None:
-        out = torch.empty_like(x)
-    _need_cuda(out, "out")
+        out = torch.empty(x.shape, dtype=x.dtype, device=x.device)
     _same_device(out, x.device, "out")
     if out.shape != x.shape or out.dtype != x.dtype:
         raise ValueError("out must match x in shape and dtype")
+    _, _, _, out_stride = _batch_layout(out, "out")
     with torch.cuda.device(x.device):
         ws, wsb = _workspace(msign_ns_workspace_size(batch, rows, cols, compute), x.device, workspace)
         c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0, _METHODS[method])
         st = _lib.lib().msign_ns(x.data_ptr(), out.data_ptr(), _dtype_code(x), _compute_code(compute), batch, rows,
-                                 cols, ctypes.byref(c) if c is not None else None, _ptr(ws), wsb,
-                                 _stream(stream, x.device))
+                                 cols, in_stride, out_stride, ctypes.byref(c) if c is not None else None, _ptr(ws),
+                                 wsb, _stream(stream, x.device))
         del keep
     check(st, "msign_ns")
     return out
@@ -176,19 +199,16 @@ def gram_ns_workspace_size(batch: int, rows: int, cols: int) -> int:
 
 
 def gram_ns(x, out=None, *, coeffs=None, eps=None, restart_after=(2,), workspace=None, stream=None):
-    """Stabilized Gram Newton-Schulz (fp16 inner iteration) of the last two dims of ``x``."""
+    """Stabilized Gram Newton-Schulz (fp16 inner iteration) of the last two dims of ``x``
+    (batched views with one batch stride accepted, as for ``msign_ns``)."""
     torch = _torch()
-    _need_cuda(x, "x")
-    if x.dim() < 2:
-        raise ValueError("x needs at least two dims")
-    rows, cols = x.shape[-2], x.shape[-1]
-    batch = math.prod(x.shape[:-2])
+    batch, rows, cols, in_stride = _batch_layout(x, "x")
     if out is None:
-        out = torch.empty_like(x)
-    _need_cuda(out, "out")
+        out = torch.empty(x.shape, dtype=x.dtype, device=x.device)
     _same_device(out, x.device, "out")
     if out.shape != x.shape or out.dtype != x.dtype:
         raise ValueError("out must match x in shape and dtype")
+    _, _, _, out_stride = _batch_layout(out, "out")
     c, keep = make_coeffs(coeffs, eps)
     if restart_after is None:
         rbuf, nr = None, -1
@@ -197,8 +217,8 @@ def gram_ns(x, out=None, *, coeffs=None, eps=None, restart_after=(2,), workspace
         rbuf, nr = (ctypes.c_int * max(1, len(r)))(*r), len(r)
     with torch.cuda.device(x.device):
         ws, wsb = _workspace(gram_ns_workspace_size(batch, rows, cols), x.device, workspace)
-        st = _lib.lib().gram_ns(x.data_ptr(), out.data_ptr(), _dtype_code(x), batch, rows, cols,
-                                ctypes.byref(c) if c is not None else None,
+        st = _lib.lib().gram_ns(x.data_ptr(), out.data_ptr(), _dtype_code(x), batch, rows, cols, in_stride,
+                                out_stride, ctypes.byref(c) if c is not None else None,
                                 ctypes.cast(rbuf, ctypes.POINTER(ctypes.c_int)) if rbuf is not None else None, nr,
                                 _ptr(ws), wsb, _stream(stream, x.device))
     del keep
@@ -257,6 +277,67 @@ def muon_step(weights, momenta, grads, *, momentum: float = 0.95, lr: float = 0.
                                   _stream(stream, device))
     del keep
     check(st, "muon_step")
+
+
+# ---------------------------------------------------------------- Mousse
+
+def mousse_inv_root(a, out=None, *, eps: float = 0.0, iters: int = 0, workspace=None, stream=None):
+    """(A + eps I)^(-1/4) of symmetric positive semidefinite fp32 matrices (the
+    last two dims of ``a``), exactly symmetric, by the coupled Newton
+    iteration in fp32-accurate arithmetic (``iters`` 0: the library default)."""
+    torch = _torch()
+    _need_cuda(a, "a")
+    if a.dtype != torch.float32 or a.dim() < 2 or a.shape[-1] != a.shape[-2]:
+        raise ValueError("a must be float32 (..., n, n)")
+    n = a.shape[-1]
+    batch = math.prod(a.shape[:-2])
+    if out is None:
+        out = torch.empty_like(a)
+    _need_cuda(out, "out")
+    _same_device(out, a.device, "out")
+    if out.shape != a.shape or out.dtype != torch.float32:
+        raise ValueError("out must match a")
+    with torch.cuda.device(a.device):
+        ws, wsb = _workspace(int(_lib.lib().mousse_inv_root_workspace_size(batch, n)), a.device, workspace)
+        st = _lib.lib().mousse_inv_root(a.data_ptr(), out.data_ptr(), batch, n, float(eps), int(iters), _ptr(ws), wsb,
+                                        _stream(stream, a.device))
+    check(st, "mousse_inv_root")
+    return out
+
+
+def mousse_direction(g, l_root, r_root, out=None, *, coeffs=None, eps=None, improved_init=False, workspace=None,
+                     stream=None):
+    """L^(-1/4) msign(L^(-1/4) G R^(-1/4)) R^(-1/4) of the last two dims of ``g``,
+    given ``l_root`` = L^(-1/4) (..., rows, rows) and ``r_root`` = R^(-1/4)
+    (..., cols, cols) as float32 (e.g. from ``mousse_inv_root``)."""
+    torch = _torch()
+    for t, nm in ((g, "g"), (l_root, "l_root"), (r_root, "r_root")):
+        _need_cuda(t, nm)
+        _same_device(t, g.device, nm)
+    if g.dim() < 2:
+        raise ValueError("g needs at least two dims")
+    rows, cols = g.shape[-2], g.shape[-1]
+    lead = tuple(g.shape[:-2])
+    if (l_root.dtype != torch.float32 or r_root.dtype != torch.float32 or tuple(l_root.shape) != lead + (rows, rows)
+            or tuple(r_root.shape) != lead + (cols, cols)):
+        raise ValueError("l_root and r_root must be float32 (..., rows, rows) and (..., cols, cols)")
+    batch = math.prod(lead)
+    if out is None:
+        out = torch.empty_like(g)
+    _need_cuda(out, "out")
+    _same_device(out, g.device, "out")
+    if out.shape != g.shape or out.dtype != g.dtype:
+        raise ValueError("out must match g")
+    c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0, 0)
+    with torch.cuda.device(g.device):
+        ws, wsb = _workspace(int(_lib.lib().mousse_direction_workspace_size(batch, rows, cols)), g.device, workspace)
+        st = _lib.lib().mousse_direction(g.data_ptr(), out.data_ptr(), _dtype_code(g), batch, rows, cols,
+                                         l_root.data_ptr(), r_root.data_ptr(),
+                                         ctypes.byref(c) if c is not None else None, _ptr(ws), wsb,
+                                         _stream(stream, g.device))
+    del keep
+    check(st, "mousse_direction")
+    return out
 
 
 # ---------------------------------------------------------------- launch records

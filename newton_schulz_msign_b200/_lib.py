@@ -26,6 +26,7 @@ EXPORTS = (
     "msign_profile_enable", "msign_profile_read", "msign_profile_reset",
     "msign_ns_noalloc_max_bytes", "msign_ns_noalloc",
     "msign_selftest_timeout",
+    "mousse_inv_root_workspace_size", "mousse_inv_root", "mousse_direction_workspace_size", "mousse_direction",
 )
 
 
@@ -66,7 +67,7 @@ def lib() -> ctypes.CDLL:
         L.msign_ns_workspace_size.restype = SZ
         L.msign_ns_workspace_size.argtypes = [I64, I64, I64, I32]
         L.msign_ns.restype = I32
-        L.msign_ns.argtypes = [P, P, I32, I32, I64, I64, I64, ctypes.POINTER(MsignCoeffs), P, SZ, P]
+        L.msign_ns.argtypes = [P, P, I32, I32, I64, I64, I64, I64, I64, ctypes.POINTER(MsignCoeffs), P, SZ, P]
         L.msign_ns_route.restype = I32
         L.msign_ns_route.argtypes = [I64, I64, I64, I32, ctypes.POINTER(MsignCoeffs)]
         L.gram_xxt_workspace_size.restype = SZ
@@ -76,7 +77,7 @@ def lib() -> ctypes.CDLL:
         L.gram_ns_workspace_size.restype = SZ
         L.gram_ns_workspace_size.argtypes = [I64, I64, I64]
         L.gram_ns.restype = I32
-        L.gram_ns.argtypes = [P, P, I32, I64, I64, I64, ctypes.POINTER(MsignCoeffs),
+        L.gram_ns.argtypes = [P, P, I32, I64, I64, I64, I64, I64, ctypes.POINTER(MsignCoeffs),
                               ctypes.POINTER(I32), I32, P, SZ, P]
         L.muon_step_workspace_size.restype = SZ
         L.muon_step_workspace_size.argtypes = [I32, ctypes.POINTER(I64), ctypes.POINTER(I64)]
@@ -97,6 +98,14 @@ def lib() -> ctypes.CDLL:
         L.msign_selftest_timeout.argtypes = [ctypes.c_uint64, P]
         L.msign_ns_noalloc.restype = I32
         L.msign_ns_noalloc.argtypes = [P, P, I32, I64, I64, I64, ctypes.POINTER(MsignCoeffs), P]
+        L.mousse_inv_root_workspace_size.restype = SZ
+        L.mousse_inv_root_workspace_size.argtypes = [I64, I64]
+        L.mousse_inv_root.restype = I32
+        L.mousse_inv_root.argtypes = [P, P, I64, I64, F32, I32, P, SZ, P]
+        L.mousse_direction_workspace_size.restype = SZ
+        L.mousse_direction_workspace_size.argtypes = [I64, I64, I64]
+        L.mousse_direction.restype = I32
+        L.mousse_direction.argtypes = [P, P, I32, I64, I64, I64, P, P, ctypes.POINTER(MsignCoeffs), P, SZ, P]
         _lib = L
     return _lib
 

@@ -60,12 +60,13 @@ __device__ __forceinline__ float block_reduce_sum(float v, float* red) {
   return v;
 }
 
-// grid (kNormParts, batch); `in` holds batch matrices of `per` elements.
+// grid (kNormParts, batch); `in` holds batch matrices of `per` elements,
+// matrix b starting at element b * bs.
 __global__ void __launch_bounds__(kNormThreads) sumsq_partial_kernel(const void* in, int in_dt, long long per,
-                                                                     int cast_dt, float* partials) {
+                                                                     long long bs, int cast_dt, float* partials) {
   __shared__ float red[32];
   const int b = blockIdx.y;
-  const char* base = reinterpret_cast<const char*>(in) + static_cast<long long>(b) * per * dtype_size(in_dt);
+  const char* base = reinterpret_cast<const char*>(in) + static_cast<long long>(b) * bs * dtype_size(in_dt);
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   float acc = 0.0f;
   const bool vec = (reinterpret_cast<uintptr_t>(base) & 15) == 0;
@@ -154,6 +155,8 @@ __global__ void __launch_bounds__(1024) norm_finalize_kernel(const float* partia
 
 struct IngestArgs {
   void* in;
+  long long in_bs;  // elements between consecutive input matrices (0: rows * cols)
+  long long ld_in;  // elements between consecutive input rows (0: cols)
   int in_dt, rows, cols, transpose, cast_dt;
   const float* pre_scale;
   void* xop;
@@ -229,7 +232,7 @@ __device__ __forceinline__ void ingest_row_chunk(const IngestArgs& a, char* src,
   const int i = static_cast<int>(tt / tc) * 32 + (tid >> 3);
   const int j = static_cast<int>(tt % tc) * 64 + 8 * (tid & 7);
   const int cnt = (i < n && j < m) ? (m - j < 8 ? m - j : 8) : 0;
-  const long long e = static_cast<long long>(i) * a.cols + j;
+  const long long e = static_cast<long long>(i) * (a.ld_in > 0 ? a.ld_in : a.cols) + j;
   load8(src + e * dtype_size(a.in_dt), a.in_dt, cnt, x);
   if (gsrc != nullptr && cnt > 0) {
     float g[8];
@@ -312,7 +315,7 @@ __global__ void __launch_bounds__(256) ingest_kernel(const IngestArgs a) {
   const int n = a.transpose ? a.cols : a.rows;
   const int m = a.transpose ? a.rows : a.cols;
   const long long per = static_cast<long long>(a.rows) * a.cols;
-  char* src = reinterpret_cast<char*>(a.in) + static_cast<long long>(b) * per * dtype_size(a.in_dt);
+  char* src = reinterpret_cast<char*>(a.in) + static_cast<long long>(b) * (a.in_bs > 0 ? a.in_bs : per) * dtype_size(a.in_dt);
   const char* gsrc = a.G ? reinterpret_cast<const char*>(a.G) + static_cast<long long>(b) * per * dtype_size(a.g_dt)
                          : nullptr;
   const float s = a.pre_scale ? a.pre_scale[b] : 1.0f;
@@ -352,7 +355,7 @@ __global__ void __launch_bounds__(256) ingest_kernel(const IngestArgs a) {
         const int jr = j0 + ty + 8 * k, ic = i0 + tx;
         float x = 0.0f;
         if (jr < m && ic < n) {
-          const long long e = static_cast<long long>(jr) * a.cols + ic;
+          const long long e = static_cast<long long>(jr) * (a.ld_in > 0 ? a.ld_in : a.cols) + ic;
           x = load_elem(src + e * dtype_size(a.in_dt), a.in_dt);
           if (gsrc != nullptr) {
             x = fmaf(a.mu, x, load_elem(gsrc + e * dtype_size(a.g_dt), a.g_dt));
@@ -448,6 +451,42 @@ __global__ void __launch_bounds__(256) improved_init_kernel(const void* A, void*
       char* q = bb + off * dtype_size(op_dt);
       store_elem(q, op_dt, kb * a + kc * load_elem(q, op_dt));
     }
+  }
+}
+
+// ---------------------------------------------------------------- Mousse preconditioner roots
+//
+// Start of the coupled Newton iteration for (A + eps I)^(-1/4), the inverse
+// fourth roots of the Mousse post's Kronecker factors: with
+// s = 1 / (||A||_F + eps) (s_in[b]) the scaled matrix M0 = s (A + eps I) has
+// its eigenvalues in (0, 1], and the first iterate is X1 = X0 (5 I - M0) / 4
+// with X0 = s^(1/4) I.  Only the upper triangle of A is read (the lower one
+// is taken as its mirror), so M0 is exactly symmetric.  Both matrices are
+// stored as tf32 (hi, lo) plane pairs for the fp32-accurate products: matrix
+// b at element 2 b plane, the lo plane `plane` elements after the hi plane,
+// rows ld apart.  Grid (blocks, batch), grid-stride over the n x n elements.
+__global__ void __launch_bounds__(256) inv_root_start_kernel(const float* A, int n, long long a_bs, const float* s_in,
+                                                             float eps, float* M, float* X, long long ld,
+                                                             long long plane) {
+  const int b = blockIdx.y;
+  const float s = s_in[b];
+  const float q = sqrtf(sqrtf(s));
+  const float* a = A + static_cast<long long>(b) * a_bs;
+  float* mh = M + 2 * plane * b;
+  float* xh = X + 2 * plane * b;
+  const long long total = static_cast<long long>(n) * n;
+  for (long long e = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; e < total;
+       e += static_cast<long long>(gridDim.x) * 256) {
+    const int i = static_cast<int>(e / n), j = static_cast<int>(e % n);
+    const float aij = i <= j ? a[e] : a[static_cast<long long>(j) * n + i];
+    const float m0 = s * (aij + (i == j ? eps : 0.0f));
+    const float x1 = q * ((i == j ? 5.0f : 0.0f) - m0) * 0.25f;
+    const long long o = static_cast<long long>(i) * ld + j;
+    const float mhi = to_tf32(m0), xhi = to_tf32(x1);
+    mh[o] = mhi;
+    mh[o + plane] = to_tf32(m0 - mhi);
+    xh[o] = xhi;
+    xh[o + plane] = to_tf32(x1 - xhi);
   }
 }
 

@@ -157,6 +157,14 @@ int to_dt(msign_dtype d) { return d == MSIGN_BF16 ? DT_BF16 : d == MSIGN_FP16 ? 
 
 bool valid_dtype(msign_dtype d) { return d == MSIGN_BF16 || d == MSIGN_FP16 || d == MSIGN_FP32; }
 
+// Batch strides: 0 (matrices back to back) or at least one matrix, so that
+// the matrices of a batch never overlap.
+bool valid_strides(int64_t rows, int64_t cols, int64_t in_stride, int64_t out_stride) {
+  const int64_t per = rows * cols;
+  return in_stride >= 0 && out_stride >= 0 && (in_stride == 0 || in_stride >= per) &&
+         (out_stride == 0 || out_stride >= per);
+}
+
 // Workspace carving: the same routine sizes and slices the workspace.
 struct Carver {
   char* base;
@@ -477,12 +485,13 @@ __global__ void selftest_timeout_kernel(int* err, unsigned long long limit_ns) {
 }
 
 // Frobenius normalisation factor of every matrix of a batch into scale[].
-msign_status launch_norm(const void* in, int in_dt, int64_t per, int64_t batch, int cast_dt, float eps, int mode,
-                         float* partials, float* scale, cudaStream_t stream) {
+// Matrix b of the batch starts at element b * bs of `in`.
+msign_status launch_norm(const void* in, int in_dt, int64_t per, int64_t bs, int64_t batch, int cast_dt, float eps,
+                         int mode, float* partials, float* scale, cudaStream_t stream) {
   const int parts = norm_parts(per);
   dim3 g(static_cast<unsigned>(parts), static_cast<unsigned>(batch));
   prof_begin(stream);
-  sumsq_partial_kernel<<<g, kNormThreads, 0, stream>>>(in, in_dt, per, cast_dt, partials);
+  sumsq_partial_kernel<<<g, kNormThreads, 0, stream>>>(in, in_dt, per, bs, cast_dt, partials);
   prof_end(1, stream, 0.0, static_cast<double>(batch) * per * dtype_size(in_dt));
   prof_begin(stream);
   norm_finalize_kernel<<<static_cast<unsigned>(batch), 1024, 0, stream>>>(partials, parts, eps, mode, scale);
@@ -1083,6 +1092,59 @@ using namespace msb;
 
 // ================================================================ C ABI
 
+// Standard NS on validated arguments: batch matrices of rows x cols, input
+// `in` (in_dt; rows in_ld apart, matrices in_bs apart) -> output `out`
+// (out_dt; out_ld, out_bs), compute dtype `compute`, the schedule `sch`, a
+// workspace of at least msign_ns_workspace_size() bytes.  [P2] eq. 4-7.
+msign_status ns_run(const void* in, int in_dt, int64_t in_ld, int64_t in_bs, void* out, int out_dt, int64_t out_ld,
+                    int64_t out_bs, msign_dtype compute_dtype, int64_t batch, int64_t rows, int64_t cols,
+                    const Schedule& sch, void* workspace, cudaStream_t stream) {
+  msign_status st = MSIGN_OK;
+  const bool tr = rows > cols;  // iterate on the side with the smaller Gram matrix
+  const int64_t n = tr ? cols : rows, m = tr ? rows : cols;
+  const int64_t ldm = round_up(m, 8);
+  const bool fp32 = compute_dtype == MSIGN_FP32;
+  const int cd = to_dt(compute_dtype);  // the input is cast to the compute dtype first
+  Carver cv(workspace);
+  NsBuffers w;
+  carve_ns(cv, batch, n, m, &w, fp32);
+
+  // bf16 and fp32-accurate operands: one fused pass writes the unscaled x and
+  // the factor s, applied by the first step.  fp16 operands must be scaled
+  // before the cast (fp16 range), so that path normalises first.
+  const bool fused = cd != DT_FP16;
+  if (fused) {
+    if (cudaMemsetAsync(w.cnt, 0, state_bytes(batch, n, kMaxClasses), stream) != cudaSuccess) return MSIGN_ERR_CUDA;
+    IngestArgs a = ingest_args(in, in_dt, rows, cols, tr, cd, w.P[0], fp32 ? DT_TF32_HI : DT_BF16, ldm,
+                               fp32 ? 2 * n * ldm : n * ldm);
+    a.op_plane = n * ldm;
+    a.in_bs = in_bs, a.ld_in = in_ld;
+    a.master = w.master, a.ld_m = blk_ld(m), a.m_bs = blk_size(n, m);
+    a.partials = w.partials, a.ticket = ns_ticket_ptr(w), a.s_out = w.scale, a.s2_out = w.scale + batch;
+    a.eps = sch.eps;
+    st = launch_ingest(a, batch, stream);
+  } else {
+    if (in_ld != cols) return MSIGN_ERR_INVALID_ARG;  // the norm pass reads whole matrices
+    st = launch_norm(in, in_dt, rows * cols, in_bs, batch, cd, sch.eps, 0, w.partials, w.scale, stream);
+    if (st != MSIGN_OK) return st;
+    IngestArgs a = ingest_args(in, in_dt, rows, cols, tr, cd, w.P[0], cd, ldm, n * ldm);
+    a.pre_scale = w.scale;
+    a.in_bs = in_bs, a.ld_in = in_ld;
+    a.master = w.master, a.ld_m = blk_ld(m), a.m_bs = blk_size(n, m);
+    st = launch_ingest(a, batch, stream);
+  }
+  if (st != MSIGN_OK) return st;
+  std::vector<NsClass> cls(1);
+  cls[0].w = w;
+  cls[0].batch = batch, cls[0].n = n, cls[0].m = m;
+  cls[0].fp32 = fp32;
+  cls[0].op_dt = fp32 ? DT_BF16 : cd;
+  cls[0].final_outs = {out_to(out, out_dt, out_ld, out_bs, tr)};
+  if (fused) cls[0].s = w.scale, cls[0].s2 = w.scale + batch;
+  cls[0].improved = sch.init == 1;
+  return ns_iterate(cls, sch, stream, fused);
+}
+
 // msign_ns's automatic route (msign_coeffs.method = 1): Gram NS where it is
 // expected to beat standard NS.  Measured on a B200 (default schedules, time
 // of Gram NS over standard NS): 0.86 at 4096 x 8192, 0.71 at 4096 x 14336,
@@ -1107,7 +1169,7 @@ bool gram_route(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute, 
 
 extern "C" {
 
-int msign_abi_version(void) { return 102; }
+int msign_abi_version(void) { return 103; }
 
 const char* msign_status_string(msign_status s) {
   switch (s) {
@@ -1201,10 +1263,11 @@ int msign_ns_route(int64_t batch, int64_t rows, int64_t cols, msign_dtype comput
 }
 
 msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dtype compute_dtype, int64_t batch,
-                      int64_t rows, int64_t cols, const msign_coeffs* coeffs, void* workspace,
-                      size_t workspace_bytes, msign_stream_t stream_) {
+                      int64_t rows, int64_t cols, int64_t in_stride, int64_t out_stride, const msign_coeffs* coeffs,
+                      void* workspace, size_t workspace_bytes, msign_stream_t stream_) {
   if (!valid_dtype(io_dtype) || !valid_dtype(compute_dtype)) return MSIGN_ERR_INVALID_ARG;
   if (batch < 0 || rows < 0 || cols < 0) return MSIGN_ERR_INVALID_ARG;
+  if (!valid_strides(rows, cols, in_stride, out_stride)) return MSIGN_ERR_INVALID_ARG;
   Schedule sch;
   msign_status st = read_schedule(coeffs, kNsEps, &sch);
   if (st != MSIGN_OK) return st;
@@ -1222,55 +1285,16 @@ msign_status msign_ns(const void* in, void* out, msign_dtype io_dtype, msign_dty
     g.steps = sch.steps();
     g.abc = sch.abc.data();
     g.eps = (coeffs != nullptr && coeffs->eps >= 0.0f) ? coeffs->eps : -1.0f;
-    return gram_ns(in, out, io_dtype, batch, rows, cols, &g, nullptr, sch.steps() >= 3 ? -1 : 0, workspace,
-                   workspace_bytes, stream_);
+    return gram_ns(in, out, io_dtype, batch, rows, cols, in_stride, out_stride, &g, nullptr, sch.steps() >= 3 ? -1 : 0,
+                   workspace, workspace_bytes, stream_);
   }
   DeviceState* dev = nullptr;
   st = device_state(&dev);
   if (st != MSIGN_OK) return st;
-
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  const bool tr = rows > cols;  // iterate on the side with the smaller Gram matrix
-  const int64_t n = tr ? cols : rows, m = tr ? rows : cols;
-  const int64_t ldm = round_up(m, 8);
   const int io = to_dt(io_dtype);
-  const bool fp32 = compute_dtype == MSIGN_FP32;
-  const int cd = to_dt(compute_dtype);  // the input is cast to the compute dtype first
-  Carver cv(workspace);
-  NsBuffers w;
-  carve_ns(cv, batch, n, m, &w, fp32);
-
-  // bf16 and fp32-accurate operands: one fused pass writes the unscaled x and
-  // the factor s, applied by the first step.  fp16 operands must be scaled
-  // before the cast (fp16 range), so that path normalises first.
-  const bool fused = cd != DT_FP16;
-  if (fused) {
-    if (cudaMemsetAsync(w.cnt, 0, state_bytes(batch, n, kMaxClasses), stream) != cudaSuccess) return MSIGN_ERR_CUDA;
-    IngestArgs a = ingest_args(in, io, rows, cols, tr, cd, w.P[0], fp32 ? DT_TF32_HI : DT_BF16, ldm,
-                               fp32 ? 2 * n * ldm : n * ldm);
-    a.op_plane = n * ldm;
-    a.master = w.master, a.ld_m = blk_ld(m), a.m_bs = blk_size(n, m);
-    a.partials = w.partials, a.ticket = ns_ticket_ptr(w), a.s_out = w.scale, a.s2_out = w.scale + batch;
-    a.eps = sch.eps;
-    st = launch_ingest(a, batch, stream);
-  } else {
-    st = launch_norm(in, io, rows * cols, batch, cd, sch.eps, 0, w.partials, w.scale, stream);
-    if (st != MSIGN_OK) return st;
-    IngestArgs a = ingest_args(in, io, rows, cols, tr, cd, w.P[0], cd, ldm, n * ldm);
-    a.pre_scale = w.scale;
-    a.master = w.master, a.ld_m = blk_ld(m), a.m_bs = blk_size(n, m);
-    st = launch_ingest(a, batch, stream);
-  }
-  if (st != MSIGN_OK) return st;
-  std::vector<NsClass> cls(1);
-  cls[0].w = w;
-  cls[0].batch = batch, cls[0].n = n, cls[0].m = m;
-  cls[0].fp32 = fp32;
-  cls[0].op_dt = fp32 ? DT_BF16 : cd;
-  cls[0].final_outs = {out_to(out, io, cols, rows * cols, tr)};
-  if (fused) cls[0].s = w.scale, cls[0].s2 = w.scale + batch;
-  cls[0].improved = sch.init == 1;
-  return ns_iterate(cls, sch, stream, fused);
+  return ns_run(in, io, cols, in_stride > 0 ? in_stride : rows * cols, out, io, cols,
+                out_stride > 0 ? out_stride : rows * cols, compute_dtype, batch, rows, cols, sch, workspace,
+                reinterpret_cast<cudaStream_t>(stream_));
 }
 
 size_t gram_xxt_workspace_size(int64_t batch, int64_t n, int64_t m, msign_dtype x_dtype, const void* X) {
@@ -1332,7 +1356,8 @@ size_t gram_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols) {
 // segment bounds of the restart schedule, a workspace of at least
 // gram_ns_workspace_size() bytes.  [P3] Algorithm 2.
 msign_status gram_run(const void* in, int in_dt, void* out, int out_dt, int64_t batch, int64_t rows, int64_t cols,
-                      const Schedule& sch, const std::vector<int>& bounds, void* workspace, cudaStream_t stream) {
+                      int64_t in_bs, int64_t out_bs, const Schedule& sch, const std::vector<int>& bounds,
+                      void* workspace, cudaStream_t stream) {
   msign_status st = MSIGN_OK;
   const bool tr = rows > cols;
   const int64_t n = tr ? cols : rows, m = tr ? rows : cols;
@@ -1346,11 +1371,12 @@ msign_status gram_run(const void* in, int in_dt, void* out, int out_dt, int64_t 
   auto sqm = [&](void* p) { return Mat{p, DT_FP16, n, n, ldn, sq}; };
 
   // [P3] Algorithm 2 steps 1-2: X <- X / (||X||_F + eps); X <- float16(X)
-  st = launch_norm(in, in_dt, rows * cols, batch, DT_FP32, sch.eps, 1, w.partials, w.scale, stream);
+  st = launch_norm(in, in_dt, rows * cols, in_bs, batch, DT_FP32, sch.eps, 1, w.partials, w.scale, stream);
   if (st != MSIGN_OK) return st;
   {
     IngestArgs a = ingest_args(in, in_dt, rows, cols, tr, DT_FP32, w.P[0], DT_FP16, ldm, rect);
     a.pre_scale = w.scale;
+    a.in_bs = in_bs;
     st = launch_ingest(a, batch, stream);
   }
   if (st != MSIGN_OK) return st;
@@ -1437,7 +1463,7 @@ msign_status gram_run(const void* in, int in_dt, void* out, int out_dt, int64_t 
       s.M = n, s.N = m, s.K = n, s.batch = batch;
       void* dst = (seg + 2 == bounds.size()) ? out : w.P[cur ^ 1];
       if (seg + 2 == bounds.size())
-        s.outs = {out_to(out, out_dt, cols, rows * cols, tr)};
+        s.outs = {out_to(out, out_dt, cols, out_bs, tr)};
       else
         s.outs = {out_to(w.P[cur ^ 1], DT_FP16, ldm, rect, false)};
       st = ch.add(s, {{w.Q[q], DEP_TM}, {w.P[cur], DEP_ALL}}, nullptr, {dst});
@@ -1451,10 +1477,11 @@ msign_status gram_run(const void* in, int in_dt, void* out, int out_dt, int64_t 
 extern "C" {
 
 msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t batch, int64_t rows, int64_t cols,
-                     const msign_coeffs* coeffs, const int* restart_after, int n_restart, void* workspace,
-                     size_t workspace_bytes, msign_stream_t stream_) {
+                     int64_t in_stride, int64_t out_stride, const msign_coeffs* coeffs, const int* restart_after,
+                     int n_restart, void* workspace, size_t workspace_bytes, msign_stream_t stream_) {
   if (!valid_dtype(io_dtype)) return MSIGN_ERR_INVALID_ARG;
   if (batch < 0 || rows < 0 || cols < 0) return MSIGN_ERR_INVALID_ARG;
+  if (!valid_strides(rows, cols, in_stride, out_stride)) return MSIGN_ERR_INVALID_ARG;
   Schedule sch;
   msign_status st = read_schedule(coeffs, kGramEps, &sch);
   if (st != MSIGN_OK) return st;
@@ -1475,7 +1502,8 @@ msign_status gram_ns(const void* in, void* out, msign_dtype io_dtype, int64_t ba
   if (st != MSIGN_OK) return st;
 
   const int io = to_dt(io_dtype);
-  return gram_run(in, io, out, io, batch, rows, cols, sch, bounds, workspace,
+  return gram_run(in, io, out, io, batch, rows, cols, in_stride > 0 ? in_stride : rows * cols,
+                  out_stride > 0 ? out_stride : rows * cols, sch, bounds, workspace,
                   reinterpret_cast<cudaStream_t>(stream_));
 }
 
@@ -1611,7 +1639,7 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
         msign_status r = launch_ok();
         if (r != MSIGN_OK) return r;
         void* o = static_cast<char*>(workspace) + muon_gram_o_offset(rows[i], cols[i]);
-        r = gram_run(M[i], DT_FP32, o, DT_BF16, 1, rows[i], cols[i], gsch, gbounds, workspace, stream);
+        r = gram_run(M[i], DT_FP32, o, DT_BF16, 1, rows[i], cols[i], ne, ne, gsch, gbounds, workspace, stream);
         if (r != MSIGN_OK) return r;
         const float coef = lr * std::sqrt(std::max(1.0f, static_cast<float>(rows[i]) / static_cast<float>(cols[i])));
         prof_begin(stream);
@@ -1688,6 +1716,229 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
 
 }  // extern "C"
 
+// ---------------------------------------------------------------- Mousse
+//
+// The Mousse post (anti-entrophic.github.io/posts/10054, section "Mousse")
+// preconditions msign with Shampoo-style Kronecker factors L and R:
+// Delta W = -L^(-1/4) msign(L^(-1/4) G R^(-1/4)) R^(-1/4).  Two entry points
+// cover it: mousse_inv_root forms the inverse fourth roots of the damped
+// factors, and mousse_direction applies the two-sided projection, msign and
+// the back-projection.
+
+namespace msb {
+
+constexpr int kRootDefaultIters = 20;
+constexpr int kRootMaxIters = 1000;
+
+struct RootBuffers {
+  float* partials;
+  float* scale;  // s = 1 / (||A||_F + eps) per matrix
+  float* X[2];   // iterates X_j, tf32 plane pairs (upper 256-blocks read)
+  float* M[2];   // M_j = X_j^4 (A + eps I), plane pairs
+  float* T2;     // ((5 I - M) / 4)^2
+  float* T4;     // its square
+  int* cnt;      // chained-launch state (see Chain)
+};
+
+void carve_root(Carver& cv, int64_t batch, int64_t n, RootBuffers* b) {
+  const uint64_t mat = 8ull * batch * n * round_up(n, 8);  // two fp32 planes per matrix
+  b->partials = static_cast<float*>(cv.take(sizeof(float) * kNormParts * batch));
+  b->scale = static_cast<float*>(cv.take(sizeof(float) * batch));
+  for (int i = 0; i < 2; ++i) b->X[i] = static_cast<float*>(cv.take(mat));
+  for (int i = 0; i < 2; ++i) b->M[i] = static_cast<float*>(cv.take(mat));
+  b->T2 = static_cast<float*>(cv.take(mat));
+  b->T4 = static_cast<float*>(cv.take(mat));
+  b->cnt = static_cast<int*>(cv.take(kSchedBytes + sizeof(int) * kMaxClasses * batch * ceil_div(n, kBM)));
+}
+
+// (A + eps I)^(-1/4) by the coupled Newton iteration for inverse p-th roots
+// (p = 4): with T_j = (5 I - M_j) / 4,
+//   X_{j+1} = X_j T_j,   M_{j+1} = T_j^4 M_j,
+// from X_0 = s^(1/4) I and M_0 = s (A + eps I), which keeps M_j = X_j^4 (A + eps I)
+// and drives M_j to I and X_j to (A + eps I)^(-1/4).  Every matrix is a
+// polynomial in A, so every product is symmetric and runs on the triangle
+// schedule, in fp32-accurate arithmetic (3xTF32 on hi/lo planes).  Per step
+// four products: M M (T^2 in the epilogue: (25 I - 10 M + M M) / 16), T^2 T^2,
+// T^4 M, and X M (X T in the epilogue: 5/4 X - 1/4 X M); X_1 comes from the
+// start kernel, and the last X M writes the user's output with exact mirrors.
+msign_status root_run(const float* A, float* out, int64_t batch, int64_t n, float eps, int iters, void* workspace,
+                      cudaStream_t stream) {
+  const int64_t ldn = round_up(n, 8), pl = n * ldn;
+  Carver cv(workspace);
+  RootBuffers w;
+  carve_root(cv, batch, n, &w);
+  msign_status st = launch_norm(A, DT_FP32, n * n, n * n, batch, DT_FP32, eps, 1, w.partials, w.scale, stream);
+  if (st != MSIGN_OK) return st;
+  {
+    const int64_t blocks = std::min<int64_t>(ceil_div(n * n, 256), 1024);
+    dim3 g(static_cast<unsigned>(blocks), static_cast<unsigned>(batch));
+    prof_begin(stream);
+    inv_root_start_kernel<<<g, 256, 0, stream>>>(A, static_cast<int>(n), n * n, w.scale, eps, w.M[0], w.X[0], ldn,
+                                                 pl);
+    prof_end(3, stream, 0.0, static_cast<double>(batch) * n * n * 20.0);
+    st = launch_ok();
+    if (st != MSIGN_OK) return st;
+  }
+  Chain ch;
+  ch.state = w.cnt, ch.batch = batch, ch.rows = ceil_div(n, kBM), ch.ab_dt = DT_FP32, ch.stream = stream;
+  const int DEP_TMN = DEP_TM | DEP_TN;
+  auto planes = [&](float* p, float gamma) {
+    std::vector<EpiOut> v = split_out(p, ldn, pl);
+    for (EpiOut& e : v) e.gamma = gamma;
+    return v;
+  };
+  auto product = [&](float* a, float* b, float alpha, float beta, float* c, std::vector<EpiOut> outs) {
+    ClassSpec s;
+    s.A = Mat{a, DT_FP32, n, n, ldn, pl}, s.B = Mat{b, DT_FP32, n, n, ldn, pl};
+    s.symmetric = true, s.a_sym = true, s.b_sym = true, s.split = true;
+    s.M = n, s.N = n, s.K = n, s.batch = batch;
+    s.alpha = alpha, s.beta = beta;
+    if (c != nullptr) s.C = c, s.c_dt = DT_FP32, s.ldc = ldn, s.c_bs = 2 * pl, s.c_plane = pl;
+    s.outs = std::move(outs);
+    return s;
+  };
+  int cm = 0, cx = 0;  // M_{j-1} in M[cm], X_j in X[cx]
+  for (int j = 1; j < iters; ++j) {
+    st = ch.add(product(w.M[cm], w.M[cm], 1.0f / 16, -10.0f / 16, w.M[cm], planes(w.T2, 25.0f / 16)),
+                {{w.M[cm], DEP_TMN}}, w.M[cm], {w.T2});
+    if (st != MSIGN_OK) return st;
+    st = ch.add(product(w.T2, w.T2, 1.0f, 0.0f, nullptr, planes(w.T4, 0.0f)), {{w.T2, DEP_TMN}}, nullptr, {w.T4});
+    if (st != MSIGN_OK) return st;
+    st = ch.add(product(w.T4, w.M[cm], 1.0f, 0.0f, nullptr, planes(w.M[cm ^ 1], 0.0f)),
+                {{w.T4, DEP_TM}, {w.M[cm], DEP_TN}}, nullptr, {w.M[cm ^ 1]});
+    if (st != MSIGN_OK) return st;
+    cm ^= 1;
+    const bool last = j + 1 == iters;
+    ClassSpec x = product(w.X[cx], w.M[cm], -0.25f, 1.25f, w.X[cx],
+                          last ? std::vector<EpiOut>{out_to(out, DT_FP32, n, n * n, false)} : planes(w.X[cx ^ 1], 0.0f));
+    x.mirror = last;  // the user gets the full, exactly symmetric matrix
+    st = ch.add(x, {{w.X[cx], DEP_TM}, {w.M[cm], DEP_TN}}, w.X[cx],
+                {last ? static_cast<const void*>(out) : static_cast<const void*>(w.X[cx ^ 1])});
+    if (st != MSIGN_OK) return st;
+    cx ^= 1;
+  }
+  return ch.flush();
+}
+
+struct MousseBuffers {
+  void* Lb;  // bf16 L^(-1/4), rows x ldr
+  void* Rb;  // bf16 R^(-1/4), cols x ldc
+  void* B1;  // bf16 rows x ldc: G, then G~, then L^(-1/4) O
+  void* B2;  // bf16 rows x ldc: L^(-1/4) G, then O = msign(G~)
+  void* ns;  // msign workspace
+};
+
+void carve_mousse(Carver& cv, int64_t batch, int64_t rows, int64_t cols, MousseBuffers* b) {
+  const int64_t ldr = round_up(rows, 8), ldc = round_up(cols, 8);
+  b->Lb = cv.take(2ull * batch * rows * ldr);
+  b->Rb = cv.take(2ull * batch * cols * ldc);
+  b->B1 = cv.take(2ull * batch * rows * ldc);
+  b->B2 = cv.take(2ull * batch * rows * ldc);
+  b->ns = cv.take(msign_ns_workspace_size(batch, rows, cols, MSIGN_BF16));
+}
+
+}  // namespace msb
+
+extern "C" {
+
+size_t mousse_inv_root_workspace_size(int64_t batch, int64_t n) {
+  if (batch <= 0 || n <= 0) return 0;
+  Carver cv(nullptr);
+  RootBuffers b;
+  carve_root(cv, batch, n, &b);
+  return cv.off + 1024;
+}
+
+msign_status mousse_inv_root(const float* A, float* out, int64_t batch, int64_t n, float eps, int iters,
+                             void* workspace, size_t workspace_bytes, msign_stream_t stream) {
+  if (batch < 0 || n < 0 || !std::isfinite(eps) || eps < 0.0f) return MSIGN_ERR_INVALID_ARG;
+  if (iters <= 0) iters = kRootDefaultIters;
+  if (iters < 2 || iters > kRootMaxIters) return MSIGN_ERR_INVALID_ARG;
+  if (batch == 0 || n == 0) return MSIGN_OK;
+  if (A == nullptr || out == nullptr) return MSIGN_ERR_INVALID_ARG;
+  if (batch > 65535 || n > (1 << 20)) return MSIGN_ERR_UNSUPPORTED;
+  const size_t need = mousse_inv_root_workspace_size(batch, n);
+  if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
+    return MSIGN_ERR_WORKSPACE;
+  DeviceState* dev = nullptr;
+  msign_status st = device_state(&dev);
+  if (st != MSIGN_OK) return st;
+  return root_run(A, out, batch, n, eps, iters, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t mousse_direction_workspace_size(int64_t batch, int64_t rows, int64_t cols) {
+  if (batch <= 0 || rows <= 0 || cols <= 0) return 0;
+  Carver cv(nullptr);
+  MousseBuffers b;
+  carve_mousse(cv, batch, rows, cols, &b);
+  return cv.off + 1024;
+}
+
+msign_status mousse_direction(const void* G, void* out, msign_dtype io_dtype, int64_t batch, int64_t rows,
+                              int64_t cols, const float* L_root, const float* R_root, const msign_coeffs* coeffs,
+                              void* workspace, size_t workspace_bytes, msign_stream_t stream_) {
+  if (!valid_dtype(io_dtype) || batch < 0 || rows < 0 || cols < 0) return MSIGN_ERR_INVALID_ARG;
+  Schedule sch;
+  msign_status st = read_schedule(coeffs, kNsEps, &sch);
+  if (st != MSIGN_OK) return st;
+  if (sch.method != 0) return MSIGN_ERR_INVALID_ARG;  // standard NS inside the whitened space
+  if (batch == 0 || rows == 0 || cols == 0) return MSIGN_OK;
+  if (G == nullptr || out == nullptr || L_root == nullptr || R_root == nullptr) return MSIGN_ERR_INVALID_ARG;
+  if (batch > 65535 || rows > (1 << 30) || cols > (1 << 30)) return MSIGN_ERR_UNSUPPORTED;
+  const size_t need = mousse_direction_workspace_size(batch, rows, cols);
+  if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
+    return MSIGN_ERR_WORKSPACE;
+  DeviceState* dev = nullptr;
+  st = device_state(&dev);
+  if (st != MSIGN_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const int io = to_dt(io_dtype);
+  const int64_t ldr = round_up(rows, 8), ldc = round_up(cols, 8);
+  const int64_t rect = rows * ldc;
+  Carver cv(workspace);
+  MousseBuffers w;
+  carve_mousse(cv, batch, rows, cols, &w);
+  // bf16 operand copies of G and of the two roots
+  st = launch_ingest(ingest_args(G, io, rows, cols, false, DT_BF16, w.B1, DT_BF16, ldc, rect), batch, stream);
+  if (st != MSIGN_OK) return st;
+  st = launch_ingest(ingest_args(L_root, DT_FP32, rows, rows, false, DT_BF16, w.Lb, DT_BF16, ldr, rows * ldr), batch,
+                     stream);
+  if (st != MSIGN_OK) return st;
+  st = launch_ingest(ingest_args(R_root, DT_FP32, cols, cols, false, DT_BF16, w.Rb, DT_BF16, ldc, cols * ldc), batch,
+                     stream);
+  if (st != MSIGN_OK) return st;
+  const Mat Lm{w.Lb, DT_BF16, rows, rows, ldr, rows * ldr};
+  const Mat Rm{w.Rb, DT_BF16, cols, cols, ldc, cols * ldc};
+  // L^(-1/4) Y: Y (rows x cols) is the MN-major B operand
+  auto left = [&](void* y, std::vector<EpiOut> outs) {
+    ClassSpec s;
+    s.A = Lm, s.B = Mat{y, DT_BF16, rows, cols, ldc, rect}, s.b_mn = true;
+    s.M = rows, s.N = cols, s.K = rows, s.batch = batch;
+    s.outs = std::move(outs);
+    return launch_grouped({s}, DT_BF16, stream);
+  };
+  // Y R^(-1/4): R^(-1/4) is symmetric, so its rows are the K-major B operand
+  auto right = [&](void* y, std::vector<EpiOut> outs) {
+    ClassSpec s;
+    s.A = Mat{y, DT_BF16, rows, cols, ldc, rect}, s.B = Rm;
+    s.M = rows, s.N = cols, s.K = cols, s.batch = batch;
+    s.outs = std::move(outs);
+    return launch_grouped({s}, DT_BF16, stream);
+  };
+  st = left(w.B1, {out_to(w.B2, DT_BF16, ldc, rect, false)});  // L^(-1/4) G
+  if (st != MSIGN_OK) return st;
+  st = right(w.B2, {out_to(w.B1, DT_BF16, ldc, rect, false)});  // G~ = L^(-1/4) G R^(-1/4)
+  if (st != MSIGN_OK) return st;
+  st = ns_run(w.B1, DT_BF16, ldc, rect, w.B2, DT_BF16, ldc, rect, MSIGN_BF16, batch, rows, cols, sch, w.ns,
+              stream);  // O = msign(G~)
+  if (st != MSIGN_OK) return st;
+  st = left(w.B2, {out_to(w.B1, DT_BF16, ldc, rect, false)});  // L^(-1/4) O
+  if (st != MSIGN_OK) return st;
+  return right(w.B1, {out_to(out, io, cols, rows * cols, false)});  // ... R^(-1/4)
+}
+
+}  // extern "C"
+
 // ---------------------------------------------------------------- no-allocation variant
 //
 // Some callers cannot allocate device memory at the point where they need
@@ -1737,7 +1988,8 @@ msign_status msign_ns_noalloc(const void* in, void* out, msign_dtype io_dtype, i
   // row-block counters) with a cudaMemsetAsync on `stream` before use, and
   // writes every other buffer it carves before reading it, so what an
   // earlier call left in the array does not matter.
-  return msign_ns(in, out, io_dtype, MSIGN_BF16, batch, rows, cols, coeffs, scratch, kNoAllocScratchBytes, stream);
+  return msign_ns(in, out, io_dtype, MSIGN_BF16, batch, rows, cols, 0, 0, coeffs, scratch, kNoAllocScratchBytes,
+                  stream);
 }
 
 }  // extern "C"

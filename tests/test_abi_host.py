@@ -45,7 +45,7 @@ def test_exported_symbols_match_nm(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.msign_abi_version() == 102
+    assert L.msign_abi_version() == 103
     assert L.msign_status_string(_lib.OK) == b"ok"
     assert b"timed out" in L.msign_status_string(_lib.ERR_TIMEOUT)
     assert L.msign_status_string(99) == b"unknown status"
@@ -70,25 +70,25 @@ def test_workspace_queries_are_host_only(L):
 
 def test_invalid_arguments_rejected_on_host(L):
     # negative sizes and bad dtypes fail before any CUDA call
-    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, -1, 4, 4, None, None, 0, None) == _lib.ERR_INVALID_ARG
-    assert L.msign_ns(None, None, 7, _lib.BF16, 1, 4, 4, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, -1, 4, 4, 0, 0, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.msign_ns(None, None, 7, _lib.BF16, 1, 4, 4, 0, 0, None, None, 0, None) == _lib.ERR_INVALID_ARG
     # empty problems are a no-op
-    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 0, 4, 4, None, None, 0, None) == _lib.OK
-    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 3, 0, 4, None, None, 0, None) == _lib.OK
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 0, 4, 4, 0, 0, None, None, 0, None) == _lib.OK
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 3, 0, 4, 0, 0, None, None, 0, None) == _lib.OK
     # null data pointers with a non-empty problem
-    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 1, 4, 4, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 1, 4, 4, 0, 0, None, None, 0, None) == _lib.ERR_INVALID_ARG
     # a coefficient table needs a positive step count
     c = _lib.MsignCoeffs()
     buf = (ctypes.c_float * 3)(1.0, 0.0, 0.0)
     c.steps, c.abc, c.eps = 0, ctypes.cast(buf, ctypes.POINTER(ctypes.c_float)), -1.0
-    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == \
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 1, 4, 4, 0, 0, ctypes.byref(c), None, 0, None) == \
         _lib.ERR_INVALID_ARG
     c.steps = 100  # beyond the built maximum
-    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == \
+    assert L.msign_ns(None, None, _lib.BF16, _lib.BF16, 1, 4, 4, 0, 0, ctypes.byref(c), None, 0, None) == \
         _lib.ERR_UNSUPPORTED
     # workspace missing for a real problem (pointer values are never dereferenced on this path)
-    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, None, None, 0, None) == _lib.ERR_WORKSPACE
-    assert L.msign_ns(16, 16, _lib.BF16, _lib.FP32, 1, 4, 4, None, None, 0, None) == _lib.ERR_WORKSPACE
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, 0, 0, None, None, 0, None) == _lib.ERR_WORKSPACE
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.FP32, 1, 4, 4, 0, 0, None, None, 0, None) == _lib.ERR_WORKSPACE
     # the fp32-accurate path keeps two fp32 planes per operand: larger workspace
     assert L.msign_ns_workspace_size(1, 512, 512, _lib.FP32) > L.msign_ns_workspace_size(1, 512, 512, _lib.BF16)
 
@@ -98,12 +98,12 @@ def test_init_option_validation(L):
     # operands and is a standard-NS option
     c = _lib.MsignCoeffs()
     c.steps, c.abc, c.eps, c.init = 0, None, -1.0, 2
-    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, 0, 0, ctypes.byref(c), None, 0, None) == _lib.ERR_INVALID_ARG
     c.init = 1
-    assert L.msign_ns(16, 16, _lib.BF16, _lib.FP32, 1, 4, 4, ctypes.byref(c), None, 0, None) == _lib.ERR_UNSUPPORTED
-    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, ctypes.byref(c), None, 0, None, 0, None) == _lib.ERR_UNSUPPORTED
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.FP32, 1, 4, 4, 0, 0, ctypes.byref(c), None, 0, None) == _lib.ERR_UNSUPPORTED
+    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, 0, 0, ctypes.byref(c), None, 0, None, 0, None) == _lib.ERR_UNSUPPORTED
     # bf16 with init = 1 passes the argument checks (fails only on the missing workspace)
-    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == _lib.ERR_WORKSPACE
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, 0, 0, ctypes.byref(c), None, 0, None) == _lib.ERR_WORKSPACE
 
 
 def _route(L, batch, rows, cols, compute=_lib.BF16, method=1, init=0, steps=0):
@@ -155,7 +155,7 @@ def test_route_workspace_fits(L):
 def test_method_field_validation(L):
     c = _lib.MsignCoeffs()
     c.steps, c.abc, c.eps, c.init, c.method = 0, None, -1.0, 0, 1
-    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, ctypes.byref(c), None, -1, 16, 1 << 20, None) == \
+    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, 0, 0, ctypes.byref(c), None, -1, 16, 1 << 20, None) == \
         _lib.ERR_INVALID_ARG
     one = (ctypes.c_void_p * 1)(16)
     rows = (ctypes.c_int64 * 1)(8)
@@ -167,7 +167,7 @@ def test_method_field_validation(L):
     c.method = 3
     assert L.muon_step(1, one, one, one, rows, cols, _lib.BF16, _lib.BF16, 0.95, 0.02, ctypes.byref(c), None, 0,
                        None) == _lib.ERR_INVALID_ARG
-    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, ctypes.byref(c), None, 0, None) == \
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 1, 4, 4, 0, 0, ctypes.byref(c), None, 0, None) == \
         _lib.ERR_INVALID_ARG
 
 
@@ -178,10 +178,10 @@ def test_selftest_timeout_validation(L):
 
 def test_gram_ns_restart_validation(L):
     r = (ctypes.c_int * 1)(5)  # must lie in 1..T-1
-    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, None, ctypes.cast(r, ctypes.POINTER(ctypes.c_int)), 1, None, 0,
+    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, 0, 0, None, ctypes.cast(r, ctypes.POINTER(ctypes.c_int)), 1, None, 0,
                      None) == _lib.ERR_INVALID_ARG
-    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, None, None, 2, None, 0, None) == _lib.ERR_INVALID_ARG
-    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, None, None, -1, None, 0, None) == _lib.ERR_WORKSPACE
+    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, 0, 0, None, None, 2, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.gram_ns(16, 16, _lib.BF16, 1, 4, 8, 0, 0, None, None, -1, None, 0, None) == _lib.ERR_WORKSPACE
 
 
 def test_muon_step_validation(L):
@@ -229,3 +229,65 @@ def test_binding_rejects_tensors_on_another_device():
         msb._same_device(torch.empty(1), torch.device("cuda", 0), "out")
     msb._same_device(torch.empty(1), torch.device("cpu"), "out")
     msb._same_device(None, torch.device("cuda", 0), "workspace")
+
+
+def test_batch_strides_validated_on_host(L):
+    # a stride is 0 (back to back) or at least one matrix; overlapping
+    # matrices are rejected before anything else is looked at
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 2, 4, 4, 15, 0, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 2, 4, 4, 0, -1, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.gram_ns(16, 16, _lib.BF16, 2, 4, 8, 31, 0, None, None, -1, None, 0, None) == _lib.ERR_INVALID_ARG
+    # valid strides pass the checks (and fail only on the missing workspace)
+    assert L.msign_ns(16, 16, _lib.BF16, _lib.BF16, 2, 4, 4, 16, 48, None, None, 0, None) == _lib.ERR_WORKSPACE
+    assert L.gram_ns(16, 16, _lib.BF16, 2, 4, 8, 64, 32, None, None, -1, None, 0, None) == _lib.ERR_WORKSPACE
+
+
+def test_binding_batch_layout():
+    import torch
+
+    import newton_schulz_msign_b200 as msb
+
+    class FakeCuda:
+        """Shape and strides of a tensor, posing as a CUDA tensor."""
+
+        is_cuda = True
+
+        def __init__(self, t):
+            self.t = t
+            self.shape = t.shape
+
+        def dim(self):
+            return self.t.dim()
+
+        def stride(self, d):
+            return self.t.stride(d)
+
+    big = torch.empty(5, 3, 7, 9)
+    assert msb._batch_layout(FakeCuda(big), "x") == (15, 7, 9, 0)
+    assert msb._batch_layout(FakeCuda(big[:, 1]), "x") == (5, 7, 9, 3 * 63)
+    assert msb._batch_layout(FakeCuda(big[1:4:2, 2]), "x") == (2, 7, 9, 2 * 3 * 63)
+    with pytest.raises(ValueError):
+        msb._batch_layout(FakeCuda(big[1:4:2]), "x")  # leading dims without one common stride
+    with pytest.raises(ValueError):
+        msb._batch_layout(FakeCuda(big[..., ::2]), "x")  # matrix not dense
+    assert msb._batch_layout(FakeCuda(big[0, 0]), "x") == (1, 7, 9, 0)
+
+
+def test_mousse_arguments_validated_on_host(L):
+    F32 = ctypes.c_float
+    # inverse root: eps must be finite and >= 0, iters in [2, 1000] (0: default)
+    assert L.mousse_inv_root(16, 16, 1, 8, F32(-1.0), 0, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.mousse_inv_root(16, 16, 1, 8, F32(0.1), 1, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.mousse_inv_root(16, 16, 1, 8, F32(0.1), 1001, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.mousse_inv_root(None, None, 0, 8, F32(0.1), 0, None, 0, None) == _lib.OK
+    assert L.mousse_inv_root(None, 16, 1, 8, F32(0.1), 0, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.mousse_inv_root(16, 16, 1, 8, F32(0.1), 0, None, 0, None) == _lib.ERR_WORKSPACE
+    assert L.mousse_inv_root_workspace_size(1, 8) > 0
+    # direction: every matrix pointer is needed; method must be 0
+    assert L.mousse_direction(16, 16, _lib.BF16, 1, 8, 16, None, 16, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    c = _lib.MsignCoeffs()
+    c.steps, c.abc, c.eps, c.init, c.method = 0, None, -1.0, 0, 1
+    assert L.mousse_direction(16, 16, _lib.BF16, 1, 8, 16, 16, 16, ctypes.byref(c), None, 0, None) == \
+        _lib.ERR_INVALID_ARG
+    assert L.mousse_direction(16, 16, _lib.BF16, 1, 8, 16, 16, 16, None, None, 0, None) == _lib.ERR_WORKSPACE
+    assert L.mousse_direction_workspace_size(1, 8, 16) > L.msign_ns_workspace_size(1, 8, 16, _lib.BF16)

@@ -288,3 +288,43 @@ def test_in_place(shape, compute, method):
     msb.msign_ns(y, y, compute=compute, method=method)
     msb.sync_status()
     assert torch.equal(y, ref)
+
+
+# ---------------------------------------------------------------- batch strides
+
+@pytest.mark.parametrize("compute,method", [("bf16", "standard"), ("fp16", "standard"), ("fp32", "standard"),
+                                            ("bf16", "auto")])
+def test_strided_batch_views(compute, method):
+    # every other matrix of a larger batch, in and out: the same result as the
+    # packed batch, matrix for matrix, and the matrices in between untouched
+    shape = (512, 4608) if method == "auto" else (96, 200)
+    big = torch.from_numpy(synth.gaussian((3, 2) + shape, seed=61)).to(torch.bfloat16).cuda()
+    x = big[:, 1]
+    assert not x.is_contiguous()
+    ref = msb.msign_ns(x.contiguous(), compute=compute, method=method)
+    out_big = torch.full_like(big, 5.0)
+    y = msb.msign_ns(x, out_big[:, 0], compute=compute, method=method)
+    msb.sync_status()
+    assert torch.equal(y, ref)
+    assert torch.equal(out_big[:, 0], ref)
+    assert bool((out_big[:, 1] == 5.0).all())
+    cast = {"bf16": "bf16", "fp16": "fp16", "fp32": None}[compute]
+    if method == "standard":
+        tol = TOL_FP32 if compute == "fp32" else TOL_BF16
+        assert rel_fro(to_np(y), O.msign_ns(to_np(x), input_cast=cast)) < tol
+    # in place on the strided view
+    z = big.clone()
+    msb.msign_ns(z[:, 1], z[:, 1], compute=compute, method=method)
+    msb.sync_status()
+    assert torch.equal(z[:, 1], ref)
+    assert torch.equal(z[:, 0], big[:, 0])
+
+
+def test_gram_ns_strided_batch_view():
+    big = torch.from_numpy(synth.gaussian((4, 3, 128, 384), seed=62)).to(torch.bfloat16).cuda()
+    x = big[:, 2]
+    ref = msb.gram_ns(x.contiguous())
+    y = msb.gram_ns(x)
+    msb.sync_status()
+    assert torch.equal(y, ref)
+    assert rel_fro(to_np(y), O.gram_ns(to_np(x))) < TOL_BF16
