@@ -14,24 +14,26 @@
 // Each SM thus streams half of B per FLOP compared with a one-SM 128 x 256
 // tile, which is what keeps the tensor pipe fed from L2.
 //
-// Roles inside each 192-thread CTA (one CTA per SM, persistent over tiles):
+// Roles inside each CTA of 2 + kEpiWarps warps (one CTA per SM, persistent
+// over tiles):
 //   warp 0      TMA producer, in both CTAs: loads this CTA's halves of A and
 //               B (128 x 64 elements each, 128-byte swizzle) into a
 //               kStages-deep ring; completion is counted on the LEADER's
 //               stage barrier, which expects the bytes of both CTAs.
 //   warp 1      allocates 512 TMEM columns in both CTAs (two 128 x 256 fp32
-//               accumulators per CTA); in the leader one thread issues the
-//               MMAs and tcgen05.commit-multicasts stage releases and
-//               accumulator-ready signals to both CTAs.
-//   warps 2..5  epilogue, in both CTAs: tcgen05.ld of this CTA's 128
-//               accumulator rows (warp w reads TMEM lanes 32*(w%4)..+31),
-//               fused arithmetic v = alpha*acc + beta*C, then up to
-//               kMaxOuts stores, each direct or transposed and each with its
-//               own gamma*I term.  Every 32x32 block moves between registers
-//               and global memory through a swizzled shared-memory block, so
-//               all global accesses are coalesced 16-byte row segments.  One
-//               lane per warp then releases the accumulator on the leader's
-//               barrier.
+//               accumulators per CTA); in the leader it issues the MMAs and
+//               tcgen05.commit-multicasts stage releases and accumulator-ready
+//               signals to both CTAs.
+//   warps 2..   epilogue, in both CTAs: tcgen05.ld of this CTA's 128
+//               accumulator rows (warp w reads TMEM lanes 32*(w%4)..+31, two
+//               warps per lane quarter, each half of the columns), fused
+//               arithmetic v = alpha*acc + beta*C, then up to kMaxOuts stores,
+//               each direct or transposed and each with its own gamma*I term.
+//               One lane per warp then releases the accumulator on the
+//               leader's barrier.
+// The producer and MMA warps run their loops warp-converged and issue each
+// TMA load, MMA and commit from one elected lane (see "warp-converged issue"
+// in ptx_sm100.cuh).
 //
 // Symmetric classes ([P1] flash-muon matmul_transpose; [P3] section 4,
 // triangular scheduler) enumerate only tiles (tm, tn) with tn >= tm.  A
@@ -616,15 +618,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
+    // The whole warp runs the loop (see "warp-converged issue" in
+    // ptx_sm100.cuh): lane 0 claims tiles and broadcasts them, every lane
+    // waits on the barriers and counters (so that each has its own acquire),
+    // and one elected lane issues each load.
+    {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t used = 0, last_phase = 0;  // per-stage bits (leader only)
       bool ok = true;
-      const uint32_t sA0 = smem_u32(sA), sB0 = smem_u32(sB);
       for (int seq = 0; ok; ++seq) {
-        int t;
-        if (!next_tile(p, pair, num_pairs, leader, seq, s_abort, limit, &t)) {
+        int t = 0, got = 1;
+        if (lane == 0) got = next_tile(p, pair, num_pairs, leader, seq, s_abort, limit, &t) ? 1 : 0;
+        got = __shfl_sync(0xFFFFFFFFu, got, 0);
+        t = __shfl_sync(0xFFFFFFFFu, t, 0);
+        if (!got) {
           ok = false;
           break;
         }
@@ -647,30 +655,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const void* tmB2 = &g.tmB2;
         if (k.num_deps > 0) {
           // operands produced earlier in this launch (and earlier readers of
-          // the buffers this tile overwrites): wait for their row blocks
-          for (int e = 0; e < k.num_deps && ok; ++e) {
+          // the buffers this tile overwrites): wait for their row blocks.
+          // Every lane waits, so the elected lane that issues the loads has
+          // its own acquire.
+          bool dok = true;
+          for (int e = 0; e < k.num_deps && dok; ++e) {
             const RowDep& d = k.deps[e];
             if (d.mode & DEP_EPI) continue;
             const int* base = d.ptr + static_cast<long long>(tc.b) * d.rows;
             if (d.mode & DEP_ALL) {
-              for (int r = 0; r < d.rows && ok; ++r) ok = wait_counter(base + r, d.target, s_abort, p.err, limit);
+              for (int r = 0; r < d.rows && dok; ++r) dok = wait_counter(base + r, d.target, s_abort, p.err, limit);
             } else {
-              if (d.mode & DEP_TM) ok = ok && wait_counter(base + tc.tm, d.target, s_abort, p.err, limit);
-              if (d.mode & DEP_TN) ok = ok && wait_counter(base + tc.tn, d.target, s_abort, p.err, limit);
+              if (d.mode & DEP_TM) dok = dok && wait_counter(base + tc.tm, d.target, s_abort, p.err, limit);
+              if (d.mode & DEP_TN) dok = dok && wait_counter(base + tc.tn, d.target, s_abort, p.err, limit);
             }
           }
-          if (!ok) break;
+          if (!__all_sync(0xFFFFFFFFu, dok)) {
+            ok = false;
+            break;
+          }
           fence_proxy_async_global();
         }
         for (int step = 0; step < nk * passes; ++step) {
           const int kb = step / passes, pass = step - kb * passes;
           const int za = passes == 1 ? tc.b : 2 * tc.b + (pass == 2 ? 1 : 0);
           const int zb = passes == 1 ? tc.b : 2 * tc.b + (pass == 1 ? 1 : 0);
-          if (!wait_bounded(&empty[stage], phase ^ 1u, s_abort, p.err, limit)) {
+          if (!__all_sync(0xFFFFFFFFu, wait_bounded(&empty[stage], phase ^ 1u, s_abort, p.err, limit))) {
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+          if (leader) mbar_arrive_expect_tx_w(&full[stage], 2 * kStageBytes);
           const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = sA + stage * kATileBytes;
           uint8_t* b_dst = sB + stage * kBTileBytes;
@@ -679,17 +693,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // stored transpose: rows k0.. of S, columns arow..arow+127 (MN-major)
 #pragma unroll
             for (int c = 0; c < OK::chunks; ++c)
-              tma_load_3d_pair(a_dst + c * OK::chunk_bytes, tmA2, fbar, arow + c * OK::mn_chunk, k0, za);
+              tma_load_3d_pair_w(a_dst + c * OK::chunk_bytes, tmA2, fbar, arow + c * OK::mn_chunk, k0, za);
           } else {
-            tma_load_3d_pair(a_dst, tmA, fbar, k0, arow, za);
+            tma_load_3d_pair_w(a_dst, tmA, fbar, k0, arow, za);
           }
           if (kb < b_tr || b_mn) {
             const void* tm = (kb < b_tr) ? tmB2 : tmB;
 #pragma unroll
             for (int c = 0; c < OK::chunks; ++c)
-              tma_load_3d_pair(b_dst + c * OK::chunk_bytes, tm, fbar, bcol + c * OK::mn_chunk, k0, zb);
+              tma_load_3d_pair_w(b_dst + c * OK::chunk_bytes, tm, fbar, bcol + c * OK::mn_chunk, k0, zb);
           } else {
-            tma_load_3d_pair(b_dst, tmB, fbar, k0, bcol, zb);
+            tma_load_3d_pair_w(b_dst, tmB, fbar, k0, bcol, zb);
           }
           used |= 1u << stage;
           last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
@@ -699,18 +713,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
       }
-      (void)sA0;
-      (void)sB0;
       // Never leave the pair with bulk copies still landing: the leader's
       // stage barriers count both CTAs' bytes, so the leader waits (bounded,
       // ignoring the abort word) for the last phase issued into each stage.
-      if (leader)
+      if (leader && lane == 0)
         for (int s = 0; s < kStages; ++s)
           if ((used >> s) & 1u) wait_bounded(&full[s], (last_phase >> s) & 1u, nullptr, p.err, limit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
-    if (lane == 0 && leader) {
+    // The whole warp runs the loop; every lane waits, one elected lane issues
+    // each MMA and commit (see "warp-converged issue" in ptx_sm100.cuh).
+    if (leader) {
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
@@ -724,9 +738,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint64_t dA_k = smem_desc_sw128(sA0, 16, 1024), dA_mn = smem_desc_sw128(sA0, OK::chunk_bytes, OK::mn_sbo, OK::mn_layout);
       const uint64_t dB_k = smem_desc_sw128(sB0, 16, 1024), dB_mn = smem_desc_sw128(sB0, OK::chunk_bytes, OK::mn_sbo, OK::mn_layout);
       for (int seq = 0; ok; ++seq) {
-        int t;
-        if (!next_tile(p, pair, num_pairs, false, seq, s_abort, limit, &t)) break;
-        if (t >= p.total_tiles) break;
+        int t = 0, got = 1;
+        if (lane == 0) got = next_tile(p, pair, num_pairs, false, seq, s_abort, limit, &t) ? 1 : 0;
+        got = __shfl_sync(0xFFFFFFFFu, got, 0);
+        t = __shfl_sync(0xFFFFFFFFu, t, 0);
+        if (!got || t >= p.total_tiles) break;
         const TileCoord tc = decode_tile(p, t);
         const ClassInfo& k = p.cls[tc.c].info;
         const int nk = (k.K + OK::bke - 1) / OK::bke;
@@ -734,12 +750,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int ko = k.k_begin / OK::bke;
         const int a_tr = k.a_sym ? (tc.tm * kBM) / OK::bke - ko : 0;
         const int b_tr = k.b_sym ? (tc.tn * kBN) / OK::bke - ko : (k.b_mn_major ? nk : 0);
-        if (!wait_bounded(&tempty[buf], bphase ^ 1u, s_abort, p.err, limit)) break;
+        if (!__all_sync(0xFFFFFFFFu, wait_bounded(&tempty[buf], bphase ^ 1u, s_abort, p.err, limit))) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
         for (int step = 0; step < nk * passes; ++step) {
           const int kb = step / passes;
-          if (!wait_bounded(&full[stage], phase, s_abort, p.err, limit)) {
+          if (!__all_sync(0xFFFFFFFFu, wait_bounded(&full[stage], phase, s_abort, p.err, limit))) {
             ok = false;
             break;
           }
@@ -755,24 +771,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < OK::bke / OK::kmma; ++kk) {
             const uint32_t acc = (step | kk) != 0 ? 1u : 0u;
             if (TF32)
-              umma_tf32_pair(d_tmem, da + kk * sa, db + kk * sb, idesc, acc);
+              umma_tf32_pair_w(d_tmem, da + kk * sa, db + kk * sb, idesc, acc);
             else
-              umma_f16_pair(d_tmem, da + kk * sa, db + kk * sb, idesc, acc);
+              umma_f16_pair_w(d_tmem, da + kk * sa, db + kk * sb, idesc, acc);
           }
-          umma_commit_pair_mc(&empty[stage], 0x3);
+          umma_commit_pair_mc_w(&empty[stage], 0x3);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit_pair_mc(&tfull[buf], 0x3);
+        umma_commit_pair_mc_w(&tfull[buf], 0x3);
         buf ^= 1;
         if (buf == 0) bphase ^= 1u;
       }
       // every MMA issued so far has finished before TMEM is released
-      umma_commit_pair_mc(drain, 0x1);
-      wait_bounded(drain, 0, nullptr, p.err, limit);
+      umma_commit_pair_mc_w(drain, 0x1);
+      if (lane == 0) wait_bounded(drain, 0, nullptr, p.err, limit);
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
