@@ -160,6 +160,7 @@ struct ClassInfo {
   int M, N, K, batch;
   int tiles_m, tiles_n, tiles_per_batch, tile_begin;
   int symmetric;   // output tiles (tm, tn) with tn >= tm only
+  int group;       // tile order: bands of `group` tile rows, column by column inside a band (1: row by row)
   int mirror;      // symmetric: every tile also stores its mirror (full, exactly symmetric matrix)
   int a_sym;       // A operand is a symmetric matrix stored by upper 256-blocks
   int b_sym;       // same for the B operand (K-major)
@@ -238,6 +239,13 @@ struct TileCoord {
   int c, b, tm, tn;
 };
 
+// Tile order inside a class.  group = 1: row by row (the order that lets a
+// chained phase start on the first finished row blocks of the one before).
+// group = G > 1: bands of G tile rows; inside a band, column by column and
+// top to bottom, so that the tiles a wave of CTA pairs works on at once share
+// G row blocks of A and a few column blocks of B -- a working set that stays
+// in L2 where the whole operand would not.  Symmetric classes keep only the
+// tiles with tn >= tm: a band's first G columns form a triangle.
 __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
   int c = 0;
   while (c + 1 < p.num_classes && t >= p.cls[c + 1].info.tile_begin) ++c;
@@ -246,19 +254,46 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
   int b = l / k.tiles_per_batch;
   int r = l - b * k.tiles_per_batch;
   int tm, tn;
-  if (!k.symmetric) {
-    tm = r / k.tiles_n;
-    tn = r - tm * k.tiles_n;
-  } else {
-    // square 256 x 256 tiles on or above the diagonal, row by row
-    tm = 0;
-    while (true) {
-      int cnt = k.tiles_n - tm;
-      if (r < cnt) break;
-      r -= cnt;
-      ++tm;
+  const int G = k.group;
+  if (G <= 1) {
+    if (!k.symmetric) {
+      tm = r / k.tiles_n;
+      tn = r - tm * k.tiles_n;
+    } else {
+      // square 256 x 256 tiles on or above the diagonal, row by row
+      tm = 0;
+      while (true) {
+        int cnt = k.tiles_n - tm;
+        if (r < cnt) break;
+        r -= cnt;
+        ++tm;
+      }
+      tn = tm + r;
     }
-    tn = tm + r;
+  } else {
+    int g0 = 0;
+    while (true) {
+      const int gh = min(G, k.tiles_m - g0);
+      // tiles of the band: symmetric, a gh-row triangle then full columns
+      const int tri = k.symmetric ? gh * (gh + 1) / 2 : 0;
+      const int first = k.symmetric ? g0 : 0;  // first column of the band
+      const int cnt = tri + gh * (k.tiles_n - first - (k.symmetric ? gh : 0));
+      if (r < cnt || g0 + gh >= k.tiles_m) {
+        if (r < tri) {
+          int col = 0;
+          while ((col + 1) * (col + 2) / 2 <= r) ++col;
+          tn = first + col;
+          tm = g0 + (r - col * (col + 1) / 2);
+        } else {
+          const int rr = r - tri;
+          tn = first + (k.symmetric ? gh : 0) + rr / gh;
+          tm = g0 + rr % gh;
+        }
+        break;
+      }
+      r -= cnt;
+      g0 += gh;
+    }
   }
   return {c, b, tm, tn};
 }

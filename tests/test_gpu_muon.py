@@ -174,3 +174,41 @@ def test_muon_auto_route_mixed():
         # and the standard-NS update agrees within the same tolerance
         w_std, _, _ = O.muon_step(to_np(W0[i]), to_np(M0[i]), to_np(G[i]), momentum=0.95, lr=0.02, input_cast="bf16")
         assert rel_fro(w_ref - to_np(W0[i]), w_std - to_np(W0[i])) < TOL_BF16
+
+
+def test_muon_llama_stack_one_step():
+    # the whole 32-layer Llama-3-8B stack (224 matrices, ~7e9 parameters) in
+    # one call, as the Muon workload runs it: bf16 weights, fp32 momenta from
+    # zero, bf16 G ~ N(0, 1e-4^2).  After the step every matrix is finite and
+    # one matrix of each distinct shape -- q (4096^2), k (1024x4096), gate
+    # (14336x4096, tall) and down (4096x14336) -- matches the oracle; the
+    # spot checks sit in different layers of the stack.
+    layer = [(r, c) for _, r, c in synth.llama3_8b_layer_shapes()]
+    shapes = layer * synth.LLAMA3_8B_LAYERS
+    W = [synth.gaussian_torch(s, seed=7000 + i, device="cuda", std=0.02, dtype=torch.bfloat16)
+         for i, s in enumerate(shapes)]
+    M = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in shapes]
+    G = [synth.gaussian_torch(s, seed=9000 + i, device="cuda", std=1e-4, dtype=torch.bfloat16)
+         for i, s in enumerate(shapes)]
+    picks = [7 * 3 + 0, 7 * 11 + 1, 7 * 20 + 4, 7 * 31 + 6]  # q, k, gate, down in layers 3, 11, 20, 31
+    W0 = {i: W[i].clone() for i in picks}
+    # the automatic route: q, k, v, o run standard NS, gate, up and down
+    # Gram NS (batched by shape), all in one call
+    method = "auto"
+    msb.muon_step(W, M, G, momentum=0.95, lr=0.02, method=method)
+    msb.sync_status()
+    for w in W:
+        assert torch.isfinite(w).all()
+    for i in picks:
+        r, c = shapes[i]
+        if method == "auto" and msb.msign_ns_route(1, r, c, method="auto") == "gram":
+            # Gram NS (fp16 inside) on the momentum M = G; the update against
+            # its own oracle and within the acceptance bound of standard NS
+            o_ref = O.gram_ns(to_np(M[i]))
+            dW_ref = -0.02 * math.sqrt(max(1.0, r / c)) * o_ref
+            w1 = to_np(W[i])
+            half_ulp = np.ldexp(1.0, np.frexp(np.abs(w1))[1] - 9)
+            excess = np.maximum(np.abs(w1 - (to_np(W0[i]) + dW_ref)) - half_ulp, 0.0)
+            assert np.linalg.norm(excess) <= TOL_BF16 * np.linalg.norm(dW_ref)
+        else:
+            check_matrix(W0[i], torch.zeros(shapes[i], device="cuda"), G[i], W[i], M[i], 0.02)
