@@ -161,6 +161,7 @@ struct ClassInfo {
   int tiles_m, tiles_n, tiles_per_batch, tile_begin;
   int symmetric;   // output tiles (tm, tn) with tn >= tm only
   int group;       // tile order: bands of `group` tile rows, column by column inside a band (1: row by row)
+  int bn;          // tile width: 256 or 128 output columns per CTA pair (N of each MMA)
   int mirror;      // symmetric: every tile also stores its mirror (full, exactly symmetric matrix)
   int a_sym;       // A operand is a symmetric matrix stored by upper 256-blocks
   int b_sym;       // same for the B operand (K-major)
@@ -237,6 +238,7 @@ static_assert(sizeof(GemmParams) <= 32764, "kernel parameter space");
 
 struct TileCoord {
   int c, b, tm, tn;
+  int tnb;  // the 256-row block of the tile's first column (= tn for 256-wide tiles)
 };
 
 // Tile order inside a class.  group = 1: row by row (the order that lets a
@@ -246,6 +248,14 @@ struct TileCoord {
 // G row blocks of A and a few column blocks of B -- a working set that stays
 // in L2 where the whole operand would not.  Symmetric classes keep only the
 // tiles with tn >= tm: a band's first G columns form a triangle.
+// Tile width of a class: a compile-time 256 in kernels built without narrow
+// tiles (the common case keeps its constant-folded code), else the class's.
+template <bool NARROW>
+__device__ __forceinline__ int tile_bn(const ClassInfo& k) {
+  return NARROW ? k.bn : kBN;
+}
+
+template <bool NARROW>
 __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
   int c = 0;
   while (c + 1 < p.num_classes && t >= p.cls[c + 1].info.tile_begin) ++c;
@@ -260,15 +270,17 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
       tm = r / k.tiles_n;
       tn = r - tm * k.tiles_n;
     } else {
-      // square 256 x 256 tiles on or above the diagonal, row by row
+      // tiles on or above the diagonal 256-block, row by row: row tm starts
+      // at the column tile of its diagonal block
+      const int per = kBM / tile_bn<NARROW>(k);
       tm = 0;
       while (true) {
-        int cnt = k.tiles_n - tm;
+        int cnt = k.tiles_n - tm * per;
         if (r < cnt) break;
         r -= cnt;
         ++tm;
       }
-      tn = tm + r;
+      tn = tm * per + r;
     }
   } else {
     int g0 = 0;
@@ -295,7 +307,7 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, int t) {
       g0 += gh;
     }
   }
-  return {c, b, tm, tn};
+  return {c, b, tm, tn, (tn * tile_bn<NARROW>(k)) / kBM};
 }
 
 // ---------------------------------------------------------------- blocked fp32 layout
@@ -595,7 +607,7 @@ __device__ __forceinline__ bool next_tile(const GemmParams& p, int pair, int num
 
 // Launched with clusters of 2 CTAs along x; gridDim.x is even.  TF32 selects
 // the operand kind (see OpKind).
-template <bool TF32>
+template <bool TF32, bool NARROW>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_sm100_kernel(const __grid_constant__ GemmParams p) {
   using OK = OpKind<TF32>;
@@ -672,16 +684,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           break;
         }
         if (t >= p.total_tiles) break;
-        const TileCoord tc = decode_tile(p, t);
+        const TileCoord tc = decode_tile<NARROW>(p, t);
         const ClassInfo& k = p.cls[tc.c].info;
         // per-tile state in registers
         const int nk = (k.K + OK::bke - 1) / OK::bke;
         const int passes = k.split ? 3 : 1;  // split: hi*hi, hi*lo, lo*hi per K slice
         const int arow = tc.tm * kBM + static_cast<int>(rank) * kHalfM;
-        const int bcol = tc.tn * kBN + static_cast<int>(rank) * kHalfN;
+        const int bn = tile_bn<NARROW>(k);
+        const int bhalf = bn / 2;  // B rows (output columns) staged per CTA
+        const int bcol = tc.tn * bn + static_cast<int>(rank) * bhalf;
+        const int bch = bhalf / OK::mn_chunk;  // MN-major chunks of B per CTA
+        const uint32_t stage_tx = 2u * static_cast<uint32_t>(kATileBytes + bhalf * kRowBytes);  // both CTAs
         const int ko = k.k_begin / OK::bke;  // first K slice of this class (split K)
         const int a_tr = k.a_sym ? (tc.tm * kBM) / OK::bke - ko : 0;  // K slices below this read A transposed
-        const int b_tr = k.b_sym ? (tc.tn * kBN) / OK::bke - ko : 0;
+        // (B is stored by upper 256-blocks: the K slices below the 256-block of
+        // the tile's columns are read from the stored transpose)
+        const int b_tr = k.b_sym ? (tc.tnb * kBM) / OK::bke - ko : 0;
         const bool b_mn = k.b_mn_major != 0;
         const GemmClass& g = p.cls[tc.c];
         const void* tmA = &g.tmA;
@@ -702,7 +720,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               for (int r = 0; r < d.rows && dok; ++r) dok = wait_counter(base + r, d.target, s_abort, p.err, limit);
             } else {
               if (d.mode & DEP_TM) dok = dok && wait_counter(base + tc.tm, d.target, s_abort, p.err, limit);
-              if (d.mode & DEP_TN) dok = dok && wait_counter(base + tc.tn, d.target, s_abort, p.err, limit);
+              if (d.mode & DEP_TN) dok = dok && wait_counter(base + tc.tnb, d.target, s_abort, p.err, limit);
             }
           }
           if (!__all_sync(0xFFFFFFFFu, dok)) {
@@ -719,7 +737,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx_w(&full[stage], 2 * kStageBytes);
+          if (leader) mbar_arrive_expect_tx_w(&full[stage], stage_tx);
           const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
           uint8_t* a_dst = sA + stage * kATileBytes;
           uint8_t* b_dst = sB + stage * kBTileBytes;
@@ -736,7 +754,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const void* tm = (kb < b_tr) ? tmB2 : tmB;
 #pragma unroll
             for (int c = 0; c < OK::chunks; ++c)
-              tma_load_3d_pair_w(b_dst + c * OK::chunk_bytes, tm, fbar, bcol + c * OK::mn_chunk, k0, zb);
+              if (c < bch) tma_load_3d_pair_w(b_dst + c * OK::chunk_bytes, tm, fbar, bcol + c * OK::mn_chunk, k0, zb);
           } else {
             tma_load_3d_pair_w(b_dst, tmB, fbar, k0, bcol, zb);
           }
@@ -778,13 +796,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         got = __shfl_sync(0xFFFFFFFFu, got, 0);
         t = __shfl_sync(0xFFFFFFFFu, t, 0);
         if (!got || t >= p.total_tiles) break;
-        const TileCoord tc = decode_tile(p, t);
+        const TileCoord tc = decode_tile<NARROW>(p, t);
         const ClassInfo& k = p.cls[tc.c].info;
         const int nk = (k.K + OK::bke - 1) / OK::bke;
         const int passes = k.split ? 3 : 1;
         const int ko = k.k_begin / OK::bke;
         const int a_tr = k.a_sym ? (tc.tm * kBM) / OK::bke - ko : 0;
-        const int b_tr = k.b_sym ? (tc.tn * kBN) / OK::bke - ko : (k.b_mn_major ? nk : 0);
+        const int b_tr = k.b_sym ? (tc.tnb * kBM) / OK::bke - ko : (k.b_mn_major ? nk : 0);
+        // the MMA's N is the class's tile width
+        const uint32_t idesc_n =
+            NARROW ? (idesc0 & ~(0x3Fu << 17)) | (static_cast<uint32_t>(k.bn >> 3) << 17) : idesc0;
         if (!__all_sync(0xFFFFFFFFu, wait_bounded(&tempty[buf], bphase ^ 1u, s_abort, p.err, limit))) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
@@ -797,7 +818,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const bool a_mn = kb < a_tr;
           const bool b_mn = kb < b_tr;
-          const uint32_t idesc = idesc0 | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16);
+          const uint32_t idesc = idesc_n | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16);
           const uint64_t da = (a_mn ? dA_mn : dA_k) + static_cast<uint64_t>((stage * kATileBytes) >> 4);
           const uint64_t db = (b_mn ? dB_mn : dB_k) + static_cast<uint64_t>((stage * kBTileBytes) >> 4);
           const uint32_t sa = a_mn ? (OK::mn_kstep >> 4) : (32 >> 4);
@@ -829,9 +850,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;  // TMEM lane quarter this warp may read
     const int ew = warp - 2;  // epilogue warp index
-    // this warp's 32-column blocks of every tile: [jbeg, jend)
-    constexpr int kBlocksPerWarp = (kBN / 32) / (kEpiWarps / 4);
-    const int jbeg = (ew >> 2) * kBlocksPerWarp, jend = jbeg + kBlocksPerWarp;
     float* scratch = reinterpret_cast<float*>(sOut + ew * kStageOutBytes);
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
@@ -843,14 +861,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       got = __shfl_sync(0xFFFFFFFFu, got, 0);
       t = __shfl_sync(0xFFFFFFFFu, t, 0);
       if (!got || t >= p.total_tiles) break;
-      const TileCoord tc = decode_tile(p, t);
+      const TileCoord tc = decode_tile<NARROW>(p, t);
       const ClassInfo& k = p.cls[tc.c].info;
       const int row0 = tc.tm * kBM + static_cast<int>(rank) * kHalfM + q * 32;
-      // mirrored tiles visit only blocks on or above the diagonal
-      const bool mirror = k.symmetric && (k.mirror || tc.tm == tc.tn);
+      // this warp's 32-column blocks of the tile: [jbeg, jend) (two warps per
+      // TMEM lane quarter, each half of the tile's columns)
+      const int bn = tile_bn<NARROW>(k);
+      const int bpw = (bn / 32) / (kEpiWarps / 4);
+      const int jbeg = (ew >> 2) * bpw, jend = jbeg + bpw;
+      const int coln = tc.tn * bn;  // the tile's first column
+      // mirrored tiles (every tile of a mirror class, and the tiles inside a
+      // diagonal 256-block) visit only blocks on or above the diagonal
+      const bool mirror = k.symmetric && (k.mirror || tc.tm == tc.tnb);
       int jfirst = jbeg;
       if (mirror)
-        while (jfirst < jend && tc.tn * kBN + jfirst * 32 < row0) ++jfirst;
+        while (jfirst < jend && coln + jfirst * 32 < row0) ++jfirst;
       const bool has_c = k.C != nullptr;
       int ok = 1;
       if (has_c && k.c_dep >= 0) {
@@ -878,7 +903,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int r = 0; r < d.rows && eok; ++r) eok = wait_counter(base + r, d.target, s_abort, p.err, limit);
           } else {
             if (d.mode & DEP_TM) eok = eok && wait_counter(base + tc.tm, d.target, s_abort, p.err, limit);
-            if (d.mode & DEP_TN) eok = eok && wait_counter(base + tc.tn, d.target, s_abort, p.err, limit);
+            if (d.mode & DEP_TN) eok = eok && wait_counter(base + tc.tnb, d.target, s_abort, p.err, limit);
           }
         }
         if (!__all_sync(0xFFFFFFFFu, eok)) break;
@@ -887,8 +912,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ready, each next block's just before its accumulator load
       float cv[32];
       float sq = 0.0f;  // this lane's part of the tile's sum of squares (sumsq classes)
-      if (has_c && row0 < k.M && jfirst < jend && tc.tn * kBN + jfirst * 32 < k.N)
-        load_c(k, tc.b, row0, tc.tn * kBN + jfirst * 32, lane, cv);
+      if (has_c && row0 < k.M && jfirst < jend && coln + jfirst * 32 < k.N)
+        load_c(k, tc.b, row0, coln + jfirst * 32, lane, cv);
       // the epilogue coefficients of this lane's row, for every block of the tile
       float alpha = k.alpha, beta = k.beta;
       if (k.row_beta != nullptr && row0 + lane < k.M)
@@ -901,7 +926,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
 #pragma unroll 1
       for (int j = jfirst; j < jend; ++j) {
-        const int col0 = tc.tn * kBN + j * 32;
+        const int col0 = coln + j * 32;
         if (row0 >= k.M || col0 >= k.N) break;
         // (issued before the accumulator load, so that the two overlap)
         if (has_c && j > jfirst) load_c(k, tc.b, row0, col0, lane, cv);
@@ -944,7 +969,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           int* sg = k.sig + static_cast<long long>(tc.b) * k.tiles_m;
           red_release_gpu_add(sg + tc.tm, 1);
-          if (k.symmetric && tc.tn != tc.tm) red_release_gpu_add(sg + tc.tn, 1);
+          if (k.symmetric && tc.tnb != tc.tm) red_release_gpu_add(sg + tc.tnb, 1);
         }
       }
       buf ^= 1;

@@ -57,10 +57,14 @@ msign_status device_state(DeviceState** out) {
     if (major != 10 || minor != 0) return MSIGN_ERR_UNSUPPORTED;  // built for sm_100a only
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MSIGN_ERR_CUDA;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_err_word) != cudaSuccess) return MSIGN_ERR_CUDA;
-    if (cudaFuncSetAttribute(gemm_sm100_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(gemm_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-            cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_sm100_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm_sm100_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm_sm100_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm_sm100_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess)
       return MSIGN_ERR_CUDA;
     {
       cudaLaunchConfig_t cfg = {};
@@ -75,7 +79,8 @@ msign_status device_state(DeviceState** out) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, gemm_sm100_kernel<false>, &cfg) != cudaSuccess || clusters < 1) {
+      if (cudaOccupancyMaxActiveClusters(&clusters, gemm_sm100_kernel<false, false>, &cfg) != cudaSuccess ||
+          clusters < 1) {
         (void)cudaGetLastError();
         clusters = d.sms / 2;
       }
@@ -289,6 +294,7 @@ struct ClassSpec {
   bool a_sym = false;      // A is a symmetric matrix stored by upper 256-blocks
   bool b_sym = false;      // B likewise
   bool split = false;      // fp32-accurate: A and B are tf32 hi/lo planes (Mat.bs = plane stride)
+  int bn = kBN;            // tile width (output columns per CTA pair): 256, or 128 (see pick_bn)
   int64_t c_plane = 0;     // > 0: C is split, lo plane at C + c_plane elements
   int64_t M = 0, N = 0, K = 0, batch = 0;
   float alpha = 1.0f, beta = 0.0f;
@@ -327,9 +333,20 @@ int64_t triangle_tiles(int64_t n) {
 
 int64_t class_tiles(const ClassSpec& s) {
   if (s.M <= 0 || s.N <= 0 || s.batch <= 0) return 0;
-  const int64_t per = s.symmetric ? triangle_tiles(s.M) : ((s.M + kBM - 1) / kBM) * ((s.N + kBN - 1) / kBN);
+  const int64_t tm = (s.M + kBM - 1) / kBM, tn = (s.N + s.bn - 1) / s.bn;
+  // symmetric: row block r keeps the column tiles from its diagonal 256-block on
+  const int64_t per = s.symmetric ? tm * tn - (kBM / s.bn) * tm * (tm - 1) / 2 : tm * tn;
   return per * s.batch;
 }
+
+// Tile width of a product of an M x N output (batch entries): 128 where its
+// 256-wide tiles would leave CTA pairs idle (fewer tiles than kPlanPairs),
+// which halves each tile's MMA and epilogue time and doubles the tiles a
+// dependent phase can spread over.  A symmetric output takes 128 only when
+// every 256-row block holds two column tiles, so that each row block is
+// touched by the same number of tiles.  From the shapes alone (kPlanPairs,
+// not the device), like the split-K plans.
+int pick_bn(int64_t M, int64_t N, int64_t batch, bool symmetric);
 
 // Encodes and launches up to kMaxClasses classes of one operand dtype.
 // `ordered`: the classes form a chain (later classes read earlier outputs
@@ -381,7 +398,7 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     if (!s.b_mn) {
       b.rows = s.N;
       b.cols = kt;
-      if (!encode(&c.tmB, b, bke, kHalfN, zb)) return MSIGN_ERR_CUDA;
+      if (!encode(&c.tmB, b, bke, s.bn / 2, zb)) return MSIGN_ERR_CUDA;
     } else {
       b.rows = kt;
       b.cols = s.N;
@@ -393,7 +410,10 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
     ci.K = static_cast<int>(s.K);
     ci.batch = static_cast<int>(s.batch);
     ci.tiles_m = static_cast<int>((s.M + kBM - 1) / kBM);
-    ci.tiles_n = static_cast<int>((s.N + kBN - 1) / kBN);
+    if (s.bn != kBN && (s.bn != kBN / 2 || (s.symmetric && ((s.N + s.bn - 1) / s.bn) % 2 != 0) || s.sumsq != nullptr))
+      return MSIGN_ERR_INVALID_ARG;
+    ci.bn = s.bn;
+    ci.tiles_n = static_cast<int>((s.N + s.bn - 1) / s.bn);
     ci.tiles_per_batch = static_cast<int>(class_tiles(s) / s.batch);
     ci.tile_begin = static_cast<int>(total);
     ci.symmetric = s.symmetric ? 1 : 0;
@@ -403,7 +423,7 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
       // (measured: the row-by-row order re-read X 5x from DRAM in 8192^2 X X^T)
       const double fp = static_cast<double>(dtype_size(ab_dt)) * (s.split ? 2.0 : 1.0) *
                         (static_cast<double>(s.M) * kt + (s.A.ptr == s.B.ptr ? 0.0 : static_cast<double>(s.N) * kt));
-      ci.group = fp > kBandBytes ? kBand : 1;
+      ci.group = (fp > kBandBytes && s.bn == kBN) ? kBand : 1;
     }
     ci.mirror = (s.symmetric && s.mirror) ? 1 : 0;
     ci.a_sym = s.a_sym ? 1 : 0;
@@ -472,10 +492,20 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
   }
   if (ab_dt == DT_FP32) flops *= 3.0;  // three tf32 products per fp32-accurate product
   prof_begin(stream);
-  if (ab_dt == DT_FP32)
-    gemm_sm100_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(p);
-  else
-    gemm_sm100_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(p);
+  // the kernel built with per-class tile widths only where a class is narrow
+  bool narrow = false;
+  for (const ClassSpec& s : specs) narrow = narrow || s.bn != kBN;
+  if (ab_dt == DT_FP32) {
+    if (narrow)
+      gemm_sm100_kernel<true, true><<<grid, kThreads, kSmemBytes, stream>>>(p);
+    else
+      gemm_sm100_kernel<true, false><<<grid, kThreads, kSmemBytes, stream>>>(p);
+  } else {
+    if (narrow)
+      gemm_sm100_kernel<false, true><<<grid, kThreads, kSmemBytes, stream>>>(p);
+    else
+      gemm_sm100_kernel<false, false><<<grid, kThreads, kSmemBytes, stream>>>(p);
+  }
   prof_end(0, stream, flops, bytes);
   return cudaGetLastError() == cudaSuccess ? MSIGN_OK : MSIGN_ERR_CUDA;
 }
@@ -584,6 +614,14 @@ inline size_t state_bytes(int64_t batch, int64_t n, int items) {
 // depend on the device, because the workspace size is a host-only query.
 constexpr int kPlanPairs = 74;
 
+int pick_bn(int64_t M, int64_t N, int64_t batch, bool symmetric) {
+  ClassSpec s;
+  s.M = M, s.N = N, s.batch = batch, s.symmetric = symmetric;
+  if (class_tiles(s) >= kPlanPairs) return kBN;
+  if (symmetric && ceil_div(N, kBN / 2) % 2 != 0) return kBN;
+  return kBN / 2;
+}
+
 // K parts of the X X^T product (K = m) of a class whose triangle tiles
 // leave CTA pairs idle: whole 256-blocks, each at least 4096 long.  In the
 // chained iteration the split pays only there: measured on 1 x 2048 x 4096
@@ -680,12 +718,17 @@ void ns_specs(const NsClass& k, int cur, float a, float b, float c, bool first, 
   ClassSpec& s = *syrk;
   s = ClassSpec();
   s.A = X, s.B = X, s.symmetric = true, s.split = sp;
+  // 128-wide tiles where 256-wide ones would leave CTA pairs idle (X X^T
+  // split in K parts keeps 256); step 0's A A of the sharper normalisation
+  // keeps 256 for its per-tile sums of squares
+  s.bn = k.w.syrk_parts > 1 ? kBN : pick_bn(n, n, k.batch, true);
   s.M = n, s.N = n, s.K = m, s.batch = k.batch;
   s.outs = outs(k.w.A, ldn, pn);
 
   ClassSpec& q = *sqr;  // both operands read from A's upper blocks
   q = ClassSpec();
   q.A = A, q.B = A, q.symmetric = true, q.a_sym = true, q.b_sym = true, q.split = sp;
+  q.bn = (first && k.improved) ? kBN : pick_bn(n, n, k.batch, true);
   q.M = n, q.N = n, q.K = n, q.batch = k.batch;
   q.alpha = c, q.beta = b;
   q.C = k.w.A, q.c_dt = od, q.ldc = ldn, q.c_bs = zn, q.c_plane = sp ? pn : 0;
@@ -695,6 +738,7 @@ void ns_specs(const NsClass& k, int cur, float a, float b, float c, bool first, 
   ClassSpec& x = *bx;  // B read from its upper blocks
   x = ClassSpec();
   x.A = B, x.a_sym = true, x.B = X, x.b_mn = true, x.split = sp;
+  x.bn = pick_bn(n, m, k.batch, false);
   x.M = n, x.N = m, x.K = n, x.batch = k.batch;
   x.alpha = 1.0f, x.beta = a;
   if (!sp) x.row_beta = k.w.diag, x.row_beta_bs = n;
@@ -831,15 +875,20 @@ msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cu
         int* const base = ns_counter_base(k.w, k.batch);
         auto ctr = [&](int slot) { return base + static_cast<int64_t>(slot) * k.batch * rb; };
         const int rows = static_cast<int>(rb);
-        const int per_block_sym = static_cast<int>(kTileSignals * rb);                 // tiles touching a block of A or B
-        const int per_block_x = static_cast<int>(kTileSignals * ceil_div(k.m, kBN));  // tiles in a row block of X'
-        // the phase this one reads: the previous one in the order
+        // arrivals that complete a row block of a phase's output: kTileSignals
+        // per tile touching it, i.e. per column tile of the phase's width
+        auto per_block = [&](int ph) {
+          return static_cast<int>(kTileSignals * ceil_div(ph == 2 ? k.m : k.n, sp[ph].bn));
+        };
+        const int per_block_sym = per_block(0);  // the X X^T parts below
+        // the phase this one reads: the previous one in the order (the B X of
+        // the step before has the same shape and tile width as this step's)
         std::vector<RowDep> reads;
         if (it - 1 >= i) {
           const int ps = done[ci][it - 1 - i];
-          if (p == 0) reads = {RowDep{ctr(ps), rows, per_block_x, DEP_TM | DEP_TN}};
-          if (p == 1) reads = {RowDep{ctr(ps), rows, per_block_sym, DEP_TM | DEP_TN}};
-          if (p == 2) reads = {RowDep{ctr(ps), rows, per_block_sym, DEP_TM}};
+          if (p == 0) reads = {RowDep{ctr(ps), rows, per_block(2), DEP_TM | DEP_TN}};
+          if (p == 1) reads = {RowDep{ctr(ps), rows, per_block(0), DEP_TM | DEP_TN}};
+          if (p == 2) reads = {RowDep{ctr(ps), rows, per_block(1), DEP_TM}};
         }
         if (p == 0 && k.w.syrk_parts > 1) {
           // split K (see Chain::add_split): parts 0 .. P-2 store fp32
@@ -849,7 +898,7 @@ msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cu
           std::vector<RowDep> epi;
           for (int qq = 0; qq + 1 < P; ++qq) {
             ClassSpec c;
-            c.A = q.A, c.B = q.B, c.symmetric = true, c.split = q.split;
+            c.A = q.A, c.B = q.B, c.symmetric = true, c.split = q.split, c.bn = q.bn;
             c.M = q.M, c.N = q.N, c.batch = q.batch;
             c.K = len, c.k_begin = qq * len, c.k_total = k.m;
             c.outs = {out_blocked(k.w.part[qq], blk_ld(k.n), blk_size(k.n, k.n))};
@@ -1030,8 +1079,10 @@ struct Chain {
     }
     if (s.deps.size() > static_cast<size_t>(kMaxDeps)) return MSIGN_ERR_UNSUPPORTED;
     s.sig = counters(me);
-    const int64_t tiles_n = ceil_div(s.N, kBN);
-    target.push_back(static_cast<int>(kTileSignals * (s.symmetric ? rows : tiles_n)));
+    const int64_t tiles_n = ceil_div(s.N, s.bn);
+    // tiles touching a row block: a row of tiles, or for a symmetric output
+    // (tiles of both 256-wide halves of a row block count) the same number
+    target.push_back(static_cast<int>(kTileSignals * tiles_n));
     cls.push_back(s);
     for (const void* w : writes) {
       Buf& b = buf(w);
@@ -1060,7 +1111,7 @@ struct Chain {
     std::vector<std::pair<const void*, int>> last_reads = reads;
     for (int q = 0; q + 1 < parts; ++q) {
       ClassSpec c;
-      c.A = s.A, c.B = s.B, c.b_mn = s.b_mn, c.symmetric = s.symmetric, c.mirror = s.mirror;
+      c.A = s.A, c.B = s.B, c.b_mn = s.b_mn, c.symmetric = s.symmetric, c.mirror = s.mirror, c.bn = s.bn;
       c.a_sym = s.a_sym, c.b_sym = s.b_sym, c.split = s.split;
       c.M = s.M, c.N = s.N, c.batch = s.batch;
       c.K = len, c.k_begin = q * len, c.k_total = K;
@@ -1348,6 +1399,7 @@ msign_status gram_xxt(const void* X, msign_dtype x_dtype, void* A, msign_dtype a
   s.symmetric = true;
   s.mirror = true;  // the user gets the full, exactly symmetric matrix
   s.M = n, s.N = n, s.K = m, s.batch = batch;
+  s.bn = pick_bn(n, n, batch, true);
   const int ad = to_dt(a_dtype);
   s.outs = {out_to(A, ad, n, n * n, false)};
   return launch_grouped({s}, xd, stream);
@@ -1418,9 +1470,12 @@ msign_status gram_run(const void* in, int in_dt, void* out, int out_dt, int64_t 
   const int DEP_TMN = DEP_TM | DEP_TN;
   // split K for the symmetric products with few tiles and a long K
   auto parts_for = [&](int64_t K) { return gram_parts(batch, n, K); };
-  auto add_sym = [&](const ClassSpec& s, const std::vector<std::pair<const void*, int>>& reads, const void* c_buf,
+  // (products split in K keep 256-wide tiles; the others take pick_bn's width)
+  auto add_sym = [&](ClassSpec s, const std::vector<std::pair<const void*, int>>& reads, const void* c_buf,
                      const std::vector<const void*>& writes) {
-    return ch.add_split(s, parts_for(s.K), reads, c_buf, writes, w.part, blk_ld(n), blk_size(n, n));
+    const int parts = parts_for(s.K);
+    s.bn = parts > 1 ? kBN : pick_bn(n, n, batch, true);
+    return ch.add_split(s, parts, reads, c_buf, writes, w.part, blk_ld(n), blk_size(n, n));
   };
   int cur = 0;
   for (size_t seg = 0; seg + 1 < bounds.size(); ++seg) {
@@ -1491,6 +1546,7 @@ msign_status gram_run(const void* in, int in_dt, void* out, int out_dt, int64_t 
       ClassSpec s;
       s.A = sqm(w.Q[q]), s.a_sym = true, s.B = X, s.b_mn = true;
       s.M = n, s.N = m, s.K = n, s.batch = batch;
+      s.bn = pick_bn(n, m, batch, false);
       const bool final = seg + 2 == bounds.size();
       if (final && out == nullptr) {
         // the previous X copy is dead: the result takes its place
@@ -1849,6 +1905,7 @@ msign_status root_run(const float* A, float* out, int64_t batch, int64_t n, floa
     s.A = Mat{a, DT_FP32, n, n, ldn, pl}, s.B = Mat{b, DT_FP32, n, n, ldn, pl};
     s.symmetric = true, s.a_sym = true, s.b_sym = true, s.split = true;
     s.M = n, s.N = n, s.K = n, s.batch = batch;
+    s.bn = pick_bn(n, n, batch, true);
     s.alpha = alpha, s.beta = beta;
     if (c != nullptr) s.C = c, s.c_dt = DT_FP32, s.ldc = ldn, s.c_bs = 2 * pl, s.c_plane = pl;
     s.outs = std::move(outs);
@@ -1971,6 +2028,7 @@ msign_status mousse_direction(const void* G, void* out, msign_dtype io_dtype, in
     ClassSpec s;
     s.A = Lm, s.B = Mat{y, DT_BF16, rows, cols, ldc, rect}, s.b_mn = true;
     s.M = rows, s.N = cols, s.K = rows, s.batch = batch;
+    s.bn = pick_bn(rows, cols, batch, false);
     s.outs = std::move(outs);
     return launch_grouped({s}, DT_BF16, stream);
   };
@@ -1979,6 +2037,7 @@ msign_status mousse_direction(const void* G, void* out, msign_dtype io_dtype, in
     ClassSpec s;
     s.A = Mat{y, DT_BF16, rows, cols, ldc, rect}, s.B = Rm;
     s.M = rows, s.N = cols, s.K = cols, s.batch = batch;
+    s.bn = pick_bn(rows, cols, batch, false);
     s.outs = std::move(outs);
     return launch_grouped({s}, DT_BF16, stream);
   };
