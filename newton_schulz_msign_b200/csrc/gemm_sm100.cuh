@@ -107,8 +107,11 @@ struct OpKind {
   static constexpr uint32_t mn_sbo = TF32 ? 512u : 1024u;
 };
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
-constexpr int kScratchStride = 33;  // padded row of the per-warp 32 x 32 fp32 transpose scratch
-constexpr int kStageOutBytes = 32 * kScratchStride * 4;
+// Per-warp epilogue scratch: a 32 x 32 fp32 transpose block (XOR-swizzled
+// rows), or two 16-bit staging boxes of staged bulk stores.  A multiple of
+// 1024 bytes from a 1024-byte aligned base, so every box is aligned to its
+// swizzle pattern.
+constexpr int kStageOutBytes = 32 * 32 * 4;
 constexpr int kEpiBytes = kEpiWarps * kStageOutBytes;  // one scratch block per epilogue warp
 constexpr int kTmemCols = 512;
 constexpr int kMaxClasses = 16;
@@ -138,6 +141,10 @@ struct EpiOut {
   // diag[b * diag_bs + i] and stored as 0 in the matrix itself
   float* diag;
   long long diag_bs;
+  // 16-bit row-major output written by bulk tensor stores of staged 32 x 32
+  // blocks through the class's tmOut[o] (a 32 x 32 box over the stored
+  // matrix, 64-byte swizzle); 0: lane-per-row stores
+  int tma;
 };
 
 // One dependency of a class on an earlier class of the launch (its row-block
@@ -211,6 +218,7 @@ struct alignas(64) GemmClass {
   CUtensorMap tmB;   // K-major: (k, col, batch) box 64 x 128; MN-major: (col, k, batch) box 64 x 64
   CUtensorMap tmA2;  // a_sym: the same matrix with a 64 x 64 box, for transposed K slices
   CUtensorMap tmB2;  // b_sym: likewise
+  CUtensorMap tmOut[kMaxOuts];  // outputs with EpiOut::tma: (col, row, batch) of the stored matrix, box 32 x 32
   ClassInfo info;
 };
 
@@ -471,6 +479,54 @@ __device__ __forceinline__ void load_c(const ClassInfo& k, int b, int row0, int 
   }
 }
 
+// ---------------------------------------------------------------- staged bulk stores
+//
+// A 16-bit output block leaves through a 32 x 32 staging box in the warp's
+// scratch, which lane 0 hands to a bulk tensor store: whole lines reach L2
+// instead of one 16-byte piece of 32 different rows per store instruction.
+// The box has 64-byte rows in the tensor map's 64-byte swizzle: 16-byte
+// piece i of row r sits at piece i ^ ((r >> 1) & 3) of the row, so when lane
+// l writes piece i of its row l, each group of 8 lanes covers the 8 16-byte
+// bank groups of a 128-byte line (one wavefront per group).  A transposed
+// box is read out of the first by columns: lane l loads column l, 32
+// two-byte loads that each stay inside one 64-byte row.
+constexpr int kBoxBytes = 32 * 32 * 2;
+static_assert(2 * kBoxBytes <= kStageOutBytes, "two staging boxes per epilogue warp");
+
+__device__ __forceinline__ void pack16(const float (&w)[32], int dt, uint32_t (&h)[16]) {
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    if (dt == DT_BF16) {
+      __nv_bfloat162 v = __floats2bfloat162_rn(w[2 * m], w[2 * m + 1]);
+      h[m] = *reinterpret_cast<uint32_t*>(&v);
+    } else {
+      __half2 v = __floats2half2_rn(w[2 * m], w[2 * m + 1]);
+      h[m] = *reinterpret_cast<uint32_t*>(&v);
+    }
+  }
+}
+
+__device__ __forceinline__ void stage_row(uint8_t* box, int lane, const uint32_t (&h)[16]) {
+  uint8_t* rowp = box + lane * 64;
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    *reinterpret_cast<uint4*>(rowp + 16 * (i ^ sw)) = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+}
+
+// Column `lane` of a staged box, packed like a row: element j of the result
+// is box[j][lane].
+__device__ __forceinline__ void stage_col(const uint8_t* box, int lane, uint32_t (&h)[16]) {
+  const int piece = lane >> 3, within = 2 * (lane & 7);
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    const int r0 = 2 * m, r1 = 2 * m + 1;
+    const uint32_t lo = *reinterpret_cast<const uint16_t*>(box + r0 * 64 + 16 * (piece ^ ((r0 >> 1) & 3)) + within);
+    const uint32_t hi = *reinterpret_cast<const uint16_t*>(box + r1 * 64 + 16 * (piece ^ ((r1 >> 1) & 3)) + within);
+    h[m] = lo | (hi << 16);
+  }
+}
+
 // One 32x32 block: this lane owns output row `row0 + lane`, columns
 // col0..col0+31, whose fp32 accumulators are in `acc` and epilogue input in
 // `cv` (when the class has one).  `mirror`: the block is stored together
@@ -480,9 +536,9 @@ __device__ __forceinline__ void load_c(const ClassInfo& k, int b, int row0, int 
 // is exactly symmetric there.
 // alpha and beta: the class's coefficients with their per-batch scales and
 // this lane's row term applied (formed once per tile).
-__device__ __forceinline__ void epilogue_block(const ClassInfo& k, int b, int row0, int col0, bool mirror,
-                                               float (&acc)[32], const float (&cv)[32], float alpha, float beta,
-                                               float* scratch, int lane, float& sq) {
+__device__ __forceinline__ void epilogue_block(const ClassInfo& k, const CUtensorMap* tmo, int b, int row0, int col0,
+                                               bool mirror, float (&acc)[32], const float (&cv)[32], float alpha,
+                                               float beta, float* scratch, int lane, float& sq) {
   const int r = row0 + lane;
   const bool diag = mirror && (col0 == row0);
   const uint32_t colmask = lane_mask(k.N - col0);
@@ -530,21 +586,62 @@ __device__ __forceinline__ void epilogue_block(const ClassInfo& k, int b, int ro
     }
     const bool direct = !e.transposed;
     const bool trans = e.transposed || mirror;
+    if (e.tma) {
+      // staged: box 0 holds the block, box 1 its transpose (or, on a diagonal
+      // block, the exactly symmetric block: the upper part and its mirror)
+      uint8_t* s0 = reinterpret_cast<uint8_t*>(scratch);
+      uint8_t* s1 = s0 + kBoxBytes;
+      if (lane == 0) bulk_wait_read_all();  // the previous stores have read both boxes
+      __syncwarp();
+      uint32_t h[16];
+      pack16(w, e.dtype, h);
+      stage_row(s0, lane, h);
+      if (trans) {
+        __syncwarp();
+        uint32_t t[16];
+        stage_col(s0, lane, t);
+        if (diag) {
+          // columns c < r take the mirror's value (row c, column r)
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            const uint32_t lo = (2 * m < lane) ? (t[m] & 0xFFFFu) : (h[m] & 0xFFFFu);
+            const uint32_t hi = (2 * m + 1 < lane) ? (t[m] & 0xFFFF0000u) : (h[m] & 0xFFFF0000u);
+            t[m] = lo | hi;
+          }
+        }
+        stage_row(s1, lane, t);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const void* tm = tmo + o;
+        if (diag) {
+          tma_store_3d(tm, s1, col0, row0, b);
+        } else {
+          if (direct) tma_store_3d(tm, s0, col0, row0, b);
+          if (trans) tma_store_3d(tm, s1, row0, col0, b);
+        }
+        bulk_commit_group();
+      }
+      continue;
+    }
     if (direct && r < k.M) {
       uint32_t m = colmask;
       if (diag) m &= (0xFFFFFFFFu << lane);  // columns c >= r; the mirror supplies c < r
       store_row32(gaddr(e.ptr, e.dtype, e.ld, e.bs, b, r, col0), e.dtype, m, w);
     }
     if (trans) {
-      // scratch[i][lane] = w(row0 + lane, col0 + i) in rows padded to 33
-      // words (conflict-free both ways); lane l then reads its column l,
-      // which is row col0 + l of the transposed block
+      // scratch[i][lane] = w(row0 + lane, col0 + i), word lane ^ i of row i
+      // (conflict-free both ways); lane l then reads its column l, which is
+      // row col0 + l of the transposed block
+      if (lane == 0) bulk_wait_read_all();  // staged stores of an earlier output have read the scratch
+      __syncwarp();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) scratch[i * kScratchStride + lane] = w[i];
+      for (int i = 0; i < 32; ++i) scratch[i * 32 + (lane ^ i)] = w[i];
       __syncwarp();
       // w now takes the transposed block's row
 #pragma unroll
-      for (int j = 0; j < 32; ++j) w[j] = scratch[lane * kScratchStride + j];
+      for (int j = 0; j < 32; ++j) w[j] = scratch[lane * 32 + (j ^ lane)];
       __syncwarp();
       const int tr = col0 + lane;  // row of the transposed block
       if (tr < k.N) {
@@ -949,7 +1046,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             acc[4 * j4 + 3] += f.w;
           }
         }
-        epilogue_block(k, tc.b, row0, col0, mirror, acc, cv, alpha, beta, scratch, lane, sq);
+        epilogue_block(k, p.cls[tc.c].tmOut, tc.b, row0, col0, mirror, acc, cv, alpha, beta, scratch, lane, sq);
       }
       if (k.sumsq != nullptr) {
 #pragma unroll
@@ -963,6 +1060,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
       if (k.sig != nullptr) {
         // publish this warp's rows of the tile to later classes of the launch
+        // (lane 0's staged stores complete first)
+        if (lane == 0) bulk_wait_all();
         fence_proxy_async_global();
         __threadfence();
         __syncwarp();
@@ -975,6 +1074,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       buf ^= 1;
       if (buf == 0) bphase ^= 1u;
     }
+    // the staging boxes stay in use until the last stores have completed
+    if (lane == 0) bulk_wait_all();
   }
 
   // Reconverge every warp first: in the producer and MMA warps only lane 0

@@ -260,6 +260,20 @@ bool encode(CUtensorMap* tm, const Mat& m, int box0, int box_rows, int64_t batch
   return r == CUDA_SUCCESS;
 }
 
+// 3-D tensor map (cols, rows, batch) of a 16-bit output for the epilogue's
+// staged bulk stores: a 32 x 32 box (64-byte rows) in the 64-byte swizzle.
+bool encode_out(CUtensorMap* tm, const Mat& m, int64_t batch) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(m.cols), static_cast<cuuint64_t>(m.rows),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(m.ld * 2), static_cast<cuuint64_t>(m.bs * 2)};
+  cuuint32_t box[3] = {32u, 32u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUtensorMapDataType dt = m.dt == DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = g_encode(tm, dt, 3, const_cast<void*>(m.ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // fp32 in the blocked layout of blk_off(): padded width and per-matrix size
 inline int64_t blk_ld(int64_t cols) { return round_up(cols, 32); }
 inline int64_t blk_size(int64_t rows, int64_t cols) { return round_up(rows, 32) * round_up(cols, 32); }
@@ -447,7 +461,19 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
       return MSIGN_ERR_INVALID_ARG;
     for (const EpiOut& e : s.outs)
       if (e.blocked && (e.dtype != DT_FP32 || e.transposed || e.ld % 32 != 0)) return MSIGN_ERR_INVALID_ARG;
-    for (size_t o = 0; o < s.outs.size(); ++o) ci.out[o] = s.outs[o];
+    for (size_t o = 0; o < s.outs.size(); ++o) {
+      EpiOut& e = ci.out[o];
+      e = s.outs[o];
+      // 16-bit row-major outputs leave by staged bulk stores where the
+      // buffer's address and strides allow a tensor map (16-byte multiples);
+      // the rest, and transposed outputs of symmetric classes, by lane stores
+      e.tma = 0;
+      if (!e.blocked && (e.dtype == DT_BF16 || e.dtype == DT_FP16) && !(e.transposed && s.symmetric)) {
+        Mat d{e.ptr, e.dtype, e.transposed ? s.N : s.M, e.transposed ? s.M : s.N, e.ld, e.bs};
+        if (s.batch == 1) d.bs = d.rows * d.ld;
+        if (d.ld >= d.cols && d.bs > 0 && tma_ok(d) && encode_out(&c.tmOut[o], d, s.batch)) e.tma = 1;
+      }
+    }
     if (s.deps.size() > static_cast<size_t>(kMaxDeps) || s.c_dep >= static_cast<int>(s.deps.size()))
       return MSIGN_ERR_INVALID_ARG;
     for (size_t e = 0; e < s.deps.size(); ++e) ci.deps[e] = s.deps[e];
