@@ -46,7 +46,7 @@ FLUSH_BYTES = 256 << 20
 # launch (all 15 products, chained) of a 4096^2 msign call, from the ncu
 # capture summarised in profiles/gemm_sm100_msign4096.md; valid only for the
 # kernel source whose hash is recorded with it.
-NCU_TRAFFIC = {"bytes_per_launch": 1237.99e6, "kernel_sha": "ddde70953a48874a"}
+NCU_TRAFFIC = {"bytes_per_launch": 1264.21e6, "kernel_sha": "7fd2afb8fa99d499"}
 
 
 def useful_flops(n: int, m: int, steps: int) -> float:
@@ -372,6 +372,9 @@ WORKLOADS = {
     "msign_1024x4096": ("msign", dict(batch=1, rows=1024, cols=4096)),
     "msign_4096_fp32": ("msign", dict(batch=1, rows=4096, cols=4096, compute="fp32")),
     "msign_4096_improved_init": ("msign", dict(batch=1, rows=4096, cols=4096, improved=True)),
+    # the headline call with its phases as separate launches (msign_set_chaining(0)),
+    # for per-phase timing and profiles of X X^T, the A^2 product and B X
+    "msign_4096_phases": ("msign", dict(batch=1, rows=4096, cols=4096, chaining=False)),
     "gram_xxt_1024": ("gram_xxt", dict(n=1024)),
     "gram_xxt_2048": ("gram_xxt", dict(n=2048)),
     "gram_xxt_4096": ("gram_xxt", dict(n=4096)),
@@ -424,6 +427,9 @@ def run_workload(args):
         imp = cfg.get("improved", False)
         meth = cfg.get("method", "standard")
         call = lambda: msb.msign_ns(x, out, compute=comp, improved_init=imp, method=meth, workspace=ws)
+        if not cfg.get("chaining", True):
+            msb.set_chaining(False)
+            desc.update(chaining="one launch per product")
         desc.update(batch=b, rows=r, cols=c, compute=comp,
                     input=("N(0,1) seed 0, " if cfg.get("gaussian") else "momentum-like, ") + cfg.get("io", "bf16"),
                     improved_init=imp, method=meth,

@@ -147,6 +147,16 @@ msign_status msign_profile_read(int kind, int *launches, double *total_ms, doubl
 
 msign_status msign_profile_reset(void);
 
+/* Diagnostics (no counterpart on the pages): msign_set_chaining(0) makes
+ * later msign_ns and muon_step calls on the standard route run each product
+ * of an iteration step (X X^T, the A^2 product with its combine b A + c A^2,
+ * B X with its a X term) as a launch of its own, so that a profiler sees the
+ * three phases apart; msign_set_chaining(1) restores the default, the phases
+ * of up to five steps chained in one launch.  Results agree with the chained
+ * ones to rounding (X X^T is not split along K then).  Process-wide; returns
+ * the previous setting.  Added in ABI 104. */
+int msign_set_chaining(int enable);
+
 /* ------------------------------------------------------------------------
  * msign_ns: batched standard Newton-Schulz msign ([P2] eq. 4-7, section
  * 参考实现).

@@ -352,6 +352,14 @@ def selftest_timeout(limit_ns: int = 50_000_000, stream=None) -> None:
     check(_lib.lib().msign_selftest_timeout(int(limit_ns), _stream(stream)), "msign_selftest_timeout")
 
 
+def set_chaining(enable: bool) -> bool:
+    """Diagnostics (msign_set_chaining): False runs each product of a
+    standard-route iteration step as a launch of its own, for profiling the
+    phases apart; True (the default) chains them.  Returns the previous
+    setting."""
+    return bool(_lib.lib().msign_set_chaining(1 if enable else 0))
+
+
 def profile_enable(enable: bool = True) -> None:
     check(_lib.lib().msign_profile_enable(1 if enable else 0), "msign_profile_enable")
 

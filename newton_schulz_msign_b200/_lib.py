@@ -25,7 +25,7 @@ EXPORTS = (
     "muon_step_workspace_size", "muon_step",
     "msign_profile_enable", "msign_profile_read", "msign_profile_reset",
     "msign_ns_noalloc_max_bytes", "msign_ns_noalloc",
-    "msign_selftest_timeout",
+    "msign_selftest_timeout", "msign_set_chaining",
     "mousse_inv_root_workspace_size", "mousse_inv_root", "mousse_direction_workspace_size", "mousse_direction",
 )
 
@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
         L.msign_ns_noalloc_max_bytes.argtypes = []
         L.msign_selftest_timeout.restype = I32
         L.msign_selftest_timeout.argtypes = [ctypes.c_uint64, P]
+        L.msign_set_chaining.restype = I32
+        L.msign_set_chaining.argtypes = [I32]
         L.msign_ns_noalloc.restype = I32
         L.msign_ns_noalloc.argtypes = [P, P, I32, I64, I64, I64, ctypes.POINTER(MsignCoeffs), P]
         L.mousse_inv_root_workspace_size.restype = SZ

@@ -9,6 +9,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -849,6 +850,9 @@ msign_status ns_step(const std::vector<NsClass>& cls, const Schedule& sch, int c
 // needs B rows i and j of step t, i.e. every SQR tile that read A rows i, j).
 //   `zeroed`: the classes' state regions were zeroed for this call (and only
 // the tickets used since), so the first chained launch needs no memset.
+// msign_set_chaining(0): every phase as a launch of its own (diagnostics)
+std::atomic<int> g_chaining{1};
+
 msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cudaStream_t stream,
                         bool zeroed = false) {
   const int T = sch.steps();
@@ -861,7 +865,7 @@ msign_status ns_iterate(const std::vector<NsClass>& cls, const Schedule& sch, cu
     for (const NsClass& k : cls) c += p == 0 ? k.w.syrk_parts : 1;
     return c;
   };
-  const bool chained = uniform && std::max({phase_classes(0), phase_classes(1), phase_classes(2)}) <= kMaxClasses &&
+  const bool chained = g_chaining.load() != 0 && uniform && std::max({phase_classes(0), phase_classes(1), phase_classes(2)}) <= kMaxClasses &&
                        3 * ncls <= kMaxClasses;
   if (!chained) {
     for (int t = 0; t < T; ++t) {
@@ -1259,7 +1263,9 @@ bool gram_route(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute, 
 
 extern "C" {
 
-int msign_abi_version(void) { return 103; }
+int msign_abi_version(void) { return 104; }
+
+int msign_set_chaining(int enable) { return msb::g_chaining.exchange(enable != 0 ? 1 : 0); }
 
 const char* msign_status_string(msign_status s) {
   switch (s) {

@@ -93,6 +93,45 @@ def test_syrk_split_k(shape):
     assert rel_fro(got, ref) < TOL_BF16
 
 
+@pytest.mark.parametrize("shape", [(2, 520, 1300), (300, 9000)])
+def test_unchained_phases(shape):
+    # msign_set_chaining(0): one launch per product (three per step) instead
+    # of chained launches; the same iteration, so the same oracle bound and
+    # agreement with the chained result to rounding (the long-K X X^T of
+    # 300 x 9000 is split along K only when chained)
+    x = torch.from_numpy(synth.gaussian(shape, seed=sum(shape))).to(torch.bfloat16).cuda()
+    msb.profile_reset()
+    msb.profile_enable(True)
+    chained = msb.msign_ns(x)
+    msb.profile_enable(False)
+    msb.sync_status()
+    n_chained = msb.profile_read("gemm")["launches"]
+    assert 1 <= n_chained < 15
+    msb.profile_reset()
+    msb.profile_enable(True)
+    prev = msb.set_chaining(False)
+    try:
+        apart = msb.msign_ns(x)
+    finally:
+        msb.set_chaining(prev)
+        msb.profile_enable(False)
+    msb.sync_status()
+    assert prev is True
+    assert msb.profile_read("gemm")["launches"] == 15  # 5 steps x (X X^T, A^2 + combine, B X)
+    msb.profile_reset()
+    ref = O.msign_ns(to_np(x), input_cast="bf16")
+    assert rel_fro(to_np(apart), ref) < TOL_BF16
+    assert rel_fro(to_np(apart), to_np(chained)) < 1e-2
+    # the default is back: chained launches again
+    msb.profile_enable(True)
+    again = msb.msign_ns(x)
+    msb.profile_enable(False)
+    msb.sync_status()
+    assert msb.profile_read("gemm")["launches"] == n_chained
+    msb.profile_reset()
+    assert torch.equal(again, chained)
+
+
 def test_momentum_like_spectrum():
     x = synth.momentum_like(512, 1024, seed=6)
     got, ref = run_case(x)
