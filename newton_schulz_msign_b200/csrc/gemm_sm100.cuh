@@ -1060,10 +1060,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
       if (k.sig != nullptr) {
         // publish this warp's rows of the tile to later classes of the launch
-        // (lane 0's staged stores complete first)
+        // (lane 0's staged stores complete first).  Every lane orders its
+        // generic stores before later async-proxy reads; the warp barrier
+        // orders all lanes' stores before lane 0's release, which is
+        // cumulative, so no lane needs a gpu-scope fence of its own
+        // (measured: one such fence per tile cost 1-2.5% on chains of small
+        // products)
         if (lane == 0) bulk_wait_all();
         fence_proxy_async_global();
-        __threadfence();
         __syncwarp();
         if (lane == 0) {
           int* sg = k.sig + static_cast<long long>(tc.b) * k.tiles_m;

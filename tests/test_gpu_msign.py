@@ -368,3 +368,50 @@ def test_gram_ns_strided_batch_view():
     msb.sync_status()
     assert torch.equal(y, ref)
     assert rel_fro(to_np(y), O.gram_ns(to_np(x))) < TOL_BF16
+
+
+# ---------------------------------------------------------------- output store paths
+
+@pytest.mark.parametrize("shape,method", [((2, 384, 640), "standard"), ((2, 640, 384), "standard"),
+                                          ((2, 520, 4700), "auto")])
+def test_staged_and_lane_stores_agree(shape, method):
+    # a 16-bit output whose batch stride is a multiple of 8 elements leaves the
+    # epilogue by staged bulk tensor stores; an odd batch stride forces the
+    # lane-per-row stores.  Same fp32 values, same rounding: the same bits,
+    # transposed (tall input) or not
+    b, r, c = shape
+    x = torch.from_numpy(synth.gaussian(shape, seed=r + c)).to(torch.bfloat16).cuda()
+    staged = msb.msign_ns(x, method=method)
+    pad = r * c + 3
+    flat = torch.full((b * pad,), 9.0, dtype=torch.bfloat16, device="cuda")
+    lanes = flat.as_strided((b, r, c), (pad, c, 1))
+    msb.msign_ns(x, lanes, method=method)
+    msb.sync_status()
+    assert torch.equal(lanes, staged)
+    # the 3 elements after each matrix are untouched
+    tail = flat.as_strided((b, 3), (pad, 1), r * c)
+    assert bool((tail == 9.0).all())
+    ref = O.msign_ns(to_np(x[0]), input_cast="bf16") if method == "standard" else O.gram_ns(to_np(x[0]))
+    assert rel_fro(to_np(staged[0]), ref) < TOL_BF16
+
+
+# ---------------------------------------------------------------- hand-off stress
+
+@pytest.mark.parametrize("kind,shape", [("msign", (1024, 4096)), ("msign", (8, 256, 512)), ("gram_ns", (1024, 4096)),
+                                        ("msign", (2, 2048, 2048))])
+def test_chained_handoffs_are_deterministic(kind, shape):
+    # every chained launch hands row blocks from one product to the next
+    # through release/acquire counters; a missing order would let a tile read
+    # a stale operand now and then.  Thirty back-to-back calls (no sync in
+    # between) must give the same bits every time, and the first must match
+    # the oracle.
+    x = torch.from_numpy(synth.gaussian(shape, seed=sum(shape))).to(torch.bfloat16).cuda()
+    run = (lambda: msb.msign_ns(x)) if kind == "msign" else (lambda: msb.gram_ns(x))
+    first = run()
+    outs = [run() for _ in range(30)]
+    msb.sync_status()
+    for y in outs:
+        assert torch.equal(y, first)
+    x0 = to_np(x.reshape((-1,) + shape[-2:])[0])
+    ref = O.msign_ns(x0, input_cast="bf16") if kind == "msign" else O.gram_ns(x0)
+    assert rel_fro(to_np(first.reshape((-1,) + shape[-2:])[0]), ref) < TOL_BF16
