@@ -705,6 +705,11 @@ struct NsClass {
   const float* s = nullptr;
   const float* s2 = nullptr;
   bool improved = false;  // sharper step-0 normalisation (Schedule::init)
+  // the first step's a X term reads the 16-bit operand copy P[0] instead of
+  // the fp32 master: the fused ingest writes the unscaled x rounded to the
+  // operand type, which the copy holds exactly, so the ingest skips the
+  // master and the first B X epilogue writes it
+  bool c0_op = false;
 };
 
 // Hi and lo plane outputs of a split matrix at `p` (planes of `plane` elements).
@@ -770,6 +775,7 @@ void ns_specs(const NsClass& k, int cur, float a, float b, float c, bool first, 
   x.alpha = 1.0f, x.beta = a;
   if (!sp) x.row_beta = k.w.diag, x.row_beta_bs = n;
   x.C = k.w.master, x.c_dt = DT_FP32, x.ldc = blk_ld(m), x.c_bs = blk_size(n, m), x.c_blocked = true;
+  if (first && k.c0_op && !sp) x.C = k.w.P[cur], x.c_dt = k.op_dt, x.ldc = ldm, x.c_bs = pm, x.c_blocked = false;
   if (!last) {
     x.outs = outs(k.w.P[cur ^ 1], ldm, pm);
     x.outs.insert(x.outs.begin(), out_blocked(k.w.master, blk_ld(m), blk_size(n, m)));
@@ -1213,7 +1219,7 @@ msign_status ns_run(const void* in, int in_dt, int64_t in_ld, int64_t in_bs, voi
                                fp32 ? 2 * n * ldm : n * ldm);
     a.op_plane = n * ldm;
     a.in_bs = in_bs, a.ld_in = in_ld;
-    a.master = w.master, a.ld_m = blk_ld(m), a.m_bs = blk_size(n, m);
+    if (fp32) a.master = w.master, a.ld_m = blk_ld(m), a.m_bs = blk_size(n, m);  // else see NsClass::c0_op
     a.partials = w.partials, a.ticket = ns_ticket_ptr(w), a.s_out = w.scale, a.s2_out = w.scale + batch;
     a.eps = sch.eps;
     st = launch_ingest(a, batch, stream);
@@ -1235,6 +1241,7 @@ msign_status ns_run(const void* in, int in_dt, int64_t in_ld, int64_t in_bs, voi
   cls[0].op_dt = fp32 ? DT_BF16 : cd;
   cls[0].final_outs = {out_to(out, out_dt, out_ld, out_bs, tr)};
   if (fused) cls[0].s = w.scale, cls[0].s2 = w.scale + batch;
+  cls[0].c0_op = fused && !fp32;
   cls[0].improved = sch.init == 1;
   return ns_iterate(cls, sch, stream, fused);
 }
@@ -1812,6 +1819,7 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
       ns[c].s = ns[c].w.scale;
       ns[c].s2 = ns[c].w.scale + counts[c];
       ns[c].improved = sch.init == 1;
+      ns[c].c0_op = true;  // the ingest below writes no master
       if (cudaMemsetAsync(ns[c].w.cnt, 0, state_bytes(counts[c], ns[c].n, kMaxClasses), stream) != cudaSuccess)
         return MSIGN_ERR_CUDA;
     }
@@ -1823,10 +1831,9 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
       const int64_t slot = slots[i - begin];
       const NsClass& k = ns[c];
       const bool tr = rows[i] > cols[i];
-      const int64_t ldm = round_up(k.m, 8), per = k.n * ldm, mb = blk_size(k.n, k.m);
+      const int64_t ldm = round_up(k.m, 8), per = k.n * ldm;
       IngestArgs a = ingest_args(M[i], DT_FP32, rows[i], cols[i], tr, DT_BF16,
                                  static_cast<char*>(k.w.P[0]) + 2 * slot * per, DT_BF16, ldm, per);
-      a.master = k.w.master + slot * mb, a.ld_m = blk_ld(k.m), a.m_bs = mb;
       a.partials = k.w.partials + slot * kNormParts, a.ticket = ns_ticket_ptr(k.w) + slot;
       a.s_out = k.w.scale + slot, a.s2_out = k.w.scale + k.batch + slot, a.eps = sch.eps;
       a.G = G[i], a.g_dt = gd, a.mu = momentum;
