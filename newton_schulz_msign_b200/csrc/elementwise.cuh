@@ -225,14 +225,12 @@ __device__ __forceinline__ void load8(const char* p, int dt, int cnt, float* x) 
   for (int e = 0; e < 8; ++e) x[e] = e < cnt ? load_elem(p + e * es, dt) : 0.0f;
 }
 
-// The values this thread owns in output tile `tt` of the non-transposed
-// path: row i0 + tid/8, columns j0 + 8 (tid%8) .. +7 (0 outside the matrix).
-__device__ __forceinline__ void ingest_row_chunk(const IngestArgs& a, char* src, const char* gsrc, float s, int n,
-                                                 int m, int tc, long long tt, int tid, float* x) {
-  const int i = static_cast<int>(tt / tc) * 32 + (tid >> 3);
-  const int j = static_cast<int>(tt % tc) * 64 + 8 * (tid & 7);
-  const int cnt = (i < n && j < m) ? (m - j < 8 ? m - j : 8) : 0;
-  const long long e = static_cast<long long>(i) * (a.ld_in > 0 ? a.ld_in : a.cols) + j;
+// Input elements (row, col .. col+7) after the momentum update, the cast and
+// the scale (ingest_value); 0 outside the input's rows x cols.
+__device__ __forceinline__ void ingest_load8(const IngestArgs& a, char* src, const char* gsrc, float s, int row,
+                                             int col, float* x) {
+  const int cnt = (row < a.rows && col < a.cols) ? (a.cols - col < 8 ? a.cols - col : 8) : 0;
+  const long long e = static_cast<long long>(row) * (a.ld_in > 0 ? a.ld_in : a.cols) + col;
   load8(src + e * dtype_size(a.in_dt), a.in_dt, cnt, x);
   if (gsrc != nullptr && cnt > 0) {
     float g[8];
@@ -244,11 +242,23 @@ __device__ __forceinline__ void ingest_row_chunk(const IngestArgs& a, char* src,
       reinterpret_cast<float4*>(mp)[0] = make_float4(x[0], x[1], x[2], x[3]);
       reinterpret_cast<float4*>(mp)[1] = make_float4(x[4], x[5], x[6], x[7]);
     } else {
-      for (int t = 0; t < cnt; ++t) mp[t] = x[t];
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+        if (t < cnt) mp[t] = x[t];
     }
   }
 #pragma unroll
   for (int t = 0; t < 8; ++t) x[t] = t < cnt ? ingest_value(x[t], a, s) : 0.0f;
+}
+
+// The values this thread owns in output tile `tt` of the non-transposed
+// path: row i0 + tid/8, columns j0 + 8 (tid%8) .. +7 (0 outside the matrix).
+// Tile indices fit in 32 bits (fewer than 2^31 tiles of 2048 elements for
+// any matrix a device holds); 32-bit division measured 10% faster here.
+__device__ __forceinline__ void ingest_row_chunk(const IngestArgs& a, char* src, const char* gsrc, float s, int tc,
+                                                 long long tt, int tid, float* x) {
+  const int t32 = static_cast<int>(tt);
+  ingest_load8(a, src, gsrc, s, (t32 / tc) * 32 + (tid >> 3), (t32 % tc) * 64 + 8 * (tid & 7), x);
 }
 
 // Operand-copy store of 8 consecutive values at (i, j); cnt of them valid.
@@ -284,7 +294,9 @@ __device__ __forceinline__ void ingest_store_op(const IngestArgs& a, int b, int 
     }
     return;
   }
-  for (int e = 0; e < cnt; ++e) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    if (e >= cnt) break;
     store_elem(dst + e * es, a.op_dt, v[e]);
     if (a.op_dt == DT_TF32_HI) store_elem(dst + a.op_plane * 4 + e * es, DT_TF32_LO, v[e]);
   }
@@ -306,7 +318,7 @@ __device__ __forceinline__ void ingest_store_master(const IngestArgs& a, int b, 
   }
 }
 
-__global__ void __launch_bounds__(256) ingest_kernel(const IngestArgs a) {
+__global__ void __launch_bounds__(256, 5) ingest_kernel(const IngestArgs a) {
   __shared__ float tile[32][65];
   __shared__ float red[32];
   __shared__ int last;
@@ -327,13 +339,13 @@ __global__ void __launch_bounds__(256) ingest_kernel(const IngestArgs a) {
     // row chunks in registers, the next tile's loads issued before this
     // tile's stores
     float nxt[8];
-    if (blockIdx.x < ntiles) ingest_row_chunk(a, src, gsrc, s, n, m, tc, blockIdx.x, tid, nxt);
+    if (blockIdx.x < ntiles) ingest_row_chunk(a, src, gsrc, s, tc, blockIdx.x, tid, nxt);
     for (long long tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
       float v[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = nxt[e];
-      if (tt + gridDim.x < ntiles) ingest_row_chunk(a, src, gsrc, s, n, m, tc, tt + gridDim.x, tid, nxt);
-      const int i0 = static_cast<int>(tt / tc) * 32, j0 = static_cast<int>(tt % tc) * 64;
+      if (tt + gridDim.x < ntiles) ingest_row_chunk(a, src, gsrc, s, tc, tt + gridDim.x, tid, nxt);
+      const int i0 = (static_cast<int>(tt) / tc) * 32, j0 = (static_cast<int>(tt) % tc) * 64;
       const int r = tid >> 3, c0 = 8 * (tid & 7);
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc = fmaf(v[e], v[e], acc);
@@ -348,23 +360,19 @@ __global__ void __launch_bounds__(256) ingest_kernel(const IngestArgs a) {
     }
   } else {
     for (long long tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
-      const int i0 = static_cast<int>(tt / tc) * 32, j0 = static_cast<int>(tt % tc) * 64;
-      // output (i, j) = in (j, i): input rows j0 + ty + 8k, columns i0 + tx
+      const int i0 = (static_cast<int>(tt) / tc) * 32, j0 = (static_cast<int>(tt) % tc) * 64;
+      // output (i, j) = in (j, i): this thread loads input row j0 + tid/4,
+      // columns i0 + 8 (tid%4) .. +7 with 16-byte accesses and stores them
+      // transposed into the tile (rows padded to 65 words: the 32 lanes hit
+      // 32 different banks)
+      {
+        float x[8];
+        ingest_load8(a, src, gsrc, s, j0 + (tid >> 2), i0 + 8 * (tid & 3), x);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int jr = j0 + ty + 8 * k, ic = i0 + tx;
-        float x = 0.0f;
-        if (jr < m && ic < n) {
-          const long long e = static_cast<long long>(jr) * (a.ld_in > 0 ? a.ld_in : a.cols) + ic;
-          x = load_elem(src + e * dtype_size(a.in_dt), a.in_dt);
-          if (gsrc != nullptr) {
-            x = fmaf(a.mu, x, load_elem(gsrc + e * dtype_size(a.g_dt), a.g_dt));
-            reinterpret_cast<float*>(src)[e] = x;
-          }
-          x = ingest_value(x, a, s);
+        for (int e = 0; e < 8; ++e) {
+          acc = fmaf(x[e], x[e], acc);
+          tile[8 * (tid & 3) + e][tid >> 2] = x[e];
         }
-        acc = fmaf(x, x, acc);
-        tile[tx][ty + 8 * k] = x;
       }
       __syncthreads();
       const int r = tid >> 3, c0 = 8 * (tid & 7);
