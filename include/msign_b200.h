@@ -42,6 +42,9 @@
  * - Coefficient schedules are HOST arrays.  NULL selects Jordan's triple
  *   for T = 5 steps ([P2] eq. 7).
  * - Empty problems (batch, rows or cols = 0) are valid and do nothing.
+ * - Size limits: batch <= 65535 and every matrix dimension <= 2^30
+ *   (mousse_inv_root: n <= 2^20); beyond them an entry point returns
+ *   MSIGN_ERR_UNSUPPORTED before enqueuing anything.
  * - Entry points run on the CURRENT device (cudaGetDevice) and every pointer
  *   of a call must belong to it.  The library keeps per-device addresses
  *   (its device error word, the msign_ns_noalloc scratch) for the life of

@@ -415,3 +415,26 @@ def test_chained_handoffs_are_deterministic(kind, shape):
     x0 = to_np(x.reshape((-1,) + shape[-2:])[0])
     ref = O.msign_ns(x0, input_cast="bf16") if kind == "msign" else O.gram_ns(x0)
     assert rel_fro(to_np(first.reshape((-1,) + shape[-2:])[0]), ref) < TOL_BF16
+
+
+# ---------------------------------------------------------------- size limits
+
+def test_largest_batch():
+    # batch = 65535, the documented maximum: one tile per matrix and phase,
+    # 983025 tiles in the chained launch, 65535 sets of row-block counters;
+    # a sample of matrices (first, last, across the range) against the oracle
+    b = 65535
+    x = torch.from_numpy(synth.gaussian((b, 4, 8), seed=14)).to(torch.bfloat16).cuda()
+    y = msb.msign_ns(x)
+    msb.sync_status()
+    for i in (0, 1, 4097, 32768, 65533, 65534):
+        ref = O.msign_ns(to_np(x[i]), input_cast="bf16")
+        assert rel_fro(to_np(y[i]), ref) < TOL_BF16, i
+    # one more matrix is beyond the built limits: refused on the host,
+    # nothing enqueued
+    big = torch.full((65536, 4, 8), 3.0, dtype=torch.bfloat16, device="cuda")
+    out = torch.full_like(big, 7.0)
+    with pytest.raises(msb.MsignError):
+        msb.msign_ns(big, out)
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all())
