@@ -46,7 +46,7 @@ FLUSH_BYTES = 256 << 20
 # launch (all 15 products, chained) of a 4096^2 msign call, from the ncu
 # capture summarised in profiles/gemm_sm100_msign4096.md; valid only for the
 # kernel source whose hash is recorded with it.
-NCU_TRAFFIC = {"bytes_per_launch": 1187.72e6, "kernel_sha": "3558db7261745c7a"}
+NCU_TRAFFIC = {"bytes_per_launch": 1186.81e6, "kernel_sha": "293a2f59ad5eb25a"}
 
 
 def useful_flops(n: int, m: int, steps: int) -> float:

@@ -759,6 +759,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  // Launched as a programmatic dependent of the previous kernel on the
+  // stream: the set-up above overlaps that kernel's tail, and nothing below
+  // touches global memory before it has completed.  (Without the launch
+  // attribute the wait returns at once.)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)

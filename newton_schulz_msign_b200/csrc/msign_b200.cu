@@ -522,17 +522,22 @@ msign_status launch_grouped(std::vector<ClassSpec> specs, int ab_dt, cudaStream_
   // the kernel built with per-class tile widths only where a class is narrow
   bool narrow = false;
   for (const ClassSpec& s : specs) narrow = narrow || s.bn != kBN;
-  if (ab_dt == DT_FP32) {
-    if (narrow)
-      gemm_sm100_kernel<true, true><<<grid, kThreads, kSmemBytes, stream>>>(p);
-    else
-      gemm_sm100_kernel<true, false><<<grid, kThreads, kSmemBytes, stream>>>(p);
-  } else {
-    if (narrow)
-      gemm_sm100_kernel<false, true><<<grid, kThreads, kSmemBytes, stream>>>(p);
-    else
-      gemm_sm100_kernel<false, false><<<grid, kThreads, kSmemBytes, stream>>>(p);
-  }
+  // a programmatic dependent launch: the CTAs set up while the previous
+  // kernel drains, then wait for it (griddepcontrol.wait in the kernel)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  if (ab_dt == DT_FP32)
+    (void)cudaLaunchKernelEx(&cfg, narrow ? gemm_sm100_kernel<true, true> : gemm_sm100_kernel<true, false>, p);
+  else
+    (void)cudaLaunchKernelEx(&cfg, narrow ? gemm_sm100_kernel<false, true> : gemm_sm100_kernel<false, false>, p);
   prof_end(0, stream, flops, bytes);
   return cudaGetLastError() == cudaSuccess ? MSIGN_OK : MSIGN_ERR_CUDA;
 }
