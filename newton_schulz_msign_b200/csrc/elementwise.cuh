@@ -335,7 +335,34 @@ __global__ void __launch_bounds__(256, 5) ingest_kernel(const IngestArgs a) {
   const long long ntiles = static_cast<long long>(tr) * tc;
   const int mpad = (m + 31) / 32 * 32;
   float acc = 0.0f;
-  if (!a.transpose) {
+  const long long ld_in = a.ld_in > 0 ? a.ld_in : a.cols;
+  uint16_t* dop = reinterpret_cast<uint16_t*>(a.xop) + static_cast<long long>(b) * a.op_bs;
+  // bf16 in and out, nothing else to do: the operand copy is the input
+  // itself (its cast to bf16 is exact), moved row by row in 16-byte pieces
+  // with the sum of squares on the way (the general path below spends ~40
+  // instructions per element on conversions it does not need here)
+  const bool copy16 = a.in_dt == DT_BF16 && a.op_dt == DT_BF16 && a.cast_dt == DT_BF16 && !a.transpose &&
+                      a.pre_scale == nullptr && gsrc == nullptr && a.master == nullptr && (m & 7) == 0 &&
+                      (ld_in & 7) == 0 && (a.ld_op & 7) == 0 && (a.op_bs & 7) == 0 &&
+                      (reinterpret_cast<uintptr_t>(src) & 15) == 0 && (reinterpret_cast<uintptr_t>(dop) & 15) == 0;
+  if (copy16) {
+    const int mc = m >> 3;
+    for (int row = blockIdx.x; row < n; row += gridDim.x) {
+      const uint4* srow = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(src) + row * ld_in);
+      uint4* drow = reinterpret_cast<uint4*>(dop + row * a.ld_op);
+      for (int c = tid; c < mc; c += 256) {
+        const uint4 u = srow[c];
+        drow[c] = u;
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float lo = __uint_as_float(w[t] << 16), hi = __uint_as_float(w[t] & 0xFFFF0000u);
+          acc = fmaf(lo, lo, acc);
+          acc = fmaf(hi, hi, acc);
+        }
+      }
+    }
+  } else if (!a.transpose) {
     // row chunks in registers, the next tile's loads issued before this
     // tile's stores
     float nxt[8];
