@@ -362,6 +362,42 @@ __global__ void __launch_bounds__(256, 5) ingest_kernel(const IngestArgs a) {
         }
       }
     }
+  } else if (a.in_dt == DT_FP32 && a.op_dt == DT_BF16 && a.cast_dt == DT_BF16 && !a.transpose &&
+             a.pre_scale == nullptr && a.master == nullptr && (m & 7) == 0 && (ld_in & 7) == 0 &&
+             (a.ld_op & 7) == 0 && (a.op_bs & 7) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0 &&
+             (reinterpret_cast<uintptr_t>(dop) & 15) == 0 &&
+             (gsrc == nullptr || (reinterpret_cast<uintptr_t>(gsrc) & 15) == 0)) {
+    // fp32 in (Muon's momentum M, optionally updated by M <- mu M + G in
+    // place), bf16 operands: the same row-wise walk, eight elements per step
+    const int mc = m >> 3;
+    for (int row = blockIdx.x; row < n; row += gridDim.x) {
+      float* srow = reinterpret_cast<float*>(src) + row * ld_in;
+      const char* grow = gsrc != nullptr ? gsrc + row * ld_in * dtype_size(a.g_dt) : nullptr;
+      uint4* drow = reinterpret_cast<uint4*>(dop + row * a.ld_op);
+      for (int c = tid; c < mc; c += 256) {
+        const float4 u = reinterpret_cast<const float4*>(srow)[2 * c], v = reinterpret_cast<const float4*>(srow)[2 * c + 1];
+        float x[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
+        if (grow != nullptr) {
+          float g[8];
+          load8(grow + static_cast<long long>(8 * c) * dtype_size(a.g_dt), a.g_dt, 8, g);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) x[t] = fmaf(a.mu, x[t], g[t]);
+          reinterpret_cast<float4*>(srow)[2 * c] = make_float4(x[0], x[1], x[2], x[3]);
+          reinterpret_cast<float4*>(srow)[2 * c + 1] = make_float4(x[4], x[5], x[6], x[7]);
+        }
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * t], x[2 * t + 1]);
+          w[t] = *reinterpret_cast<uint32_t*>(&h);
+          // the norm of the rounded values, as the general path forms it
+          const float lo = __uint_as_float(w[t] << 16), hi = __uint_as_float(w[t] & 0xFFFF0000u);
+          acc = fmaf(lo, lo, acc);
+          acc = fmaf(hi, hi, acc);
+        }
+        drow[c] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
   } else if (!a.transpose) {
     // row chunks in registers, the next tile's loads issued before this
     // tile's stores
