@@ -421,6 +421,72 @@ __global__ void __launch_bounds__(256, 5) ingest_kernel(const IngestArgs a) {
         __syncthreads();
       }
     }
+  } else if (a.op_dt == DT_BF16 && a.cast_dt == DT_BF16 && a.pre_scale == nullptr && a.master == nullptr &&
+             (a.in_dt == DT_BF16 || a.in_dt == DT_FP32) && (n & 7) == 0 && (ld_in & 7) == 0 &&
+             (a.ld_op & 7) == 0 && (a.op_bs & 7) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0 &&
+             (reinterpret_cast<uintptr_t>(dop) & 15) == 0) {
+    // transposing, bf16 operands, nothing else (tall inputs, Muon's tall
+    // momenta): the tiles of the general path below without its dtype
+    // dispatch per element; input rows of a multiple of 8 elements
+    for (long long tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
+      const int i0 = (static_cast<int>(tt) / tc) * 32, j0 = (static_cast<int>(tt) % tc) * 64;
+      {
+        const int jr = j0 + (tid >> 2), ic = i0 + 8 * (tid & 3);  // input row and first column
+        float x[8];
+        if (jr < a.rows && ic < a.cols) {
+          const long long e = static_cast<long long>(jr) * ld_in + ic;
+          if (a.in_dt == DT_BF16) {
+            const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(src) + e);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+              x[2 * t] = __uint_as_float(w[t] << 16), x[2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
+          } else {
+            float* mp = reinterpret_cast<float*>(src) + e;
+            const float4 u = reinterpret_cast<const float4*>(mp)[0], v = reinterpret_cast<const float4*>(mp)[1];
+            x[0] = u.x, x[1] = u.y, x[2] = u.z, x[3] = u.w, x[4] = v.x, x[5] = v.y, x[6] = v.z, x[7] = v.w;
+            if (gsrc != nullptr) {
+              float g[8];
+              load8(gsrc + e * dtype_size(a.g_dt), a.g_dt, 8, g);
+#pragma unroll
+              for (int t = 0; t < 8; ++t) x[t] = fmaf(a.mu, x[t], g[t]);
+              reinterpret_cast<float4*>(mp)[0] = make_float4(x[0], x[1], x[2], x[3]);
+              reinterpret_cast<float4*>(mp)[1] = make_float4(x[4], x[5], x[6], x[7]);
+            }
+#pragma unroll
+            for (int t = 0; t < 8; ++t) x[t] = __bfloat162float(__float2bfloat16_rn(x[t]));
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) x[t] = 0.0f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          acc = fmaf(x[e], x[e], acc);
+          tile[8 * (tid & 3) + e][tid >> 2] = x[e];
+        }
+      }
+      __syncthreads();
+      const int r = tid >> 3, c0 = 8 * (tid & 7);
+      if (i0 + r < n && j0 + c0 < m) {
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(tile[r][c0 + 2 * t], tile[r][c0 + 2 * t + 1]);
+          w[t] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        uint16_t* d = dop + static_cast<long long>(i0 + r) * a.ld_op + j0 + c0;
+        const int cnt = m - j0 - c0 < 8 ? m - j0 - c0 : 8;
+        if (cnt == 8) {
+          *reinterpret_cast<uint4*>(d) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if (e < cnt) d[e] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
+        }
+      }
+      __syncthreads();  // the tile is rewritten by the next iteration
+    }
   } else {
     for (long long tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
       const int i0 = (static_cast<int>(tt) / tc) * 32, j0 = (static_cast<int>(tt) % tc) * 64;
