@@ -258,6 +258,31 @@ msign_status msign_ns_noalloc(const void *in, void *out, msign_dtype io_dtype,
                               msign_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * msign_ns_host: msign_ns on HOST buffers (no counterpart on the pages).
+ *
+ * Enqueues on `stream`: the copy of the input from in_host into the
+ * workspace, msign_ns in place there (same arguments and results as
+ * msign_ns with back-to-back matrices), and the copy of the result to
+ * out_host.  in_host and out_host are host pointers to batch x rows x cols
+ * values in io_dtype, dense; they must stay valid, and out_host unread,
+ * until the stream has passed the call.  With page-locked (pinned) host
+ * memory the copies are asynchronous and calls on two streams overlap one
+ * call's copies with the other's kernels; pageable memory works, with the
+ * copies synchronous to the host.  out_host may equal in_host.
+ *   workspace   device scratch of at least msign_ns_host_workspace_size()
+ *               bytes (the device copy of the matrices, then msign_ns's
+ *               workspace), 256-byte aligned
+ * Errors as for msign_ns; the argument checks come before any copy is
+ * enqueued.  Added in ABI 105.
+ * ------------------------------------------------------------------------ */
+size_t msign_ns_host_workspace_size(int64_t batch, int64_t rows, int64_t cols, msign_dtype io_dtype,
+                                    msign_dtype compute_dtype);
+
+msign_status msign_ns_host(const void *in_host, void *out_host, msign_dtype io_dtype, msign_dtype compute_dtype,
+                           int64_t batch, int64_t rows, int64_t cols, const msign_coeffs *coeffs,
+                           void *workspace, size_t workspace_bytes, msign_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * gram_xxt: symmetric Gram product A = X X^T ([P1] flash-muon
  * matmul_transpose; [P3] section 4, triangular scheduling).
  *

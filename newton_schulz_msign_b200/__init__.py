@@ -16,7 +16,8 @@ from . import _lib
 from ._lib import BF16, FP16, FP32, MsignError, check, make_coeffs
 
 __all__ = [
-    "MsignError", "msign_ns", "msign_ns_workspace_size", "gram_xxt", "gram_xxt_workspace_size", "gram_ns",
+    "MsignError", "msign_ns", "msign_ns_workspace_size", "msign_ns_host", "msign_ns_host_workspace_size",
+    "gram_xxt", "gram_xxt_workspace_size", "gram_ns",
     "gram_ns_workspace_size", "muon_step", "muon_step_workspace_size", "mousse_inv_root", "mousse_direction",
     "sync_status", "selftest_timeout", "library_path",
 ]
@@ -161,6 +162,45 @@ def msign_ns(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, impro
                                  wsb, _stream(stream, x.device))
         del keep
     check(st, "msign_ns")
+    return out
+
+
+def msign_ns_host_workspace_size(batch: int, rows: int, cols: int, io: str = "bf16", compute: str = "bf16") -> int:
+    return int(_lib.lib().msign_ns_host_workspace_size(batch, rows, cols, _compute_code(io), _compute_code(compute)))
+
+
+def msign_ns_host(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, improved_init=False,
+                  method="standard", workspace=None, stream=None, device=None):
+    """msign_ns of HOST matrices (``x``: a CPU tensor, dense, bf16/fp16/fp32;
+    page-locked for asynchronous copies): the call enqueues the copy in, the
+    iteration and the copy out on ``stream`` (default: the current stream of
+    ``device``, default the current device) and returns ``out`` (a CPU
+    tensor, page-locked when allocated here) BEFORE the result is there:
+    synchronize the stream before reading it.  ``workspace``: a device uint8
+    tensor of at least msign_ns_host_workspace_size() bytes."""
+    torch = _torch()
+    if x.is_cuda or out is not None and out.is_cuda:
+        raise ValueError("msign_ns_host takes host (CPU) tensors; use msign_ns for device tensors")
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    if x.dim() < 2:
+        raise ValueError("x needs at least two dims")
+    rows, cols = x.shape[-2], x.shape[-1]
+    batch = x.numel() // max(rows * cols, 1) if rows * cols else 0
+    if out is None:
+        out = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+    if out.shape != x.shape or out.dtype != x.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CPU tensor matching x in shape and dtype")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    io = _dtype_code(x)
+    with torch.cuda.device(dev):
+        need = int(_lib.lib().msign_ns_host_workspace_size(batch, rows, cols, io, _compute_code(compute)))
+        ws, wsb = _workspace(need, dev, workspace)
+        c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0, _METHODS[method])
+        st = _lib.lib().msign_ns_host(x.data_ptr(), out.data_ptr(), io, _compute_code(compute), batch, rows, cols,
+                                      ctypes.byref(c) if c is not None else None, _ptr(ws), wsb, _stream(stream, dev))
+        del keep
+    check(st, "msign_ns_host")
     return out
 
 

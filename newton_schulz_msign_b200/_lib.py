@@ -25,7 +25,7 @@ EXPORTS = (
     "muon_step_workspace_size", "muon_step",
     "msign_profile_enable", "msign_profile_read", "msign_profile_reset",
     "msign_ns_noalloc_max_bytes", "msign_ns_noalloc",
-    "msign_selftest_timeout", "msign_set_chaining",
+    "msign_selftest_timeout", "msign_set_chaining", "msign_ns_host_workspace_size", "msign_ns_host",
     "mousse_inv_root_workspace_size", "mousse_inv_root", "mousse_direction_workspace_size", "mousse_direction",
 )
 
@@ -68,6 +68,10 @@ def lib() -> ctypes.CDLL:
         L.msign_ns_workspace_size.argtypes = [I64, I64, I64, I32]
         L.msign_ns.restype = I32
         L.msign_ns.argtypes = [P, P, I32, I32, I64, I64, I64, I64, I64, ctypes.POINTER(MsignCoeffs), P, SZ, P]
+        L.msign_ns_host_workspace_size.restype = SZ
+        L.msign_ns_host_workspace_size.argtypes = [I64, I64, I64, I32, I32]
+        L.msign_ns_host.restype = I32
+        L.msign_ns_host.argtypes = [P, P, I32, I32, I64, I64, I64, ctypes.POINTER(MsignCoeffs), P, SZ, P]
         L.msign_ns_route.restype = I32
         L.msign_ns_route.argtypes = [I64, I64, I64, I32, ctypes.POINTER(MsignCoeffs)]
         L.gram_xxt_workspace_size.restype = SZ

@@ -1275,7 +1275,7 @@ bool gram_route(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute, 
 
 extern "C" {
 
-int msign_abi_version(void) { return 104; }
+int msign_abi_version(void) { return 105; }
 
 int msign_set_chaining(int enable) { return msb::g_chaining.exchange(enable != 0 ? 1 : 0); }
 
@@ -2121,6 +2121,44 @@ void* g_noalloc_ptr[64] = {};
 }  // namespace msb
 
 extern "C" {
+
+size_t msign_ns_host_workspace_size(int64_t batch, int64_t rows, int64_t cols, msign_dtype io_dtype,
+                                    msign_dtype compute_dtype) {
+  if (batch <= 0 || rows <= 0 || cols <= 0 || !valid_dtype(io_dtype)) return 0;
+  const uint64_t xb = static_cast<uint64_t>(batch) * rows * cols * (io_dtype == MSIGN_FP32 ? 4 : 2);
+  return round_up(xb, 256) + msign_ns_workspace_size(batch, rows, cols, compute_dtype);
+}
+
+msign_status msign_ns_host(const void* in_host, void* out_host, msign_dtype io_dtype, msign_dtype compute_dtype,
+                           int64_t batch, int64_t rows, int64_t cols, const msign_coeffs* coeffs, void* workspace,
+                           size_t workspace_bytes, msign_stream_t stream_) {
+  // msign_ns's checks first: nothing is enqueued on an argument error
+  if (!valid_dtype(io_dtype) || !valid_dtype(compute_dtype)) return MSIGN_ERR_INVALID_ARG;
+  if (batch < 0 || rows < 0 || cols < 0) return MSIGN_ERR_INVALID_ARG;
+  Schedule sch;
+  msign_status st = read_schedule(coeffs, kNsEps, &sch);
+  if (st != MSIGN_OK) return st;
+  if (sch.init != 0 && compute_dtype == MSIGN_FP32) return MSIGN_ERR_UNSUPPORTED;
+  if (batch == 0 || rows == 0 || cols == 0) return MSIGN_OK;
+  if (in_host == nullptr || out_host == nullptr) return MSIGN_ERR_INVALID_ARG;
+  if (batch > 65535 || rows > (1 << 30) || cols > (1 << 30)) return MSIGN_ERR_UNSUPPORTED;
+  const size_t need = msign_ns_host_workspace_size(batch, rows, cols, io_dtype, compute_dtype);
+  if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 256) != 0)
+    return MSIGN_ERR_WORKSPACE;
+  DeviceState* dev = nullptr;
+  st = device_state(&dev);
+  if (st != MSIGN_OK) return st;
+  const size_t xb = static_cast<size_t>(batch) * rows * cols * (io_dtype == MSIGN_FP32 ? 4 : 2);
+  const size_t xr = round_up(xb, 256);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  void* dx = workspace;
+  if (cudaMemcpyAsync(dx, in_host, xb, cudaMemcpyHostToDevice, stream) != cudaSuccess) return MSIGN_ERR_CUDA;
+  st = msign_ns(dx, dx, io_dtype, compute_dtype, batch, rows, cols, 0, 0, coeffs, static_cast<char*>(workspace) + xr,
+                workspace_bytes - xr, stream_);
+  if (st != MSIGN_OK) return st;
+  if (cudaMemcpyAsync(out_host, dx, xb, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return MSIGN_ERR_CUDA;
+  return MSIGN_OK;
+}
 
 size_t msign_ns_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
 

@@ -45,7 +45,7 @@ def test_exported_symbols_match_nm(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.msign_abi_version() == 104
+    assert L.msign_abi_version() == 105
     assert L.msign_status_string(_lib.OK) == b"ok"
     assert b"timed out" in L.msign_status_string(_lib.ERR_TIMEOUT)
     assert L.msign_status_string(99) == b"unknown status"

@@ -441,3 +441,66 @@ def test_largest_batch():
         msb.msign_ns(big, out)
     torch.cuda.synchronize()
     assert bool((out == 7.0).all())
+
+
+# ---------------------------------------------------------------- host buffers
+
+def test_host_buffers_match_device_call():
+    # msign_ns_host: copy in, msign_ns in place in the workspace, copy out,
+    # all on the stream; the same kernels on the same values as msign_ns
+    x = torch.from_numpy(synth.gaussian((2, 384, 640), seed=81)).to(torch.bfloat16)
+    xp = x.pin_memory()
+    ref = msb.msign_ns(xp.cuda()).cpu()
+    out = msb.msign_ns_host(xp)
+    torch.cuda.current_stream().synchronize()
+    msb.sync_status()
+    assert torch.equal(out, ref)
+    assert rel_fro(to_np(out[0]), O.msign_ns(to_np(x[0]), input_cast="bf16")) < TOL_BF16
+    # pageable memory, in place
+    y = x.clone()
+    msb.msign_ns_host(y, y)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
+
+
+@pytest.mark.parametrize("shape,io,method", [((3, 520, 200), torch.float32, "standard"),
+                                             ((1, 512, 4608), torch.bfloat16, "auto")])
+def test_host_buffers_tall_and_auto(shape, io, method):
+    x = torch.from_numpy(synth.gaussian(shape, seed=shape[-1])).to(io).pin_memory()
+    ref = msb.msign_ns(x.cuda(), method=method).cpu()
+    out = msb.msign_ns_host(x, method=method)
+    torch.cuda.synchronize()
+    msb.sync_status()
+    assert torch.equal(out, ref)
+
+
+def test_host_buffers_two_streams():
+    # calls alternating between two streams, each with its own workspace and
+    # host buffers, as a pipelined caller runs them: every result as alone
+    xs = [torch.from_numpy(synth.gaussian((256, 768), seed=90 + i)).to(torch.bfloat16).pin_memory() for i in range(6)]
+    refs = [msb.msign_ns(x.cuda()).cpu() for x in xs]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    need = msb.msign_ns_host_workspace_size(1, 256, 768)
+    wss = [torch.empty(need, dtype=torch.uint8, device="cuda") for _ in streams]
+    outs = [torch.empty_like(x).pin_memory() for x in xs]
+    torch.cuda.synchronize()
+    for i, x in enumerate(xs):
+        msb.msign_ns_host(x, outs[i], workspace=wss[i % 2], stream=streams[i % 2])
+        # the next call on this stream reuses its workspace: stream order keeps
+        # them apart
+    torch.cuda.synchronize()
+    msb.sync_status()
+    for o, r in zip(outs, refs):
+        assert torch.equal(o, r)
+
+
+def test_host_buffers_errors_enqueue_nothing():
+    x = torch.from_numpy(synth.gaussian((128, 256), seed=95)).to(torch.bfloat16).pin_memory()
+    out = torch.full_like(x, 5.0)
+    small = torch.empty(4096, dtype=torch.uint8, device="cuda")
+    with pytest.raises(msb.MsignError):
+        msb.msign_ns_host(x, out, workspace=small)
+    with pytest.raises(ValueError):
+        msb.msign_ns_host(x.cuda())
+    torch.cuda.synchronize()
+    assert bool((out == 5.0).all())
