@@ -346,19 +346,36 @@ __global__ void __launch_bounds__(256, 5) ingest_kernel(const IngestArgs a) {
                       (ld_in & 7) == 0 && (a.ld_op & 7) == 0 && (a.op_bs & 7) == 0 &&
                       (reinterpret_cast<uintptr_t>(src) & 15) == 0 && (reinterpret_cast<uintptr_t>(dop) & 15) == 0;
   if (copy16) {
+    // (up to four pieces, from two rows, loaded before any is stored: the
+    // loads are in flight together, which the compiler cannot arrange across
+    // possibly aliasing stores)
     const int mc = m >> 3;
-    for (int row = blockIdx.x; row < n; row += gridDim.x) {
-      const uint4* srow = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(src) + row * ld_in);
-      uint4* drow = reinterpret_cast<uint4*>(dop + row * a.ld_op);
-      for (int c = tid; c < mc; c += 256) {
-        const uint4 u = srow[c];
-        drow[c] = u;
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    for (int row = blockIdx.x; row < n; row += 2 * gridDim.x) {
+      const bool has2 = row + static_cast<int>(gridDim.x) < n;
+      const int row2 = has2 ? row + static_cast<int>(gridDim.x) : row;
+      const uint4* s0 = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(src) + row * ld_in);
+      const uint4* s1 = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(src) + row2 * ld_in);
+      uint4* d0 = reinterpret_cast<uint4*>(dop + row * a.ld_op);
+      uint4* d1 = reinterpret_cast<uint4*>(dop + row2 * a.ld_op);
+      for (int c = tid; c < mc; c += 512) {
+        const bool two = c + 256 < mc;
+        uint4 u[4];
+        const bool ok[4] = {true, two, has2, has2 && two};
+        u[0] = s0[c];
+        if (ok[1]) u[1] = s0[c + 256];
+        if (ok[2]) u[2] = s1[c];
+        if (ok[3]) u[3] = s1[c + 256];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float lo = __uint_as_float(w[t] << 16), hi = __uint_as_float(w[t] & 0xFFFF0000u);
-          acc = fmaf(lo, lo, acc);
-          acc = fmaf(hi, hi, acc);
+        for (int q = 0; q < 4; ++q) {
+          if (!ok[q]) continue;
+          (q < 2 ? d0 : d1)[c + 256 * (q & 1)] = u[q];
+          const uint32_t w[4] = {u[q].x, u[q].y, u[q].z, u[q].w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float lo = __uint_as_float(w[t] << 16), hi = __uint_as_float(w[t] & 0xFFFF0000u);
+            acc = fmaf(lo, lo, acc);
+            acc = fmaf(hi, hi, acc);
+          }
         }
       }
     }
