@@ -66,6 +66,24 @@ def test_workspace_queries_are_host_only(L):
     # aligned X with m % 8 == 0 needs no staging workspace
     assert L.gram_xxt_workspace_size(1, 100, 64, _lib.BF16, 1 << 20) == 0
     assert L.gram_xxt_workspace_size(1, 100, 63, _lib.BF16, 1 << 20) > 0
+    # host buffers: the device copy of the matrices (256-byte rounded) ahead of msign_ns's workspace
+    for io, es in ((_lib.BF16, 2), (_lib.FP32, 4)):
+        h = L.msign_ns_host_workspace_size(3, 100, 70, io, _lib.BF16)
+        assert h == -(-3 * 100 * 70 * es // 256) * 256 + L.msign_ns_workspace_size(3, 100, 70, _lib.BF16)
+    assert L.msign_ns_host_workspace_size(0, 100, 70, _lib.BF16, _lib.BF16) == 0
+
+
+def test_host_buffer_call_checks_before_any_copy(L):
+    # argument errors of msign_ns_host come back before anything is enqueued
+    # (no device is touched: these run without a GPU)
+    buf = (ctypes.c_uint16 * 16)()
+    p = ctypes.addressof(buf)
+    assert L.msign_ns_host(p, p, 7, _lib.BF16, 1, 4, 4, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.msign_ns_host(p, p, _lib.BF16, _lib.BF16, -1, 4, 4, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.msign_ns_host(None, None, _lib.BF16, _lib.BF16, 0, 4, 4, None, None, 0, None) == _lib.OK
+    assert L.msign_ns_host(None, p, _lib.BF16, _lib.BF16, 1, 4, 4, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.msign_ns_host(p, p, _lib.BF16, _lib.BF16, 65536, 4, 4, None, None, 0, None) == _lib.ERR_UNSUPPORTED
+    assert L.msign_ns_host(p, p, _lib.BF16, _lib.BF16, 1, 4, 4, None, None, 0, None) == _lib.ERR_WORKSPACE
 
 
 def test_invalid_arguments_rejected_on_host(L):
