@@ -16,10 +16,11 @@ from . import _lib
 from ._lib import BF16, FP16, FP32, MsignError, check, make_coeffs
 
 __all__ = [
-    "MsignError", "msign_ns", "msign_ns_workspace_size", "msign_ns_host", "msign_ns_host_workspace_size",
+    "MsignError", "msign_ns", "msign_ns_workspace_size", "msign_ns_route", "msign_ns_host",
+    "msign_ns_host_workspace_size", "msign_ns_noalloc", "msign_ns_noalloc_max_bytes",
     "gram_xxt", "gram_xxt_workspace_size", "gram_ns",
     "gram_ns_workspace_size", "muon_step", "muon_step_workspace_size", "mousse_inv_root", "mousse_direction",
-    "sync_status", "selftest_timeout", "library_path",
+    "sync_status", "selftest_timeout", "set_chaining", "library_path",
 ]
 
 
@@ -201,6 +202,38 @@ def msign_ns_host(x, out=None, *, compute: str = "bf16", coeffs=None, eps=None, 
                                       ctypes.byref(c) if c is not None else None, _ptr(ws), wsb, _stream(stream, dev))
         del keep
     check(st, "msign_ns_host")
+    return out
+
+
+def msign_ns_noalloc_max_bytes() -> int:
+    """Size of the scratch array built into the library (the largest
+    msign_ns_workspace_size() that msign_ns_noalloc accepts)."""
+    return int(_lib.lib().msign_ns_noalloc_max_bytes())
+
+
+def msign_ns_noalloc(x, out, *, coeffs=None, eps=None, improved_init=False, method="standard", stream=None):
+    """msign_ns (bf16 arithmetic) in the library's built-in scratch array: no
+    workspace and no device allocation.  ``x`` and ``out`` are the caller's
+    dense CUDA tensors of one shape and dtype.  Calls on one device share the
+    scratch array: order them on one stream.  Raises MsignError with status
+    ERR_WORKSPACE, before anything is enqueued, when the problem needs more
+    than msign_ns_noalloc_max_bytes() of workspace."""
+    torch = _torch()
+    _need_cuda(x, "x")
+    _need_cuda(out, "out")
+    _same_device(out, x.device, "out")
+    if x.dim() < 2:
+        raise ValueError("x needs at least two dims")
+    if out.shape != x.shape or out.dtype != x.dtype:
+        raise ValueError("out must match x in shape and dtype")
+    rows, cols = x.shape[-2], x.shape[-1]
+    batch = math.prod(x.shape[:-2])
+    c, keep = make_coeffs(coeffs, eps, 1 if improved_init else 0, _METHODS[method])
+    with torch.cuda.device(x.device):
+        st = _lib.lib().msign_ns_noalloc(x.data_ptr(), out.data_ptr(), _dtype_code(x), batch, rows, cols,
+                                         ctypes.byref(c) if c is not None else None, _stream(stream, x.device))
+    del keep
+    check(st, "msign_ns_noalloc")
     return out
 
 

@@ -223,6 +223,17 @@ def test_binding_refuses_cpu_tensors():
         msb.msign_ns(torch.zeros(4, 4))
 
 
+def test_binding_noalloc_checks_on_host():
+    # the no-allocation binding takes the caller's CUDA tensors only, and
+    # reports the built-in scratch size without a GPU
+    import torch
+    import newton_schulz_msign_b200 as msb
+    build.build()
+    assert msb.msign_ns_noalloc_max_bytes() == 32 << 20
+    with pytest.raises(ValueError, match="CUDA"):
+        msb.msign_ns_noalloc(torch.zeros(4, 4), torch.zeros(4, 4))
+
+
 def test_binding_route_query():
     # the Python binding's route query is host-only as well
     import newton_schulz_msign_b200 as msb

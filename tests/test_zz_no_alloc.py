@@ -92,6 +92,22 @@ def test_noalloc_rejects_problems_beyond_the_builtin_scratch():
     assert bool((out == 7.0).all())  # nothing was enqueued
 
 
+def test_noalloc_binding_matches_msign_ns():
+    # the Python binding of the same name: same result, and the size check
+    # raises before anything is enqueued
+    x = torch.from_numpy(synth.gaussian((3, 200, 330), seed=75)).to(torch.float16).cuda()
+    ref = msb.msign_ns(x)
+    out = torch.empty_like(x)
+    torch.cuda.synchronize()
+    assert msb.msign_ns_noalloc(x, out) is out
+    msb.sync_status()
+    assert torch.equal(out, ref)
+    big = torch.zeros(2048, 2048, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(msb.MsignError) as e:
+        msb.msign_ns_noalloc(big, torch.empty_like(big))
+    assert e.value.status == _lib.ERR_WORKSPACE
+
+
 def test_noalloc_follows_the_automatic_route():
     # msign_coeffs.method = 1 through the no-allocation entry point: a shape
     # the route sends to Gram NS fits the built-in scratch too
