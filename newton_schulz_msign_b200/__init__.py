@@ -72,11 +72,13 @@ def _batch_layout(t, name):
     if t.dim() < 2:
         raise ValueError(f"{name} needs at least two dims")
     rows, cols = t.shape[-2], t.shape[-1]
+    if rows * cols == 0:  # empty matrices have no layout to check
+        return math.prod(t.shape[:-2]), rows, cols, 0
     if (cols > 1 and t.stride(-1) != 1) or (rows > 1 and t.stride(-2) != cols):
         raise ValueError(f"{name}: each matrix (the last two dims) must be dense row-major")
     lead = [(t.shape[d], t.stride(d)) for d in range(t.dim() - 2) if t.shape[d] != 1]
     batch = math.prod(sz for sz, _ in lead)
-    if batch <= 1 or rows * cols == 0:
+    if batch <= 1:
         return batch, rows, cols, 0
     stride = lead[-1][1]
     for (sz_o, st_o), (sz_i, st_i) in zip(lead[:-1], lead[1:]):

@@ -300,6 +300,10 @@ def test_binding_batch_layout():
     with pytest.raises(ValueError):
         msb._batch_layout(FakeCuda(big[..., ::2]), "x")  # matrix not dense
     assert msb._batch_layout(FakeCuda(big[0, 0]), "x") == (1, 7, 9, 0)
+    # empty batches and empty matrices pass whatever strides torch gave them
+    assert msb._batch_layout(FakeCuda(torch.empty(0, 64, 96)), "x") == (0, 64, 96, 0)
+    assert msb._batch_layout(FakeCuda(torch.empty(5, 0, 8)), "x") == (5, 0, 8, 0)
+    assert msb._batch_layout(FakeCuda(torch.empty(4, 16, 0)), "x") == (4, 16, 0, 0)
 
 
 def test_mousse_arguments_validated_on_host(L):

@@ -145,6 +145,18 @@ def test_zero_input_gives_zero():
     assert torch.count_nonzero(y).item() == 0
 
 
+def test_empty_inputs_through_every_entry_point():
+    # an empty batch or an empty matrix is a no-op that returns an empty result
+    for shape in ((0, 64, 96), (5, 0, 8), (4, 16, 0)):
+        x = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+        assert msb.msign_ns(x).shape == shape
+        assert msb.msign_ns(x, method="auto").shape == shape
+        assert msb.gram_ns(x).shape == shape
+        assert msb.msign_ns_host(torch.empty(shape, dtype=torch.bfloat16)).shape == shape
+    msb.muon_step([], [], [])
+    msb.sync_status()
+
+
 def test_rank_one_input():
     u = synth.gaussian((200, 1), seed=7)
     v = synth.gaussian((1, 300), seed=8)
