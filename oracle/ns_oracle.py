@@ -20,6 +20,9 @@ Sources (cited by page title and section/equation):
   update (section 1.1), FLOP accounting (sections 1.2, 2.4, 3.4),
   Algorithm 1 (Naive Gram Newton-Schulz, section 2.3), Algorithm 2
   (Stabilized Gram Newton-Schulz, section 3.4), Theorem 1 (section 2.2).
+* [P5] the Mousse post (anti-entrophic.github.io/posts/10054), section
+  "Mousse": the update L^(-1/4) msign(L^(-1/4) G R^(-1/4)) R^(-1/4) with
+  Shampoo-style Kronecker factors L and R.
 
 Conventions (readings of the pages where they leave a step open):
 
@@ -40,8 +43,7 @@ Conventions (readings of the pages where they leave a step open):
 
 Parity pins: every public function here is checked in
 ``tests/test_oracle_*.py`` against closed forms, invariants, special cases
-and the figures the pages print; none is "parity unpinned" except the ones
-whose docstring says so.
+and the figures the pages print; none is "parity unpinned".
 """
 
 from __future__ import annotations
