@@ -207,14 +207,17 @@ size_t msign_ns_workspace_size(int64_t batch, int64_t rows, int64_t cols, msign_
  * With coeffs->method = 1 the call takes Gram NS when all of these hold:
  * 16-bit compute (Gram NS iterates in fp16; the fp32-accurate path stays
  * standard), init = 0 (the sharper normalisation is a standard-NS option),
- * m - n >= 4096 and n >= 512 after orientation (n <= m), and Gram NS's
- * workspace is no larger than msign_ns_workspace_size().  [P3] section 2
- * counts (17 + 3 alpha) n^3 FLOPs for Gram NS against T (3 alpha + 1) n^3
- * for standard NS with symmetric products, alpha = m / n, so Gram NS does
- * less work whenever alpha > 1; measured on a B200, its chain of n x n fp16
- * products pays once m - n reaches about 4096 (e.g. 4096 x 8192, 2048 x 6144,
- * 1024 x 6144), and below n = 512 both are latency-bound.  The two results
- * agree within 2e-2 (relative Frobenius). */
+ * after orientation (n <= m) n >= 512 and m - n >= 3072, or m - n >= 2048
+ * where n <= 2048, and Gram NS's workspace is no larger than
+ * msign_ns_workspace_size() (2048 x 4096 alone is not routed for that
+ * reason).  [P3] section 2 counts (17 + 3 alpha) n^3 FLOPs for Gram NS
+ * against T (3 alpha + 1) n^3 for standard NS with symmetric products,
+ * alpha = m / n, so Gram NS does less work whenever alpha > 1; measured on a
+ * B200, its chain of n x n fp16 products pays from the widths above (e.g.
+ * 0.91 of standard NS's time at 1024 x 4096, 0.98 at 4096 x 7168, 1.04 at
+ * 4096 x 6144), and below n = 512 both are latency-bound.  The two results
+ * agree within 2e-2 (relative Frobenius).  Changed in ABI 106 (before it:
+ * m - n >= 4096 for every n). */
 int msign_ns_route(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute_dtype,
                    const msign_coeffs *coeffs);
 
@@ -339,10 +342,9 @@ msign_status gram_ns(const void *in, void *out, msign_dtype io_dtype,
  *   W_i <- W_i - lr * sqrt(max(1, rows_i / cols_i)) * O_i
  * Matrices of equal (oriented) shape share grouped launches; all shapes in
  * one call are scheduled together.
- * With coeffs->method = 1, a matrix for which msign_ns_route(1, rows_i,
- * cols_i, MSIGN_BF16, coeffs) is 1 runs Gram NS instead, when Gram NS's
- * workspace fits in this matrix's standard-route workspace (4096 x 11008 and
- * 4096 x 14336 do): M_i is updated by its own elementwise pass,
+ * With coeffs->method = 1, a matrix for which muon_step_route(rows_i,
+ * cols_i, coeffs) is 1 runs Gram NS instead (4096 x 11008 and 4096 x 14336
+ * do; 1024 x 4096 does not): M_i is updated by its own elementwise pass,
  * O_i = gram_ns(M_i) (restart after step 2 when T >= 3) is stored in bf16
  * in place of Gram NS's dead copy of X, and W_i is updated from it.
  * Matrices of equal shape (rows, cols) share one batched Gram-NS chain,
@@ -357,6 +359,17 @@ msign_status gram_ns(const void *in, void *out, msign_dtype io_dtype,
  *               the call process the list in several groups.
  * ------------------------------------------------------------------------ */
 size_t muon_step_workspace_size(int num, const int64_t *rows, const int64_t *cols);
+
+/* The iteration muon_step runs for one rows x cols matrix: 0 standard NS,
+ * 1 Gram NS, or a negated status for a schedule muon_step would reject.
+ * Host only.  A matrix takes Gram NS when msign_ns_route(1, rows, cols,
+ * MSIGN_BF16, coeffs) is 1, m - n >= 4096 after orientation, and Gram NS's
+ * workspace with a bf16 O fits in the matrix's standard-route workspace.
+ * The width is larger than msign_ns's because muon_step runs its Gram-NS
+ * matrices after the grouped standard-route launch, where a small matrix
+ * would otherwise share the launch with the large ones (a Llama layer's
+ * 1024 x 4096 k and v stay standard).  Added in ABI 106. */
+int muon_step_route(int64_t rows, int64_t cols, const msign_coeffs *coeffs);
 
 msign_status muon_step(int num, void *const *W, float *const *M, const void *const *G,
                        const int64_t *rows, const int64_t *cols,

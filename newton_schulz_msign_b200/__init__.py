@@ -19,7 +19,8 @@ __all__ = [
     "MsignError", "msign_ns", "msign_ns_workspace_size", "msign_ns_route", "msign_ns_host",
     "msign_ns_host_workspace_size", "msign_ns_noalloc", "msign_ns_noalloc_max_bytes",
     "gram_xxt", "gram_xxt_workspace_size", "gram_ns",
-    "gram_ns_workspace_size", "muon_step", "muon_step_workspace_size", "mousse_inv_root", "mousse_direction",
+    "gram_ns_workspace_size", "muon_step", "muon_step_workspace_size", "muon_step_route", "mousse_inv_root",
+    "mousse_direction",
     "sync_status", "selftest_timeout", "set_chaining", "library_path",
 ]
 
@@ -307,6 +308,16 @@ def _i64_array(vals):
     return (ctypes.c_int64 * len(vals))(*[int(v) for v in vals])
 
 
+def muon_step_route(rows: int, cols: int, *, coeffs=None, improved_init=False, method="auto") -> str:
+    """The iteration ``muon_step`` runs for one rows x cols matrix: "standard" or "gram" (host only)."""
+    c, keep = make_coeffs(coeffs, None, 1 if improved_init else 0, _METHODS[method])
+    r = _lib.lib().muon_step_route(rows, cols, ctypes.byref(c) if c is not None else None)
+    del keep
+    if r < 0:
+        check(-r, "muon_step_route")
+    return "gram" if r == 1 else "standard"
+
+
 def muon_step_workspace_size(shapes) -> int:
     rows = _i64_array([s[0] for s in shapes])
     cols = _i64_array([s[1] for s in shapes])
@@ -317,8 +328,8 @@ def muon_step(weights, momenta, grads, *, momentum: float = 0.95, lr: float = 0.
               improved_init=False, method="standard", workspace=None, stream=None):
     """In-place Muon update of lists of weights (bf16/fp32), fp32 momenta and grads (bf16/fp32).
 
-    ``method="auto"``: matrices the msign route gives to Gram NS take it here too
-    (msign_coeffs.method = 1; see ``msign_ns_route``)."""
+    ``method="auto"``: the matrices ``muon_step_route`` gives to Gram NS take it
+    (msign_coeffs.method = 1)."""
     torch = _torch()
     num = len(weights)
     if not (len(momenta) == num and len(grads) == num):

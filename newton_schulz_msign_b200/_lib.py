@@ -19,7 +19,7 @@ BF16, FP16, FP32 = 0, 1, 2
 
 EXPORTS = (
     "msign_abi_version", "msign_status_string", "msign_sync_status",
-    "msign_ns_workspace_size", "msign_ns", "msign_ns_route",
+    "msign_ns_workspace_size", "msign_ns", "msign_ns_route", "muon_step_route",
     "gram_xxt_workspace_size", "gram_xxt",
     "gram_ns_workspace_size", "gram_ns",
     "muon_step_workspace_size", "muon_step",
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.msign_ns_host.argtypes = [P, P, I32, I32, I64, I64, I64, ctypes.POINTER(MsignCoeffs), P, SZ, P]
         L.msign_ns_route.restype = I32
         L.msign_ns_route.argtypes = [I64, I64, I64, I32, ctypes.POINTER(MsignCoeffs)]
+        L.muon_step_route.restype = I32
+        L.muon_step_route.argtypes = [I64, I64, ctypes.POINTER(MsignCoeffs)]
         L.gram_xxt_workspace_size.restype = SZ
         L.gram_xxt_workspace_size.argtypes = [I64, I64, I64, I32, P]
         L.gram_xxt.restype = I32

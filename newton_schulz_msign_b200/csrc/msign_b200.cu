@@ -1252,30 +1252,47 @@ msign_status ns_run(const void* in, int in_dt, int64_t in_ld, int64_t in_bs, voi
 }
 
 // msign_ns's automatic route (msign_coeffs.method = 1): Gram NS where it is
-// expected to beat standard NS.  Measured on a B200 (default schedules, time
-// of Gram NS over standard NS): 0.86 at 4096 x 8192, 0.71 at 4096 x 14336,
-// 0.91 at 2048 x 6144, 0.92 at 1024 x 6144, 0.75 at 1024 x 16384, 0.92 at
-// 512 x 8192, all with m - n >= 4096; 1.04 at 1024 x 4096, 1.05 at
-// 2048 x 4096, 0.98 at 512 x 4096, 0.99 at 256 x 4096, 1.13 at 256 x 2048,
-// all below it.  Gram NS saves FLOPs in proportion to m - n (it touches the
-// n x m operand only in its first and last products), while its n x n chain
-// costs latency that only large problems hide.  Only shapes whose Gram-NS
-// workspace fits in msign_ns's qualify, so the workspace query stays the
-// same for both routes.
-constexpr int64_t kGramMinExcess = 4096;  // m - n
-constexpr int64_t kGramMinRows = 512;     // n
+// expected to beat standard NS.  Gram NS saves FLOPs in proportion to m - n
+// (it touches the n x m operand only in its first and last products), while
+// its chain of n x n products costs latency that only larger problems hide;
+// at n = 4096 the n x n products fill under two waves of CTA pairs, so the
+// saving must be larger there.  Measured on a B200 (default schedules, L2
+// flushed, median of 20; time of Gram NS over standard NS):
+//   m - n >= 3072:        0.93 at 512 x 3584, 0.91 at 1024 x 4096, 0.87 at
+//                         2048 x 5120, 0.96 at 3072 x 6144, 0.98 at
+//                         4096 x 7168, 0.87 at 6144 x 9216, 0.86 at
+//                         4096 x 8192, 0.71 at 4096 x 14336;
+//   m - n = 2048, n <= 2048: 0.98 at 512 x 2560, 0.94 at 1024 x 3072, 0.95 at
+//                         2048 x 4096 (0.94 for a batch of 4);
+//   below the rule:       1.04 at 4096 x 6144, 1.13 at 4096 x 5120, 0.99 at
+//                         2048 x 3072, 1.09 at 1024 x 2048, 1.08 at
+//                         512 x 1536, 0.99 at 256 x 4096, 1.13 at 256 x 2048.
+// Only shapes whose Gram-NS workspace fits in msign_ns's qualify, so the
+// workspace query stays the same for both routes (2048 x 4096 alone does
+// not fit).
+constexpr int64_t kGramMinRows = 512;          // n
+constexpr int64_t kGramMinExcess = 3072;       // m - n, any n
+constexpr int64_t kGramMinExcessSmall = 2048;  // m - n, n <= kGramSmallRows
+constexpr int64_t kGramSmallRows = 2048;
+// muon_step runs its Gram-NS matrices after the grouped standard-route launch
+// instead of inside it, where a small matrix shares the launch with the large
+// ones: there a matrix takes Gram NS only from m - n >= 4096 (a Llama layer's
+// 1024 x 4096 k and v stay in the group).
+constexpr int64_t kGramMuonMinExcess = 4096;
 
-bool gram_route(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute, const Schedule& sch) {
+bool gram_route(int64_t batch, int64_t rows, int64_t cols, msign_dtype compute, const Schedule& sch,
+                int64_t min_excess = 0) {
   if (sch.method != 1 || compute == MSIGN_FP32 || sch.init != 0) return false;
   if (batch <= 0 || rows <= 0 || cols <= 0) return false;
   const int64_t n = std::min(rows, cols), m = std::max(rows, cols);
-  if (n < kGramMinRows || m - n < kGramMinExcess) return false;
+  const int64_t need = std::max(n <= kGramSmallRows ? kGramMinExcessSmall : kGramMinExcess, min_excess);
+  if (n < kGramMinRows || m - n < need) return false;
   return gram_ns_workspace_size(batch, rows, cols) <= msign_ns_workspace_size(batch, rows, cols, compute);
 }
 
 extern "C" {
 
-int msign_abi_version(void) { return 105; }
+int msign_abi_version(void) { return 106; }
 
 int msign_set_chaining(int enable) { return msb::g_chaining.exchange(enable != 0 ? 1 : 0); }
 
@@ -1687,6 +1704,24 @@ static size_t muon_gram_bytes(int64_t batch, int64_t rows, int64_t cols) {
   return gram_ns_workspace_size(batch, rows, cols);
 }
 
+// muon_step's per-matrix route (msign_coeffs.method = 1): Gram NS for a
+// matrix that msign_ns's route gives to it and whose m - n is at least
+// kGramMuonMinExcess, when Gram NS's workspace (O in bf16 over its dead copy
+// of X) fits in the matrix's standard-route workspace.
+static bool muon_gram_route(int64_t rows, int64_t cols, const Schedule& sch) {
+  if (rows <= 0 || cols <= 0 || !gram_route(1, rows, cols, MSIGN_BF16, sch, kGramMuonMinExcess)) return false;
+  const std::pair<int64_t, int64_t> sh{std::min(rows, cols), std::max(rows, cols)};
+  return muon_gram_bytes(1, rows, cols) <= muon_group_bytes({sh}, {1});
+}
+
+int muon_step_route(int64_t rows, int64_t cols, const msign_coeffs* coeffs) {
+  if (rows < 0 || cols < 0) return -MSIGN_ERR_INVALID_ARG;
+  Schedule sch;
+  const msign_status st = read_schedule(coeffs, kNsEps, &sch);
+  if (st != MSIGN_OK) return -static_cast<int>(st);
+  return muon_gram_route(rows, cols, sch) ? 1 : 0;
+}
+
 size_t muon_step_workspace_size(int num, const int64_t* rows, const int64_t* cols) {
   if (num <= 0 || rows == nullptr || cols == nullptr) return 0;
   std::vector<std::pair<int64_t, int64_t>> shapes;
@@ -1727,18 +1762,14 @@ msign_status muon_step(int num, void* const* W, float* const* M, const void* con
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   const int wd = to_dt(w_dtype), gd = to_dt(g_dtype);
 
-  // msign_coeffs.method = 1: matrices that msign_ns's route would give to
-  // Gram NS take it here too, when Gram NS's workspace and a bf16 O fit in
-  // the standard route's workspace for the same matrix (so the workspace
-  // query is the same for both routes)
+  // msign_coeffs.method = 1: the matrices muon_step_route gives to Gram NS
+  // (the workspace query stays the same for both routes)
   std::vector<char> gram(num, 0);
   Schedule gsch;
   std::vector<int> gbounds;
   if (sch.method == 1) {
     for (int i = 0; i < num; ++i) {
-      if (rows[i] == 0 || cols[i] == 0 || !gram_route(1, rows[i], cols[i], MSIGN_BF16, sch)) continue;
-      const std::pair<int64_t, int64_t> sh{std::min(rows[i], cols[i]), std::max(rows[i], cols[i])};
-      gram[i] = muon_gram_bytes(1, rows[i], cols[i]) <= muon_group_bytes({sh}, {1}) ? 1 : 0;
+      gram[i] = muon_gram_route(rows[i], cols[i], sch) ? 1 : 0;
     }
     gsch.abc = sch.abc;
     gsch.eps = (coeffs != nullptr && coeffs->eps >= 0.0f) ? coeffs->eps : kGramEps;

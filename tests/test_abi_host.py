@@ -45,7 +45,7 @@ def test_exported_symbols_match_nm(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.msign_abi_version() == 105
+    assert L.msign_abi_version() == 106
     assert L.msign_status_string(_lib.OK) == b"ok"
     assert b"timed out" in L.msign_status_string(_lib.ERR_TIMEOUT)
     assert L.msign_status_string(99) == b"unknown status"
@@ -132,8 +132,8 @@ def _route(L, batch, rows, cols, compute=_lib.BF16, method=1, init=0, steps=0):
 
 def test_route_rule(L):
     # the automatic route takes Gram NS only for 16-bit problems with
-    # n >= 512 and m - n >= 4096, in either orientation, whose Gram-NS
-    # workspace fits in msign_ns's
+    # n >= 512 and m - n >= 3072 (>= 2048 where n <= 2048), in either
+    # orientation, whose Gram-NS workspace fits in msign_ns's
     assert _route(L, 1, 1024, 16384) == 1
     assert _route(L, 1, 16384, 1024) == 1
     assert _route(L, 3, 512, 4608) == 1
@@ -141,9 +141,18 @@ def test_route_rule(L):
     assert _route(L, 4, 4096, 11008) == 1
     assert _route(L, 1, 14336, 4096) == 1
     assert _route(L, 1, 1024, 16384, compute=_lib.FP16) == 1
-    assert _route(L, 1, 1024, 5119) == 0    # m - n < 4096
-    assert _route(L, 1, 1024, 4096) == 0
-    assert _route(L, 1, 2048, 4096) == 0
+    assert _route(L, 1, 1024, 4096) == 1
+    assert _route(L, 1, 4096, 1024) == 1
+    assert _route(L, 1, 512, 2560) == 1     # m - n = 2048 at n <= 2048
+    assert _route(L, 4, 2048, 4096) == 1
+    assert _route(L, 1, 3072, 6144) == 1    # m - n = 3072 at n > 2048
+    assert _route(L, 1, 4096, 7168) == 1
+    assert _route(L, 1, 512, 2559) == 0     # m - n < 2048
+    assert _route(L, 1, 1024, 3071) == 0
+    assert _route(L, 1, 4096, 6144) == 0    # m - n < 3072 at n > 2048
+    assert _route(L, 1, 3072, 5119) == 0
+    assert _route(L, 1, 2048, 4096) == 0    # Gram NS's workspace would not fit
+    assert L.gram_ns_workspace_size(1, 2048, 4096) > L.msign_ns_workspace_size(1, 2048, 4096, _lib.BF16)
     assert _route(L, 1, 511, 8192) == 0     # n < 512
     assert _route(L, 1, 4096, 4096) == 0
     assert _route(L, 1, 1024, 16384, compute=_lib.FP32) == 0   # fp32-accurate stays standard
@@ -157,13 +166,38 @@ def test_route_rule(L):
     assert L.msign_ns_route(-1, 4, 4, _lib.BF16, None) == -_lib.ERR_INVALID_ARG
 
 
+def test_muon_route_rule(L):
+    # muon_step takes Gram NS only where msign_ns's route does and m - n >= 4096
+    c = _lib.MsignCoeffs()
+    c.steps, c.abc, c.eps, c.init, c.method = 0, None, -1.0, 0, 1
+    assert L.muon_step_route(4096, 14336, ctypes.byref(c)) == 1
+    assert L.muon_step_route(14336, 4096, ctypes.byref(c)) == 1
+    assert L.muon_step_route(4096, 11008, ctypes.byref(c)) == 1
+    assert L.muon_step_route(600, 5000, ctypes.byref(c)) == 1
+    assert _route(L, 1, 1024, 4096) == 1 and L.muon_step_route(1024, 4096, ctypes.byref(c)) == 0
+    assert L.muon_step_route(4096, 4096, ctypes.byref(c)) == 0
+    assert L.muon_step_route(0, 4096, ctypes.byref(c)) == 0
+    assert L.muon_step_route(4096, 14336, None) == 0  # NULL coeffs: standard
+    c.init = 1
+    assert L.muon_step_route(4096, 14336, ctypes.byref(c)) == 0  # the sharper init is standard-only
+    c.init, c.method = 0, 2
+    assert L.muon_step_route(4096, 14336, ctypes.byref(c)) == -_lib.ERR_INVALID_ARG
+    assert L.muon_step_route(-1, 4, None) == -_lib.ERR_INVALID_ARG
+    # every matrix the Muon route takes is one msign_ns's route takes
+    c.method = 1
+    for n in (256, 512, 1024, 2048, 3072, 4096):
+        for m in (n + 2048, n + 3072, n + 4096, 2 * n, 4 * n):
+            if L.muon_step_route(n, m, ctypes.byref(c)) == 1:
+                assert _route(L, 1, n, m) == 1 and m - n >= 4096
+
+
 def test_route_workspace_fits(L):
     # wherever the route picks Gram NS, its workspace fits in msign_ns's
     # (the one query a caller makes)
     routed = 0
     for batch in (1, 2, 8):
         for n in (512, 640, 1024, 1536, 2048, 3072, 4096, 8192, 16384):
-            for m in (n + 4096, n + 5000, 2 * n, 3 * n, 4 * n, 8 * n, 16 * n):
+            for m in (n + 2048, n + 3072, n + 4096, n + 5000, 2 * n, 3 * n, 4 * n, 8 * n, 16 * n):
                 if _route(L, batch, n, m) == 1:
                     routed += 1
                     assert L.gram_ns_workspace_size(batch, n, m) <= L.msign_ns_workspace_size(batch, n, m, _lib.BF16)
@@ -244,6 +278,9 @@ def test_binding_route_query():
     assert msb.msign_ns_route(1, 1024, 16384, improved_init=True) == "standard"
     assert msb.msign_ns_route(4, 4096, 11008) == "gram"
     assert msb.msign_ns_route(8, 4096, 4096) == "standard"
+    assert msb.muon_step_route(4096, 14336) == "gram"
+    assert msb.muon_step_route(1024, 4096) == "standard"
+    assert msb.muon_step_route(4096, 14336, method="standard") == "standard"
     with pytest.raises(msb.MsignError):
         msb.msign_ns_route(1, 1024, 16384, coeffs=[(1.0, 0.0, 0.0)] * 100)
 

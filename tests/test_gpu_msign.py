@@ -282,9 +282,10 @@ def test_improved_init_full_size():
 
 # ---------------------------------------------------------------- automatic route (msign_coeffs.method = 1)
 
-@pytest.mark.parametrize("shape", [(600, 5000), (5000, 600), (2, 512, 4608)])
+@pytest.mark.parametrize("shape", [(600, 5000), (5000, 600), (2, 512, 4608), (1024, 3072), (2, 2560, 512)])
 def test_auto_route_runs_gram_ns(shape):
-    # wide enough for the route (m - n >= 4096): the call is Gram NS with its defaults
+    # wide enough for the route (m - n >= 3072, or >= 2048 where n <= 2048):
+    # the call is Gram NS with its defaults
     x = torch.from_numpy(synth.gaussian(shape, seed=shape[-1] + 3 * shape[-2])).to(torch.bfloat16).cuda()
     batch = x.numel() // (shape[-2] * shape[-1])
     assert msb.msign_ns_route(batch, shape[-2], shape[-1], method="auto") == "gram"
@@ -318,9 +319,11 @@ def test_auto_route_short_schedule_has_no_restart():
     assert rel_fro(to_np(y), O.gram_ns(to_np(x), coeffs, restart_after=())) < TOL_BF16
 
 
-@pytest.mark.parametrize("shape,compute", [((512, 1024), "bf16"), ((512, 4096), "bf16"), ((1024, 16384), "fp32")])
+@pytest.mark.parametrize("shape,compute", [((512, 1024), "bf16"), ((512, 2048), "bf16"), ((4096, 6144), "bf16"),
+                                           ((2048, 4096), "bf16"), ((1024, 16384), "fp32")])
 def test_auto_route_keeps_standard_ns(shape, compute):
-    # not wide enough, or the fp32-accurate path: the call is standard NS
+    # not wide enough, Gram NS's workspace larger than msign_ns's (2048 x 4096),
+    # or the fp32-accurate path: the call is standard NS
     x = torch.from_numpy(synth.gaussian(shape, seed=41)).to(torch.bfloat16).cuda()
     assert msb.msign_ns_route(1, *shape, compute, method="auto") == "standard"
     a = msb.msign_ns(x, compute=compute, method="auto")

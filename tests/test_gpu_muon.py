@@ -145,12 +145,15 @@ def test_muon_improved_init():
 
 def test_muon_auto_route_mixed():
     # method="auto": the wide matrices (m - n >= 4096, n >= 512) run Gram NS,
-    # the others standard NS, in one call; each against its fp64 oracle
-    shapes = [(600, 5000), (256, 384), (5000, 600), (512, 512)]
+    # the others standard NS, in one call; each against its fp64 oracle.
+    # 1024 x 3072 is one msign_ns's route gives to Gram NS and muon_step's
+    # keeps in the standard group.
+    shapes = [(600, 5000), (256, 384), (5000, 600), (512, 512), (1024, 3072)]
     gram_shapes = {(600, 5000), (5000, 600)}
     for r, c in shapes:
         want = "gram" if (r, c) in gram_shapes else "standard"
-        assert msb.msign_ns_route(1, r, c, method="auto") == want
+        assert msb.muon_step_route(r, c, method="auto") == want
+    assert msb.msign_ns_route(1, 1024, 3072, method="auto") == "gram"
     W, M, G = make(shapes, torch.bfloat16, torch.bfloat16, seed=900)
     W0 = [w.clone() for w in W]
     M0 = [m.clone() for m in M]
@@ -194,6 +197,7 @@ def test_muon_llama_stack_one_step():
     W0 = {i: W[i].clone() for i in picks}
     # the automatic route: q, k, v, o run standard NS, gate, up and down
     # Gram NS (batched by shape), all in one call
+    assert [msb.muon_step_route(r, c) for r, c in layer] == ["standard"] * 4 + ["gram"] * 3
     method = "auto"
     msb.muon_step(W, M, G, momentum=0.95, lr=0.02, method=method)
     msb.sync_status()
@@ -201,7 +205,7 @@ def test_muon_llama_stack_one_step():
         assert torch.isfinite(w).all()
     for i in picks:
         r, c = shapes[i]
-        if method == "auto" and msb.msign_ns_route(1, r, c, method="auto") == "gram":
+        if method == "auto" and msb.muon_step_route(r, c, method="auto") == "gram":
             # Gram NS (fp16 inside) on the momentum M = G; the update against
             # its own oracle and within the acceptance bound of standard NS
             o_ref = O.gram_ns(to_np(M[i]))
