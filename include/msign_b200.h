@@ -19,6 +19,9 @@
  *        (section 3.4) with its restart (section 3.2), fp16 arithmetic
  *        (section 3.3), and the fused symmetric kernel C <- aAB + bC + gI
  *        (section 4).
+ *   [P5] the Mousse post (anti-entrophic.github.io/posts/10054), section
+ *        "Mousse": L^(-1/4) msign(L^(-1/4) G R^(-1/4)) R^(-1/4) with
+ *        Shampoo-style Kronecker factors L and R.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -41,7 +44,8 @@
  *   reports it as MSIGN_ERR_TIMEOUT.
  * - Coefficient schedules are HOST arrays.  NULL selects Jordan's triple
  *   for T = 5 steps ([P2] eq. 7).
- * - Empty problems (batch, rows or cols = 0) are valid and do nothing.
+ * - Empty problems (batch, rows or cols = 0) are valid and do nothing,
+ *   except gram_xxt with m = 0 and n > 0, which writes the zero n x n result.
  * - Size limits: batch <= 65535 and every matrix dimension <= 2^30
  *   (mousse_inv_root: n <= 2^20); beyond them an entry point returns
  *   MSIGN_ERR_UNSUPPORTED before enqueuing anything.
