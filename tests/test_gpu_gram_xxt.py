@@ -34,6 +34,22 @@ def test_gram_xxt_fp32_out_matches_oracle(n, m, dt):
     assert torch.equal(A, A.transpose(-1, -2))
 
 
+@pytest.mark.parametrize("n,m", [(8, 200000), (300, 70000)])
+def test_gram_xxt_long_inner_dimension(n, m):
+    # few tiles over a very long K: the product splits along K and the last
+    # part adds the fp32 partials.  The tensor cores' fp32 accumulation
+    # truncates instead of rounding, so a sum of m positive products (the
+    # diagonal) drifts low by up to about 2^-22 of the running sum per
+    # 16-wide MMA step: the bound is (m / 16) * 2^-22, 3e-3 at m = 200000
+    # (measured 9.4e-4 there, every diagonal entry below the fp64 value)
+    x = _x(n, m, "bf16", seed=n + m)
+    A = msb.gram_xxt(x, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref = O.gram_xxt(to_np(x))
+    assert rel_fro(to_np(A), ref) < (m / 16) * 2.0 ** -22
+    assert torch.equal(A, A.transpose(-1, -2))
+
+
 @pytest.mark.parametrize("n,m", [(256, 512), (384, 128), (100, 300), (7, 129)])
 @pytest.mark.parametrize("dt", ["bf16", "fp16"])
 def test_gram_xxt_same_dtype_out(n, m, dt):

@@ -39,7 +39,8 @@ def test_gaussian_256x512_fp32_in():
 
 
 @pytest.mark.parametrize("shape", [(64, 64), (128, 384), (384, 128), (100, 300), (300, 100), (1, 64), (64, 1),
-                                   (7, 129), (129, 7), (33, 257), (256, 2048), (520, 600), (1000, 1000)])
+                                   (7, 129), (129, 7), (33, 257), (256, 2048), (520, 600), (1000, 1000),
+                                   (1, 1), (2, 3), (3, 40000), (40000, 3)])
 def test_shapes(shape):
     x = synth.gaussian(shape, seed=shape[0] * 131 + shape[1])
     got, ref = run_case(x)
